@@ -1,0 +1,457 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 DashAttention forward pass (prefill + decode), one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 16k|32k|96k] [--no-decode]
+    python bench.py --impl reference ...      # the fp64 CPU oracle timed on this host
+
+A step is one full prefill (block summaries, coarse scores + alpha-entmax thresholds +
+block lists, prior-weighted fine attention) of the workload (default: the 16K prefill
+at 75 % block sparsity).  `value` is prefill tokens/s over all ranks with inputs resident
+in HBM; `e2e` is the same through the C ABI's host-buffer entry point (host<->device
+copies inside the timed region).  The `decode` object times one decode step of the 96K
+workload (B=8, cache 98304) the same way.  L2 is flushed (256 MiB write) before every
+timed step; times are CUDA events on the launching stream, max over ranks.
+
+Multi-GPU: one process per GPU (torchrun), every rank runs its own replica of the
+workload (work units are independent: weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill tok/s & decode tok/s at 16K–96K ctx; % of BF16 TC / HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def calibrated(name):
+    with open(os.path.join(ROOT, "tests", "golden", "coarse_scale.json")) as f:
+        return json.load(f)[name]
+
+
+def source_sha(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "sparse_hierarchical_attention_pool_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, sha):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel is unchanged since."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f).get(kernel)
+    if not d or d.get("source_sha256_16") != sha:
+        return None
+    return d.get("traffic_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms during a timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import torch
+        ident = str(self.dev)
+        try:
+            ident = str(torch.cuda.get_device_properties(self.dev).uuid)
+            if not ident.startswith("GPU-"):
+                ident = "GPU-" + ident
+        except Exception:
+            pass
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={ident}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = sorted(float(r[1]) for r in rows if r[1].replace(".", "").isdigit())
+        mx = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if _num(r[3]))}
+
+
+def _num(s):
+    try:
+        float(s)
+        return True
+    except ValueError:
+        return False
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_setup(n_gpus):
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(ws, x):
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ GPU arms
+
+def bench_prefill(args, ws, rank, local):
+    import torch
+    from sparse_hierarchical_attention_pool_b200 import dash_attn as da
+    from sparse_hierarchical_attention_pool_b200 import inputs
+
+    wl, (q, k, v) = inputs.make(args.workload)
+    cal = calibrated(args.workload)
+    cs, alpha = cal["coarse_scale"], wl.alpha
+    B, Hq, Hkv, T, d = wl.B, wl.Hq, wl.Hkv, wl.T, wl.d
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    out = torch.empty_like(qd)
+    wsb = da.alloc_workspace(da.prefill_workspace_size(B, Hq, Hkv, T, d))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup):
+        flush.zero_()
+        da.dash_prefill(qd, kd, vd, out, alpha, cs, wsb)
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.3)
+    evs = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        da.dash_prefill_profiled(qd, kd, vd, out, alpha, cs, wsb, e)
+        evs.append(e)
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    clocks = clk.stop()
+    tot = [e[0].elapsed_time(e[3]) for e in evs]
+    summ = [e[0].elapsed_time(e[1]) for e in evs]
+    coarse = [e[1].elapsed_time(e[2]) for e in evs]
+    fine = [e[2].elapsed_time(e[3]) for e in evs]
+    mean = lambda xs: sum(xs) / len(xs)  # noqa: E731
+    step_ms = max_over_ranks(ws, mean(tot))
+    st = da.dash_prefill_stats(wsb)
+    if da.dash_get_device_status(wsb) != 0:
+        raise RuntimeError("device status not clean after the timed prefill")
+
+    # algorithmic work: fine FLOPs = 4 d * sum_rows |L_row|; coarse FLOPs = 2 d * sum_rows bt
+    diag_tokens = sum((t % 64) + 1 for t in range(T)) * B * Hq
+    fine_alg = 4.0 * d * (64.0 * st["selected_pairs"] + diag_tokens)
+    coarse_alg = 2.0 * d * st["scored_pairs"]
+    P = min(64, 1 << (max(1, 128 // (Hq // Hkv)).bit_length() - 1))
+    ntiles = B * Hkv * ((T + P - 1) // P)
+    fine_exec = 4.0 * d * 64.0 * 128.0 * (st["union_blocks"] + ntiles)
+    pk, pk_kind = peaks()
+    peak = pk["bf16_tflops"]
+    fine_ms = mean(fine)
+    achieved = fine_alg / (fine_ms * 1e-3) / 1e12
+    traffic = recorded_traffic("fine_mma_kernel", source_sha("fine_mma.cu", "common.cuh"))
+    res = {
+        "step_ms": step_ms,
+        "tok_s": ws * B * T / (step_ms * 1e-3),
+        "stage_ms": {"block_summary": mean(summ), "coarse_select": mean(coarse), "fine_attention": fine_ms},
+        "clocks": clocks,
+        "stats": st,
+        "sparsity": 1.0 - st["selected_pairs"] / max(1, st["scored_pairs"]),
+        "roofline": {"bound": "tensor", "kernel": "fine_mma_kernel", "achieved": round(achieved, 2),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": traffic, "peak_source": f"{pk_kind} bf16_tflops (burst)",
+                     "algorithmic_flops_per_launch": fine_alg,
+                     "executed_flops_per_launch": fine_exec,
+                     "executed_tflops": round(fine_exec / (fine_ms * 1e-3) / 1e12, 2),
+                     "executed_frac": round(fine_exec / (fine_ms * 1e-3) / 1e12 / peak, 4),
+                     "inflation": round(fine_exec / fine_alg, 3)},
+        "coarse_algorithmic_flops": coarse_alg,
+        "launches_per_step": 3,
+        "wl": wl, "cs": cs,
+    }
+    # end-to-end through the host-buffer entry point
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = torch.empty_like(q).pin_memory()
+    for _ in range(2):
+        da.dash_prefill_host(qh, kh, vh, oh, qd, kd, vd, out, alpha, cs, wsb)
+    torch.cuda.synchronize()
+    barrier(ws)
+    e2e_ms = []
+    ne2e = max(3, min(args.steps, 20))
+    for _ in range(ne2e):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        da.dash_prefill_host(qh, kh, vh, oh, qd, kd, vd, out, alpha, cs, wsb)
+        e1.record()
+        e2e_ms.append((e0, e1))
+    torch.cuda.synchronize()
+    e2e_step = max_over_ranks(ws, mean([a.elapsed_time(b) for a, b in e2e_ms]))
+    res["e2e"] = {"value": ws * B * T / (e2e_step * 1e-3), "unit": "tok/s",
+                  "h2d_bytes_per_step": q.numel() * 2 + k.numel() * 2 + v.numel() * 2,
+                  "d2h_bytes_per_step": q.numel() * 2, "ms_per_step": e2e_step}
+    del flush, wsb
+    return res
+
+
+def bench_decode(args, ws, rank, local):
+    import torch
+    from sparse_hierarchical_attention_pool_b200 import dash_attn as da
+    from sparse_hierarchical_attention_pool_b200 import inputs
+
+    wl, (q, kc, vc, kv_len) = inputs.make("decode96k")
+    cs = calibrated("decode96k")["coarse_scale"]
+    B, Hq, Hkv, T, d = wl.B, wl.Hq, wl.Hkv, wl.T, wl.d
+    qd, kcd, vcd, lens = q.cuda(), kc.cuda(), vc.cuda(), kv_len.cuda()
+    del kc, vc
+    ksum = da.dash_block_summary(kcd)
+    out = torch.empty_like(qd)
+    wsb = da.alloc_workspace(da.decode_workspace_size(B, Hq, Hkv, T, d))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        da.dash_decode(qd, kcd, vcd, ksum, lens, out, wl.alpha, cs, wsb)
+    torch.cuda.synchronize()
+    barrier(ws)
+    steps = max(args.steps, 20)
+    evs = []
+    for _ in range(steps):
+        flush.zero_()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        da.dash_decode_profiled(qd, kcd, vcd, ksum, lens, out, wl.alpha, cs, wsb, e)
+        evs.append(e)
+    torch.cuda.synchronize()
+    barrier(ws)
+    mean = lambda xs: sum(xs) / len(xs)  # noqa: E731
+    tot = max_over_ranks(ws, mean([e[0].elapsed_time(e[4]) for e in evs]))
+    st_ms = [mean([e[i].elapsed_time(e[i + 1]) for e in evs]) for i in range(4)]
+    st = da.dash_decode_stats(wsb)
+    if da.dash_get_device_status(wsb) != 0:
+        raise RuntimeError("device status not clean after the timed decode")
+    blk_bytes = 64 * d * 2 * 2
+    gathered = (st["union_blocks"] + B * Hkv) * blk_bytes
+    other = B * Hkv * (T // 64) * d * 4 + 2 * B * Hq * d * 2
+    pk, pk_kind = peaks()
+    attn_gbs = gathered / (st_ms[2] * 1e-3) / 1e9
+    step_gbs = (gathered + other) / (tot * 1e-3) / 1e9
+    traffic = recorded_traffic("decode_attn_kernel", source_sha("decode.cu", "common.cuh"))
+    # end to end: the new query goes up, the output comes back (the cache stays resident)
+    qh, oh = q.pin_memory(), torch.empty_like(q).pin_memory()
+    e2e = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        qd.copy_(qh, non_blocking=True)
+        da.dash_decode(qd, kcd, vcd, ksum, lens, out, wl.alpha, cs, wsb)
+        oh.copy_(out, non_blocking=True)
+        e1.record()
+        e2e.append((e0, e1))
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(ws, mean([a.elapsed_time(b) for a, b in e2e]))
+    return {
+        "workload": wl.name, "coarse_scale": cs, "seed": wl.seed,
+        "value": ws * B / (tot * 1e-3), "unit": "tok/s", "ms_per_step": tot,
+        "stage_ms": dict(zip(["scores", "select", "attention", "combine"], st_ms)),
+        "sparsity": 1.0 - st["selected_pairs"] / max(1, st["scored_pairs"]),
+        "union_blocks_per_group": st["union_blocks"] / (B * Hkv),
+        "roofline": {"bound": "hbm", "kernel": "decode_attn_kernel", "achieved": round(attn_gbs, 1),
+                     "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(attn_gbs / pk["hbm_gbs"], 4),
+                     "traffic": traffic, "peak_source": f"{pk_kind} hbm_gbs",
+                     "algorithmic_bytes_per_launch": gathered,
+                     "step_bytes": gathered + other, "step_frac": round(step_gbs / pk["hbm_gbs"], 4)},
+        "e2e": {"value": ws * B / (e2e_ms * 1e-3), "unit": "tok/s", "h2d_bytes_per_step": q.numel() * 2,
+                "d2h_bytes_per_step": q.numel() * 2},
+        "launches_per_step": 4,
+        "stats": st,
+    }
+
+
+# ------------------------------------------------------------------ CPU oracle (baseline / reference arm)
+
+def oracle_rows_per_s(workload, n_rows, seed, tensors=None):
+    """Time the fp64 oracle on n_rows random rows of the workload; returns (rows/s, cores, wl)."""
+    import oracle
+    from sparse_hierarchical_attention_pool_b200 import inputs
+    oracle.build()
+    if tensors is None:
+        wl, (q, k, v) = inputs.make(workload)
+    else:
+        wl, (q, k, v) = tensors
+    cs = calibrated(workload)["coarse_scale"]
+    rows = inputs.sample_rows(wl.B, wl.Hq, wl.T, n_rows, seed)
+    qr = oracle.gather_q_rows(q, rows)
+    t0 = time.perf_counter()
+    oracle.forward_rows(qr, k, v, rows, wl.Hq, 64, wl.alpha, cs)
+    dt = time.perf_counter() - t0
+    return n_rows / dt, os.cpu_count(), wl, dt
+
+
+def cpu_baseline(args):
+    from sparse_hierarchical_attention_pool_b200 import inputs
+    tensors = inputs.make(args.workload)
+    r, cores, wl, dt = oracle_rows_per_s(args.workload, 64, 1, tensors)
+    n = int(max(64, min(20000, r * 10.0)))            # about 10 s of oracle work
+    r, cores, wl, dt = oracle_rows_per_s(args.workload, n, 2, tensors)
+    return {"value": r / wl.Hq, "unit": "tok/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} uniformly drawn rows (b, h, t) of the {wl.name} workload, fp64 C oracle "
+                      f"with OpenMP over rows, {dt:.1f} s; tok/s = rows/s / Hq (extrapolated)"}
+
+
+def run_reference(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from sparse_hierarchical_attention_pool_b200 import inputs
+    tensors = inputs.make(args.workload)
+    wl = tensors[0]
+    r, cores, _, _ = oracle_rows_per_s(args.workload, 32, 1, tensors)
+    n = int(max(16, min(5000, r * 2.0)))               # about 2 s per step
+    for i in range(args.warmup):
+        oracle_rows_per_s(args.workload, max(8, n // 4), 100 + i, tensors)
+    times = []
+    for i in range(args.steps):
+        rr, cores, _, dt = oracle_rows_per_s(args.workload, n, 200 + i, tensors)
+        times.append(dt)
+    step_s = sum(times) / len(times)
+    value = n / step_s / wl.Hq
+    line = {"metric": METRIC, "value": value, "unit": "tok/s", "impl": "reference", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "T": wl.T, "d": wl.d,
+                       "block": wl.block, "alpha": wl.alpha, "coarse_scale": calibrated(args.workload)["coarse_scale"],
+                       "seed": wl.seed},
+            "cpu_baseline": {"value": value, "unit": "tok/s", "cores": cores, "kind": "oracle",
+                             "sample": f"each step: {n} uniformly drawn rows of the workload (fp64 C oracle, "
+                                       "OpenMP over rows); tok/s = rows/s / Hq (extrapolated)"},
+            "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="16k", choices=["16k", "32k", "96k"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+    ws, rank, local = dist_setup(args.gpus)
+    from sparse_hierarchical_attention_pool_b200 import build as _b
+    if rank == 0:
+        _b.build()
+    barrier(ws)
+    pre = bench_prefill(args, ws, rank, local)
+    dec = None if args.no_decode else bench_decode(args, ws, rank, local)
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args)
+    if rank == 0:
+        wl = pre["wl"]
+        line = {
+            "metric": METRIC, "value": pre["tok_s"], "unit": "tok/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": pre["step_ms"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "T": wl.T, "d": wl.d,
+                       "block": wl.block, "alpha": wl.alpha, "coarse_scale": pre["cs"], "seed": wl.seed,
+                       "realised_sparsity": round(pre["sparsity"], 5),
+                       "l2": "flushed before every timed step (256 MiB write, outside the step's events)",
+                       "parallelism": f"independent replica per GPU x{ws}"},
+            "roofline": pre["roofline"],
+            "e2e": pre["e2e"],
+            "cpu_baseline": cpu,
+            "clocks": pre["clocks"],
+            "gpu_launches": pre["launches_per_step"] * args.steps,
+            "stage_ms": pre["stage_ms"],
+            "prefill_stats": pre["stats"],
+            "decode": dec,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        barrier(ws)
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

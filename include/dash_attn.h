@@ -1,0 +1,196 @@
+/*
+ * dash_attn.h -- C ABI of the B200 (sm_100a) DashAttention forward pass.
+ *
+ * DashAttention (pages: "DashAttention: Making Sparse Attention Fully Differentiable with
+ * Adaptive Block Selection", sections "Core Mechanism" and "Key Concepts"; "DashAttention
+ * and the year sparse attention became a field", section "What alpha-entmax changes"):
+ *   Stage 0  keys are split into blocks of `block` tokens and mean-pooled into summaries
+ *            kbar_j (a zero-initialised learned summary head is exactly mean pooling);
+ *   Stage 1  per query head, coarse scores s_j = coarse_scale * (q . kbar_j) / sqrt(d) over
+ *            the complete blocks strictly before the query's own block; alpha-entmax
+ *            p_j = [(alpha-1) s_j - tau]_+^(1/(alpha-1)), tau chosen so that sum_j p_j = 1,
+ *            gives a sparse, variable-size block set;
+ *   Stage 2  softmax attention over the tokens of the selected blocks plus the query's own
+ *            block (causal, prior weight 1), with logits (q . k_i)/sqrt(d) + log p_block(i).
+ * Query head h reads KV head h / (Hq / Hkv).
+ *
+ * Conventions for every entry point:
+ *   - q, k, v, out, caches are bf16, row-major, last dimension d contiguous:
+ *       q, out [B, Hq, T, d];  k, v [B, Hkv, T, d];  caches [B, Hkv, Tmax, d].
+ *     Every tensor pointer must be 16-byte aligned.
+ *   - All pointers are DEVICE pointers owned by the caller unless stated otherwise.  The
+ *     library allocates no memory and keeps no state between calls; scratch lives in a
+ *     caller-provided workspace whose size the *_workspace_size functions return.
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream).  Argument errors
+ *     are returned at once and nothing is launched.  Calls that use the same workspace
+ *     concurrently race.
+ *   - Supported: d in {64, 128}; block == 64; Hq % Hkv == 0 and Hq / Hkv <= 128;
+ *     1 <= T <= 1048576; alpha > 1 and finite; coarse_scale finite.
+ *   - Device-side conditions (a threshold solve that hit its iteration cap) set a status
+ *     word inside the workspace; dash_get_device_status reads it.
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef DASH_ATTN_H
+#define DASH_ATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define DASH_API __attribute__((visibility("default")))
+#else
+#define DASH_API
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* dash_stream_t;   /* same handle as cudaStream_t */
+
+typedef enum {
+    DASH_OK = 0,
+    DASH_ERR_ARG = -1,           /* null / misaligned pointer, bad alpha or scale */
+    DASH_ERR_SHAPE = -2,         /* unsupported B, H, T, d or block */
+    DASH_ERR_DTYPE = -3,         /* reserved: every tensor is bf16 */
+    DASH_ERR_UNSUPPORTED = -4,   /* valid request the library does not implement */
+    DASH_ERR_WORKSPACE = -5,     /* workspace null, misaligned (256 B) or too small */
+    DASH_ERR_CUDA = -6,          /* a CUDA runtime call failed (launch, copy) */
+    DASH_ERR_NO_CONVERGE = -7    /* device status: a tau solve hit its iteration cap */
+} dash_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+DASH_API const char* dash_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+DASH_API int dash_version(void);
+
+/*
+ * Stage 0 (block summaries).  ksum[b, g, j, :] = mean of k[b, g, j*block : (j+1)*block, :]
+ * for every COMPLETE block j < T / block, accumulated and stored in fp32.
+ *   k     device bf16 [B, Hkv, T, d]
+ *   ksum  device fp32 [B, Hkv, T / block, d]   (nothing is written when T < block)
+ * Decode callers keep ksum for their KV cache by calling this on the cache (T = Tmax) or
+ * on each block as it fills.
+ */
+DASH_API int dash_block_summary(const void* k, float* ksum, int B, int Hkv, int T, int d, int block,
+                       dash_stream_t stream);
+
+/* Bytes of workspace dash_prefill needs (0 when the shape is unsupported). */
+DASH_API size_t dash_prefill_workspace_size(int B, int Hq, int Hkv, int T, int d, int block);
+
+/*
+ * Full causal prefill: Stages 0-2 for every query row (b, h, t), t in [0, T).
+ *   q [B,Hq,T,d], k, v [B,Hkv,T,d] -> out [B,Hq,T,d], all device bf16.
+ *   alpha > 1 (1.5 is the pages' inference value); coarse_scale multiplies the coarse
+ *   scores only (fine logits always use 1/sqrt(d)).
+ *   workspace: device, 256-byte aligned, >= dash_prefill_workspace_size(...) bytes.  It
+ *   holds the block summaries, per-row thresholds, per-tile block lists and counters of
+ *   this call until the next call that uses it.
+ * Rows in block 0 have no past blocks and attend causally to their own block only.
+ */
+DASH_API int dash_prefill(const void* q, const void* k, const void* v, void* out,
+                 int B, int Hq, int Hkv, int T, int d, int block,
+                 float alpha, float coarse_scale,
+                 void* workspace, size_t ws_bytes, dash_stream_t stream);
+
+/*
+ * dash_prefill with HOST inputs and output: copies q, k, v from host memory into the
+ * caller's device buffers, runs dash_prefill, copies out back to host memory, all
+ * asynchronously on `stream` (host buffers should be pinned for the copies to overlap).
+ * Host pointers: q_host, k_host, v_host (read), out_host (written).  Device pointers:
+ * q_dev, k_dev, v_dev, out_dev (same shapes as dash_prefill) and the workspace.
+ */
+DASH_API int dash_prefill_host(const void* q_host, const void* k_host, const void* v_host, void* out_host,
+                      void* q_dev, void* k_dev, void* v_dev, void* out_dev,
+                      int B, int Hq, int Hkv, int T, int d, int block,
+                      float alpha, float coarse_scale,
+                      void* workspace, size_t ws_bytes, dash_stream_t stream);
+
+/*
+ * dash_prefill that also records four caller-created CUDA events on `stream`:
+ * events[0] before the block-summary kernel, events[1] before the coarse (Stage 1) kernel,
+ * events[2] before the fine (Stage 2) kernel and events[3] after it.  `events` is a host
+ * array of cudaEvent_t handles; the elapsed times between them are the per-kernel times.
+ */
+DASH_API int dash_prefill_profiled(const void* q, const void* k, const void* v, void* out,
+                                   int B, int Hq, int Hkv, int T, int d, int block,
+                                   float alpha, float coarse_scale,
+                                   void* workspace, size_t ws_bytes, dash_stream_t stream,
+                                   void* const* events);
+
+/* Counters the last dash_prefill or dash_decode wrote into its workspace. */
+typedef struct {
+    long long scored_pairs;    /* sum over rows of the number of scored past blocks */
+    long long selected_pairs;  /* sum over rows of #{j : p_j > 0} */
+    long long union_blocks;    /* sum over work tiles of the union of their rows' blocks */
+    long long tiles;           /* work tiles with at least one past block */
+    int status;                /* device status bits (0 = clean) */
+} dash_stats;
+
+/* Synchronises `stream`, then copies the counters out of `workspace` into *out (host). */
+DASH_API int dash_prefill_stats(const void* workspace, size_t ws_bytes, dash_stats* out, dash_stream_t stream);
+DASH_API int dash_decode_stats(const void* workspace, size_t ws_bytes, dash_stats* out, dash_stream_t stream);
+
+/*
+ * Per-row thresholds the last dash_prefill computed: tau_out[b, h, t] (device fp32,
+ * [B, Hq, T]) in the (alpha-1)*s space of the entmax formula.  Rows in block 0 get NaN.
+ * Same shape arguments as the dash_prefill call that filled the workspace.
+ */
+DASH_API int dash_prefill_tau(const void* workspace, size_t ws_bytes, float* tau_out,
+                     int B, int Hq, int Hkv, int T, int d, int block, dash_stream_t stream);
+
+/*
+ * Block-weight dump (parity hook for Stage 1).  For each listed row (b, h, t):
+ *   rows      device int64 [nrows, 3]
+ *   ksum      device fp32 [B, Hkv, T / block, d]  (from dash_block_summary)
+ *   out_idx   device int32 [nrows, max_sel]  selected past blocks, ascending
+ *   out_p     device fp32  [nrows, max_sel]  their entmax weights
+ *   out_count device int32 [nrows]           full support size (may exceed max_sel;
+ *                                            only the first max_sel entries are written)
+ *   out_tau   device fp32  [nrows]           threshold (NaN when t < block)
+ * Uses the same score arithmetic and threshold solver as dash_prefill.
+ */
+DASH_API int dash_select_dump(const void* q, const float* ksum, const long long* rows, int nrows, int max_sel,
+                     int* out_idx, float* out_p, int* out_count, float* out_tau,
+                     int B, int Hq, int Hkv, int T, int d, int block,
+                     float alpha, float coarse_scale, dash_stream_t stream);
+
+/* Bytes of workspace dash_decode needs (0 when the shape is unsupported). */
+DASH_API size_t dash_decode_workspace_size(int B, int Hq, int Hkv, int Tmax, int d, int block);
+
+/*
+ * One decode step: for each sequence b the new token's K/V are already in the cache at
+ * position kv_len[b] - 1, and the query attends exactly as row t = kv_len[b] - 1 of a
+ * prefill over the first kv_len[b] cache entries would.
+ *   q        device bf16 [B, Hq, d]
+ *   k_cache, v_cache  device bf16 [B, Hkv, Tmax, d]
+ *   ksum     device fp32 [B, Hkv, Tmax / block, d]; blocks j < (kv_len[b]-1)/block must
+ *            hold the summaries of the cache (dash_block_summary)
+ *   kv_len   device int32 [B], 1 <= kv_len[b] <= Tmax (rows outside the range output 0
+ *            and set no status)
+ *   out      device bf16 [B, Hq, d]
+ */
+DASH_API int dash_decode(const void* q, const void* k_cache, const void* v_cache, const float* ksum,
+                const int* kv_len, void* out, int B, int Hq, int Hkv, int Tmax, int d, int block,
+                float alpha, float coarse_scale, void* workspace, size_t ws_bytes,
+                dash_stream_t stream);
+
+/*
+ * dash_decode that also records five caller-created CUDA events on `stream`: before the
+ * score, select, attention and combine kernels, and after the combine kernel.
+ */
+DASH_API int dash_decode_profiled(const void* q, const void* k_cache, const void* v_cache, const float* ksum,
+                                  const int* kv_len, void* out, int B, int Hq, int Hkv, int Tmax, int d,
+                                  int block, float alpha, float coarse_scale, void* workspace,
+                                  size_t ws_bytes, dash_stream_t stream, void* const* events);
+
+/* Synchronises `stream` and returns DASH_OK, or DASH_ERR_NO_CONVERGE when a kernel that
+ * used `workspace` recorded a failed threshold solve, or DASH_ERR_CUDA. */
+DASH_API int dash_get_device_status(const void* workspace, dash_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DASH_ATTN_H */

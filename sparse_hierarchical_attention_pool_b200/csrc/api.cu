@@ -1,0 +1,212 @@
+// api.cu -- the extern "C" entry points declared in include/dash_attn.h.
+//
+// Argument checks happen here, before any launch; kernels live in summary.cu, coarse.cu,
+// fine_mma.cu, decode.cu and dump.cu.  Nothing here allocates memory.
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/dash_attn.h"
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace dash;
+
+namespace {
+
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool al256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+inline cudaStream_t S(dash_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+inline bool good_params(float alpha, float cs) {
+    return isfinite(alpha) && alpha > 1.0f && isfinite(cs);
+}
+
+int read_stats(const void* ws, size_t ws_bytes, dash_stats* out, dash_stream_t stream) {
+    if (!ws || !out || ws_bytes < sizeof(WsHeader)) return DASH_ERR_ARG;
+    if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return DASH_ERR_CUDA;
+    WsHeader h;
+    if (cudaMemcpy(&h, ws, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess) return DASH_ERR_CUDA;
+    out->scored_pairs = (long long)h.scored_pairs;
+    out->selected_pairs = (long long)h.selected_pairs;
+    out->union_blocks = (long long)h.union_blocks;
+    out->tiles = (long long)h.tiles;
+    out->status = h.status;
+    return DASH_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dash_status_string(int status) {
+    switch (status) {
+        case DASH_OK: return "DASH_OK";
+        case DASH_ERR_ARG: return "DASH_ERR_ARG: null or misaligned pointer, or bad alpha / coarse_scale";
+        case DASH_ERR_SHAPE: return "DASH_ERR_SHAPE: unsupported B, H, T, d or block";
+        case DASH_ERR_DTYPE: return "DASH_ERR_DTYPE";
+        case DASH_ERR_UNSUPPORTED: return "DASH_ERR_UNSUPPORTED";
+        case DASH_ERR_WORKSPACE: return "DASH_ERR_WORKSPACE: workspace null, misaligned or too small";
+        case DASH_ERR_CUDA: return "DASH_ERR_CUDA: a CUDA runtime call failed";
+        case DASH_ERR_NO_CONVERGE: return "DASH_ERR_NO_CONVERGE: a threshold solve hit its iteration cap";
+        default: return "unknown dash status";
+    }
+}
+
+int dash_version(void) { return 100; }
+
+int dash_block_summary(const void* k, float* ksum, int B, int Hkv, int T, int d, int block,
+                       dash_stream_t stream) {
+    if (!k || !ksum || !al16(k) || !al16(ksum)) return DASH_ERR_ARG;
+    if (block != kBlock || (d != 64 && d != 128) || B < 1 || Hkv < 1 || T < 1 || T > kMaxT)
+        return DASH_ERR_SHAPE;
+    return launch_block_summary(k, ksum, B, Hkv, T, d, S(stream)) == cudaSuccess ? DASH_OK : DASH_ERR_CUDA;
+}
+
+size_t dash_prefill_workspace_size(int B, int Hq, int Hkv, int T, int d, int block) {
+    PrefillGeom g;
+    if (block != kBlock || !make_prefill_geom(B, Hq, Hkv, T, d, &g)) return 0;
+    return g.total;
+}
+
+static int prefill_impl(const void* q, const void* k, const void* v, void* out, int B, int Hq,
+                        int Hkv, int T, int d, int block, float alpha, float coarse_scale,
+                        void* workspace, size_t ws_bytes, dash_stream_t stream, void* const* events) {
+    if (!q || !k || !v || !out || !al16(q) || !al16(k) || !al16(v) || !al16(out)) return DASH_ERR_ARG;
+    if (!good_params(alpha, coarse_scale)) return DASH_ERR_ARG;
+    PrefillGeom g;
+    if (block != kBlock || !make_prefill_geom(B, Hq, Hkv, T, d, &g)) return DASH_ERR_SHAPE;
+    if (!workspace || !al256(workspace) || ws_bytes < g.total) return DASH_ERR_WORKSPACE;
+    char* ws = static_cast<char*>(workspace);
+    cudaStream_t s = S(stream);
+    auto mark = [&](int i) {
+        return !events || cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[i]), s) == cudaSuccess;
+    };
+    if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), s) != cudaSuccess) return DASH_ERR_CUDA;
+    if (!mark(0)) return DASH_ERR_CUDA;
+    if (g.nbs > 0 && launch_block_summary(k, reinterpret_cast<float*>(ws + g.off_ksum), B, Hkv, T, d, s) != cudaSuccess)
+        return DASH_ERR_CUDA;
+    if (!mark(1)) return DASH_ERR_CUDA;
+    if (launch_coarse(q, g, ws, alpha, coarse_scale, s) != cudaSuccess) return DASH_ERR_CUDA;
+    if (!mark(2)) return DASH_ERR_CUDA;
+    if (launch_fine(q, k, v, out, g, ws, alpha, coarse_scale, s) != cudaSuccess) return DASH_ERR_CUDA;
+    if (!mark(3)) return DASH_ERR_CUDA;
+    return DASH_OK;
+}
+
+int dash_prefill(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv,
+                 int T, int d, int block, float alpha, float coarse_scale, void* workspace,
+                 size_t ws_bytes, dash_stream_t stream) {
+    return prefill_impl(q, k, v, out, B, Hq, Hkv, T, d, block, alpha, coarse_scale, workspace,
+                        ws_bytes, stream, nullptr);
+}
+
+int dash_prefill_profiled(const void* q, const void* k, const void* v, void* out, int B, int Hq,
+                          int Hkv, int T, int d, int block, float alpha, float coarse_scale,
+                          void* workspace, size_t ws_bytes, dash_stream_t stream, void* const* events) {
+    if (!events) return DASH_ERR_ARG;
+    return prefill_impl(q, k, v, out, B, Hq, Hkv, T, d, block, alpha, coarse_scale, workspace,
+                        ws_bytes, stream, events);
+}
+
+int dash_prefill_host(const void* q_host, const void* k_host, const void* v_host, void* out_host,
+                      void* q_dev, void* k_dev, void* v_dev, void* out_dev, int B, int Hq, int Hkv,
+                      int T, int d, int block, float alpha, float coarse_scale, void* workspace,
+                      size_t ws_bytes, dash_stream_t stream) {
+    if (!q_host || !k_host || !v_host || !out_host) return DASH_ERR_ARG;
+    PrefillGeom g;
+    if (block != kBlock || !make_prefill_geom(B, Hq, Hkv, T, d, &g)) return DASH_ERR_SHAPE;
+    if (!q_dev || !k_dev || !v_dev || !out_dev) return DASH_ERR_ARG;
+    const size_t qb = (size_t)B * Hq * T * d * 2, kb = (size_t)B * Hkv * T * d * 2;
+    cudaStream_t s = S(stream);
+    if (cudaMemcpyAsync(q_dev, q_host, qb, cudaMemcpyHostToDevice, s) != cudaSuccess) return DASH_ERR_CUDA;
+    if (cudaMemcpyAsync(k_dev, k_host, kb, cudaMemcpyHostToDevice, s) != cudaSuccess) return DASH_ERR_CUDA;
+    if (cudaMemcpyAsync(v_dev, v_host, kb, cudaMemcpyHostToDevice, s) != cudaSuccess) return DASH_ERR_CUDA;
+    int rc = dash_prefill(q_dev, k_dev, v_dev, out_dev, B, Hq, Hkv, T, d, block, alpha, coarse_scale,
+                          workspace, ws_bytes, stream);
+    if (rc != DASH_OK) return rc;
+    if (cudaMemcpyAsync(out_host, out_dev, qb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return DASH_ERR_CUDA;
+    return DASH_OK;
+}
+
+int dash_prefill_stats(const void* workspace, size_t ws_bytes, dash_stats* out, dash_stream_t stream) {
+    return read_stats(workspace, ws_bytes, out, stream);
+}
+
+int dash_decode_stats(const void* workspace, size_t ws_bytes, dash_stats* out, dash_stream_t stream) {
+    return read_stats(workspace, ws_bytes, out, stream);
+}
+
+int dash_prefill_tau(const void* workspace, size_t ws_bytes, float* tau_out, int B, int Hq, int Hkv,
+                     int T, int d, int block, dash_stream_t stream) {
+    if (!workspace || !tau_out) return DASH_ERR_ARG;
+    PrefillGeom g;
+    if (block != kBlock || !make_prefill_geom(B, Hq, Hkv, T, d, &g)) return DASH_ERR_SHAPE;
+    if (ws_bytes < g.total) return DASH_ERR_WORKSPACE;
+    const char* ws = static_cast<const char*>(workspace);
+    return cudaMemcpyAsync(tau_out, ws + g.off_tau, (size_t)B * Hq * T * sizeof(float),
+                           cudaMemcpyDeviceToDevice, S(stream)) == cudaSuccess ? DASH_OK : DASH_ERR_CUDA;
+}
+
+int dash_select_dump(const void* q, const float* ksum, const long long* rows, int nrows, int max_sel,
+                     int* out_idx, float* out_p, int* out_count, float* out_tau, int B, int Hq, int Hkv,
+                     int T, int d, int block, float alpha, float coarse_scale, dash_stream_t stream) {
+    if (nrows < 0 || max_sel < 0) return DASH_ERR_ARG;
+    if (nrows > 0 && (!q || !ksum || !rows || !out_count || !out_tau || !al16(q))) return DASH_ERR_ARG;
+    if (nrows > 0 && max_sel > 0 && (!out_idx || !out_p)) return DASH_ERR_ARG;
+    if (!good_params(alpha, coarse_scale)) return DASH_ERR_ARG;
+    PrefillGeom g;
+    if (block != kBlock || !make_prefill_geom(B, Hq, Hkv, T, d, &g)) return DASH_ERR_SHAPE;
+    return launch_select_dump(q, ksum, rows, nrows, max_sel, out_idx, out_p, out_count, out_tau, B, Hq,
+                              Hkv, T, d, alpha, coarse_scale, S(stream)) == cudaSuccess
+               ? DASH_OK : DASH_ERR_CUDA;
+}
+
+size_t dash_decode_workspace_size(int B, int Hq, int Hkv, int Tmax, int d, int block) {
+    DecodeGeom g;
+    if (block != kBlock || !make_decode_geom(B, Hq, Hkv, Tmax, d, &g)) return 0;
+    return g.total;
+}
+
+static int decode_impl(const void* q, const void* k_cache, const void* v_cache, const float* ksum,
+                       const int* kv_len, void* out, int B, int Hq, int Hkv, int Tmax, int d, int block,
+                       float alpha, float coarse_scale, void* workspace, size_t ws_bytes,
+                       dash_stream_t stream, void* const* events) {
+    if (!q || !k_cache || !v_cache || !ksum || !kv_len || !out) return DASH_ERR_ARG;
+    if (!al16(q) || !al16(k_cache) || !al16(v_cache) || !al16(ksum) || !al16(out)) return DASH_ERR_ARG;
+    if (!good_params(alpha, coarse_scale)) return DASH_ERR_ARG;
+    DecodeGeom g;
+    if (block != kBlock || !make_decode_geom(B, Hq, Hkv, Tmax, d, &g)) return DASH_ERR_SHAPE;
+    if (!workspace || !al256(workspace) || ws_bytes < g.total) return DASH_ERR_WORKSPACE;
+    char* ws = static_cast<char*>(workspace);
+    cudaStream_t s = S(stream);
+    if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), s) != cudaSuccess) return DASH_ERR_CUDA;
+    return launch_decode(q, k_cache, v_cache, ksum, kv_len, out, g, ws, alpha, coarse_scale, s,
+                         reinterpret_cast<cudaEvent_t const*>(events)) == cudaSuccess
+               ? DASH_OK : DASH_ERR_CUDA;
+}
+
+int dash_decode(const void* q, const void* k_cache, const void* v_cache, const float* ksum,
+                const int* kv_len, void* out, int B, int Hq, int Hkv, int Tmax, int d, int block,
+                float alpha, float coarse_scale, void* workspace, size_t ws_bytes, dash_stream_t stream) {
+    return decode_impl(q, k_cache, v_cache, ksum, kv_len, out, B, Hq, Hkv, Tmax, d, block, alpha,
+                       coarse_scale, workspace, ws_bytes, stream, nullptr);
+}
+
+int dash_decode_profiled(const void* q, const void* k_cache, const void* v_cache, const float* ksum,
+                         const int* kv_len, void* out, int B, int Hq, int Hkv, int Tmax, int d, int block,
+                         float alpha, float coarse_scale, void* workspace, size_t ws_bytes,
+                         dash_stream_t stream, void* const* events) {
+    if (!events) return DASH_ERR_ARG;
+    return decode_impl(q, k_cache, v_cache, ksum, kv_len, out, B, Hq, Hkv, Tmax, d, block, alpha,
+                       coarse_scale, workspace, ws_bytes, stream, events);
+}
+
+int dash_get_device_status(const void* workspace, dash_stream_t stream) {
+    if (!workspace) return DASH_ERR_ARG;
+    if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return DASH_ERR_CUDA;
+    int st = 0;
+    if (cudaMemcpy(&st, workspace, sizeof st, cudaMemcpyDeviceToHost) != cudaSuccess) return DASH_ERR_CUDA;
+    return (st & kStNoConverge) ? DASH_ERR_NO_CONVERGE : DASH_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,145 @@
+// common.cuh -- shared device helpers and the workspace layout of the DashAttention kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dash {
+
+constexpr int kBlock = 64;        // tokens per key block (the only supported block size)
+constexpr int kTileRows = 128;    // query rows per work tile (positions x heads of one group)
+constexpr int kMaxT = 1 << 20;    // longest supported sequence
+constexpr int kCoarseCTAs = 296;  // persistent coarse grid: 2 CTAs on each of 148 SMs
+constexpr int kSolveMaxIt = 64;   // iteration cap of the threshold solve
+
+// Device status bits (workspace header).
+enum : int { kStNoConverge = 1 };
+
+// First 256 bytes of every workspace.
+struct WsHeader {
+    int status;
+    int pad;
+    unsigned long long scored_pairs;
+    unsigned long long selected_pairs;
+    unsigned long long union_blocks;
+    unsigned long long tiles;
+    unsigned long long reserved[27];
+};
+static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
+
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Geometry of a prefill call.  Work tiles are P consecutive positions (inside one key
+// block) x the G query heads of one KV head: rows r = head_local * P + pos_local.
+struct PrefillGeom {
+    int B, Hq, Hkv, T, d, G, P, M;   // M = G * P rows used of the 128-row tile
+    int ntile_bg;                    // tiles per (b, kv head) = ceil(T / P)
+    int ntiles;                      // B * Hkv * ntile_bg
+    int nbs;                         // complete blocks = T / 64
+    int cap;                         // list capacity per tile = max(1, nbs)
+    size_t off_ksum, off_tau, off_list, off_count, off_scratch, total;
+};
+
+inline int pow2_floor(int x) {
+    int p = 1;
+    while (p * 2 <= x) p *= 2;
+    return p;
+}
+
+inline bool make_prefill_geom(int B, int Hq, int Hkv, int T, int d, PrefillGeom* g) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || T < 1 || T > kMaxT || (Hq % Hkv) != 0) return false;
+    if (d != 64 && d != 128) return false;
+    int G = Hq / Hkv;
+    if (G > kTileRows) return false;
+    g->B = B; g->Hq = Hq; g->Hkv = Hkv; g->T = T; g->d = d; g->G = G;
+    int P = pow2_floor(kTileRows / G);
+    if (P > kBlock) P = kBlock;
+    g->P = P;
+    g->M = G * P;
+    g->ntile_bg = (T + P - 1) / P;
+    g->ntiles = B * Hkv * g->ntile_bg;
+    g->nbs = T / kBlock;
+    g->cap = g->nbs > 0 ? g->nbs : 1;
+    size_t off = align256(sizeof(WsHeader));
+    g->off_ksum = off;    off = align256(off + (size_t)B * Hkv * (g->nbs > 0 ? g->nbs : 1) * d * sizeof(float));
+    g->off_tau = off;     off = align256(off + (size_t)B * Hq * T * sizeof(float));
+    g->off_list = off;    off = align256(off + (size_t)g->ntiles * g->cap * sizeof(int));
+    g->off_count = off;   off = align256(off + (size_t)g->ntiles * sizeof(int));
+    int cgrid = g->ntiles < kCoarseCTAs ? g->ntiles : kCoarseCTAs;
+    g->off_scratch = off; off = align256(off + (size_t)cgrid * kTileRows * g->cap * sizeof(float));
+    g->total = off;
+    return true;
+}
+
+// Geometry of a decode call.
+struct DecodeGeom {
+    int B, Hq, Hkv, Tmax, d, G, nbs, chunk, maxchunks;
+    size_t off_x, off_tau, off_list, off_count, off_part, total;
+};
+
+constexpr int kDecodeChunk = 16;   // list entries (key blocks) per split-KV work item
+
+inline bool make_decode_geom(int B, int Hq, int Hkv, int Tmax, int d, DecodeGeom* g) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Tmax < 1 || Tmax > kMaxT || (Hq % Hkv) != 0) return false;
+    if (d != 64 && d != 128) return false;
+    int G = Hq / Hkv;
+    if (G > 32) return false;
+    g->B = B; g->Hq = Hq; g->Hkv = Hkv; g->Tmax = Tmax; g->d = d; g->G = G;
+    g->nbs = Tmax / kBlock;
+    g->chunk = kDecodeChunk;
+    g->maxchunks = (g->nbs + 1 + kDecodeChunk - 1) / kDecodeChunk;
+    int cap = g->nbs + 1;
+    size_t off = align256(sizeof(WsHeader));
+    g->off_x = off;     off = align256(off + (size_t)B * Hq * cap * sizeof(float));
+    g->off_tau = off;   off = align256(off + (size_t)B * Hq * sizeof(float));
+    g->off_list = off;  off = align256(off + (size_t)B * Hkv * cap * sizeof(int));
+    g->off_count = off; off = align256(off + (size_t)B * Hkv * sizeof(int));
+    // partial (m, l, o[d]) per (b, kv head, chunk, head in group)
+    g->off_part = off;  off = align256(off + (size_t)B * Hkv * g->maxchunks * G * (d + 2) * sizeof(float));
+    g->total = off;
+    return true;
+}
+
+// ------------------------------------------------------------------ small device helpers
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_min(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ void bf16x8_to_float(const uint4& u, float* f) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 t = __bfloat1622float2(h[i]);
+        f[2 * i] = t.x;
+        f[2 * i + 1] = t.y;
+    }
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 16-byte asynchronous global->shared copy; src_bytes = 0 zero-fills the destination.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n"
+                 :: "r"(smem_u32(dst)), "l"(src), "r"(src_bytes));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" :: "n"(N)); }
+
+}  // namespace dash

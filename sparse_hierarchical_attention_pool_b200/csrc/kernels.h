@@ -1,0 +1,33 @@
+// kernels.h -- host-side launchers of the DashAttention kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace dash {
+
+cudaError_t launch_block_summary(const void* k, float* ksum, int B, int Hkv, int T, int d,
+                                 cudaStream_t stream);
+
+// Stage 1 for prefill: scores of every work tile against the block summaries, per-row
+// thresholds and the per-tile union of selected blocks.
+cudaError_t launch_coarse(const void* q, const PrefillGeom& g, char* ws, float alpha,
+                          float coarse_scale, cudaStream_t stream);
+
+// Stage 2 for prefill: prior-weighted softmax attention over each tile's listed blocks.
+cudaError_t launch_fine(const void* q, const void* k, const void* v, void* out,
+                        const PrefillGeom& g, char* ws, float alpha, float coarse_scale,
+                        cudaStream_t stream);
+
+cudaError_t launch_select_dump(const void* q, const float* ksum, const long long* rows, int nrows,
+                               int max_sel, int* out_idx, float* out_p, int* out_count,
+                               float* out_tau, int B, int Hq, int Hkv, int T, int d, float alpha,
+                               float coarse_scale, cudaStream_t stream);
+
+cudaError_t launch_decode(const void* q, const void* kc, const void* vc, const float* ksum,
+                          const int* kv_len, void* out, const DecodeGeom& g, char* ws,
+                          float alpha, float coarse_scale, cudaStream_t stream,
+                          const cudaEvent_t* events);
+
+}  // namespace dash

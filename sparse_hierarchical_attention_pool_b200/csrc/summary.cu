@@ -1,0 +1,74 @@
+// summary.cu -- Stage 0: block summaries (mean pooling of each complete 64-key block).
+//
+// "DashAttention and the year sparse attention became a field", section "What
+// alpha-entmax changes": the chunk summary is a small learned attention head initialised
+// at zero, i.e. uniform weights over the chunk's keys -- the arithmetic mean.
+//
+// One warp per (b, kv head, block): the block is 64 * d * 2 bytes contiguous in k.  Lane
+// l reads 16-byte vectors (8 bf16) of column group l % (d/8) from rows l / (d/8), + 32/(d/8),
+// ...; partial sums are combined with shuffles; fp32 accumulation throughout.  HBM-bound:
+// bytes per block = 64 * d * 2 read + d * 4 written.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dash {
+
+template <int D>
+__global__ void __launch_bounds__(256)
+block_summary_kernel(const __nv_bfloat16* __restrict__ k, float* __restrict__ ksum,
+                     long long nblocks_total, int nbs, int T) {
+    constexpr int CH = D / 8;          // 16-byte column groups per row
+    constexpr int RPS = 32 / CH;       // rows covered by one warp-wide load
+    constexpr int STEPS = kBlock / RPS;
+    const int lane = threadIdx.x & 31;
+    long long wid = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (wid >= nblocks_total) return;
+    long long bg = wid / nbs;
+    int j = (int)(wid % nbs);
+    const int cg = lane % CH, r0 = lane / CH;
+    const uint4* src = reinterpret_cast<const uint4*>(k + ((size_t)bg * T + (size_t)j * kBlock) * D);
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    constexpr int BATCH = 8;           // loads in flight per lane
+#pragma unroll
+    for (int s0 = 0; s0 < STEPS; s0 += BATCH) {
+        uint4 buf[BATCH];
+#pragma unroll
+        for (int s = 0; s < BATCH; ++s) buf[s] = __ldg(src + (size_t)(r0 + (s0 + s) * RPS) * CH + cg);
+#pragma unroll
+        for (int s = 0; s < BATCH; ++s) {
+            float f[8];
+            bf16x8_to_float(buf[s], f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] += f[i];
+        }
+    }
+#pragma unroll
+    for (int o = CH; o < 32; o <<= 1)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+    if (lane < CH) {
+        float4* dst = reinterpret_cast<float4*>(ksum + ((size_t)bg * nbs + j) * D + lane * 8);
+        const float s = 1.0f / kBlock;
+        dst[0] = make_float4(acc[0] * s, acc[1] * s, acc[2] * s, acc[3] * s);
+        dst[1] = make_float4(acc[4] * s, acc[5] * s, acc[6] * s, acc[7] * s);
+    }
+}
+
+cudaError_t launch_block_summary(const void* k, float* ksum, int B, int Hkv, int T, int d,
+                                 cudaStream_t stream) {
+    int nbs = T / kBlock;
+    long long total = (long long)B * Hkv * nbs;
+    if (total == 0) return cudaSuccess;
+    unsigned grid = (unsigned)((total + 7) / 8);
+    if (d == 128)
+        block_summary_kernel<128><<<grid, 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(k), ksum, total, nbs, T);
+    else
+        block_summary_kernel<64><<<grid, 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(k), ksum, total, nbs, T);
+    return cudaGetLastError();
+}
+
+}  // namespace dash

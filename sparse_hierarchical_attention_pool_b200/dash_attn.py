@@ -1,0 +1,270 @@
+"""Thin Python binding over libdash_attn.so (the C ABI of include/dash_attn.h).
+
+Every function here only checks tensors and marshals pointers; all computation runs in
+the library's CUDA kernels on the current torch stream.  There is no CPU fallback: when
+the library is missing or fails to load, the first call raises.
+
+Tensor conventions follow the header: bf16, contiguous, q/out [B, Hq, T, d], k/v
+[B, Hkv, T, d], caches [B, Hkv, Tmax, d], block summaries fp32 [B, Hkv, T // 64, d].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdash_attn.so")
+
+DASH_OK = 0
+STATUS = {0: "DASH_OK", -1: "DASH_ERR_ARG", -2: "DASH_ERR_SHAPE", -3: "DASH_ERR_DTYPE",
+          -4: "DASH_ERR_UNSUPPORTED", -5: "DASH_ERR_WORKSPACE", -6: "DASH_ERR_CUDA",
+          -7: "DASH_ERR_NO_CONVERGE"}
+
+EXPORTS = ("dash_status_string", "dash_version", "dash_block_summary", "dash_prefill_workspace_size",
+           "dash_prefill", "dash_prefill_host", "dash_prefill_stats", "dash_decode_stats",
+           "dash_prefill_tau", "dash_select_dump", "dash_decode_workspace_size", "dash_decode",
+           "dash_get_device_status", "dash_prefill_profiled", "dash_decode_profiled")
+
+
+class DashError(RuntimeError):
+    def __init__(self, fn, code):
+        self.code = code
+        super().__init__(f"{fn} failed: {STATUS.get(code, code)}")
+
+
+class dash_stats(ctypes.Structure):
+    _fields_ = [("scored_pairs", ctypes.c_longlong), ("selected_pairs", ctypes.c_longlong),
+                ("union_blocks", ctypes.c_longlong), ("tiles", ctypes.c_longlong),
+                ("status", ctypes.c_int)]
+
+
+_lib = None
+_i = ctypes.c_int
+_f = ctypes.c_float
+_p = ctypes.c_void_p
+_sz = ctypes.c_size_t
+
+
+def lib():
+    """Load libdash_attn.so (raises if it is missing: there is no fallback path)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libdash_attn.so not found at {LIB_PATH}; build it with "
+                           "`python -m sparse_hierarchical_attention_pool_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    L.dash_status_string.restype = ctypes.c_char_p
+    L.dash_status_string.argtypes = [_i]
+    L.dash_version.restype = _i
+    L.dash_block_summary.argtypes = [_p, _p, _i, _i, _i, _i, _i, _p]
+    L.dash_prefill_workspace_size.argtypes = [_i] * 6
+    L.dash_prefill_workspace_size.restype = _sz
+    L.dash_prefill.argtypes = [_p] * 4 + [_i] * 6 + [_f, _f, _p, _sz, _p]
+    L.dash_prefill_host.argtypes = [_p] * 8 + [_i] * 6 + [_f, _f, _p, _sz, _p]
+    L.dash_prefill_stats.argtypes = [_p, _sz, ctypes.POINTER(dash_stats), _p]
+    L.dash_decode_stats.argtypes = [_p, _sz, ctypes.POINTER(dash_stats), _p]
+    L.dash_prefill_tau.argtypes = [_p, _sz, _p] + [_i] * 6 + [_p]
+    L.dash_select_dump.argtypes = [_p, _p, _p, _i, _i, _p, _p, _p, _p] + [_i] * 6 + [_f, _f, _p]
+    L.dash_decode_workspace_size.argtypes = [_i] * 6
+    L.dash_decode_workspace_size.restype = _sz
+    L.dash_decode.argtypes = [_p] * 6 + [_i] * 6 + [_f, _f, _p, _sz, _p]
+    L.dash_get_device_status.argtypes = [_p, _p]
+    L.dash_prefill_profiled.argtypes = [_p] * 4 + [_i] * 6 + [_f, _f, _p, _sz, _p, _p]
+    L.dash_decode_profiled.argtypes = [_p] * 6 + [_i] * 6 + [_f, _f, _p, _sz, _p, _p]
+    for name in EXPORTS:
+        if name not in ("dash_status_string", "dash_prefill_workspace_size", "dash_decode_workspace_size"):
+            getattr(L, name).restype = _i
+    _lib = L
+    return L
+
+
+def _check(fn, rc):
+    if rc != DASH_OK:
+        raise DashError(fn, rc)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t, dtype, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def version() -> int:
+    return lib().dash_version()
+
+
+def dash_block_summary(k, ksum=None, block=64, stream=None):
+    """Mean of every complete 64-key block: k [B, Hkv, T, d] -> ksum fp32 [B, Hkv, T // 64, d]."""
+    B, Hkv, T, d = k.shape
+    if ksum is None:
+        ksum = torch.empty(B, Hkv, max(T // block, 1), d, device=k.device, dtype=torch.float32)
+    _check("dash_block_summary", lib().dash_block_summary(
+        _dev(k, torch.bfloat16, "k"), _dev(ksum, torch.float32, "ksum"), B, Hkv, T, d, block, _stream(stream)))
+    return ksum
+
+
+def prefill_workspace_size(B, Hq, Hkv, T, d, block=64) -> int:
+    n = lib().dash_prefill_workspace_size(B, Hq, Hkv, T, d, block)
+    if n == 0:
+        raise DashError("dash_prefill_workspace_size", -2)
+    return n
+
+
+def decode_workspace_size(B, Hq, Hkv, Tmax, d, block=64) -> int:
+    n = lib().dash_decode_workspace_size(B, Hq, Hkv, Tmax, d, block)
+    if n == 0:
+        raise DashError("dash_decode_workspace_size", -2)
+    return n
+
+
+def alloc_workspace(nbytes, device="cuda"):
+    """A 256-byte aligned uint8 device buffer (torch's caching allocator aligns to 512)."""
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    assert ws.data_ptr() % 256 == 0
+    return ws
+
+
+def dash_prefill(q, k, v, out=None, alpha=1.5, coarse_scale=1.0, workspace=None, block=64, stream=None):
+    """Causal DashAttention prefill.  Returns (out, workspace)."""
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, T, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Hkv, T, d] matching q")
+    if out is None:
+        out = torch.empty_like(q)
+    need = prefill_workspace_size(B, Hq, Hkv, T, d, block)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    rc = lib().dash_prefill(_dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"),
+                            _dev(v, torch.bfloat16, "v"), _dev(out, torch.bfloat16, "out"),
+                            B, Hq, Hkv, T, d, block, float(alpha), float(coarse_scale),
+                            ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream))
+    _check("dash_prefill", rc)
+    return out, workspace
+
+
+def _events(evs):
+    arr = (ctypes.c_void_p * len(evs))(*[ctypes.c_void_p(e.cuda_event) for e in evs])
+    return arr
+
+
+def dash_prefill_profiled(q, k, v, out, alpha, coarse_scale, workspace, events, block=64, stream=None):
+    """dash_prefill recording torch.cuda.Event objects events[0..3] around its three kernels."""
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    rc = lib().dash_prefill_profiled(_dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"),
+                                     _dev(v, torch.bfloat16, "v"), _dev(out, torch.bfloat16, "out"),
+                                     B, Hq, Hkv, T, d, block, float(alpha), float(coarse_scale),
+                                     ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream),
+                                     _events(events))
+    _check("dash_prefill_profiled", rc)
+    return out
+
+
+def dash_decode_profiled(q, k_cache, v_cache, ksum, kv_len, out, alpha, coarse_scale, workspace, events,
+                         block=64, stream=None):
+    """dash_decode recording torch.cuda.Event objects events[0..4] around its four kernels."""
+    B, Hq, d = q.shape
+    Hkv, Tmax = k_cache.shape[1], k_cache.shape[2]
+    rc = lib().dash_decode_profiled(_dev(q, torch.bfloat16, "q"), _dev(k_cache, torch.bfloat16, "k_cache"),
+                                    _dev(v_cache, torch.bfloat16, "v_cache"), _dev(ksum, torch.float32, "ksum"),
+                                    _dev(kv_len, torch.int32, "kv_len"), _dev(out, torch.bfloat16, "out"),
+                                    B, Hq, Hkv, Tmax, d, block, float(alpha), float(coarse_scale),
+                                    ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream),
+                                    _events(events))
+    _check("dash_decode_profiled", rc)
+    return out
+
+
+def dash_prefill_host(q_host, k_host, v_host, out_host, q_dev, k_dev, v_dev, out_dev, alpha, coarse_scale,
+                      workspace, block=64, stream=None):
+    """Prefill from host tensors (pinned for overlap): H2D copies, prefill, D2H copy, async."""
+    B, Hq, T, d = q_dev.shape
+    Hkv = k_dev.shape[1]
+    for name, t in (("q_host", q_host), ("k_host", k_host), ("v_host", v_host), ("out_host", out_host)):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 host tensor")
+    rc = lib().dash_prefill_host(
+        ctypes.c_void_p(q_host.data_ptr()), ctypes.c_void_p(k_host.data_ptr()),
+        ctypes.c_void_p(v_host.data_ptr()), ctypes.c_void_p(out_host.data_ptr()),
+        _dev(q_dev, torch.bfloat16, "q_dev"), _dev(k_dev, torch.bfloat16, "k_dev"),
+        _dev(v_dev, torch.bfloat16, "v_dev"), _dev(out_dev, torch.bfloat16, "out_dev"),
+        B, Hq, Hkv, T, d, block, float(alpha), float(coarse_scale),
+        ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream))
+    _check("dash_prefill_host", rc)
+    return out_host
+
+
+def _stats(fn, workspace, stream):
+    st = dash_stats()
+    _check(fn, getattr(lib(), fn)(ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
+                                  ctypes.byref(st), _stream(stream)))
+    return {f: getattr(st, f) for f, _ in dash_stats._fields_}
+
+
+def dash_prefill_stats(workspace, stream=None):
+    return _stats("dash_prefill_stats", workspace, stream)
+
+
+def dash_decode_stats(workspace, stream=None):
+    return _stats("dash_decode_stats", workspace, stream)
+
+
+def dash_prefill_tau(workspace, B, Hq, Hkv, T, d, block=64, stream=None):
+    tau = torch.empty(B, Hq, T, device=workspace.device, dtype=torch.float32)
+    _check("dash_prefill_tau", lib().dash_prefill_tau(
+        ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), ctypes.c_void_p(tau.data_ptr()),
+        B, Hq, Hkv, T, d, block, _stream(stream)))
+    return tau
+
+
+def dash_select_dump(q, ksum, rows, max_sel, alpha, coarse_scale, Hkv, block=64, stream=None):
+    """Selected blocks, weights, support size and tau of rows (b, h, t) [n, 3] int64."""
+    B, Hq, T, d = q.shape
+    rows = torch.as_tensor(rows, dtype=torch.int64, device=q.device).reshape(-1, 3).contiguous()
+    n = rows.shape[0]
+    idx = torch.full((n, max(max_sel, 1)), -1, dtype=torch.int32, device=q.device)
+    p = torch.zeros((n, max(max_sel, 1)), dtype=torch.float32, device=q.device)
+    cnt = torch.zeros(n, dtype=torch.int32, device=q.device)
+    tau = torch.zeros(n, dtype=torch.float32, device=q.device)
+    _check("dash_select_dump", lib().dash_select_dump(
+        _dev(q, torch.bfloat16, "q"), _dev(ksum, torch.float32, "ksum"), ctypes.c_void_p(rows.data_ptr()),
+        n, max_sel, ctypes.c_void_p(idx.data_ptr()), ctypes.c_void_p(p.data_ptr()),
+        ctypes.c_void_p(cnt.data_ptr()), ctypes.c_void_p(tau.data_ptr()),
+        B, Hq, Hkv, T, d, block, float(alpha), float(coarse_scale), _stream(stream)))
+    return idx, p, cnt, tau
+
+
+def dash_decode(q, k_cache, v_cache, ksum, kv_len, out=None, alpha=1.5, coarse_scale=1.0,
+                workspace=None, block=64, stream=None):
+    """One decode step.  q [B, Hq, d]; caches [B, Hkv, Tmax, d]; kv_len int32 [B] (device)."""
+    B, Hq, d = q.shape
+    Hkv, Tmax = k_cache.shape[1], k_cache.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    need = decode_workspace_size(B, Hq, Hkv, Tmax, d, block)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    rc = lib().dash_decode(_dev(q, torch.bfloat16, "q"), _dev(k_cache, torch.bfloat16, "k_cache"),
+                           _dev(v_cache, torch.bfloat16, "v_cache"), _dev(ksum, torch.float32, "ksum"),
+                           _dev(kv_len, torch.int32, "kv_len"), _dev(out, torch.bfloat16, "out"),
+                           B, Hq, Hkv, Tmax, d, block, float(alpha), float(coarse_scale),
+                           ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream))
+    _check("dash_decode", rc)
+    return out, workspace
+
+
+def dash_get_device_status(workspace, stream=None) -> int:
+    return lib().dash_get_device_status(ctypes.c_void_p(workspace.data_ptr()), _stream(stream))

@@ -1,0 +1,131 @@
+"""Shared helpers of the GPU parity tests: run the CUDA path through the C ABI, run the fp64
+oracle on the same seeded inputs, and compare with the tolerances of the specification.
+
+Tolerances (bf16 inputs, fp32 accumulation):
+  outputs        max-abs <= 2e-2 and mean-abs <= 2e-3 against the fp64 oracle;
+  block weights  within 1e-4 absolute;
+  block sets     identical except blocks whose (alpha-1) s_j - tau lies within 1e-4 of 0.
+"""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+import torch
+
+import oracle
+from sparse_hierarchical_attention_pool_b200 import dash_attn as da
+from sparse_hierarchical_attention_pool_b200 import inputs
+
+OUT_MAX_ABS = 2e-2
+OUT_MEAN_ABS = 2e-3
+P_ABS = 1e-4
+BAND = 1e-4
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "coarse_scale.json")
+
+
+def calibrated_scale(name):
+    with open(GOLDEN) as f:
+        return json.load(f)[name]["coarse_scale"]
+
+
+def all_rows(B, Hq, T):
+    return [(b, h, t) for b in range(B) for h in range(Hq) for t in range(T)]
+
+
+def stratified_rows(B, Hq, T, n_random, seed):
+    fixed = sorted({0, 1, 63, 64, 65, 127, 128, 129, 1023, 1024, 4095, 4096, T // 2, T - 65, T - 64, T - 2, T - 1})
+    return inputs.sample_rows(B, Hq, T, n_random, seed, t_fixed=fixed)
+
+
+def gpu_prefill(q, k, v, alpha, cs):
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    out, ws = da.dash_prefill(qd, kd, vd, alpha=alpha, coarse_scale=cs)
+    torch.cuda.synchronize()
+    return qd, kd, vd, out, ws
+
+
+def compare_out(got, ref, what=""):
+    got = np.asarray(got, dtype=np.float64)
+    err = np.abs(got - ref)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    mx, mean = float(err.max()), float(err.mean())
+    assert mx <= OUT_MAX_ABS, f"{what}: max-abs {mx:.3e} > {OUT_MAX_ABS}"
+    assert mean <= OUT_MEAN_ABS, f"{what}: mean-abs {mean:.3e} > {OUT_MEAN_ABS}"
+    return mx, mean
+
+
+def rows_of(t4, rows):
+    r = torch.as_tensor(np.asarray(rows, dtype=np.int64))
+    return t4[r[:, 0], r[:, 1], r[:, 2]]
+
+
+def check_prefill(q, k, v, alpha, cs, rows, what="", check_selection=True, nthreads=0):
+    """Full parity of one prefill call: outputs, thresholds, block sets and weights."""
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    qd, kd, vd, out, ws = gpu_prefill(q, k, v, alpha, cs)
+    st = da.dash_get_device_status(ws)
+    assert st == 0, f"{what}: device status {st}"
+    qr = oracle.gather_q_rows(q, rows)
+    ref, tau_ref, nsel_ref = oracle.forward_rows(qr, k, v, rows, Hq, 64, alpha, cs, nthreads)
+    got = rows_of(out.float().cpu(), rows).numpy()
+    res = {"out": compare_out(got, ref, what)}
+    tau_gpu = rows_of(da.dash_prefill_tau(ws, B, Hq, Hkv, T, d).cpu(), rows).numpy()
+    has_past = np.array([t >= 64 for _, _, t in rows])
+    if has_past.any():
+        dt = np.abs(tau_gpu[has_past] - tau_ref[has_past])
+        assert dt.max() <= 1e-4, f"{what}: tau differs by {dt.max():.3e}"
+    assert np.all(np.isnan(tau_gpu[~has_past]))
+    if check_selection and has_past.any():
+        res["sel"] = check_dump(qd, kd, rows, q, k, alpha, cs, Hkv, tau_gpu, what)
+    return res, out, ws
+
+
+def check_dump(qd, kd, rows, q, k, alpha, cs, Hkv, tau_prefill=None, what=""):
+    """Block sets and weights of the dump against the oracle (band-exempt set parity)."""
+    B, Hq, T, d = q.shape
+    nbs = T // 64
+    ksum = da.dash_block_summary(kd)
+    idx, p, cnt, tau = da.dash_select_dump(qd, ksum, rows, max(nbs, 1), alpha, cs, Hkv)
+    idx, p, cnt, tau = idx.cpu().numpy(), p.cpu().numpy(), cnt.cpu().numpy(), tau.cpu().numpy()
+    sel = oracle.select_rows(oracle.gather_q_rows(q, rows), k, rows, Hq, 64, alpha, cs)
+    worst_p, n_band = 0.0, 0
+    for r, (b, h, t) in enumerate(rows):
+        bt = t // 64
+        if bt == 0:
+            assert cnt[r] == 0 and np.isnan(tau[r])
+            continue
+        x, tr = sel["x"][r, :bt], sel["tau"][r]
+        s_gpu = set(idx[r, :cnt[r]].tolist())
+        s_ref = set(np.nonzero(x > tr)[0].tolist())
+        diff = s_gpu ^ s_ref
+        for j in diff:
+            assert abs(x[j] - tr) < BAND, f"{what}: row {(b, h, t)} block {j} differs outside the band"
+        n_band += len(diff)
+        pg = np.zeros(bt)
+        pg[idx[r, :cnt[r]]] = p[r, :cnt[r]]
+        worst_p = max(worst_p, float(np.abs(pg - sel["p"][r, :bt]).max()))
+        if tau_prefill is not None:
+            assert abs(tau[r] - tau_prefill[r]) <= 1e-6, f"{what}: dump tau != prefill tau"
+    assert worst_p <= P_ABS, f"{what}: block weight error {worst_p:.3e}"
+    return {"p_max_err": worst_p, "band_differences": n_band}
+
+
+def check_decode(q, kc, vc, kv_len, alpha, cs, what=""):
+    """Decode step on the GPU vs the oracle row t = kv_len - 1 of each sequence."""
+    B, Hq, d = q.shape
+    Hkv, Tmax = kc.shape[1], kc.shape[2]
+    qd, kcd, vcd = q.cuda(), kc.cuda(), vc.cuda()
+    lens = torch.as_tensor(kv_len, dtype=torch.int32)
+    ksum = da.dash_block_summary(kcd)
+    out, ws = da.dash_decode(qd, kcd, vcd, ksum, lens.cuda(), alpha=alpha, coarse_scale=cs)
+    torch.cuda.synchronize()
+    assert da.dash_get_device_status(ws) == 0
+    rows = [(b, h, int(lens[b]) - 1) for b in range(B) for h in range(Hq) if 1 <= int(lens[b]) <= Tmax]
+    qr = torch.stack([q[b, h] for b, h, _ in rows])
+    ref, _, _ = oracle.forward_rows(qr, kc, vc, rows, Hq, 64, alpha, cs)
+    got = torch.stack([out[b, h].float().cpu() for b, h, _ in rows]).numpy()
+    return compare_out(got, ref, what), out, ws
