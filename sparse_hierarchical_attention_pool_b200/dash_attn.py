@@ -156,8 +156,10 @@ def dash_prefill(q, k, v, out=None, alpha=1.5, coarse_scale=1.0, workspace=None,
 
 
 def _events(evs):
-    arr = (ctypes.c_void_p * len(evs))(*[ctypes.c_void_p(e.cuda_event) for e in evs])
-    return arr
+    for e in evs:
+        if e.cuda_event == 0:      # torch creates the CUDA event on its first record
+            e.record()
+    return (ctypes.c_void_p * len(evs))(*[ctypes.c_void_p(e.cuda_event) for e in evs])
 
 
 def dash_prefill_profiled(q, k, v, out, alpha, coarse_scale, workspace, events, block=64, stream=None):
