@@ -56,7 +56,9 @@ typedef enum {
     DASH_ERR_UNSUPPORTED = -4,   /* valid request the library does not implement */
     DASH_ERR_WORKSPACE = -5,     /* workspace null, misaligned (256 B) or too small */
     DASH_ERR_CUDA = -6,          /* a CUDA runtime call failed (launch, copy) */
-    DASH_ERR_NO_CONVERGE = -7    /* device status: a tau solve hit its iteration cap */
+    DASH_ERR_NO_CONVERGE = -7,   /* device status: a tau solve hit its iteration cap */
+    DASH_ERR_SCRATCH_LIMIT = -8  /* dash_decode_noalloc: the step needs more scratch than
+                                    the library's fixed array holds */
 } dash_status;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -184,6 +186,32 @@ DASH_API int dash_decode_profiled(const void* q, const void* k_cache, const void
                                   const int* kv_len, void* out, int B, int Hq, int Hkv, int Tmax, int d,
                                   int block, float alpha, float coarse_scale, void* workspace,
                                   size_t ws_bytes, dash_stream_t stream, void* const* events);
+
+/*
+ * dash_decode without a workspace argument, for callers that cannot allocate device memory
+ * where they decode: code running while a CUDA graph is captured (cudaMalloc cannot be
+ * captured), real-time loops that must not take the device-wide synchronisation
+ * cudaMalloc / cudaFree can cause, and hosts whose device memory belongs to an allocator
+ * this library cannot call.  The pages describe no such entry point; it has no
+ * counterpart in the paper.
+ *   Arguments, layouts and results are those of dash_decode; the caller still owns and
+ *   passes every input and output buffer.
+ *   Scratch is one 32 MiB array in device memory that the library declares statically:
+ *   every GPU that loads the library holds it until the process exits.  A decode step
+ *   whose scratch (dash_decode_workspace_size) exceeds 32 MiB is rejected with
+ *   DASH_ERR_SCRATCH_LIMIT before anything is launched (the 96K workload, B=8, Hq=32,
+ *   Hkv=8, d=128, needs about 15 MiB).
+ *   The first call on a device looks the array's device address up (cudaGetSymbolAddress)
+ *   and caches it; make that first call before any stream capture begins.
+ *   No memory is allocated or freed.  Every call, on every stream, shares the one array
+ *   and leaves its contents behind; the counters that must start at zero are cleared at
+ *   the start of each call.  Calls whose executions overlap on the GPU (other streams,
+ *   other host threads) race on the array and give wrong results: serialise them.
+ *   dash_decode_stats / dash_get_device_status do not see this array.
+ */
+DASH_API int dash_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, const float* ksum,
+                                 const int* kv_len, void* out, int B, int Hq, int Hkv, int Tmax, int d,
+                                 int block, float alpha, float coarse_scale, dash_stream_t stream);
 
 /* Synchronises `stream` and returns DASH_OK, or DASH_ERR_NO_CONVERGE when a kernel that
  * used `workspace` recorded a failed threshold solve, or DASH_ERR_CUDA. */

@@ -20,12 +20,13 @@ LIB_PATH = os.path.join(_HERE, "libdash_attn.so")
 DASH_OK = 0
 STATUS = {0: "DASH_OK", -1: "DASH_ERR_ARG", -2: "DASH_ERR_SHAPE", -3: "DASH_ERR_DTYPE",
           -4: "DASH_ERR_UNSUPPORTED", -5: "DASH_ERR_WORKSPACE", -6: "DASH_ERR_CUDA",
-          -7: "DASH_ERR_NO_CONVERGE"}
+          -7: "DASH_ERR_NO_CONVERGE", -8: "DASH_ERR_SCRATCH_LIMIT"}
 
 EXPORTS = ("dash_status_string", "dash_version", "dash_block_summary", "dash_prefill_workspace_size",
            "dash_prefill", "dash_prefill_host", "dash_prefill_stats", "dash_decode_stats",
            "dash_prefill_tau", "dash_select_dump", "dash_decode_workspace_size", "dash_decode",
-           "dash_get_device_status", "dash_prefill_profiled", "dash_decode_profiled")
+           "dash_get_device_status", "dash_prefill_profiled", "dash_decode_profiled",
+           "dash_decode_noalloc")
 
 
 class DashError(RuntimeError):
@@ -74,6 +75,7 @@ def lib():
     L.dash_get_device_status.argtypes = [_p, _p]
     L.dash_prefill_profiled.argtypes = [_p] * 4 + [_i] * 6 + [_f, _f, _p, _sz, _p, _p]
     L.dash_decode_profiled.argtypes = [_p] * 6 + [_i] * 6 + [_f, _f, _p, _sz, _p, _p]
+    L.dash_decode_noalloc.argtypes = [_p] * 6 + [_i] * 6 + [_f, _f, _p]
     for name in EXPORTS:
         if name not in ("dash_status_string", "dash_prefill_workspace_size", "dash_decode_workspace_size"):
             getattr(L, name).restype = _i
@@ -266,6 +268,23 @@ def dash_decode(q, k_cache, v_cache, ksum, kv_len, out=None, alpha=1.5, coarse_s
                            ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream))
     _check("dash_decode", rc)
     return out, workspace
+
+
+def dash_decode_noalloc(q, k_cache, v_cache, ksum, kv_len, out=None, alpha=1.5, coarse_scale=1.0,
+                        block=64, stream=None):
+    """dash_decode on the library's fixed 32 MiB device scratch array, for callers that cannot
+    allocate device memory where they decode (graph capture, real-time loops, foreign
+    allocators).  No workspace; calls that overlap on the GPU race on the shared array."""
+    B, Hq, d = q.shape
+    Hkv, Tmax = k_cache.shape[1], k_cache.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    rc = lib().dash_decode_noalloc(_dev(q, torch.bfloat16, "q"), _dev(k_cache, torch.bfloat16, "k_cache"),
+                                   _dev(v_cache, torch.bfloat16, "v_cache"), _dev(ksum, torch.float32, "ksum"),
+                                   _dev(kv_len, torch.int32, "kv_len"), _dev(out, torch.bfloat16, "out"),
+                                   B, Hq, Hkv, Tmax, d, block, float(alpha), float(coarse_scale), _stream(stream))
+    _check("dash_decode_noalloc", rc)
+    return out
 
 
 def dash_get_device_status(workspace, stream=None) -> int:
