@@ -57,8 +57,10 @@ typedef enum {
     DASH_ERR_WORKSPACE = -5,     /* workspace null, misaligned (256 B) or too small */
     DASH_ERR_CUDA = -6,          /* a CUDA runtime call failed (launch, copy) */
     DASH_ERR_NO_CONVERGE = -7,   /* device status: a tau solve hit its iteration cap */
-    DASH_ERR_SCRATCH_LIMIT = -8  /* dash_decode_noalloc: the step needs more scratch than
+    DASH_ERR_SCRATCH_LIMIT = -8, /* dash_decode_noalloc: the step needs more scratch than
                                     the library's fixed array holds */
+    DASH_ERR_DEVICE_TIMEOUT = -9 /* device status: a kernel's bounded wait gave up (about 2 s);
+                                    the outputs of that call are invalid */
 } dash_status;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -213,8 +215,9 @@ DASH_API int dash_decode_noalloc(const void* q, const void* k_cache, const void*
                                  const int* kv_len, void* out, int B, int Hq, int Hkv, int Tmax, int d,
                                  int block, float alpha, float coarse_scale, dash_stream_t stream);
 
-/* Synchronises `stream` and returns DASH_OK, or DASH_ERR_NO_CONVERGE when a kernel that
- * used `workspace` recorded a failed threshold solve, or DASH_ERR_CUDA. */
+/* Synchronises `stream` and returns DASH_OK, DASH_ERR_DEVICE_TIMEOUT when a kernel that used
+ * `workspace` gave up a bounded wait, DASH_ERR_NO_CONVERGE when one recorded a failed
+ * threshold solve, or DASH_ERR_CUDA. */
 DASH_API int dash_get_device_status(const void* workspace, dash_stream_t stream);
 
 #ifdef __cplusplus

@@ -48,6 +48,7 @@ const char* dash_status_string(int status) {
         case DASH_ERR_WORKSPACE: return "DASH_ERR_WORKSPACE: workspace null, misaligned or too small";
         case DASH_ERR_CUDA: return "DASH_ERR_CUDA: a CUDA runtime call failed";
         case DASH_ERR_NO_CONVERGE: return "DASH_ERR_NO_CONVERGE: a threshold solve hit its iteration cap";
+        case DASH_ERR_DEVICE_TIMEOUT: return "DASH_ERR_DEVICE_TIMEOUT: a device-side wait gave up; outputs invalid";
         case DASH_ERR_SCRATCH_LIMIT: return "DASH_ERR_SCRATCH_LIMIT: the decode step needs more than the 32 MiB static scratch";
         default: return "unknown dash status";
     }
@@ -207,6 +208,7 @@ int dash_get_device_status(const void* workspace, dash_stream_t stream) {
     if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return DASH_ERR_CUDA;
     int st = 0;
     if (cudaMemcpy(&st, workspace, sizeof st, cudaMemcpyDeviceToHost) != cudaSuccess) return DASH_ERR_CUDA;
+    if (st & kStWaitTimeout) return DASH_ERR_DEVICE_TIMEOUT;
     return (st & kStNoConverge) ? DASH_ERR_NO_CONVERGE : DASH_OK;
 }
 

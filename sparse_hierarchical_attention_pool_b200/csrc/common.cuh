@@ -14,7 +14,7 @@ constexpr int kCoarseCTAs = 296;  // persistent coarse grid: 2 CTAs on each of 1
 constexpr int kSolveMaxIt = 64;   // iteration cap of the threshold solve
 
 // Device status bits (workspace header).
-enum : int { kStNoConverge = 1 };
+enum : int { kStNoConverge = 1, kStWaitTimeout = 2 };
 
 // First 256 bytes of every workspace.
 struct WsHeader {
@@ -50,6 +50,7 @@ inline int pow2_floor(int x) {
 inline bool make_prefill_geom(int B, int Hq, int Hkv, int T, int d, PrefillGeom* g) {
     if (B < 1 || Hq < 1 || Hkv < 1 || T < 1 || T > kMaxT || (Hq % Hkv) != 0) return false;
     if (d != 64 && d != 128) return false;
+    if ((long long)B * Hq * T >= (1ll << 31)) return false;
     int G = Hq / Hkv;
     if (G > kTileRows) return false;
     g->B = B; g->Hq = Hq; g->Hkv = Hkv; g->T = T; g->d = d; g->G = G;

@@ -16,6 +16,9 @@
 // first.  8 warps x 16 rows; bf16 mma.sync m16n8k16 with fp32 accumulators; K/V blocks
 // streamed through a two-stage cp.async pipeline into XOR-swizzled shared memory; the
 // gathered block serves all G heads of the group.  Online softmax in the log2 domain.
+#include <stdlib.h>
+#include <string.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -246,9 +249,22 @@ fine_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     }
 }
 
+// Which Stage-2 kernel runs: the tcgen05 kernel wherever it supports the shape, unless
+// DASH_FINE_KERNEL=mma selects the mma.sync kernel (kept for comparison and for groups of
+// more than 16 query heads per KV head).
+static bool use_mma_kernel() {
+    static const int choice = [] {
+        const char* e = getenv("DASH_FINE_KERNEL");
+        return (e && strcmp(e, "mma") == 0) ? 1 : 0;
+    }();
+    return choice == 1;
+}
+
 cudaError_t launch_fine(const void* q, const void* k, const void* v, void* out,
                         const PrefillGeom& g, char* ws, float alpha, float coarse_scale,
                         cudaStream_t stream) {
+    if (!use_mma_kernel() && fine_tc_supported(g))
+        return launch_fine_tc(q, k, v, out, g, ws, alpha, coarse_scale, stream);
     const float cxm = (alpha - 1.0f) * coarse_scale / sqrtf((float)g.d) / (float)kBlock;
     const float e_pow = 1.0f / (alpha - 1.0f);
     const float sm2 = 1.4426950408889634f / sqrtf((float)g.d);

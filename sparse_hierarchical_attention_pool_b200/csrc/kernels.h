@@ -20,6 +20,12 @@ cudaError_t launch_fine(const void* q, const void* k, const void* v, void* out,
                         const PrefillGeom& g, char* ws, float alpha, float coarse_scale,
                         cudaStream_t stream);
 
+// tcgen05 variant of launch_fine (needs P >= 8, i.e. at most 16 query heads per KV head)
+bool fine_tc_supported(const PrefillGeom& g);
+cudaError_t launch_fine_tc(const void* q, const void* k, const void* v, void* out,
+                           const PrefillGeom& g, char* ws, float alpha, float coarse_scale,
+                           cudaStream_t stream);
+
 cudaError_t launch_select_dump(const void* q, const float* ksum, const long long* rows, int nrows,
                                int max_sel, int* out_idx, float* out_p, int* out_count,
                                float* out_tau, int B, int Hq, int Hkv, int T, int d, float alpha,

@@ -20,7 +20,8 @@ LIB_PATH = os.path.join(_HERE, "libdash_attn.so")
 DASH_OK = 0
 STATUS = {0: "DASH_OK", -1: "DASH_ERR_ARG", -2: "DASH_ERR_SHAPE", -3: "DASH_ERR_DTYPE",
           -4: "DASH_ERR_UNSUPPORTED", -5: "DASH_ERR_WORKSPACE", -6: "DASH_ERR_CUDA",
-          -7: "DASH_ERR_NO_CONVERGE", -8: "DASH_ERR_SCRATCH_LIMIT"}
+          -7: "DASH_ERR_NO_CONVERGE", -8: "DASH_ERR_SCRATCH_LIMIT",
+          -9: "DASH_ERR_DEVICE_TIMEOUT"}
 
 EXPORTS = ("dash_status_string", "dash_version", "dash_block_summary", "dash_prefill_workspace_size",
            "dash_prefill", "dash_prefill_host", "dash_prefill_stats", "dash_decode_stats",
