@@ -7,17 +7,24 @@
 // own block (causal, prior 1), times V.  x_j, hence p_j, comes from the row sums of the
 // Q K^T block the kernel computes anyway (q . kbar_j is the mean of q . k_i).
 //
-// One CTA per tile, 192 threads in three roles:
-//   warp 4 (one lane)  TMA producer: the Q tile once (one 64-column box per head and half
-//                      of d), then K and V of every listed block through a 3-stage ring;
-//   warp 5 (one lane)  MMA issuer: S_s = Q K_s^T into one of two TMEM S buffers (M=128,
-//                      N=64), then O += P_{s-1} V_{s-1} into the TMEM O accumulator
-//                      (M=128, N=d), so the tensor core computes S_s while the softmax
-//                      warps work on S_{s-1};
-//   warps 0-3          softmax, one thread per tile row = TMEM lane: load S, block weight,
-//                      online softmax in the log2 domain, P (bf16) into shared memory in the
-//                      128-byte-swizzled K-major layout the MMA reads; O is rescaled in TMEM
-//                      only when the running max grows by more than 2^8 (lazy rescale).
+// One CTA per tile.  The tile's listed blocks (steps s = 0 .. n-1, own block last) are
+// dealt alternately to two softmax groups (group s & 1), each with its own TMEM S buffer,
+// P buffer, O accumulator, row-sum column and running max; the two partial softmaxes are
+// merged in the epilogue (exactly as split-KV partials).  The per-step work of a row is a
+// serial chain (load S, row stats, weights, exponentials, P), so two groups keep two chains
+// in flight while sharing the Q tile and every K/V load.  Warps:
+//   8 SPLIT            TMA producer (one lane): the Q tile once (one 64-column box per head
+//                      and half of d), then K and V of every listed block, 4-stage ring;
+//   8 SPLIT + 1        MMA issuer (one lane): S_s = Q K_s^T (M=128, N=64) into the S buffer
+//                      of group s & 1 as soon as that group has read S_{s-2}, so S_{s+2} is
+//                      computed while the group works on step s; O_g += P_s V_s (M=128, N=d)
+//                      and L_g += P_s 1 (N=16, an all-ones B tile: the softmax denominator
+//                      summed by the tensor core over exactly the bf16 P it multiplies);
+//   0 .. 8 SPLIT - 1   softmax, group = warp / (4 SPLIT); SPLIT threads per tile row (warps
+//                      of one group sharing TMEM lanes 32 (warp % 4).. split the row's keys
+//                      and exchange partial row sums and maxima through shared memory behind
+//                      a named barrier).  Online softmax in the log2 domain; O_g is rescaled
+//                      in TMEM only when the running max grows by more than 2^8.
 // Operands: Q, K, P K-major and V MN-major, all 128-byte swizzled (TMA writes that layout).
 // Every wait is bounded (~2 s); a CTA that gives up sets a status bit and exits cleanly.
 #include <cudaTypedefs.h>
@@ -30,8 +37,8 @@
 
 namespace dash {
 
-constexpr int kTcStages = 3;
-constexpr int kTcThreads = 192;
+constexpr int kTcStages = 4;
+constexpr int kFineSplit = 1;          // threads per tile row in each softmax group
 constexpr float kLazyRescale = 8.0f;   // log2 units: p values stay below 2^8 between rescales
 
 template <int D>
@@ -44,27 +51,41 @@ struct TcLayout {
     static constexpr uint32_t kP = 128 * 128;                   // 128 rows x 64 keys bf16
     static constexpr uint32_t off_q = 0;
     static constexpr uint32_t off_kv = kQ;
-    static constexpr uint32_t off_p = kQ + kTcStages * kStage;
-    static constexpr uint32_t bytes = off_p + 2 * kP + 1024;    // + alignment slack
+    static constexpr uint32_t off_p = kQ + kTcStages * kStage;  // one P buffer per group
+    static constexpr uint32_t off_ones = off_p + 2 * kP;        // 16 x 64 bf16 ones (B of the row sum)
+    static constexpr uint32_t bytes = off_ones + 2048 + 1024;   // + alignment slack
+    // TMEM columns: S of group 0 and 1, O of group 0 and 1, row sums of group 0 and 1
+    static constexpr uint32_t colO = 128;
+    static constexpr uint32_t colL = 128 + 2 * D;
 };
+constexpr uint32_t kTmemCols = 512;
 
 // barrier slots
 enum : int { B_Q = 0, B_KV_FULL = 1, B_KV_EMPTY = 1 + kTcStages, B_S_FULL = 1 + 2 * kTcStages,
              B_S_FREE = B_S_FULL + 2, B_P_FULL = B_S_FREE + 2, B_PV_DONE = B_P_FULL + 2,
              B_DRAIN = B_PV_DONE + 2, B_COUNT = B_DRAIN + 1 };
 
-template <int D>
-__global__ void __launch_bounds__(kTcThreads, 1)
+template <int D, int SPLIT>
+__global__ void __launch_bounds__((8 * SPLIT + 2) * 32, 1)
 fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
                const float* __restrict__ tau, const int* __restrict__ list, const int* __restrict__ count,
                WsHeader* __restrict__ hdr, PrefillGeom g, float cxm, float e_pow, float sm2) {
     using L = TcLayout<D>;
     using namespace sm100;
+    constexpr int kGroupThreads = 128 * SPLIT;  // softmax threads per group
+    constexpr int KEYS = 64 / SPLIT;            // keys of a block per softmax thread
+    constexpr int OCOLS = D / (2 * SPLIT);      // epilogue output columns per softmax thread
+    constexpr int OCW = OCOLS < 32 ? OCOLS : 32;
+    constexpr int RCOLS = D / SPLIT;            // O columns a thread rescales in its group
+    constexpr int RCW = RCOLS < 32 ? RCOLS : 32;
+    constexpr int kProducerWarp = 8 * SPLIT, kMmaWarp = 8 * SPLIT + 1;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t bars[B_COUNT];
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
+    __shared__ float2 xch[2][2][SPLIT][kTileRows]; // [step parity][group][split][row]: partial (sum, max)
+    __shared__ float m_sh[2][kTileRows];        // running max of each group, for the merge
 
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -94,8 +115,8 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(B_S_FULL + i), 1);
-            mbar_init(bar(B_S_FREE + i), 128);
-            mbar_init(bar(B_P_FULL + i), 128);
+            mbar_init(bar(B_S_FREE + i), kGroupThreads);
+            mbar_init(bar(B_P_FULL + i), kGroupThreads);
             mbar_init(bar(B_PV_DONE + i), 1);
         }
         mbar_init(bar(B_DRAIN), 1);
@@ -109,9 +130,14 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int c = 0; c < 8; ++c) p[c] = make_uint4(0u, 0u, 0u, 0u);
         }
     }
+    // the all-ones B operand of the row-sum MMA (any layout: every element is 1)
+    if (tid < 128) {
+        uint4* p = reinterpret_cast<uint4*>(base_ptr + L::off_ones) + tid;
+        *p = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    }
     fence_proxy_async_smem();
     if (warp == 0) {
-        tmem_alloc(smem_u32(&tmem_base_sh), 256);
+        tmem_alloc(smem_u32(&tmem_base_sh), kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -120,7 +146,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t tmem = tmem_base_sh;
     volatile int* abort_flag = &abort_sh;
 
-    if (warp == 4) {
+    if (warp == kProducerWarp) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             prefetch_tmap(&tm_q);
@@ -154,31 +180,16 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     if (last_armed[st] >= 0) { dummy = 0; mbar_wait(bar(B_KV_FULL + st), (last_armed[st] / kTcStages) & 1, &dummy); }
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc_s = idesc_bf16(128, 64, false);
             const uint32_t idesc_pv = idesc_bf16(128, D, true);
-            auto issue_pv = [&](int p) -> bool {
-                const int bp = p & 1, stp = p % kTcStages;
-                if (!mbar_wait(bar(B_P_FULL + bp), (p >> 1) & 1, abort_flag)) return false;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t a = smem_desc_sw128(base + L::off_p + bp * L::kP + kk * 32, 16, 1024);
-                    const uint64_t bv = smem_desc_sw128(kv_addr(stp) + L::kKV + kk * 2048, L::kKVHalf, 1024);
-                    mma_bf16_ss(tmem + 128, a, bv, idesc_pv, (p > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(bar(B_PV_DONE + bp));
-                mma_commit(bar(B_KV_EMPTY + stp));
-                return true;
-            };
-            bool ok = mbar_wait(bar(B_Q), 0, abort_flag);
-            tc_fence_after();
-            for (int s = 0; ok && s < n; ++s) {
+            const uint32_t idesc_l = idesc_bf16(128, 16, false);
+            auto issue_s = [&](int s) -> bool {
                 const int st = s % kTcStages, sb = s & 1;
-                if (!mbar_wait(bar(B_KV_FULL + st), (s / kTcStages) & 1, abort_flag)) { ok = false; break; }
-                if (s >= 2 && !mbar_wait(bar(B_S_FREE + sb), ((s - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(bar(B_KV_FULL + st), (s / kTcStages) & 1, abort_flag)) return false;
+                if (s >= 2 && !mbar_wait(bar(B_S_FREE + sb), ((s - 2) >> 1) & 1, abort_flag)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -188,9 +199,38 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     mma_bf16_ss(tmem + sb * 64, a, bk, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar(B_S_FULL + sb));
-                if (s >= 1 && !issue_pv(s - 1)) { ok = false; break; }
+                return true;
+            };
+            auto issue_pv = [&](int p) -> bool {
+                const int bp = p & 1, stp = p % kTcStages;
+                if (!mbar_wait(bar(B_P_FULL + bp), (p >> 1) & 1, abort_flag)) return false;
+                tc_fence_after();
+                const uint32_t acc = p >= 2 ? 1u : 0u;          // first step of a group overwrites
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t a = smem_desc_sw128(base + L::off_p + bp * L::kP + kk * 32, 16, 1024);
+                    const uint64_t bv = smem_desc_sw128(kv_addr(stp) + L::kKV + kk * 2048, L::kKVHalf, 1024);
+                    mma_bf16_ss(tmem + L::colO + bp * D, a, bv, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t a = smem_desc_sw128(base + L::off_p + bp * L::kP + kk * 32, 16, 1024);
+                    const uint64_t bo = smem_desc_sw128(base + L::off_ones + kk * 32, 16, 1024);
+                    mma_bf16_ss(tmem + L::colL + bp * 32, a, bo, idesc_l, (acc || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(bar(B_PV_DONE + bp));
+                mma_commit(bar(B_KV_EMPTY + stp));
+                return true;
+            };
+            bool ok = mbar_wait(bar(B_Q), 0, abort_flag);
+            tc_fence_after();
+            if (ok) ok = issue_s(0);
+            if (ok && n > 1) ok = issue_s(1);
+            for (int p = 0; ok && p < n; ++p) {
+                // S_{p+2} reuses the S buffer of group p & 1 as soon as that group has read S_p
+                if (p + 2 < n && !issue_s(p + 2)) { ok = false; break; }
+                if (!issue_pv(p)) { ok = false; break; }
             }
-            if (ok) ok = issue_pv(n - 1);
             if (!ok) {
                 // every MMA this thread issued must finish before TMEM is released
                 mma_commit(bar(B_DRAIN));
@@ -199,51 +239,94 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
         }
     } else {
-        // ------------------------------------------------------------ softmax warps 0..3
-        const int r = tid;
+        // ------------------------------------------------------------ softmax groups
+        const int grp = warp / (4 * SPLIT);
+        const int wg = warp % (4 * SPLIT);
+        const int quarter = wg & 3, sp = wg >> 2;          // TMEM lane quarter, key split
+        const int r = quarter * 32 + lane;                  // tile row = TMEM lane
         const int hl = r / g.P, t = t0 + r % g.P;
         const bool valid = r < g.M && t < g.T;
         const int tpos = valid ? t : -1;
         const float tau_r = (valid && bt > 0) ? tau[(size_t)(b * g.Hq + kvh * g.G + hl) * g.T + t] : INFINITY;
-        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-        uint8_t* const prow_base = base_ptr + L::off_p + (r >> 3) * 1024 + (r & 7) * 128;
-        float m_run = -INFINITY, l_run = 0.f;
+        const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+        const uint32_t s_col = grp * 64 + sp * KEYS;        // this thread's keys in its group's S buffer
+        const uint32_t o_col = L::colO + grp * D + sp * RCOLS;   // O columns it rescales
+        const uint32_t l_col = L::colL + grp * 32;
+        uint8_t* const prow = base_ptr + L::off_p + grp * L::kP + (r >> 3) * 1024 + (r & 7) * 128;
+        const int row_bar = 1 + grp * 4 + quarter;          // named barrier of the row's SPLIT warps
+        float m_run = -INFINITY;
         bool ok = true;
         // TMEM loads and stores are warp-collective: every wait result is made warp-uniform
         auto wwait = [&](uint32_t bar_addr, uint32_t parity) -> bool {
             const bool got = mbar_wait(bar_addr, parity, abort_flag);
             return __all_sync(0xffffffffu, got);
         };
-        for (int s = 0; s < n; ++s) {
-            const int sb = s & 1;
+        auto row_sync = [&]() {
+            if constexpr (SPLIT > 1) asm volatile("bar.sync %0, %1;" :: "r"(row_bar), "n"(32 * SPLIT) : "memory");
+        };
+        // Each warp executes exactly one row barrier per step, even after a failed wait (a
+        // failed step skips its work but still synchronises), so the named barriers of the
+        // row's warps always match.
+        for (int s = grp; s < n; s += 2) {
+            const int i2 = s >> 1;                          // this group's step index
             const int j = s < U ? lst[s] : bt;
             const bool diag = (j == bt);
-            if (!wwait(bar(B_S_FULL + sb), (s >> 1) & 1)) { ok = false; break; }
-            tc_fence_after();
-            uint32_t sr[64];
-            tmem_ld32(lane_addr + sb * 64, sr);
-            tmem_ld32(lane_addr + sb * 64 + 32, sr + 32);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(bar(B_S_FREE + sb));
-            float rs = 0.f;
+            const bool okw = ok && wwait(bar(B_S_FULL + grp), i2 & 1);
+            uint32_t sr[KEYS];
+            float ps_own = 0.f, pm_own = -INFINITY;
+            if (okw) {
+                tc_fence_after();
+                tmem_ld<KEYS>(lane_addr + s_col, sr);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(bar(B_S_FREE + grp));
+                // partial row sum (for x_j): packed pairwise adds
+                uint64_t a2[4];
 #pragma unroll
-            for (int i = 0; i < 64; ++i) rs += __uint_as_float(sr[i]);
+                for (int i = 0; i < 4; ++i) a2[i] = f2_pack(sr[2 * i], sr[2 * i + 1]);
+#pragma unroll
+                for (int i = 4; i < KEYS / 2; ++i) a2[i & 3] = f2_add(a2[i & 3], f2_pack(sr[2 * i], sr[2 * i + 1]));
+                float s0, s1, s2, s3;
+                f2_unpack(f2_add(a2[0], a2[1]), s0, s1);
+                f2_unpack(f2_add(a2[2], a2[3]), s2, s3);
+                ps_own = (s0 + s1) + (s2 + s3);
+                // own block: keys after the query position are masked
+                if (diag) {
+                    const int key0 = j * kBlock + sp * KEYS;
+#pragma unroll
+                    for (int i = 0; i < KEYS; ++i)
+                        if (key0 + i > tpos) sr[i] = __float_as_uint(-INFINITY);
+                }
+                // partial raw max with three-input max
+                float m4[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) m4[i] = fmaxf(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
+#pragma unroll
+                for (int i = 4; i < KEYS / 2; ++i) m4[i & 3] = max3(m4[i & 3], __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
+                pm_own = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            }
+            float rs = ps_own, smax = pm_own;
+            if constexpr (SPLIT > 1) {
+                // every thread of the row combines the partials in the same order: identical x.
+                // Slots alternate with the step parity: a slot is rewritten two steps later,
+                // after every thread of the row has passed the barrier in between.
+                xch[i2 & 1][grp][sp][r] = make_float2(ps_own, pm_own);
+                row_sync();
+                rs = 0.f;
+                smax = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < SPLIT; ++k) {
+                    const float2 e = xch[i2 & 1][grp][k][r];
+                    rs += e.x;
+                    smax = fmaxf(smax, e.y);
+                }
+            }
+            if (!okw) { ok = false; continue; }
             const float x = rs * cxm;
             const float lp2 = diag ? (tpos >= 0 ? 0.f : -INFINITY)
                                    : (x > tau_r ? e_pow * __log2f(x - tau_r) : -INFINITY);
             const bool active = lp2 > -INFINITY;
-            float mx = -INFINITY;
-            if (active) {
-#pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    float l2 = fmaf(__uint_as_float(sr[i]), sm2, lp2);
-                    if (diag && j * kBlock + i > tpos) l2 = -INFINITY;
-                    sr[i] = __float_as_uint(l2);
-                    mx = fmaxf(mx, l2);
-                }
-            }
-            // running max and lazy rescale of the O row in TMEM
+            const float mx = active ? fmaf(smax, sm2, lp2) : -INFINITY;
             float factor = 1.f;
             bool resc = false;
             if (active) {
@@ -251,72 +334,98 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     m_run = mx;
                 } else if (mx > m_run + kLazyRescale) {
                     factor = exp2f(m_run - mx);
-                    l_run *= factor;
                     m_run = mx;
                     resc = true;
                 }
             }
+            // O_grp, L_grp and the P buffer were last used by this group's previous PV
+            if (i2 >= 1 && !wwait(bar(B_PV_DONE + grp), (i2 - 1) & 1)) { ok = false; continue; }
             if (__any_sync(0xffffffffu, resc)) {
-                // O must include PV_{s-1} before it is scaled
-                if (!wwait(bar(B_PV_DONE + ((s - 1) & 1)), ((s - 1) >> 1) & 1)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(lane_addr + 128 + c * 32, o);
+                for (int c = 0; c < RCOLS / RCW; ++c) {
+                    uint32_t o[RCW];
+                    tmem_ld<RCW>(lane_addr + o_col + c * RCW, o);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
-                    tmem_st32(lane_addr + 128 + c * 32, o);
+                    for (int i = 0; i < RCW; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
+                    tmem_st<RCW>(lane_addr + o_col + c * RCW, o);
+                }
+                if (sp == 0) {
+                    uint32_t o[16];
+                    tmem_ld16(lane_addr + l_col, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
+                    tmem_st16(lane_addr + l_col, o);
                 }
                 tmem_wait_st();
             }
-            // P buffer sb was last read by PV_{s-2}
-            if (s >= 2 && !wwait(bar(B_PV_DONE + sb), ((s - 2) >> 1) & 1)) { ok = false; break; }
-            float psum = 0.f;
-            uint8_t* prow = prow_base + sb * L::kP;
+            // p = 2^(s sm2 + log2 p_j - m): packed FMA, SFU exponent, bf16 pairs
+            const float c0 = lp2 - m_run;
+            const uint64_t sm2x2 = f2_pack(__float_as_uint(sm2), __float_as_uint(sm2));
+            const uint64_t c0x2 = f2_pack(__float_as_uint(c0), __float_as_uint(c0));
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint32_t pk[4];
+            for (int c = 0; c < KEYS / 8; ++c) {
+                uint32_t pk[4] = {0u, 0u, 0u, 0u};
+                if (active) {
 #pragma unroll
-                for (int q2 = 0; q2 < 4; ++q2) {
-                    float p0 = 0.f, p1 = 0.f;
-                    if (active) {
-                        p0 = exp2f(__uint_as_float(sr[c * 8 + 2 * q2]) - m_run);
-                        p1 = exp2f(__uint_as_float(sr[c * 8 + 2 * q2 + 1]) - m_run);
+                    for (int q2 = 0; q2 < 4; ++q2) {
+                        float e0, e1;
+                        f2_unpack(f2_fma(f2_pack(sr[c * 8 + 2 * q2], sr[c * 8 + 2 * q2 + 1]), sm2x2, c0x2), e0, e1);
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(fast_exp2(e0), fast_exp2(e1));
+                        pk[q2] = *reinterpret_cast<uint32_t*>(&h2);
                     }
-                    psum += p0 + p1;
-                    __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                    pk[q2] = *reinterpret_cast<uint32_t*>(&h2);
                 }
-                *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                const int chunk = sp * (KEYS / 8) + c;
+                *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
-            l_run += psum;
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(bar(B_P_FULL + sb));
+            mbar_arrive(bar(B_P_FULL + grp));
         }
-        // ---- epilogue: O / l -> bf16
-        if (ok && wwait(bar(B_PV_DONE + ((n - 1) & 1)), ((n - 1) >> 1) & 1)) {
+        // ---- merge the two groups: out = (O_0 2^(m_0-M) + O_1 2^(m_1-M)) / (L_0 ... + L_1 ...)
+        if (sp == 0) m_sh[grp][r] = m_run;
+        asm volatile("bar.sync %0, %1;" :: "r"(9), "n"(256 * SPLIT) : "memory");
+        const bool has1 = n >= 2;                           // group 1 ran at least one step
+        const int last0 = (n - 1) & ~1;                     // last step of group 0
+        const int last1 = (n - 1) - ((n - 1) & 1 ? 0 : 1);  // last step of group 1
+        bool done = ok && wwait(bar(B_PV_DONE + 0), (last0 >> 1) & 1);
+        if (has1) done = done && wwait(bar(B_PV_DONE + 1), (last1 >> 1) & 1);
+        if (done) {
             tc_fence_after();
-            const float inv = 1.0f / l_run;
-            __nv_bfloat16* dst = valid ? out + ((size_t)(b * g.Hq + kvh * g.G + hl) * g.T + t) * D : nullptr;
+            const float m0 = m_sh[0][r], m1 = has1 ? m_sh[1][r] : -INFINITY;
+            const float M = fmaxf(m0, m1);
+            const float w0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M);
+            const float w1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M);
+            const float l0 = __uint_as_float(tmem_ld1(lane_addr + L::colL));
+            float l1 = 0.f;
+            if (has1) l1 = __uint_as_float(tmem_ld1(lane_addr + L::colL + 32));
+            tmem_wait_ld();
+            const float inv = 1.0f / (l0 * w0 + (w1 > 0.f ? l1 * w1 : 0.f));
+            const int col0 = (grp * SPLIT + sp) * OCOLS;    // this thread's output columns
+            __nv_bfloat16* dst = valid ? out + ((size_t)(b * g.Hq + kvh * g.G + hl) * g.T + t) * D + col0 : nullptr;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t o[32];
-                tmem_ld32(lane_addr + 128 + c * 32, o);
+            for (int c = 0; c < OCOLS / OCW; ++c) {
+                uint32_t o0[OCW], o1[OCW];
+                tmem_ld<OCW>(lane_addr + L::colO + col0 + c * OCW, o0);
+                if (has1) tmem_ld<OCW>(lane_addr + L::colO + D + col0 + c * OCW, o1);
                 tmem_wait_ld();
                 if (valid) {
-                    uint32_t pk[16];
+                    uint32_t pk[OCW / 2];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(o[2 * i]) * inv,
-                                                                  __uint_as_float(o[2 * i + 1]) * inv);
+                    for (int i = 0; i < OCW / 2; ++i) {
+                        float a0 = __uint_as_float(o0[2 * i]) * w0, a1 = __uint_as_float(o0[2 * i + 1]) * w0;
+                        if (w1 > 0.f) {
+                            a0 = fmaf(__uint_as_float(o1[2 * i]), w1, a0);
+                            a1 = fmaf(__uint_as_float(o1[2 * i + 1]), w1, a1);
+                        }
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(a0 * inv, a1 * inv);
                         pk[i] = *reinterpret_cast<uint32_t*>(&h2);
                     }
-                    uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+                    uint4* d4 = reinterpret_cast<uint4*>(dst + c * OCW);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    for (int i = 0; i < OCW / 8; ++i) d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
                 }
             }
         }
@@ -325,7 +434,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, kTmemCols);
     }
     if (tid == 0 && abort_sh) atomicOr(&hdr->status, kStWaitTimeout);
 }
@@ -380,16 +489,17 @@ cudaError_t launch_fine_tc(const void* q, const void* k, const void* v, void* ou
     const int* count = reinterpret_cast<const int*>(ws + g.off_count);
     WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
     auto* ob = static_cast<__nv_bfloat16*>(out);
+    constexpr int threads = (8 * kFineSplit + 2) * 32;
     if (g.d == 128) {
         const int sm = (int)TcLayout<128>::bytes;
-        cudaError_t e = cudaFuncSetAttribute(fine_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+        cudaError_t e = cudaFuncSetAttribute(fine_tc_kernel<128, kFineSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
         if (e != cudaSuccess) return e;
-        fine_tc_kernel<128><<<g.ntiles, kTcThreads, sm, stream>>>(tq, tk, tv, ob, tau, list, count, hdr, g, cxm, e_pow, sm2);
+        fine_tc_kernel<128, kFineSplit><<<g.ntiles, threads, sm, stream>>>(tq, tk, tv, ob, tau, list, count, hdr, g, cxm, e_pow, sm2);
     } else {
         const int sm = (int)TcLayout<64>::bytes;
-        cudaError_t e = cudaFuncSetAttribute(fine_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+        cudaError_t e = cudaFuncSetAttribute(fine_tc_kernel<64, kFineSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
         if (e != cudaSuccess) return e;
-        fine_tc_kernel<64><<<g.ntiles, kTcThreads, sm, stream>>>(tq, tk, tv, ob, tau, list, count, hdr, g, cxm, e_pow, sm2);
+        fine_tc_kernel<64, kFineSplit><<<g.ntiles, threads, sm, stream>>>(tq, tk, tv, ob, tau, list, count, hdr, g, cxm, e_pow, sm2);
     }
     return cudaGetLastError();
 }
