@@ -15,11 +15,15 @@
 // in flight while sharing the Q tile and every K/V load.  Warps:
 //   8 SPLIT            TMA producer (one lane): the Q tile once (one 64-column box per head
 //                      and half of d), then K and V of every listed block, 4-stage ring;
-//   8 SPLIT + 1        MMA issuer (one lane): S_s = Q K_s^T (M=128, N=64) into the S buffer
-//                      of group s & 1 as soon as that group has read S_{s-2}, so S_{s+2} is
-//                      computed while the group works on step s; O_g += P_s V_s (M=128, N=d)
-//                      and L_g += P_s 1 (N=16, an all-ones B tile: the softmax denominator
-//                      summed by the tensor core over exactly the bf16 P it multiplies);
+//   8 SPLIT + 1        S issuer (one lane): S_s = Q K_s^T (M=128, N=64) into the S buffer of
+//                      group s & 1 as soon as block s is loaded and that group has read
+//                      S_{s-2}, so S_{s+2} is computed while the group works on step s;
+//   8 SPLIT + 2        PV issuer (one lane): O_g += P_s V_s (M=128, N=d) and L_g += P_s 1
+//                      (N=16, an all-ones B tile: the softmax denominator summed by the
+//                      tensor core over exactly the bf16 P it multiplies) as soon as P_s is
+//                      written.  Two issuing threads keep a slow K/V load of a later block
+//                      from delaying the PV of an earlier one (tcgen05.commit tracks each
+//                      thread's own MMAs);
 //   0 .. 8 SPLIT - 1   softmax, group = warp / (4 SPLIT); SPLIT threads per tile row (warps
 //                      of one group sharing TMEM lanes 32 (warp % 4).. split the row's keys
 //                      and exchange partial row sums and maxima through shared memory behind
@@ -63,10 +67,10 @@ constexpr uint32_t kTmemCols = 512;
 // barrier slots
 enum : int { B_Q = 0, B_KV_FULL = 1, B_KV_EMPTY = 1 + kTcStages, B_S_FULL = 1 + 2 * kTcStages,
              B_S_FREE = B_S_FULL + 2, B_P_FULL = B_S_FREE + 2, B_PV_DONE = B_P_FULL + 2,
-             B_DRAIN = B_PV_DONE + 2, B_COUNT = B_DRAIN + 1 };
+             B_DRAIN = B_PV_DONE + 2, B_DRAIN2 = B_DRAIN + 1, B_COUNT = B_DRAIN2 + 1 };
 
 template <int D, int SPLIT>
-__global__ void __launch_bounds__((8 * SPLIT + 2) * 32, 1)
+__global__ void __launch_bounds__((8 * SPLIT + 3) * 32, 1)
 fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
                const float* __restrict__ tau, const int* __restrict__ list, const int* __restrict__ count,
@@ -79,7 +83,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     constexpr int OCW = OCOLS < 32 ? OCOLS : 32;
     constexpr int RCOLS = D / SPLIT;            // O columns a thread rescales in its group
     constexpr int RCW = RCOLS < 32 ? RCOLS : 32;
-    constexpr int kProducerWarp = 8 * SPLIT, kMmaWarp = 8 * SPLIT + 1;
+    constexpr int kProducerWarp = 8 * SPLIT, kMmaSWarp = 8 * SPLIT + 1, kMmaPvWarp = 8 * SPLIT + 2;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t bars[B_COUNT];
     __shared__ uint32_t tmem_base_sh;
@@ -120,6 +124,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(bar(B_PV_DONE + i), 1);
         }
         mbar_init(bar(B_DRAIN), 1);
+        mbar_init(bar(B_DRAIN2), 1);
         fence_mbar_init();
     }
     // rows of the Q tile beyond G * P are never loaded: zero them once
@@ -180,16 +185,17 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     if (last_armed[st] >= 0) { dummy = 0; mbar_wait(bar(B_KV_FULL + st), (last_armed[st] / kTcStages) & 1, &dummy); }
             }
         }
-    } else if (warp == kMmaWarp) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == kMmaSWarp) {
+        // ------------------------------------------------------------ S issuer
+        // S_s = Q K_s^T into the S buffer of group s & 1, as soon as block s is loaded and the
+        // group has read S_{s-2}: it runs ahead of the softmax by up to one step per group.
         if (lane == 0) {
             const uint32_t idesc_s = idesc_bf16(128, 64, false);
-            const uint32_t idesc_pv = idesc_bf16(128, D, true);
-            const uint32_t idesc_l = idesc_bf16(128, 16, false);
-            auto issue_s = [&](int s) -> bool {
+            bool ok = mbar_wait(bar(B_Q), 0, abort_flag);
+            for (int s = 0; ok && s < n; ++s) {
                 const int st = s % kTcStages, sb = s & 1;
-                if (!mbar_wait(bar(B_KV_FULL + st), (s / kTcStages) & 1, abort_flag)) return false;
-                if (s >= 2 && !mbar_wait(bar(B_S_FREE + sb), ((s - 2) >> 1) & 1, abort_flag)) return false;
+                if (!mbar_wait(bar(B_KV_FULL + st), (s / kTcStages) & 1, abort_flag)) { ok = false; break; }
+                if (s >= 2 && !mbar_wait(bar(B_S_FREE + sb), ((s - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -199,11 +205,25 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     mma_bf16_ss(tmem + sb * 64, a, bk, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar(B_S_FULL + sb));
-                return true;
-            };
-            auto issue_pv = [&](int p) -> bool {
+            }
+            if (!ok) {
+                // every MMA this thread issued must finish before TMEM is released
+                mma_commit(bar(B_DRAIN));
+                volatile int dummy = 0;
+                mbar_wait(bar(B_DRAIN), 0, &dummy);
+            }
+        }
+    } else if (warp == kMmaPvWarp) {
+        // ------------------------------------------------------------ PV issuer
+        // O_g += P_p V_p and L_g += P_p 1 as soon as P_p is written; then the K/V stage of
+        // block p is free (S_p finished before the softmax could write P_p).
+        if (lane == 0) {
+            const uint32_t idesc_pv = idesc_bf16(128, D, true);
+            const uint32_t idesc_l = idesc_bf16(128, 16, false);
+            bool ok = true;
+            for (int p = 0; p < n; ++p) {
                 const int bp = p & 1, stp = p % kTcStages;
-                if (!mbar_wait(bar(B_P_FULL + bp), (p >> 1) & 1, abort_flag)) return false;
+                if (!mbar_wait(bar(B_P_FULL + bp), (p >> 1) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t acc = p >= 2 ? 1u : 0u;          // first step of a group overwrites
 #pragma unroll
@@ -220,22 +240,11 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
                 mma_commit(bar(B_PV_DONE + bp));
                 mma_commit(bar(B_KV_EMPTY + stp));
-                return true;
-            };
-            bool ok = mbar_wait(bar(B_Q), 0, abort_flag);
-            tc_fence_after();
-            if (ok) ok = issue_s(0);
-            if (ok && n > 1) ok = issue_s(1);
-            for (int p = 0; ok && p < n; ++p) {
-                // S_{p+2} reuses the S buffer of group p & 1 as soon as that group has read S_p
-                if (p + 2 < n && !issue_s(p + 2)) { ok = false; break; }
-                if (!issue_pv(p)) { ok = false; break; }
             }
             if (!ok) {
-                // every MMA this thread issued must finish before TMEM is released
-                mma_commit(bar(B_DRAIN));
+                mma_commit(bar(B_DRAIN2));
                 volatile int dummy = 0;
-                mbar_wait(bar(B_DRAIN), 0, &dummy);
+                mbar_wait(bar(B_DRAIN2), 0, &dummy);
             }
         }
     } else {
@@ -340,6 +349,26 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             // O_grp, L_grp and the P buffer were last used by this group's previous PV
             if (i2 >= 1 && !wwait(bar(B_PV_DONE + grp), (i2 - 1) & 1)) { ok = false; continue; }
+            // p = 2^(s sm2 + log2 p_j - m): packed FMA, SFU exponent, bf16 pairs
+            const float c0 = lp2 - m_run;
+            const uint64_t sm2x2 = f2_pack(__float_as_uint(sm2), __float_as_uint(sm2));
+            const uint64_t c0x2 = f2_pack(__float_as_uint(c0), __float_as_uint(c0));
+#pragma unroll
+            for (int c = 0; c < KEYS / 8; ++c) {
+                uint32_t pk[4] = {0u, 0u, 0u, 0u};
+                if (active) {
+#pragma unroll
+                    for (int q2 = 0; q2 < 4; ++q2) {
+                        float e0, e1;
+                        f2_unpack(f2_fma(f2_pack(sr[c * 8 + 2 * q2], sr[c * 8 + 2 * q2 + 1]), sm2x2, c0x2), e0, e1);
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(fast_exp2(e0), fast_exp2(e1));
+                        pk[q2] = *reinterpret_cast<uint32_t*>(&h2);
+                    }
+                }
+                const int chunk = sp * (KEYS / 8) + c;
+                *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+            // rescale after P: the S registers are dead by now
             if (__any_sync(0xffffffffu, resc)) {
                 tc_fence_after();
 #pragma unroll
@@ -360,25 +389,6 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     tmem_st16(lane_addr + l_col, o);
                 }
                 tmem_wait_st();
-            }
-            // p = 2^(s sm2 + log2 p_j - m): packed FMA, SFU exponent, bf16 pairs
-            const float c0 = lp2 - m_run;
-            const uint64_t sm2x2 = f2_pack(__float_as_uint(sm2), __float_as_uint(sm2));
-            const uint64_t c0x2 = f2_pack(__float_as_uint(c0), __float_as_uint(c0));
-#pragma unroll
-            for (int c = 0; c < KEYS / 8; ++c) {
-                uint32_t pk[4] = {0u, 0u, 0u, 0u};
-                if (active) {
-#pragma unroll
-                    for (int q2 = 0; q2 < 4; ++q2) {
-                        float e0, e1;
-                        f2_unpack(f2_fma(f2_pack(sr[c * 8 + 2 * q2], sr[c * 8 + 2 * q2 + 1]), sm2x2, c0x2), e0, e1);
-                        __nv_bfloat162 h2 = __floats2bfloat162_rn(fast_exp2(e0), fast_exp2(e1));
-                        pk[q2] = *reinterpret_cast<uint32_t*>(&h2);
-                    }
-                }
-                const int chunk = sp * (KEYS / 8) + c;
-                *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -489,7 +499,7 @@ cudaError_t launch_fine_tc(const void* q, const void* k, const void* v, void* ou
     const int* count = reinterpret_cast<const int*>(ws + g.off_count);
     WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
     auto* ob = static_cast<__nv_bfloat16*>(out);
-    constexpr int threads = (8 * kFineSplit + 2) * 32;
+    constexpr int threads = (8 * kFineSplit + 3) * 32;
     if (g.d == 128) {
         const int sm = (int)TcLayout<128>::bytes;
         cudaError_t e = cudaFuncSetAttribute(fine_tc_kernel<128, kFineSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
