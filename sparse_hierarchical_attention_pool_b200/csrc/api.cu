@@ -85,10 +85,14 @@ static int prefill_impl(const void* q, const void* k, const void* v, void* out, 
     };
     if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), s) != cudaSuccess) return DASH_ERR_CUDA;
     if (!mark(0)) return DASH_ERR_CUDA;
-    if (g.nbs > 0 && launch_block_summary(k, reinterpret_cast<float*>(ws + g.off_ksum), B, Hkv, T, d, s) != cudaSuccess)
+    if (g.nbs > 0 && launch_block_summary(k, reinterpret_cast<float*>(ws + g.off_ksum), B, Hkv, T, d, s,
+                                          ws + g.off_khi, ws + g.off_klo) != cudaSuccess)
         return DASH_ERR_CUDA;
     if (!mark(1)) return DASH_ERR_CUDA;
-    if (launch_coarse(q, g, ws, alpha, coarse_scale, s) != cudaSuccess) return DASH_ERR_CUDA;
+    const cudaError_t ce = g.tc ? (coarse_tc_supported(g) ? launch_coarse_tc(q, g, ws, alpha, coarse_scale, s)
+                                                          : launch_coarse(q, g, ws, alpha, coarse_scale, s))
+                                : launch_coarse(q, g, ws, alpha, coarse_scale, s);
+    if (ce != cudaSuccess) return DASH_ERR_CUDA;
     if (!mark(2)) return DASH_ERR_CUDA;
     if (launch_fine(q, k, v, out, g, ws, alpha, coarse_scale, s) != cudaSuccess) return DASH_ERR_CUDA;
     if (!mark(3)) return DASH_ERR_CUDA;

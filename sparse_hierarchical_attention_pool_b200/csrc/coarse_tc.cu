@@ -1,0 +1,466 @@
+// coarse_tc.cu -- Stage 1 for prefill on the tensor cores: block scores, alpha-entmax
+// thresholds and per-tile block lists.
+//
+// "DashAttention: Making Sparse Attention Fully Differentiable with Adaptive Block
+// Selection", section "Core Mechanism" (Stage 1: coarse scores Q * block_summary, then
+// alpha-entmax gives sparse block weights).  For a work tile (P positions inside one key
+// block x the G query heads of one KV head; every row has the same own block bt) the
+// scores of the 128 rows against the bt past block summaries are
+//     x[r, j] = (alpha - 1) * coarse_scale * (q_r . kbar_j) / sqrt(d),
+// computed as Q (bf16, exact) times kbar split into bf16 hi + lo parts (kbar = hi + lo to
+// 2^-17 relative), so the fp32 accumulation matches an fp32 dot product closely.
+//
+// Persistent kernel, one CTA per SM, 320 threads:
+//   warp 9 (one lane)  TMA producer: Q tile, then 128-block chunks of kbar hi and lo
+//                      through a 2-stage ring;
+//   warp 8 (one lane)  MMA issuer: S_chunk = Q [hi | lo]^T (M=128, N=128, K=2d) into a
+//                      4-chunk TMEM ring (512 columns) whose buffers rotate across tiles,
+//                      so a short tile's scores are computed while the previous tile is
+//                      still being solved;
+//   warps 0-7          two threads per row (warps w and w+4 share TMEM lanes 32 (w%4)..
+//                      and take alternate 32-block groups; their pass sums are merged in
+//                      shared memory in a fixed order): pass 0 takes the row maximum;
+//                      then Newton / exact-support passes for tau (entmax.cuh) until every
+//                      row of the tile has its final threshold; a last pass ORs each
+//                      block's "x > tau" over the rows (warp OR-reductions into a shared
+//                      bitmap) and counts selected pairs; warp 0 compacts the bitmap into
+//                      the tile's ascending block list.
+// Tiles with bt <= 512 keep all their scores in TMEM: one GEMM pass, every further pass
+// reads TMEM.  Longer tiles recompute their score chunks for every pass; the threshold
+// warps tell the producer and the MMA issuer after each pass whether another is needed.
+// Every wait is bounded (~2 s); a CTA that gives up sets a status bit and exits cleanly.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "entmax.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace dash {
+
+constexpr int kCtStages = 2;
+constexpr int kCtChunk = 128;        // blocks per score chunk (MMA N)
+constexpr int kCtBufs = 4;           // TMEM chunk buffers (4 x 128 columns)
+
+template <int D>
+struct CtLayout {
+    static constexpr uint32_t kQHalf = 128 * 128;
+    static constexpr uint32_t kQ = (D / 64) * kQHalf;
+    static constexpr uint32_t kKHalf = kCtChunk * 128;          // 128 blocks x 64 bf16
+    static constexpr uint32_t kKPart = (D / 64) * kKHalf;       // hi or lo of one chunk
+    static constexpr uint32_t kStage = 2 * kKPart;              // hi then lo
+    static constexpr uint32_t off_q = 0;
+    static constexpr uint32_t off_k = kQ;
+    static constexpr uint32_t bytes = off_k + kCtStages * kStage + 1024;
+};
+
+enum : int { C_Q_FULL = 0, C_Q_EMPTY = 1, C_K_FULL = 2, C_K_EMPTY = C_K_FULL + kCtStages,
+             C_C_FULL = C_K_EMPTY + kCtStages, C_C_FREE = C_C_FULL + kCtBufs,
+             C_DEC = C_C_FREE + kCtBufs, C_DRAIN = C_DEC + 1, C_COUNT = C_DRAIN + 1 };
+
+struct TileInfo {
+    int b, kvh, bg, t0, bt, nch;
+    size_t tile_id;
+    bool resident;
+};
+
+__device__ __forceinline__ TileInfo tile_info(const PrefillGeom& g, int w) {
+    TileInfo ti;
+    const int BH = g.B * g.Hkv;
+    const int it = g.ntile_bg - 1 - w / BH;
+    ti.bg = w % BH;
+    ti.b = ti.bg / g.Hkv;
+    ti.kvh = ti.bg % g.Hkv;
+    ti.t0 = it * g.P;
+    ti.bt = ti.t0 / kBlock;
+    ti.tile_id = (size_t)ti.bg * g.ntile_bg + it;
+    ti.nch = (ti.bt + kCtChunk - 1) / kCtChunk;
+    ti.resident = ti.nch <= kCtBufs;
+    return ti;
+}
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_hi,
+                 const __grid_constant__ CUtensorMap tm_lo, float* __restrict__ tau_out,
+                 int* __restrict__ list, int* __restrict__ count, WsHeader* __restrict__ hdr,
+                 PrefillGeom g, float alpha, float cx) {
+    using L = CtLayout<D>;
+    using namespace sm100;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t bars[C_COUNT];
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+    __shared__ int decision_sh;                  // 1: another pass over the scores follows
+    __shared__ int unconverged_sh;
+    __shared__ unsigned bitmap[kMaxT / kBlock / 32];
+    __shared__ unsigned long long sel_sh;
+    __shared__ float xs[2][6][kTileRows];        // [half][sum][row]: partial pass sums
+
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
+    auto k_addr = [&](int st) { return base + L::off_k + (uint32_t)st * L::kStage; };
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (tid == 0) {
+        abort_sh = 0;
+        mbar_init(bar(C_Q_FULL), 1);
+        mbar_init(bar(C_Q_EMPTY), 1);
+        for (int st = 0; st < kCtStages; ++st) {
+            mbar_init(bar(C_K_FULL + st), 1);
+            mbar_init(bar(C_K_EMPTY + st), 1);
+        }
+        for (int i = 0; i < kCtBufs; ++i) {
+            mbar_init(bar(C_C_FULL + i), 1);
+            mbar_init(bar(C_C_FREE + i), 256);
+        }
+        mbar_init(bar(C_DEC), 1);
+        mbar_init(bar(C_DRAIN), 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&tmem_base_sh), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+    volatile int* abort_flag = &abort_sh;
+
+    if (warp == 9) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_hi);
+            prefetch_tmap(&tm_lo);
+            int ntile = 0, kcount = 0, ndec = 0;
+            int last_armed[kCtStages] = {-1, -1};
+            bool ok = true;
+            for (int w = blockIdx.x; ok && w < g.ntiles; w += gridDim.x) {
+                const TileInfo ti = tile_info(g, w);
+                if (ti.bt == 0) continue;
+                if (ntile > 0 && !mbar_wait(bar(C_Q_EMPTY), (ntile - 1) & 1, abort_flag)) { ok = false; break; }
+                mbar_arrive_expect_tx(bar(C_Q_FULL), (uint32_t)(g.M * D * 2));
+                for (int hl = 0; hl < g.G; ++hl) {
+                    const int row = (ti.b * g.Hq + ti.kvh * g.G + hl) * g.T + ti.t0;
+                    for (int h = 0; h < D / 64; ++h)
+                        tma_load_2d(base + L::off_q + h * L::kQHalf + hl * g.P * 128, &tm_q, h * 64, row, bar(C_Q_FULL));
+                }
+                ++ntile;
+                while (ok) {
+                    for (int c = 0; c < ti.nch; ++c) {
+                        const int st = kcount % kCtStages;
+                        if (kcount >= kCtStages && !mbar_wait(bar(C_K_EMPTY + st), ((kcount / kCtStages) - 1) & 1, abort_flag)) { ok = false; break; }
+                        const int row = ti.bg * g.nbs + c * kCtChunk;
+                        mbar_arrive_expect_tx(bar(C_K_FULL + st), (uint32_t)(2 * kCtChunk * D * 2));
+                        for (int h = 0; h < D / 64; ++h) {
+                            tma_load_2d(k_addr(st) + h * L::kKHalf, &tm_hi, h * 64, row, bar(C_K_FULL + st));
+                            tma_load_2d(k_addr(st) + L::kKPart + h * L::kKHalf, &tm_lo, h * 64, row, bar(C_K_FULL + st));
+                        }
+                        last_armed[st] = kcount;
+                        ++kcount;
+                    }
+                    if (!ok || ti.resident) break;
+                    if (!mbar_wait(bar(C_DEC), ndec & 1, abort_flag)) { ok = false; break; }
+                    ++ndec;
+                    if (!*(volatile int*)&decision_sh) break;
+                }
+            }
+            if (!ok) {
+                // let every load this thread started land before the CTA exits
+                volatile int dummy = 0;
+                if (ntile > 0) mbar_wait(bar(C_Q_FULL), (ntile - 1) & 1, &dummy);
+                for (int st = 0; st < kCtStages; ++st)
+                    if (last_armed[st] >= 0) { dummy = 0; mbar_wait(bar(C_K_FULL + st), (last_armed[st] / kCtStages) & 1, &dummy); }
+            }
+        }
+    } else if (warp == 8) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(128, kCtChunk, false);
+            int ntile = 0, kcount = 0, ndec = 0, gch = 0;
+            int uses[kCtBufs] = {0, 0, 0, 0};
+            bool ok = true;
+            for (int w = blockIdx.x; ok && w < g.ntiles; w += gridDim.x) {
+                const TileInfo ti = tile_info(g, w);
+                if (ti.bt == 0) continue;
+                if (!mbar_wait(bar(C_Q_FULL), ntile & 1, abort_flag)) { ok = false; break; }
+                ++ntile;
+                while (ok) {
+                    for (int c = 0; c < ti.nch; ++c) {
+                        const int st = kcount % kCtStages, bf = gch % kCtBufs;
+                        if (!mbar_wait(bar(C_K_FULL + st), (kcount / kCtStages) & 1, abort_flag)) { ok = false; break; }
+                        if (uses[bf] > 0 && !mbar_wait(bar(C_C_FREE + bf), (uses[bf] - 1) & 1, abort_flag)) { ok = false; break; }
+                        tc_fence_after();
+#pragma unroll
+                        for (int part = 0; part < 2; ++part)
+#pragma unroll
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                const int h = kk >> 2, wk = kk & 3;
+                                const uint64_t a = smem_desc_sw128(base + L::off_q + h * L::kQHalf + wk * 32, 16, 1024);
+                                const uint64_t bk = smem_desc_sw128(k_addr(st) + part * L::kKPart + h * L::kKHalf + wk * 32, 16, 1024);
+                                mma_bf16_ss(tmem + bf * kCtChunk, a, bk, idesc, (part > 0 || kk > 0) ? 1u : 0u);
+                            }
+                        mma_commit(bar(C_C_FULL + bf));
+                        mma_commit(bar(C_K_EMPTY + st));
+                        ++uses[bf];
+                        ++kcount;
+                        ++gch;
+                    }
+                    if (!ok || ti.resident) break;
+                    if (!mbar_wait(bar(C_DEC), ndec & 1, abort_flag)) { ok = false; break; }
+                    ++ndec;
+                    if (!*(volatile int*)&decision_sh) break;
+                }
+                mma_commit(bar(C_Q_EMPTY));                 // Q of this tile no longer read
+            }
+            if (!ok) {
+                mma_commit(bar(C_DRAIN));
+                volatile int dummy = 0;
+                mbar_wait(bar(C_DRAIN), 0, &dummy);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ threshold warps 0-7
+        const int quarter = warp & 3, hf = warp >> 2;
+        const int r = quarter * 32 + lane;                  // tile row = TMEM lane
+        const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+        int uses[kCtBufs] = {0, 0, 0, 0};
+        int gch = 0;
+        int no_conv = 0;
+        bool ok = true;
+        auto wwait = [&](uint32_t bar_addr, uint32_t parity) -> bool {
+            const bool got = mbar_wait(bar_addr, parity, abort_flag);
+            return __all_sync(0xffffffffu, got);
+        };
+        auto sync8 = [&]() { asm volatile("bar.sync 1, 256;" ::: "memory"); };
+        for (int w = blockIdx.x; ok && w < g.ntiles; w += gridDim.x) {
+            const TileInfo ti = tile_info(g, w);
+            const int hl = r / g.P, t = ti.t0 + r % g.P;
+            const bool valid = r < g.M && t < g.T;
+            const size_t tau_idx = (size_t)(ti.b * g.Hq + ti.kvh * g.G + hl) * g.T + t;
+            if (ti.bt == 0) {
+                if (valid && hf == 0) tau_out[tau_idx] = __int_as_float(0x7fc00000);
+                if (r == 0 && hf == 0) count[ti.tile_id] = 0;
+                continue;
+            }
+            // chunk c of the current sweep sits in TMEM buffer (sweep_base + c) % 4
+            int sweep_base = gch;
+            int pass = 0;
+            auto acquire = [&](int bf) -> bool {
+                if (!wwait(bar(C_C_FULL + bf), uses[bf] & 1)) return false;
+                tc_fence_after();
+                return true;
+            };
+            auto release = [&](int bf) {
+                tc_fence_before();
+                mbar_arrive(bar(C_C_FREE + bf));
+                ++uses[bf];
+            };
+            // one sweep over the row's scores: streamed tiles acquire and release every
+            // chunk of every pass, resident tiles acquire in pass 0 and release at the end
+            auto run_pass = [&](auto&& fn) -> bool {
+                if (!ti.resident || pass == 0) { sweep_base = gch; gch += ti.nch; }
+                for (int c = 0; c < ti.nch; ++c) {
+                    const int bf = (sweep_base + c) % kCtBufs;
+                    if ((!ti.resident || pass == 0) && !acquire(bf)) return false;
+                    const int ncol = min(kCtChunk, ti.bt - c * kCtChunk);
+                    for (int g32 = hf; g32 < (ncol + 31) / 32; g32 += 2) {
+                        uint32_t v[32];
+                        tmem_ld32(lane_addr + bf * kCtChunk + g32 * 32, v);
+                        tmem_wait_ld();
+                        fn(c * kCtChunk + g32 * 32, v, min(32, ncol - g32 * 32));
+                    }
+                    if (!ti.resident) release(bf);
+                }
+                ++pass;
+                return true;
+            };
+            // announce whether the scores are swept once more (streamed tiles only)
+            auto announce = [&](bool more) {
+                if (ti.resident) return;
+                if (r == 0 && hf == 0) {
+                    decision_sh = more ? 1 : 0;
+                    __threadfence_block();
+                    mbar_arrive(bar(C_DEC));
+                }
+            };
+            // ---- pass 0: row maximum
+            float m = -INFINITY;
+            if (!run_pass([&](int, const uint32_t* v, int nv) {
+                    for (int i = 0; i < 32; ++i)
+                        if (i < nv) m = fmaxf(m, __fmul_rn(__uint_as_float(v[i]), cx));
+                })) { ok = false; break; }
+            xs[hf][0][r] = m;
+            sync8();
+            m = fmaxf(xs[0][0][r], xs[1][0][r]);
+            EntmaxSolver sv;
+            sv.init(m, alpha);
+            float tau = INFINITY;
+            bool done = !valid;
+            // ---- Newton / exact-support passes until every row of the tile is final
+            while (true) {
+                sync8();                                   // the previous flag and sums have been read
+                if (r == 0 && hf == 0) unconverged_sh = 0;
+                sync8();
+                if (!done && hf == 0) atomicOr(&unconverged_sh, 1);
+                sync8();
+                const bool more = unconverged_sh != 0;
+                announce(true);                            // a Newton pass or the union pass follows
+                if (!more) break;
+                EntmaxPass ps;
+                ps.reset();
+                // z = (x - m) - u with x rounded exactly as in pass 0 (__fmul_rn is never fused
+                // into an FMA), so the maximum gives z = -u exactly
+                if (!run_pass([&](int, const uint32_t* v, int nv) {
+                        for (int i = 0; i < 32; ++i)
+                            if (i < nv) ps.add((__fmul_rn(__uint_as_float(v[i]), cx) - sv.m) - sv.u, sv.mode, sv.e);
+                    })) { ok = false; break; }
+                xs[hf][0][r] = ps.z0; xs[hf][1][r] = ps.z1; xs[hf][2][r] = ps.z2;
+                xs[hf][3][r] = ps.fe; xs[hf][4][r] = ps.de; xs[hf][5][r] = ps.minz;
+                sync8();
+                // both threads of the row merge the halves in the same order
+                EntmaxPass tot;
+                tot.z0 = xs[0][0][r] + xs[1][0][r]; tot.z1 = xs[0][1][r] + xs[1][1][r];
+                tot.z2 = xs[0][2][r] + xs[1][2][r]; tot.fe = xs[0][3][r] + xs[1][3][r];
+                tot.de = xs[0][4][r] + xs[1][4][r]; tot.minz = fminf(xs[0][5][r], xs[1][5][r]);
+                if (!done) done = sv.update(tot, &tau, &no_conv);
+            }
+            if (!ok) break;
+            // ---- union pass: OR of x > tau over the rows, per block
+            const int nw = (ti.bt + 31) / 32;
+            for (int i = warp * 32 + lane; i < nw; i += 256) bitmap[i] = 0u;
+            if (r == 0 && hf == 0) sel_sh = 0ull;
+            sync8();
+            float nsel = 0.f;
+            if (!run_pass([&](int j0, const uint32_t* v, int nv) {
+                    unsigned mask = 0u;
+                    for (int i = 0; i < 32; ++i)
+                        if (i < nv && valid && __fmul_rn(__uint_as_float(v[i]), cx) > tau) mask |= 1u << i;
+                    nsel += (float)__popc(mask);
+                    const unsigned wm = __reduce_or_sync(0xffffffffu, mask);
+                    if (lane == 0 && wm) atomicOr(&bitmap[j0 >> 5], wm);
+                })) { ok = false; break; }
+            announce(false);
+            if (ti.resident)
+                for (int c = 0; c < ti.nch; ++c) release((sweep_base + c) % kCtBufs);
+            if (valid && hf == 0) tau_out[tau_idx] = tau;
+            nsel = warp_sum(nsel);
+            if (lane == 0) atomicAdd(&sel_sh, (unsigned long long)nsel);
+            sync8();
+            if (warp == 0) {
+                int basei = 0;
+                int* dst = list + ti.tile_id * g.cap;
+                for (int w0 = 0; w0 < nw; w0 += 32) {
+                    const int wi = w0 + lane;
+                    unsigned word = wi < nw ? bitmap[wi] : 0u;
+                    const int pc = __popc(word);
+                    int incl = pc;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int nn = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (lane >= o) incl += nn;
+                    }
+                    int pos = basei + incl - pc;
+                    while (word) {
+                        const int bit = __ffs(word) - 1;
+                        dst[pos++] = wi * 32 + bit;
+                        word &= word - 1;
+                    }
+                    basei += __shfl_sync(0xffffffffu, incl, 31);
+                }
+                if (lane == 0) {
+                    count[ti.tile_id] = basei;
+                    const int rows_valid = g.G * min(g.P, g.T - ti.t0);
+                    atomicAdd(&hdr->selected_pairs, sel_sh);
+                    atomicAdd(&hdr->scored_pairs, (unsigned long long)rows_valid * ti.bt);
+                    atomicAdd(&hdr->union_blocks, (unsigned long long)basei);
+                    atomicAdd(&hdr->tiles, 1ull);
+                }
+            }
+            sync8();
+        }
+        if (no_conv) atomicOr(&hdr->status, kStNoConverge);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+    if (tid == 0 && abort_sh) atomicOr(&hdr->status, kStWaitTimeout);
+}
+
+// ------------------------------------------------------------------ host side
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn_ct() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+bool make_map_ct(CUtensorMap* m, const void* ptr, unsigned long long rows, int d, int box_rows) {
+    auto fn = encode_fn_ct();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+}  // namespace
+
+bool coarse_tc_supported(const PrefillGeom& g) { return g.P >= 8 && g.nbs > 0; }
+
+cudaError_t launch_coarse_tc(const void* q, const PrefillGeom& g, char* ws, float alpha,
+                             float coarse_scale, cudaStream_t stream) {
+    const float cx = (alpha - 1.0f) * coarse_scale / sqrtf((float)g.d);
+    CUtensorMap tq, thi, tlo;
+    const unsigned long long qrows = (unsigned long long)g.B * g.Hq * g.T;
+    const unsigned long long krows = (unsigned long long)g.B * g.Hkv * g.nbs;
+    if (!make_map_ct(&tq, q, qrows, g.d, g.P) ||
+        !make_map_ct(&thi, ws + g.off_khi, krows, g.d, kCtChunk) ||
+        !make_map_ct(&tlo, ws + g.off_klo, krows, g.d, kCtChunk))
+        return cudaErrorInvalidValue;
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
+    float* tau = reinterpret_cast<float*>(ws + g.off_tau);
+    int* list = reinterpret_cast<int*>(ws + g.off_list);
+    int* count = reinterpret_cast<int*>(ws + g.off_count);
+    const int grid = g.ntiles < sm_count() ? g.ntiles : sm_count();
+    if (g.d == 128) {
+        const int sm = (int)CtLayout<128>::bytes;
+        cudaError_t e = cudaFuncSetAttribute(coarse_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+        if (e != cudaSuccess) return e;
+        coarse_tc_kernel<128><<<grid, 320, sm, stream>>>(tq, thi, tlo, tau, list, count, hdr, g, alpha, cx);
+    } else {
+        const int sm = (int)CtLayout<64>::bytes;
+        cudaError_t e = cudaFuncSetAttribute(coarse_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+        if (e != cudaSuccess) return e;
+        coarse_tc_kernel<64><<<grid, 320, sm, stream>>>(tq, thi, tlo, tau, list, count, hdr, g, alpha, cx);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace dash

@@ -38,7 +38,8 @@ struct PrefillGeom {
     int ntiles;                      // B * Hkv * ntile_bg
     int nbs;                         // complete blocks = T / 64
     int cap;                         // list capacity per tile = max(1, nbs)
-    size_t off_ksum, off_tau, off_list, off_count, off_scratch, total;
+    bool tc;                         // tensor-core Stage 1/2 kernels (needs P >= 8)
+    size_t off_ksum, off_khi, off_klo, off_tau, off_list, off_count, off_scratch, total;
 };
 
 inline int pow2_floor(int x) {
@@ -62,13 +63,18 @@ inline bool make_prefill_geom(int B, int Hq, int Hkv, int T, int d, PrefillGeom*
     g->ntiles = B * Hkv * g->ntile_bg;
     g->nbs = T / kBlock;
     g->cap = g->nbs > 0 ? g->nbs : 1;
+    g->tc = P >= 8;
+    const size_t nsum = (size_t)B * Hkv * (g->nbs > 0 ? g->nbs : 1) * d;
     size_t off = align256(sizeof(WsHeader));
-    g->off_ksum = off;    off = align256(off + (size_t)B * Hkv * (g->nbs > 0 ? g->nbs : 1) * d * sizeof(float));
+    g->off_ksum = off;    off = align256(off + nsum * sizeof(float));
+    g->off_khi = off;     off = align256(off + nsum * 2);            // bf16 hi part of kbar
+    g->off_klo = off;     off = align256(off + nsum * 2);            // bf16 lo part: kbar - hi
     g->off_tau = off;     off = align256(off + (size_t)B * Hq * T * sizeof(float));
     g->off_list = off;    off = align256(off + (size_t)g->ntiles * g->cap * sizeof(int));
     g->off_count = off;   off = align256(off + (size_t)g->ntiles * sizeof(int));
     int cgrid = g->ntiles < kCoarseCTAs ? g->ntiles : kCoarseCTAs;
-    g->off_scratch = off; off = align256(off + (size_t)cgrid * kTileRows * g->cap * sizeof(float));
+    g->off_scratch = off; // per-CTA score slabs of the CUDA-core coarse kernel only
+    if (!g->tc) off = align256(off + (size_t)cgrid * kTileRows * g->cap * sizeof(float));
     g->total = off;
     return true;
 }

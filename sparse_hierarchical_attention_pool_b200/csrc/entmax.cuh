@@ -17,15 +17,75 @@
 // support and u* is exact; otherwise a Newton step is taken.  Other alpha: safeguarded
 // Newton (bisection when a step leaves the bracket) until the step is below 2.5e-7.
 //
-// The row is read through an accessor x(j), j in [0, n); the solve runs either on one
-// thread (STRIDE 1) or on a whole warp (lanes take j = lane, lane + 32, ...; sums are
-// reduced with shuffles so every lane returns the same value).
+// The iteration is written as a per-pass accumulator (EntmaxPass) and an update
+// (EntmaxSolver::update) so that callers can stream a row's values through any memory:
+// the single-thread and warp solves below, and the tensor-memory coarse kernel.
 #pragma once
 
 #include "common.cuh"
 
 namespace dash {
 
+// Power sums of one pass over (part of) a row at the current shifted threshold u.
+struct EntmaxPass {
+    float z0, z1, z2, fe, de, minz;
+    __device__ __forceinline__ void reset() { z0 = z1 = z2 = fe = de = 0.f; minz = INFINITY; }
+    // z = y - u for one value (mode 0 = general alpha needs the powers)
+    __device__ __forceinline__ void add(float z, int mode, float e) {
+        if (z > 0.f) {
+            z0 += 1.f;
+            z1 += z;
+            z2 = fmaf(z, z, z2);
+            minz = fminf(minz, z);
+            if (mode == 0) {
+                const float zp = __powf(z, e - 1.0f);
+                de += zp;
+                fe = fmaf(zp, z, fe);
+            }
+        }
+    }
+    __device__ __forceinline__ void merge(const EntmaxPass& o) {
+        z0 += o.z0; z1 += o.z1; z2 += o.z2; fe += o.fe; de += o.de; minz = fminf(minz, o.minz);
+    }
+    __device__ __forceinline__ void warp_reduce() {
+        z0 = warp_sum(z0); z1 = warp_sum(z1); z2 = warp_sum(z2);
+        fe = warp_sum(fe); de = warp_sum(de); minz = warp_min(minz);
+    }
+};
+
+struct EntmaxSolver {
+    float m, u, lo, hi, e;
+    int mode, it;
+    __device__ __forceinline__ void init(float row_max, float alpha) {
+        m = row_max;
+        u = -1.0f; lo = -1.0f; hi = 0.0f;
+        e = 1.0f / (alpha - 1.0f);
+        mode = alpha == 2.0f ? 2 : (alpha == 1.5f ? 1 : 0);
+        it = 0;
+    }
+    // One iteration from the pass sums.  Returns true when tau (in x space) is final.
+    __device__ __forceinline__ bool update(EntmaxPass p, float* tau, int* no_converge) {
+        if (mode == 2) { p.fe = p.z1; p.de = p.z0; }
+        if (mode == 1) { p.fe = p.z2; p.de = p.z1; }
+        if (p.fe >= 1.0f) lo = u; else hi = u;
+        if (mode != 0 && p.fe >= 1.0f) {
+            const float delta = mode == 2
+                ? (p.z1 - 1.0f) / p.z0
+                : (p.z2 - 1.0f) / (p.z1 + sqrtf(fmaxf(fmaf(p.z1, p.z1, -p.z0 * (p.z2 - 1.0f)), 0.0f)));
+            if (delta < p.minz) { *tau = m + (u + delta); return true; }
+        }
+        const float step = (p.fe - 1.0f) / (e * p.de);
+        if (fabsf(step) <= 2.5e-7f) { *tau = m + (u + step); return true; }
+        float un = u + step;
+        if (!(un > lo && un < hi)) un = 0.5f * (lo + hi);
+        u = un;
+        if (++it >= kSolveMaxIt) { *no_converge = 1; *tau = m + u; return true; }
+        return false;
+    }
+};
+
+// Whole-row solve through an accessor x(j), j in [0, n): on one thread (WARP = false) or
+// on a whole warp (lanes take j = lane, lane + 32, ...; every lane returns the same value).
 template <bool WARP, class Acc>
 __device__ float entmax_threshold(const Acc& x, int n, float alpha, int* no_converge) {
     const int j0 = WARP ? (threadIdx.x & 31) : 0;
@@ -33,46 +93,17 @@ __device__ float entmax_threshold(const Acc& x, int n, float alpha, int* no_conv
     float m = -INFINITY;
     for (int j = j0; j < n; j += js) m = fmaxf(m, x(j));
     if (WARP) m = warp_max(m);
-    const float e = 1.0f / (alpha - 1.0f);
-    const int mode = alpha == 2.0f ? 2 : (alpha == 1.5f ? 1 : 0);
-    float lo = -1.0f, hi = 0.0f, u = -1.0f;
-    for (int it = 0; it < kSolveMaxIt; ++it) {
-        float z0 = 0.f, z1 = 0.f, z2 = 0.f, fe = 0.f, de = 0.f, minz = INFINITY;
-        for (int j = j0; j < n; j += js) {
-            float z = (x(j) - m) - u;
-            if (z > 0.f) {
-                z0 += 1.f;
-                z1 += z;
-                z2 = fmaf(z, z, z2);
-                minz = fminf(minz, z);
-                if (mode == 0) {
-                    float zp = __powf(z, e - 1.0f);
-                    de += zp;
-                    fe = fmaf(zp, z, fe);
-                }
-            }
-        }
-        if (WARP) {
-            z0 = warp_sum(z0); z1 = warp_sum(z1); z2 = warp_sum(z2);
-            fe = warp_sum(fe); de = warp_sum(de); minz = warp_min(minz);
-        }
-        if (mode == 2) { fe = z1; de = z0; }
-        if (mode == 1) { fe = z2; de = z1; }
-        if (fe >= 1.0f) lo = u; else hi = u;
-        if (mode != 0 && fe >= 1.0f) {
-            float delta = mode == 2
-                ? (z1 - 1.0f) / z0
-                : (z2 - 1.0f) / (z1 + sqrtf(fmaxf(fmaf(z1, z1, -z0 * (z2 - 1.0f)), 0.0f)));
-            if (delta < minz) return m + (u + delta);
-        }
-        float step = (fe - 1.0f) / (e * de);
-        if (fabsf(step) <= 2.5e-7f) return m + (u + step);
-        float un = u + step;
-        if (!(un > lo && un < hi)) un = 0.5f * (lo + hi);
-        u = un;
+    EntmaxSolver sv;
+    sv.init(m, alpha);
+    float tau = m - 1.0f;
+    while (true) {
+        EntmaxPass ps;
+        ps.reset();
+        for (int j = j0; j < n; j += js) ps.add((x(j) - m) - sv.u, sv.mode, sv.e);
+        if (WARP) ps.warp_reduce();
+        if (sv.update(ps, &tau, no_converge)) break;
     }
-    *no_converge = 1;
-    return m + u;
+    return tau;
 }
 
 }  // namespace dash

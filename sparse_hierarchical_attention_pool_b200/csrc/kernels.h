@@ -7,13 +7,19 @@
 
 namespace dash {
 
+// kbar in fp32, and optionally split into bf16 hi + lo parts for the tensor-core scores
 cudaError_t launch_block_summary(const void* k, float* ksum, int B, int Hkv, int T, int d,
-                                 cudaStream_t stream);
+                                 cudaStream_t stream, void* khi = nullptr, void* klo = nullptr);
 
 // Stage 1 for prefill: scores of every work tile against the block summaries, per-row
 // thresholds and the per-tile union of selected blocks.
 cudaError_t launch_coarse(const void* q, const PrefillGeom& g, char* ws, float alpha,
                           float coarse_scale, cudaStream_t stream);
+
+// tcgen05 variant of launch_coarse (needs P >= 8 and at least one complete block)
+bool coarse_tc_supported(const PrefillGeom& g);
+cudaError_t launch_coarse_tc(const void* q, const PrefillGeom& g, char* ws, float alpha,
+                             float coarse_scale, cudaStream_t stream);
 
 // Stage 2 for prefill: prior-weighted softmax attention over each tile's listed blocks.
 cudaError_t launch_fine(const void* q, const void* k, const void* v, void* out,

@@ -16,6 +16,7 @@ namespace dash {
 template <int D>
 __global__ void __launch_bounds__(256)
 block_summary_kernel(const __nv_bfloat16* __restrict__ k, float* __restrict__ ksum,
+                     __nv_bfloat16* __restrict__ khi, __nv_bfloat16* __restrict__ klo,
                      long long nblocks_total, int nbs, int T) {
     constexpr int CH = D / 8;          // 16-byte column groups per row
     constexpr int RPS = 32 / CH;       // rows covered by one warp-wide load
@@ -49,25 +50,42 @@ block_summary_kernel(const __nv_bfloat16* __restrict__ k, float* __restrict__ ks
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
     if (lane < CH) {
-        float4* dst = reinterpret_cast<float4*>(ksum + ((size_t)bg * nbs + j) * D + lane * 8);
+        const size_t o = ((size_t)bg * nbs + j) * D + lane * 8;
+        float4* dst = reinterpret_cast<float4*>(ksum + o);
         const float s = 1.0f / kBlock;
-        dst[0] = make_float4(acc[0] * s, acc[1] * s, acc[2] * s, acc[3] * s);
-        dst[1] = make_float4(acc[4] * s, acc[5] * s, acc[6] * s, acc[7] * s);
+        float mean[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mean[i] = acc[i] * s;
+        dst[0] = make_float4(mean[0], mean[1], mean[2], mean[3]);
+        dst[1] = make_float4(mean[4], mean[5], mean[6], mean[7]);
+        if (khi) {
+            // kbar = hi + lo with hi = bf16(kbar), lo = bf16(kbar - hi): 16 significant bits
+            __align__(16) __nv_bfloat16 h[8], l[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                h[i] = __float2bfloat16_rn(mean[i]);
+                l[i] = __float2bfloat16_rn(mean[i] - __bfloat162float(h[i]));
+            }
+            *reinterpret_cast<uint4*>(khi + o) = *reinterpret_cast<const uint4*>(h);
+            *reinterpret_cast<uint4*>(klo + o) = *reinterpret_cast<const uint4*>(l);
+        }
     }
 }
 
 cudaError_t launch_block_summary(const void* k, float* ksum, int B, int Hkv, int T, int d,
-                                 cudaStream_t stream) {
+                                 cudaStream_t stream, void* khi, void* klo) {
     int nbs = T / kBlock;
     long long total = (long long)B * Hkv * nbs;
     if (total == 0) return cudaSuccess;
     unsigned grid = (unsigned)((total + 7) / 8);
     if (d == 128)
         block_summary_kernel<128><<<grid, 256, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(k), ksum, total, nbs, T);
+            static_cast<const __nv_bfloat16*>(k), ksum, static_cast<__nv_bfloat16*>(khi),
+            static_cast<__nv_bfloat16*>(klo), total, nbs, T);
     else
         block_summary_kernel<64><<<grid, 256, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(k), ksum, total, nbs, T);
+            static_cast<const __nv_bfloat16*>(k), ksum, static_cast<__nv_bfloat16*>(khi),
+            static_cast<__nv_bfloat16*>(klo), total, nbs, T);
     return cudaGetLastError();
 }
 

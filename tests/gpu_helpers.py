@@ -76,16 +76,27 @@ def check_prefill(q, k, v, alpha, cs, rows, what="", check_selection=True, nthre
     tau_gpu = rows_of(da.dash_prefill_tau(ws, B, Hq, Hkv, T, d).cpu(), rows).numpy()
     has_past = np.array([t >= 64 for _, _, t in rows])
     if has_past.any():
-        # fp32 holds tau to ~1e-7 relative: 1e-4 absolute, widened for |tau| > 1
-        dt = np.abs(tau_gpu[has_past] - tau_ref[has_past]) / np.maximum(1.0, np.abs(tau_ref[has_past]))
-        assert dt.max() <= 1e-4, f"{what}: tau differs by {dt.max():.3e} (relative to max(1, |tau|))"
+        # Auxiliary check of tau (the specified checks are the block sets, weights and
+        # outputs).  fp32 holds tau to ~1e-7 relative: 1e-4, widened for |tau| > 1.  The
+        # scores use kbar split into bf16 hi + lo parts (2^-17 relative per element), and tau
+        # moves by at most the largest score error, so the allowance adds
+        # 2^-16 (alpha-1) |cs| max_j sum_i |q_i kbar_ji| / sqrt(d).
+        kbar = np.abs(oracle.block_summary(k, 64))                      # [B, Hkv, nbs, d]
+        qa = np.abs(oracle.gather_q_rows(q, rows).double().numpy())
+        G = Hq // Hkv
+        bound = np.array([(qa[i] @ kbar[b, h // G, :max(t // 64, 1)].T).max() if t >= 64 else 0.0
+                          for i, (b, h, t) in enumerate(rows)])
+        allow = 2.0 ** -16 * (alpha - 1) * abs(cs) * bound / np.sqrt(d)
+        dt = np.abs(tau_gpu - tau_ref)[has_past]
+        lim = (1e-4 * np.maximum(1.0, np.abs(tau_ref)) + allow)[has_past]
+        assert np.all(dt <= lim), f"{what}: tau differs by {(dt / lim).max():.3f} x its tolerance"
     assert np.all(np.isnan(tau_gpu[~has_past]))
     if check_selection and has_past.any():
-        res["sel"] = check_dump(qd, kd, rows, q, k, alpha, cs, Hkv, tau_gpu, what)
+        res["sel"] = check_dump(qd, kd, rows, q, k, alpha, cs, Hkv, tau_gpu, what, tau_allow=allow)
     return res, out, ws
 
 
-def check_dump(qd, kd, rows, q, k, alpha, cs, Hkv, tau_prefill=None, what=""):
+def check_dump(qd, kd, rows, q, k, alpha, cs, Hkv, tau_prefill=None, what="", tau_allow=None):
     """Block sets and weights of the dump against the oracle (band-exempt set parity)."""
     B, Hq, T, d = q.shape
     nbs = T // 64
@@ -110,7 +121,11 @@ def check_dump(qd, kd, rows, q, k, alpha, cs, Hkv, tau_prefill=None, what=""):
         pg[idx[r, :cnt[r]]] = p[r, :cnt[r]]
         worst_p = max(worst_p, float(np.abs(pg - sel["p"][r, :bt]).max()))
         if tau_prefill is not None:
-            assert abs(tau[r] - tau_prefill[r]) <= 1e-6, f"{what}: dump tau != prefill tau"
+            # the dump takes fp32 dot products, the prefill tensor-core products of q with
+            # kbar's bf16 hi + lo parts: both fp32-accurate, not bit-identical
+            extra = 0.0 if tau_allow is None else 2.0 * tau_allow[r]
+            assert abs(tau[r] - tau_prefill[r]) <= 1e-4 * max(1.0, abs(tau_prefill[r])) + extra, \
+                f"{what}: dump tau {tau[r]} != prefill tau {tau_prefill[r]}"
     assert worst_p <= P_ABS, f"{what}: block weight error {worst_p:.3e}"
     return {"p_max_err": worst_p, "band_differences": n_band}
 
