@@ -9,8 +9,11 @@ block lists, prior-weighted fine attention) of the workload (default: the 16K pr
 at 75 % block sparsity).  `value` is prefill tokens/s over all ranks with inputs resident
 in HBM; `e2e` is the same through the C ABI's host-buffer entry point (host<->device
 copies inside the timed region).  The `decode` object times one decode step of the 96K
-workload (B=8, cache 98304) the same way.  L2 is flushed (256 MiB write) before every
-timed step; times are CUDA events on the launching stream, max over ranks.
+workload (B=8, cache 98304): its step is replayed from a CUDA graph, as a serving loop
+runs it, and a profiled eager run gives the per-kernel split.  L2 is flushed before every
+timed step (a 256 MiB write, then a 256 MiB read so that no dirty line of the flush is
+written back inside the step); times are CUDA events on the launching stream, max over
+ranks.
 
 Multi-GPU: one process per GPU (torchrun), every rank runs its own replica of the
 workload (work units are independent: weak scaling, no collective on the data path).
@@ -66,6 +69,20 @@ def recorded_traffic(kernel, sha):
     if not d or d.get("source_sha256_16") != sha:
         return None
     return d.get("traffic_bytes_per_launch")
+
+
+class L2Flush:
+    """Evicts the inputs from L2: a write pass over a buffer twice the L2 size, then a read
+    pass over another, so the timed step starts with clean lines of unrelated data."""
+
+    def __init__(self, nbytes=256 << 20):
+        import torch
+        self.w = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        self.r = torch.ones(nbytes // 4, dtype=torch.float32, device="cuda")
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.amax()
 
 
 class ClockSampler:
@@ -177,9 +194,9 @@ def bench_prefill(args, ws, rank, local):
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     out = torch.empty_like(qd)
     wsb = da.alloc_workspace(da.prefill_workspace_size(B, Hq, Hkv, T, d))
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         da.dash_prefill(qd, kd, vd, out, alpha, cs, wsb)
     torch.cuda.synchronize()
     barrier(ws)
@@ -189,7 +206,7 @@ def bench_prefill(args, ws, rank, local):
     time.sleep(0.3)
     evs = []
     for _ in range(args.steps):
-        flush.zero_()
+        flush()
         e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
         da.dash_prefill_profiled(qd, kd, vd, out, alpha, cs, wsb, e)
         evs.append(e)
@@ -218,7 +235,10 @@ def bench_prefill(args, ws, rank, local):
     peak = pk["bf16_tflops"]
     fine_ms = mean(fine)
     achieved = fine_alg / (fine_ms * 1e-3) / 1e12
-    traffic = recorded_traffic("fine_mma_kernel", source_sha("fine_mma.cu", "common.cuh"))
+    G = Hq // Hkv
+    fine_kernel = "fine_tc_kernel" if G <= 16 else "fine_mma_kernel"
+    traffic = (recorded_traffic("fine_tc_kernel", source_sha("fine_tc.cu", "sm100.cuh", "common.cuh"))
+               if G <= 16 else recorded_traffic("fine_mma_kernel", source_sha("fine_mma.cu", "common.cuh")))
     res = {
         "step_ms": step_ms,
         "tok_s": ws * B * T / (step_ms * 1e-3),
@@ -226,7 +246,7 @@ def bench_prefill(args, ws, rank, local):
         "clocks": clocks,
         "stats": st,
         "sparsity": 1.0 - st["selected_pairs"] / max(1, st["scored_pairs"]),
-        "roofline": {"bound": "tensor", "kernel": "fine_mma_kernel", "achieved": round(achieved, 2),
+        "roofline": {"bound": "tensor", "kernel": fine_kernel, "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "traffic": traffic, "peak_source": f"{pk_kind} bf16_tflops (burst)",
                      "algorithmic_flops_per_launch": fine_alg,
@@ -248,7 +268,7 @@ def bench_prefill(args, ws, rank, local):
     e2e_ms = []
     ne2e = max(3, min(args.steps, 20))
     for _ in range(ne2e):
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         da.dash_prefill_host(qh, kh, vh, oh, qd, kd, vd, out, alpha, cs, wsb)
@@ -276,24 +296,49 @@ def bench_decode(args, ws, rank, local):
     ksum = da.dash_block_summary(kcd)
     out = torch.empty_like(qd)
     wsb = da.alloc_workspace(da.decode_workspace_size(B, Hq, Hkv, T, d))
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
     for _ in range(max(3, args.warmup)):
-        flush.zero_()
+        flush()
         da.dash_decode(qd, kcd, vcd, ksum, lens, out, wl.alpha, cs, wsb)
     torch.cuda.synchronize()
     barrier(ws)
     steps = max(args.steps, 20)
+    mean = lambda xs: sum(xs) / len(xs)  # noqa: E731
+    # per-kernel split from a profiled eager run
     evs = []
     for _ in range(steps):
-        flush.zero_()
+        flush()
         e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
         da.dash_decode_profiled(qd, kcd, vcd, ksum, lens, out, wl.alpha, cs, wsb, e)
         evs.append(e)
     torch.cuda.synchronize()
-    barrier(ws)
-    mean = lambda xs: sum(xs) / len(xs)  # noqa: E731
-    tot = max_over_ranks(ws, mean([e[0].elapsed_time(e[4]) for e in evs]))
     st_ms = [mean([e[i].elapsed_time(e[i + 1]) for e in evs]) for i in range(4)]
+    eager = mean([e[0].elapsed_time(e[4]) for e in evs])
+    # the step as a serving loop runs it: one CUDA graph replay (header reset + 3 kernels)
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        da.dash_decode(qd, kcd, vcd, ksum, lens, out, wl.alpha, cs, wsb)
+    torch.cuda.current_stream().wait_stream(side)
+    with torch.cuda.graph(graph):
+        da.dash_decode(qd, kcd, vcd, ksum, lens, out, wl.alpha, cs, wsb)
+    for _ in range(3):
+        flush()
+        graph.replay()
+    torch.cuda.synchronize()
+    barrier(ws)
+    gev = []
+    for _ in range(steps):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        graph.replay()
+        e1.record()
+        gev.append((e0, e1))
+    torch.cuda.synchronize()
+    barrier(ws)
+    tot = max_over_ranks(ws, mean([a.elapsed_time(b) for a, b in gev]))
     st = da.dash_decode_stats(wsb)
     if da.dash_get_device_status(wsb) != 0:
         raise RuntimeError("device status not clean after the timed decode")
@@ -303,35 +348,39 @@ def bench_decode(args, ws, rank, local):
     pk, pk_kind = peaks()
     attn_gbs = gathered / (st_ms[2] * 1e-3) / 1e9
     step_gbs = (gathered + other) / (tot * 1e-3) / 1e9
-    traffic = recorded_traffic("decode_attn_kernel", source_sha("decode.cu", "common.cuh"))
-    # end to end: the new query goes up, the output comes back (the cache stays resident)
+    traffic = recorded_traffic("decode_attn_tc_kernel", source_sha("decode_tc.cu", "decode.cu", "common.cuh"))
+    # end to end: the new query goes up, the graph runs, the output comes back (the cache
+    # stays resident)
     qh, oh = q.pin_memory(), torch.empty_like(q).pin_memory()
     e2e = []
     for _ in range(steps):
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         qd.copy_(qh, non_blocking=True)
-        da.dash_decode(qd, kcd, vcd, ksum, lens, out, wl.alpha, cs, wsb)
+        graph.replay()
         oh.copy_(out, non_blocking=True)
         e1.record()
         e2e.append((e0, e1))
     torch.cuda.synchronize()
+    del graph
     e2e_ms = max_over_ranks(ws, mean([a.elapsed_time(b) for a, b in e2e]))
     return {
         "workload": wl.name, "coarse_scale": cs, "seed": wl.seed,
         "value": ws * B / (tot * 1e-3), "unit": "tok/s", "ms_per_step": tot,
+        "timing": "CUDA graph replay of the step; stage_ms from an eager profiled run",
+        "eager_ms_per_step": eager,
         "stage_ms": dict(zip(["scores", "select", "attention", "combine"], st_ms)),
         "sparsity": 1.0 - st["selected_pairs"] / max(1, st["scored_pairs"]),
         "union_blocks_per_group": st["union_blocks"] / (B * Hkv),
-        "roofline": {"bound": "hbm", "kernel": "decode_attn_kernel", "achieved": round(attn_gbs, 1),
+        "roofline": {"bound": "hbm", "kernel": "decode_attn_tc_kernel", "achieved": round(attn_gbs, 1),
                      "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(attn_gbs / pk["hbm_gbs"], 4),
                      "traffic": traffic, "peak_source": f"{pk_kind} hbm_gbs",
                      "algorithmic_bytes_per_launch": gathered,
                      "step_bytes": gathered + other, "step_frac": round(step_gbs / pk["hbm_gbs"], 4)},
         "e2e": {"value": ws * B / (e2e_ms * 1e-3), "unit": "tok/s", "h2d_bytes_per_step": q.numel() * 2,
                 "d2h_bytes_per_step": q.numel() * 2},
-        "launches_per_step": 4,
+        "launches_per_step": 3,
         "stats": st,
     }
 
@@ -435,7 +484,7 @@ def main():
             "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "T": wl.T, "d": wl.d,
                        "block": wl.block, "alpha": wl.alpha, "coarse_scale": pre["cs"], "seed": wl.seed,
                        "realised_sparsity": round(pre["sparsity"], 5),
-                       "l2": "flushed before every timed step (256 MiB write, outside the step's events)",
+                       "l2": "flushed before every timed step (256 MiB write + 256 MiB read, outside the step's events)",
                        "parallelism": f"independent replica per GPU x{ws}"},
             "roofline": pre["roofline"],
             "e2e": pre["e2e"],

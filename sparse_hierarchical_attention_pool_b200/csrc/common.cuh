@@ -19,7 +19,7 @@ enum : int { kStNoConverge = 1, kStWaitTimeout = 2 };
 // First 256 bytes of every workspace.
 struct WsHeader {
     int status;
-    int pad;
+    int ticket;                   // CTAs of the decode select pass that have finished
     unsigned long long scored_pairs;
     unsigned long long selected_pairs;
     unsigned long long union_blocks;
@@ -82,10 +82,11 @@ inline bool make_prefill_geom(int B, int Hq, int Hkv, int T, int d, PrefillGeom*
 // Geometry of a decode call.
 struct DecodeGeom {
     int B, Hq, Hkv, Tmax, d, G, nbs, chunk, maxchunks;
-    size_t off_x, off_tau, off_list, off_count, off_part, total;
+    size_t off_x, off_tau, off_list, off_count, off_done, off_offs, off_plan, off_part, total;
 };
 
-constexpr int kDecodeChunk = 16;   // list entries (key blocks) per split-KV work item
+constexpr int kDecodeChunk = 16;     // list entries (key blocks) per split-KV work item
+constexpr int kDecodeMaxCtas = 256;  // CTAs of the balanced split-KV attention pass
 
 inline bool make_decode_geom(int B, int Hq, int Hkv, int Tmax, int d, DecodeGeom* g) {
     if (B < 1 || Hq < 1 || Hkv < 1 || Tmax < 1 || Tmax > kMaxT || (Hq % Hkv) != 0) return false;
@@ -102,8 +103,14 @@ inline bool make_decode_geom(int B, int Hq, int Hkv, int Tmax, int d, DecodeGeom
     g->off_tau = off;   off = align256(off + (size_t)B * Hq * sizeof(float));
     g->off_list = off;  off = align256(off + (size_t)B * Hkv * cap * sizeof(int));
     g->off_count = off; off = align256(off + (size_t)B * Hkv * sizeof(int));
-    // partial (m, l, o[d]) per (b, kv head, chunk, head in group)
-    g->off_part = off;  off = align256(off + (size_t)B * Hkv * g->maxchunks * G * (d + 2) * sizeof(float));
+    g->off_done = off;  off = align256(off + (size_t)B * Hkv * sizeof(int));   // partials finished per group
+    g->off_offs = off;  off = align256(off + ((size_t)B * Hkv + 1) * sizeof(int));   // prefix of counts
+    g->off_plan = off;  off = align256(off + (size_t)kDecodeMaxCtas * sizeof(int));  // first group per CTA
+    // partial (m, l, o[d]) per head in group and (b, kv head, chunk) -- or, for the balanced
+    // pass, per (CTA + group) slot
+    const size_t slots_chunk = (size_t)B * Hkv * g->maxchunks, slots_bal = (size_t)B * Hkv + kDecodeMaxCtas;
+    const size_t slots = slots_chunk > slots_bal ? slots_chunk : slots_bal;
+    g->off_part = off;  off = align256(off + slots * G * (d + 2) * sizeof(float));
     g->total = off;
     return true;
 }
@@ -111,6 +118,11 @@ inline bool make_decode_geom(int B, int Hq, int Hkv, int Tmax, int d, DecodeGeom
 // ------------------------------------------------------------------ small device helpers
 
 __device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ int warp_sum_int(int v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;

@@ -37,6 +37,13 @@ cudaError_t launch_select_dump(const void* q, const float* ksum, const long long
                                float* out_tau, int B, int Hq, int Hkv, int T, int d, float alpha,
                                float coarse_scale, cudaStream_t stream);
 
+// split-KV attention of a decode step on TMA + mma.sync, balanced over the CTAs (at most 8
+// heads per group); decode_tc_ctas() is the grid it is launched with
+bool decode_tc_supported(const DecodeGeom& g);
+int decode_tc_ctas();
+cudaError_t launch_decode_attn_tc(const void* q, const void* kc, const void* vc, const int* kv_len,
+                                  void* out, const DecodeGeom& g, char* ws, float e_pow, float sm2,
+                                  int nctas, cudaStream_t stream);
 cudaError_t launch_decode(const void* q, const void* kc, const void* vc, const float* ksum,
                           const int* kv_len, void* out, const DecodeGeom& g, char* ws,
                           float alpha, float coarse_scale, cudaStream_t stream,

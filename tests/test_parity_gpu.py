@@ -200,6 +200,20 @@ def test_decode_invalid_lengths_write_zeros():
     assert da.dash_get_device_status(ws) == 0
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,Tmax,d,lens", [
+    (2, 2, 2, 400000, 64, [400000, 123457]),   # G = 1: a row longer than the select registers
+    (2, 4, 2, 20000, 128, [20000, 4097]),      # G = 2
+    (2, 16, 2, 70000, 128, [70000, 65]),       # G = 8, one warp per head, row spills to memory
+    (1, 16, 1, 5000, 64, [5000]),              # G = 16: CUDA-core attention path
+    (3, 8, 8, 3000, 128, [3000, 64, 129]),     # G = 1, short and block-boundary lengths
+])
+def test_decode_group_sizes(B, Hq, Hkv, Tmax, d, lens):
+    _, (q, kc, vc, _) = inputs.make("decode96k", B=B, Hq=Hq, Hkv=Hkv, T=Tmax, d=d, seed=77 + Hq)
+    (mx, mean), _, ws = check_decode(q, kc, vc, lens, 1.5, calibrated_scale("decode96k"),
+                                     f"decode G={Hq // Hkv} d={d}")
+    print("decode groups", Hq // Hkv, d, mx, mean)
+
+
 def test_decode_96k_workload_all_rows():
     wl, (q, kc, vc, kv_len) = inputs.make("decode96k")
     (mx, mean), _, ws = check_decode(q, kc, vc, kv_len.tolist(), wl.alpha, calibrated_scale("decode96k"), "decode96k")
