@@ -288,7 +288,8 @@ def bench_decode(args, ws, rank, local):
     from sparse_hierarchical_attention_pool_b200 import dash_attn as da
     from sparse_hierarchical_attention_pool_b200 import inputs
 
-    wl, (q, kc, vc, kv_len) = inputs.make("decode96k")
+    over = {"B": args.decode_batch} if args.decode_batch else {}
+    wl, (q, kc, vc, kv_len) = inputs.make("decode96k", **over)
     cs = calibrated("decode96k")["coarse_scale"]
     B, Hq, Hkv, T, d = wl.B, wl.Hq, wl.Hkv, wl.T, wl.d
     qd, kcd, vcd, lens = q.cuda(), kc.cuda(), vc.cuda(), kv_len.cuda()
@@ -308,13 +309,13 @@ def bench_decode(args, ws, rank, local):
     evs = []
     for _ in range(steps):
         flush()
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
         da.dash_decode_profiled(qd, kcd, vcd, ksum, lens, out, wl.alpha, cs, wsb, e)
         evs.append(e)
     torch.cuda.synchronize()
-    st_ms = [mean([e[i].elapsed_time(e[i + 1]) for e in evs]) for i in range(4)]
-    eager = mean([e[0].elapsed_time(e[4]) for e in evs])
-    # the step as a serving loop runs it: one CUDA graph replay (header reset + 3 kernels)
+    st_ms = [mean([e[i].elapsed_time(e[i + 1]) for e in evs]) for i in range(3)]
+    eager = mean([e[0].elapsed_time(e[3]) for e in evs])
+    # the step as a serving loop runs it: one CUDA graph replay (header reset + 2 kernels)
     graph = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
@@ -346,9 +347,9 @@ def bench_decode(args, ws, rank, local):
     gathered = (st["union_blocks"] + B * Hkv) * blk_bytes
     other = B * Hkv * (T // 64) * d * 4 + 2 * B * Hq * d * 2
     pk, pk_kind = peaks()
-    attn_gbs = gathered / (st_ms[2] * 1e-3) / 1e9
+    attn_gbs = gathered / (st_ms[1] * 1e-3) / 1e9
     step_gbs = (gathered + other) / (tot * 1e-3) / 1e9
-    traffic = recorded_traffic("decode_attn_tc_kernel", source_sha("decode_tc.cu", "decode.cu", "common.cuh"))
+    traffic = recorded_traffic("decode_attn_tc_kernel", source_sha("decode_tc.cu", "common.cuh"))
     # end to end: the new query goes up, the graph runs, the output comes back (the cache
     # stays resident)
     qh, oh = q.pin_memory(), torch.empty_like(q).pin_memory()
@@ -370,7 +371,7 @@ def bench_decode(args, ws, rank, local):
         "value": ws * B / (tot * 1e-3), "unit": "tok/s", "ms_per_step": tot,
         "timing": "CUDA graph replay of the step; stage_ms from an eager profiled run",
         "eager_ms_per_step": eager,
-        "stage_ms": dict(zip(["scores", "select", "attention", "combine"], st_ms)),
+        "stage_ms": dict(zip(["coarse_select", "attention", "merge"], st_ms)),
         "sparsity": 1.0 - st["selected_pairs"] / max(1, st["scored_pairs"]),
         "union_blocks_per_group": st["union_blocks"] / (B * Hkv),
         "roofline": {"bound": "hbm", "kernel": "decode_attn_tc_kernel", "achieved": round(attn_gbs, 1),
@@ -380,7 +381,7 @@ def bench_decode(args, ws, rank, local):
                      "step_bytes": gathered + other, "step_frac": round(step_gbs / pk["hbm_gbs"], 4)},
         "e2e": {"value": ws * B / (e2e_ms * 1e-3), "unit": "tok/s", "h2d_bytes_per_step": q.numel() * 2,
                 "d2h_bytes_per_step": q.numel() * 2},
-        "launches_per_step": 3,
+        "launches_per_step": 2,
         "stats": st,
     }
 
@@ -457,6 +458,10 @@ def main():
     ap.add_argument("--workload", default="16k", choices=["16k", "32k", "96k"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="time only the decode step and print its object (for profiling runs)")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="decode batch other than the workload's 8 (smaller profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -469,6 +474,15 @@ def main():
     if rank == 0:
         _b.build()
     barrier(ws)
+    if args.decode_only:
+        dec = bench_decode(args, ws, rank, local)
+        if rank == 0:
+            print(json.dumps(dec), flush=True)
+        if ws > 1:
+            import torch.distributed as dist
+            barrier(ws)
+            dist.destroy_process_group()
+        return
     pre = bench_prefill(args, ws, rank, local)
     dec = None if args.no_decode else bench_decode(args, ws, rank, local)
     cpu = None

@@ -181,8 +181,10 @@ DASH_API int dash_decode(const void* q, const void* k_cache, const void* v_cache
                 dash_stream_t stream);
 
 /*
- * dash_decode that also records five caller-created CUDA events on `stream`: before the
- * score, select, attention and combine kernels, and after the combine kernel.
+ * dash_decode that also records four caller-created CUDA events on `stream`: events[0]
+ * before the coarse kernels (scores, then thresholds and block lists), events[1] before the
+ * attention kernel, events[2] after it (before the partial merge kernel, which only the
+ * path for more than 8 query heads per KV group launches) and events[3] at the end.
  */
 DASH_API int dash_decode_profiled(const void* q, const void* k_cache, const void* v_cache, const float* ksum,
                                   const int* kv_len, void* out, int B, int Hq, int Hkv, int Tmax, int d,

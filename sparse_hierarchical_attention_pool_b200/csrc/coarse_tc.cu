@@ -32,6 +32,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "entmax.cuh"
@@ -317,8 +318,15 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 // z = (x - m) - u with x rounded exactly as in pass 0 (__fmul_rn is never fused
                 // into an FMA), so the maximum gives z = -u exactly
                 if (!run_pass([&](int, const uint32_t* v, int nv) {
-                        for (int i = 0; i < 32; ++i)
-                            if (i < nv) ps.add((__fmul_rn(__uint_as_float(v[i]), cx) - sv.m) - sv.u, sv.mode, sv.e);
+                        auto sweep = [&](auto mode) {
+                            constexpr int MODE = decltype(mode)::value;
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (i < nv) ps.add_t<MODE>((__fmul_rn(__uint_as_float(v[i]), cx) - sv.m) - sv.u, sv.e);
+                        };
+                        if (sv.mode == 1) sweep(std::integral_constant<int, 1>{});
+                        else if (sv.mode == 2) sweep(std::integral_constant<int, 2>{});
+                        else sweep(std::integral_constant<int, 0>{});
                     })) { ok = false; break; }
                 xs[hf][0][r] = ps.z0; xs[hf][1][r] = ps.z1; xs[hf][2][r] = ps.z2;
                 xs[hf][3][r] = ps.fe; xs[hf][4][r] = ps.de; xs[hf][5][r] = ps.minz;

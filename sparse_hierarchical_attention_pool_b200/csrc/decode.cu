@@ -4,17 +4,19 @@
 // Fully Differentiable with Adaptive Block Selection", section "Core Mechanism"): coarse
 // scores over the cached block summaries of blocks j < bt = t / 64, alpha-entmax weights,
 // then softmax over the selected blocks' tokens plus the own block (causal, prior 1) with
-// log p as the prior.  Four kernels, all launched with shapes known on the host:
-//   1. decode_scores : x[b, h, j] for every head of a KV group, four threads per block
-//                      summary (the summary is read once for the whole group);
-//   2. decode_select : per (b, kv head): a team of warps per head solves tau with the row
-//                      in registers, the selected blocks of the group's heads are OR-ed
-//                      into one list, the own block last;
-//   3. decode_attn   : split-KV over chunks of 16 listed blocks: K/V blocks (16 KB each at
-//                      d = 128) stream through a two-stage cp.async pipeline; each listed
-//                      block is read once and serves every head of the group; partial
-//                      (max, sum, output) per chunk and head;
-//   4. decode_combine: merges the partials of each (b, h) and writes bf16.
+// log p as the prior.  Kernels, all launched with shapes known on the host:
+//   1. decode_scores : x[b, h, j] for every head of a KV group, each block summary read once
+//                      for all G heads (a warp streams 16 summaries of one group);
+//   2. decode_select : per (b, kv head): one warp per head solves tau with the row in
+//                      registers, the union of the heads' selected blocks becomes the
+//                      group's list (own block last), and the last CTA writes the work plan
+//                      of the balanced attention pass;
+//   3. attention     : decode_attn_tc_kernel (decode_tc.cu) for G <= 8, which also merges
+//                      the split groups; otherwise decode_attn below, split-KV over chunks of
+//                      16 listed blocks with a two-stage cp.async pipeline, each listed block
+//                      read once for every head of the group, partial (max, sum, output) per
+//                      chunk and head, and
+//   4. decode_combine: merging those partials of each (b, h) into bf16.
 // The HBM traffic that matters is step 3: (union blocks + 1) * 64 * d * 2 bytes * 2 per
 // (b, kv head).
 #include "common.cuh"
@@ -23,15 +25,134 @@
 
 namespace dash {
 
-// Four threads per block summary, each holding a quarter of its d values (8 float4 loads
-// issued together, so a CTA keeps 32 KB of summaries in flight); every head's partial dot
-// product is reduced over the four threads with two shuffles.  The query rows of the group
-// sit in shared memory with each quarter padded by one float4 so that the four quarters read
-// in one instruction fall in different banks.
-template <int D>
+constexpr int kSelRegs = 48;        // row values a select lane keeps in registers
+
+// ------------------------------------------------------------------ scores
+//
+// x[b, h, j] = cx * q[b, h] . kbar[b, g, j] for the G heads of every group and every past
+// block j < bt.  A warp takes RW consecutive block summaries of one group and issues all
+// their loads at once (lane l holds dims [l D/32, (l + 1) D/32) of each row: one coalesced
+// row per instruction); the group's query rows sit in registers (heads padded to GP, a
+// power of two <= 8).  Per task of R = 32/GP rows (at most 8) a lane has R * GP partial sums,
+// and a butterfly reduce-scatter over the 32 lanes leaves every (row, head) sum complete on
+// its own lane with 31 shuffles in all.  Each summary is read from HBM once for all heads.
+
+// Butterfly reduce-scatter of C values per lane over lane offsets O, O/2, ..., 1: at each
+// level the lane with bit O set keeps the upper half of its values and receives the
+// partner's copy of it; once one value is left, the remaining levels sum it.
+template <int C, int O>
+__device__ __forceinline__ void reduce_scatter(float* v, int lane) {
+    if constexpr (O >= 1) {
+        if constexpr (C >= 2) {
+            const bool up = (lane & O) != 0;
+#pragma unroll
+            for (int i = 0; i < C / 2; ++i) {
+                const float send = up ? v[i] : v[i + C / 2];
+                const float keep = up ? v[i + C / 2] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+            }
+            reduce_scatter<C / 2, O / 2>(v, lane);
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], O);
+            reduce_scatter<1, O / 2>(v, lane);
+        }
+    }
+}
+
+template <int D, int GP>
+struct ScoreShape {
+    static constexpr int DPL = D / 32;                 // dims per lane
+    static constexpr int R = GP >= 4 ? 32 / GP : 8;    // rows per reduce-scatter
+    static constexpr int V = R * GP;                   // partial sums per lane (<= 32)
+    static constexpr int RW = 2 * R;                   // rows per warp, loads issued together
+    static constexpr int LOGV = V >= 32 ? 5 : V >= 16 ? 4 : V >= 8 ? 3 : V >= 4 ? 2 : V >= 2 ? 1 : 0;
+};
+
+template <int D, int GP>
 __global__ void __launch_bounds__(256)
 decode_scores_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ ksum,
                      const int* __restrict__ kv_len, float* __restrict__ xs, DecodeGeom g, float cx) {
+    using S = ScoreShape<D, GP>;
+    const int lane = threadIdx.x & 31;
+    const long long wtask = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int tpg = (g.nbs + S::RW - 1) / S::RW;
+    const int bg = (int)(wtask / tpg);
+    if (bg >= g.B * g.Hkv) return;
+    const int j0 = (int)(wtask % tpg) * S::RW;
+    const int b = bg / g.Hkv, kvh = bg % g.Hkv;
+    const int L = kv_len[b];
+    if (L < 1 || L > g.Tmax) return;
+    const int bt = (L - 1) / kBlock;
+    if (j0 >= bt) return;
+    const size_t qrow0 = (size_t)b * g.Hq + (size_t)kvh * g.G;
+    // rows past bt load row bt - 1 again (in bounds; their sums are not written)
+    const float* src = ksum + (size_t)bg * g.nbs * D + lane * S::DPL;
+    float kv[S::RW][S::DPL];
+#pragma unroll
+    for (int r = 0; r < S::RW; ++r) {
+        const size_t jr = (size_t)min(j0 + r, bt - 1);
+        if constexpr (S::DPL == 4) {
+            const float4 t = __ldg(reinterpret_cast<const float4*>(src + jr * D));
+            kv[r][0] = t.x; kv[r][1] = t.y; kv[r][2] = t.z; kv[r][3] = t.w;
+        } else {
+            const float2 t = __ldg(reinterpret_cast<const float2*>(src + jr * D));
+            kv[r][0] = t.x; kv[r][1] = t.y;
+        }
+    }
+    // query rows of the group (heads past G repeat head 0; their sums are not written)
+    float qv[GP][S::DPL];
+#pragma unroll
+    for (int h = 0; h < GP; ++h) {
+        const __nv_bfloat16* qh = q + (qrow0 + (h < g.G ? h : 0)) * D + lane * S::DPL;
+        if constexpr (S::DPL == 4) {
+            const uint2 t = __ldg(reinterpret_cast<const uint2*>(qh));
+            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&t.x));
+            const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&t.y));
+            qv[h][0] = a.x; qv[h][1] = a.y; qv[h][2] = c.x; qv[h][3] = c.y;
+        } else {
+            const uint32_t t = __ldg(reinterpret_cast<const unsigned int*>(qh));
+            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&t));
+            qv[h][0] = a.x; qv[h][1] = a.y;
+        }
+    }
+    const size_t cap = (size_t)g.nbs + 1;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        float v[S::V];
+#pragma unroll
+        for (int r = 0; r < S::R; ++r)
+#pragma unroll
+            for (int h = 0; h < GP; ++h) {
+                float acc = 0.f;
+#pragma unroll
+                for (int d = 0; d < S::DPL; ++d) acc = fmaf(kv[half * S::R + r][d], qv[h][d], acc);
+                v[r * GP + h] = acc;
+            }
+        reduce_scatter<S::V, 16>(v, lane);
+        // value index held by this lane (see reduce_scatter): lane * V/32 + k when V >= 32,
+        // else lane >> (5 - log2 V), replicated on 32/V lanes
+        if constexpr (S::V >= 32) {
+#pragma unroll
+            for (int k = 0; k < S::V / 32; ++k) {
+                const int idx = lane * (S::V / 32) + k, r = idx / GP, h = idx % GP;
+                const int j = j0 + half * S::R + r;
+                if (h < g.G && j < bt) xs[(qrow0 + h) * cap + j] = v[k] * cx;
+            }
+        } else {
+            const int idx = lane >> (5 - S::LOGV), r = idx / GP, h = idx % GP;
+            const int j = j0 + half * S::R + r;
+            if ((lane & ((32 >> S::LOGV) - 1)) == 0 && h < g.G && j < bt) xs[(qrow0 + h) * cap + j] = v[0] * cx;
+        }
+    }
+}
+
+// Groups of more than 8 heads: four threads per block summary, each with a quarter of its d
+// values; every head's partial dot product is reduced over the four threads with two
+// shuffles.
+template <int D>
+__global__ void __launch_bounds__(256)
+decode_scores_wide_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ ksum,
+                          const int* __restrict__ kv_len, float* __restrict__ xs, DecodeGeom g, float cx) {
     constexpr int QD = D / 4;                 // dims per thread
     constexpr int QV = QD / 4;                // float4 per thread
     constexpr int QS = D + 16;                // padded row stride of a query head (floats)
@@ -44,6 +165,8 @@ decode_scores_kernel(const __nv_bfloat16* __restrict__ q, const float* __restric
     if (j0 >= bt) return;
     const int part = threadIdx.x & 3, j = j0 + (threadIdx.x >> 2);
     float4 kv[QV];
+#pragma unroll
+    for (int i = 0; i < QV; ++i) kv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     if (j < bt) {
         const float4* kb = reinterpret_cast<const float4*>(ksum + ((size_t)bg * g.nbs + j) * D + part * QD);
 #pragma unroll
@@ -54,10 +177,6 @@ decode_scores_kernel(const __nv_bfloat16* __restrict__ q, const float* __restric
         qs[h * QS + (c / QD) * (QD + 4) + c % QD] = __bfloat162float(q[(size_t)(b * g.Hq + kvh * g.G) * D + i]);
     }
     __syncthreads();
-    if (j >= bt) {
-#pragma unroll
-        for (int i = 0; i < QV; ++i) kv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
     const int cap = g.nbs + 1;
     for (int h0 = 0; h0 < g.G; h0 += 4) {
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -85,40 +204,77 @@ decode_scores_kernel(const __nv_bfloat16* __restrict__ q, const float* __restric
     }
 }
 
-constexpr int kSelRegs = 24;   // row values a select lane keeps in registers
+template <int D, int GP>
+void launch_scores_gp(const __nv_bfloat16* q, const float* ksum, const int* kv_len, float* xs,
+                      const DecodeGeom& g, float cx, cudaStream_t stream) {
+    using S = ScoreShape<D, GP>;
+    const long long warps = (long long)g.B * g.Hkv * ((g.nbs + S::RW - 1) / S::RW);
+    const unsigned grid = (unsigned)((warps + 7) / 8);
+    if (grid > 0) decode_scores_kernel<D, GP><<<grid, 256, 0, stream>>>(q, ksum, kv_len, xs, g, cx);
+}
 
-// Row values of one head, spread over a team of W warps: lane tl of the team holds
-// x[tl + k * 32W] for k < kSelRegs in registers; values past that are read from memory.
-struct TeamRow {
+template <int D>
+void launch_scores(const __nv_bfloat16* q, const float* ksum, const int* kv_len, float* xs,
+                   const DecodeGeom& g, float cx, cudaStream_t stream) {
+    if (g.G == 1) launch_scores_gp<D, 1>(q, ksum, kv_len, xs, g, cx, stream);
+    else if (g.G == 2) launch_scores_gp<D, 2>(q, ksum, kv_len, xs, g, cx, stream);
+    else if (g.G <= 4) launch_scores_gp<D, 4>(q, ksum, kv_len, xs, g, cx, stream);
+    else if (g.G <= 8) launch_scores_gp<D, 8>(q, ksum, kv_len, xs, g, cx, stream);
+    else {
+        dim3 gs(g.B * g.Hkv, (g.nbs + 63) / 64 > 0 ? (g.nbs + 63) / 64 : 1);
+        decode_scores_wide_kernel<D><<<gs, 256, 0, stream>>>(q, ksum, kv_len, xs, g, cx);
+    }
+}
+
+// ------------------------------------------------------------------ select
+
+// Row values of one head on one warp: lane l holds x[l + 32 k] for k < kSelRegs in
+// registers (-inf past the row's end, which no pass counts); values past that are read from
+// memory.
+struct WarpRow {
     float r[kSelRegs];
     const float* p;
-    int tl, stride, n;
-    __device__ __forceinline__ void load(const float* row, int team_lane, int team_threads, int count) {
-        p = row; tl = team_lane; stride = team_threads; n = count;
+    int lane, n;
+    __device__ __forceinline__ void load(const float* row, int ln, int count) {
+        p = row; lane = ln; n = count;
 #pragma unroll
         for (int k = 0; k < kSelRegs; ++k) {
-            const int j = tl + k * stride;
+            const int j = lane + 32 * k;
             r[k] = j < n ? row[j] : -INFINITY;
         }
     }
     template <class F>
     __device__ __forceinline__ void each(F&& f) const {
 #pragma unroll
-        for (int k = 0; k < kSelRegs; ++k) {
-            const int j = tl + k * stride;
-            if (j < n) f(j, r[k]);
-        }
-        for (int j = tl + kSelRegs * stride; j < n; j += stride) f(j, p[j]);
+        for (int k = 0; k < kSelRegs; ++k) f(lane + 32 * k, r[k]);
+        for (int j = lane + 32 * kSelRegs; j < n; j += 32) f(j, p[j]);
     }
 };
+
+// Threshold of one row held by a warp (every lane returns it); MODE as in EntmaxPass::add_t.
+template <int MODE>
+__device__ __forceinline__ float warp_row_tau(const WarpRow& xr, float m, float alpha, int* no_conv) {
+    EntmaxSolver sv;
+    sv.init(m, alpha);
+    float t = m;
+    while (true) {
+        EntmaxPass ps;
+        ps.reset();
+        xr.each([&](int, float v) { ps.add_t<MODE>((v - sv.m) - sv.u, sv.e); });
+        ps.warp_reduce_t<MODE>();
+        if (sv.update(ps, &t, no_conv)) break;
+    }
+    return t;
+}
 
 // Work plan of the balanced attention pass, built by the last select CTA to finish (a
 // ticket in the workspace header): offs = exclusive prefix of the list lengths (U = offs[BH]
 // blocks in all), and plan[c] = the group holding position floor(U c / n), where CTA c's
-// range starts (n = min(nctas, U)).  Called by every thread of every select CTA after its count is written.
+// range starts (n = min(nctas, U)).  Called by every thread of every CTA once its count is
+// written.
 __device__ void decode_plan_tail(const int* count, int* offs, int* plan, WsHeader* hdr, int BH, int nctas) {
     __shared__ int last_sh;
-    __shared__ int wsum[8];
+    __shared__ int wsum[32];
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();                              // this CTA's count before its ticket
@@ -129,7 +285,7 @@ __device__ void decode_plan_tail(const int* count, int* offs, int* plan, WsHeade
     __threadfence();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
     const int slice = (BH + nwarp - 1) / nwarp;
-    const int lo = warp * slice, hi = min(BH, lo + slice);
+    const int lo = min(BH, warp * slice), hi = min(BH, lo + slice);
     int sum = 0;
     for (int i = lo + lane; i < hi; i += 32) sum += __ldcg(count + i);
     sum = warp_sum_int(sum);
@@ -165,78 +321,55 @@ __device__ void decode_plan_tail(const int* count, int* offs, int* plan, WsHeade
     }
 }
 
-// One CTA per (b, kv head).  The 8 warps form G teams (W = 8 / G warps each, one warp per
-// head when G >= 8); a team solves its head's threshold with the row in registers, summing
-// each pass over the team through shared memory (double-buffered, one named barrier per
-// pass).  Selected blocks of all heads are OR-ed into a bitmap and compacted into the
-// group's list, the own block last.
-__global__ void __launch_bounds__(256)
+// One CTA of 8 warps per (b, kv head).  Warp w solves the thresholds of heads w, w + 8, ...
+// with the row in registers (one warp per head: no cross-warp reduction in a pass).  The
+// heads' selected blocks are OR-ed into a bitmap; every thread then takes bitmap words
+// w, w + 256, ..., a block-wide scan of their popcounts places the words, and each thread
+// writes its words' blocks into the group's list, the own block last.
+constexpr int kSelThreads = 256;
+
+__global__ void __launch_bounds__(kSelThreads)
 decode_select_kernel(const int* __restrict__ kv_len, const float* __restrict__ xs,
                      float* __restrict__ tau, int* __restrict__ list, int* __restrict__ count,
                      int* __restrict__ done, int* __restrict__ offs, int* __restrict__ plan,
                      __nv_bfloat16* __restrict__ out, WsHeader* __restrict__ hdr, DecodeGeom g,
                      float alpha, int nctas) {
-    __shared__ unsigned bitmap[kMaxT / kBlock / 32];
-    __shared__ EntmaxPass red[2][8];
-    __shared__ float redm[8];
+    constexpr int kWords = kMaxT / kBlock / 32;
+    constexpr int kWpt = kWords / kSelThreads;        // bitmap words per thread
+    __shared__ unsigned bitmap[kWords];
+    __shared__ int wtot[kSelThreads / 32];
     const int bg = blockIdx.x, b = bg / g.Hkv, kvh = bg % g.Hkv;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarp = blockDim.x >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarp = kSelThreads / 32;
     const int cap = g.nbs + 1;
     const int L = kv_len[b];
-    if (threadIdx.x == 0) done[bg] = 0;
+    const size_t qrow0 = (size_t)b * g.Hq + (size_t)kvh * g.G;
+    if (tid == 0) done[bg] = 0;
     if (L < 1 || L > g.Tmax) {
         // no keys: the group's heads get a zero output and no work
-        if (threadIdx.x == 0) count[bg] = 0;
-        __nv_bfloat16* o = out + ((size_t)b * g.Hq + (size_t)kvh * g.G) * g.d;
-        for (int i = threadIdx.x; i < g.G * g.d; i += blockDim.x) o[i] = __float2bfloat16(0.f);
+        if (tid == 0) count[bg] = 0;
+        for (int i = tid; i < g.G * g.d; i += kSelThreads) out[qrow0 * g.d + i] = __float2bfloat16(0.f);
         if (nctas > 0) decode_plan_tail(count, offs, plan, hdr, g.B * g.Hkv, nctas);
         return;
     }
     const int bt = (L - 1) / kBlock;
     const int nw = (bt + 31) / 32;
-    for (int i = threadIdx.x; i < nw; i += blockDim.x) bitmap[i] = 0u;
+    for (int i = tid; i < nw; i += kSelThreads) bitmap[i] = 0u;
     __syncthreads();
-    // team geometry: W warps per head (a power of two), nteam heads in flight
-    int W = 1;
-    while (W * 2 * g.G <= nwarp) W *= 2;
-    const int nteam = nwarp / W, team = warp / W, tw = warp % W;
-    const int tl = tw * 32 + lane, tthreads = W * 32;
-    auto team_sync = [&]() {
-        if (W > 1) asm volatile("bar.sync %0, %1;" :: "r"(team + 1), "r"(tthreads) : "memory");
-    };
     int no_conv = 0;
-    for (int hl = team; hl < g.G; hl += nteam) {
-        const size_t row = (size_t)(b * g.Hq + kvh * g.G + hl);
+    for (int hl = warp; hl < g.G; hl += nwarp) {
+        const size_t row = qrow0 + hl;
         float t = __int_as_float(0x7fc00000);
-        TeamRow xr;
-        xr.load(xs + row * cap, tl, tthreads, bt);
+        WarpRow xr;
+        xr.load(xs + row * cap, lane, bt);
         if (bt > 0) {
             float m = -INFINITY;
             xr.each([&](int, float v) { m = fmaxf(m, v); });
             m = warp_max(m);
-            if (W > 1) {
-                if (lane == 0) redm[warp] = m;
-                team_sync();
-                m = -INFINITY;
-                for (int v = 0; v < W; ++v) m = fmaxf(m, redm[team * W + v]);
-            }
-            EntmaxSolver sv;
-            sv.init(m, alpha);
-            for (int pass = 0;; ++pass) {
-                EntmaxPass ps;
-                ps.reset();
-                xr.each([&](int, float v) { ps.add((v - sv.m) - sv.u, sv.mode, sv.e); });
-                ps.warp_reduce();
-                if (W > 1) {
-                    if (lane == 0) red[pass & 1][warp] = ps;
-                    team_sync();
-                    ps = red[pass & 1][team * W];
-                    for (int v = 1; v < W; ++v) ps.merge(red[pass & 1][team * W + v]);
-                }
-                if (sv.update(ps, &t, &no_conv)) break;
-            }
+            t = alpha == 1.5f ? warp_row_tau<1>(xr, m, alpha, &no_conv)
+              : alpha == 2.0f ? warp_row_tau<2>(xr, m, alpha, &no_conv)
+                              : warp_row_tau<0>(xr, m, alpha, &no_conv);
         }
-        if (tw == 0 && lane == 0) tau[row] = t;
+        if (lane == 0) tau[row] = t;
         float nsel = 0.f;
         xr.each([&](int j, float v) {
             if (v > t) {
@@ -247,39 +380,50 @@ decode_select_kernel(const int* __restrict__ kv_len, const float* __restrict__ x
         nsel = warp_sum(nsel);
         if (lane == 0) {
             atomicAdd(&hdr->selected_pairs, (unsigned long long)nsel);
-            if (tw == 0) atomicAdd(&hdr->scored_pairs, (unsigned long long)bt);
+            atomicAdd(&hdr->scored_pairs, (unsigned long long)bt);
         }
-        team_sync();                      // the team's reduction slots are reused by its next head
     }
     if (no_conv) atomicOr(&hdr->status, kStNoConverge);
     __syncthreads();
-    if (warp == 0) {
-        int base = 0;
-        int* dst = list + (size_t)bg * cap;
-        for (int w0 = 0; w0 < nw; w0 += 32) {
-            const int wi = w0 + lane;
-            unsigned word = wi < nw ? bitmap[wi] : 0u;
-            const int pc = __popc(word);
-            int incl = pc;
+    // compaction: thread tid owns words tid * kWpt .. + kWpt - 1
+    unsigned wv[kWpt];
+    int pc = 0;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                int n = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += n;
-            }
-            int pos = base + incl - pc;
-            while (word) {
-                const int bit = __ffs(word) - 1;
-                dst[pos++] = wi * 32 + bit;
-                word &= word - 1;
-            }
-            base += __shfl_sync(0xffffffffu, incl, 31);
+    for (int k = 0; k < kWpt; ++k) {
+        const int wi = tid * kWpt + k;
+        wv[k] = wi < nw ? bitmap[wi] : 0u;
+        pc += __popc(wv[k]);
+    }
+    int incl = pc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+    }
+    if (lane == 31) wtot[warp] = incl;
+    __syncthreads();
+    int base = 0, total = 0;
+    for (int w = 0; w < nwarp; ++w) {
+        if (w < warp) base += wtot[w];
+        total += wtot[w];
+    }
+    int pos = base + incl - pc;
+    int* dst = list + (size_t)bg * cap;
+#pragma unroll
+    for (int k = 0; k < kWpt; ++k) {
+        unsigned word = wv[k];
+        const int wi = tid * kWpt + k;
+        while (word) {
+            const int bit = __ffs(word) - 1;
+            dst[pos++] = wi * 32 + bit;
+            word &= word - 1;
         }
-        if (lane == 0) {
-            dst[base] = bt;                  // own block, always last
-            count[bg] = base + 1;
-            atomicAdd(&hdr->union_blocks, (unsigned long long)base);
-            if (bt > 0) atomicAdd(&hdr->tiles, 1ull);
-        }
+    }
+    if (tid == 0) {
+        dst[total] = bt;                  // own block, always last
+        count[bg] = total + 1;
+        atomicAdd(&hdr->union_blocks, (unsigned long long)total);
+        if (bt > 0) atomicAdd(&hdr->tiles, 1ull);
     }
     if (nctas > 0) decode_plan_tail(count, offs, plan, hdr, g.B * g.Hkv, nctas);
 }
@@ -465,47 +609,45 @@ cudaError_t launch_decode(const void* q, const void* kc, const void* vc, const f
     float* tau = reinterpret_cast<float*>(ws + g.off_tau);
     int* list = reinterpret_cast<int*>(ws + g.off_list);
     int* count = reinterpret_cast<int*>(ws + g.off_count);
+    int* done = reinterpret_cast<int*>(ws + g.off_done);
+    int* offs = reinterpret_cast<int*>(ws + g.off_offs);
+    int* plan = reinterpret_cast<int*>(ws + g.off_plan);
     float* part = reinterpret_cast<float*>(ws + g.off_part);
     const auto* qb = static_cast<const __nv_bfloat16*>(q);
     const auto* kb = static_cast<const __nv_bfloat16*>(kc);
     const auto* vb = static_cast<const __nv_bfloat16*>(vc);
     auto* ob = static_cast<__nv_bfloat16*>(out);
     const int BH = g.B * g.Hkv;
-    dim3 gs(BH, (g.nbs + 63) / 64 > 0 ? (g.nbs + 63) / 64 : 1);
-    const size_t sm_attn = (size_t)4 * kBlock * g.d * sizeof(__nv_bfloat16)
-                         + (size_t)(2 * g.G * g.d + g.G * kBlock + 4 * 32) * sizeof(float);
-    cudaError_t e = cudaSuccess;
-    if (g.d == 128) e = cudaFuncSetAttribute(decode_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_attn);
-    else e = cudaFuncSetAttribute(decode_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_attn);
-    if (e != cudaSuccess) return e;
-    dim3 ga(BH, g.maxchunks);
-    if (!mark(0)) return cudaErrorUnknown;
-    if (g.d == 128) decode_scores_kernel<128><<<gs, 256, 0, stream>>>(qb, ksum, kv_len, xs, g, cx);
-    else decode_scores_kernel<64><<<gs, 256, 0, stream>>>(qb, ksum, kv_len, xs, g, cx);
-    if (!mark(1)) return cudaErrorUnknown;
-    int* done = reinterpret_cast<int*>(ws + g.off_done);
-    int* offs = reinterpret_cast<int*>(ws + g.off_offs);
-    int* plan = reinterpret_cast<int*>(ws + g.off_plan);
     const bool fused = decode_tc_supported(g);
     const int nctas = fused ? decode_tc_ctas() : 0;
-    decode_select_kernel<<<BH, 256, 0, stream>>>(kv_len, xs, tau, list, count, done, offs, plan, ob, hdr, g,
-                                                 alpha, nctas);
-    if (!mark(2)) return cudaErrorUnknown;
+    cudaError_t e = cudaSuccess;
+    if (!mark(0)) return cudaErrorUnknown;
+    if (g.d == 128) launch_scores<128>(qb, ksum, kv_len, xs, g, cx, stream);
+    else launch_scores<64>(qb, ksum, kv_len, xs, g, cx, stream);
+    decode_select_kernel<<<BH, kSelThreads, 0, stream>>>(kv_len, xs, tau, list, count, done, offs, plan, ob, hdr, g,
+                                                         alpha, nctas);
+    if (!mark(1)) return cudaErrorUnknown;
     if (fused) {
         e = launch_decode_attn_tc(q, kc, vc, kv_len, out, g, ws, e_pow, sm2, nctas, stream);
         if (e != cudaSuccess) return e;
-    } else if (g.d == 128) {
+        if (!mark(2) || !mark(3)) return cudaErrorUnknown;   // no separate merge pass
+        return cudaGetLastError();
+    }
+    const size_t sm_attn = (size_t)4 * kBlock * g.d * sizeof(__nv_bfloat16)
+                         + (size_t)(2 * g.G * g.d + g.G * kBlock + 4 * 32) * sizeof(float);
+    e = g.d == 128
+        ? cudaFuncSetAttribute(decode_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_attn)
+        : cudaFuncSetAttribute(decode_attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_attn);
+    if (e != cudaSuccess) return e;
+    dim3 ga(BH, g.maxchunks);
+    if (g.d == 128)
         decode_attn_kernel<128><<<ga, 128, sm_attn, stream>>>(qb, kb, vb, kv_len, xs, tau, list, count, part, g, e_pow, sm2);
-    } else {
+    else
         decode_attn_kernel<64><<<ga, 128, sm_attn, stream>>>(qb, kb, vb, kv_len, xs, tau, list, count, part, g, e_pow, sm2);
-    }
+    if (!mark(2)) return cudaErrorUnknown;
+    if (g.d == 128) decode_combine_kernel<128><<<g.B * g.Hq, 128, 0, stream>>>(count, part, ob, g);
+    else decode_combine_kernel<64><<<g.B * g.Hq, 128, 0, stream>>>(count, part, ob, g);
     if (!mark(3)) return cudaErrorUnknown;
-    // the tensor-core attention kernel merges the chunk partials itself
-    if (!fused) {
-        if (g.d == 128) decode_combine_kernel<128><<<g.B * g.Hq, 128, 0, stream>>>(count, part, ob, g);
-        else decode_combine_kernel<64><<<g.B * g.Hq, 128, 0, stream>>>(count, part, ob, g);
-    }
-    if (!mark(4)) return cudaErrorUnknown;
     return cudaGetLastError();
 }
 

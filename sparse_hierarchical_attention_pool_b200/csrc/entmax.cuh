@@ -44,6 +44,30 @@ struct EntmaxPass {
             }
         }
     }
+    // Branch-free form for a solver mode known at compile time (1: alpha = 1.5, 2: alpha = 2,
+    // 0: any other alpha), accumulating only the sums that mode's update reads.
+    template <int MODE>
+    __device__ __forceinline__ void add_t(float z, float e) {
+        const bool pos = z > 0.f;
+        const float zp = pos ? z : 0.f;
+        if constexpr (MODE != 0) {
+            z0 += pos ? 1.f : 0.f;
+            z1 += zp;
+            minz = fminf(minz, pos ? z : INFINITY);
+        }
+        if constexpr (MODE == 1) z2 = fmaf(zp, zp, z2);
+        if constexpr (MODE == 0) {
+            const float zq = pos ? __powf(z, e - 1.0f) : 0.f;
+            de += zq;
+            fe = fmaf(zq, zp, fe);
+        }
+    }
+    template <int MODE>
+    __device__ __forceinline__ void warp_reduce_t() {
+        if constexpr (MODE != 0) { z0 = warp_sum(z0); z1 = warp_sum(z1); minz = warp_min(minz); }
+        if constexpr (MODE == 1) z2 = warp_sum(z2);
+        if constexpr (MODE == 0) { fe = warp_sum(fe); de = warp_sum(de); }
+    }
     __device__ __forceinline__ void merge(const EntmaxPass& o) {
         z0 += o.z0; z1 += o.z1; z2 += o.z2; fe += o.fe; de += o.de; minz = fminf(minz, o.minz);
     }

@@ -180,7 +180,8 @@ def dash_prefill_profiled(q, k, v, out, alpha, coarse_scale, workspace, events, 
 
 def dash_decode_profiled(q, k_cache, v_cache, ksum, kv_len, out, alpha, coarse_scale, workspace, events,
                          block=64, stream=None):
-    """dash_decode recording torch.cuda.Event objects events[0..4] around its four kernels."""
+    """dash_decode recording torch.cuda.Event objects events[0..3]: before the coarse kernels,
+    before the attention kernel, after it, and after the merge kernel (if any)."""
     B, Hq, d = q.shape
     Hkv, Tmax = k_cache.shape[1], k_cache.shape[2]
     rc = lib().dash_decode_profiled(_dev(q, torch.bfloat16, "q"), _dev(k_cache, torch.bfloat16, "k_cache"),
