@@ -235,6 +235,31 @@ def bench_prefill(args, ws, rank, local):
     peak = pk["bf16_tflops"]
     fine_ms = mean(fine)
     achieved = fine_alg / (fine_ms * 1e-3) / 1e12
+    # block-summary kernel: reads K, writes the fp32 means and their bf16 hi/lo parts
+    nb = T // 64
+    sum_bytes = B * Hkv * T * d * 2 + B * Hkv * nb * d * (4 + 2 + 2)
+    sum_gbs = sum_bytes / (mean(summ) * 1e-3) / 1e9
+    summary_roofline = {"bound": "hbm", "kernel": "block_summary_kernel", "bytes_per_launch": sum_bytes,
+                        "achieved": round(sum_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                        "frac": round(sum_gbs / pk["hbm_gbs"], 4)}
+    # context only: dense causal attention FLOPs and torch's SDPA (flash) on the same tensors
+    dense_flops = 4.0 * d * B * Hq * T * (T + 1) / 2
+    import torch.nn.functional as F
+    for _ in range(2):
+        F.scaled_dot_product_attention(qd, kd, vd, is_causal=True, enable_gqa=True)
+    sd = []
+    for _ in range(5):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        F.scaled_dot_product_attention(qd, kd, vd, is_causal=True, enable_gqa=True)
+        e1.record()
+        sd.append((e0, e1))
+    torch.cuda.synchronize()
+    sdpa_ms = mean([a.elapsed_time(b) for a, b in sd])
+    context = {"dense_causal_flops": dense_flops, "torch_sdpa_dense_causal_ms": round(sdpa_ms, 4),
+               "torch_sdpa_tflops": round(dense_flops / (sdpa_ms * 1e-3) / 1e12, 1),
+               "note": "library dense attention on the same inputs, for context only"}
     G = Hq // Hkv
     fine_kernel = "fine_tc_kernel" if G <= 16 else "fine_mma_kernel"
     traffic = (recorded_traffic("fine_tc_kernel", source_sha("fine_tc.cu", "sm100.cuh", "common.cuh"))
@@ -255,6 +280,8 @@ def bench_prefill(args, ws, rank, local):
                      "executed_frac": round(fine_exec / (fine_ms * 1e-3) / 1e12 / peak, 4),
                      "inflation": round(fine_exec / fine_alg, 3)},
         "coarse_algorithmic_flops": coarse_alg,
+        "summary_roofline": summary_roofline,
+        "context": context,
         "launches_per_step": 3,
         "wl": wl, "cs": cs,
     }
@@ -400,10 +427,11 @@ def oracle_rows_per_s(workload, n_rows, seed, tensors=None):
     cs = calibrated(workload)["coarse_scale"]
     rows = inputs.sample_rows(wl.B, wl.Hq, wl.T, n_rows, seed)
     qr = oracle.gather_q_rows(q, rows)
+    threads = len(os.sched_getaffinity(0))
     t0 = time.perf_counter()
-    oracle.forward_rows(qr, k, v, rows, wl.Hq, 64, wl.alpha, cs)
+    oracle.forward_rows(qr, k, v, rows, wl.Hq, 64, wl.alpha, cs, nthreads=threads)
     dt = time.perf_counter() - t0
-    return n_rows / dt, os.cpu_count(), wl, dt
+    return n_rows / dt, threads, wl, dt
 
 
 def cpu_baseline(args):
@@ -413,8 +441,10 @@ def cpu_baseline(args):
     n = int(max(64, min(20000, r * 10.0)))            # about 10 s of oracle work
     r, cores, wl, dt = oracle_rows_per_s(args.workload, n, 2, tensors)
     return {"value": r / wl.Hq, "unit": "tok/s", "cores": cores, "kind": "oracle",
+            "rows_per_s": r, "rows_per_s_per_core": r / cores,
             "sample": f"{n} uniformly drawn rows (b, h, t) of the {wl.name} workload, fp64 C oracle "
-                      f"with OpenMP over rows, {dt:.1f} s; tok/s = rows/s / Hq (extrapolated)"}
+                      f"with OpenMP over rows on {cores} threads, {dt:.1f} s; tok/s = rows/s / Hq "
+                      "(extrapolated); per core = all-thread rate / threads"}
 
 
 def run_reference(args):
@@ -506,6 +536,8 @@ def main():
             "clocks": pre["clocks"],
             "gpu_launches": pre["launches_per_step"] * args.steps,
             "stage_ms": pre["stage_ms"],
+            "summary_roofline": pre["summary_roofline"],
+            "context": pre["context"],
             "prefill_stats": pre["stats"],
             "decode": dec,
         }

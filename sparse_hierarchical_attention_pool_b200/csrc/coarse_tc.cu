@@ -98,7 +98,8 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __shared__ int unconverged_sh;
     __shared__ unsigned bitmap[kMaxT / kBlock / 32];
     __shared__ unsigned long long sel_sh;
-    __shared__ float xs[2][6][kTileRows];        // [half][sum][row]: partial pass sums
+    __shared__ float xp[2][2][6][kTileRows];     // [pass parity][half][sum][row]: partial pass sums
+    __shared__ int wtot_sh[8];
 
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -229,6 +230,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // ------------------------------------------------------------ threshold warps 0-7
         const int quarter = warp & 3, hf = warp >> 2;
         const int r = quarter * 32 + lane;                  // tile row = TMEM lane
+        const int st = warp * 32 + lane;                    // 0 .. 255
         const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
         int uses[kCtBufs] = {0, 0, 0, 0};
         int gch = 0;
@@ -239,6 +241,8 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             return __all_sync(0xffffffffu, got);
         };
         auto sync8 = [&]() { asm volatile("bar.sync 1, 256;" ::: "memory"); };
+        // the two warps (w, w + 4) that share a quarter of the tile rows
+        auto sync_pair = [&]() { asm volatile("bar.sync %0, 64;" :: "r"(2 + quarter) : "memory"); };
         for (int w = blockIdx.x; ok && w < g.ntiles; w += gridDim.x) {
             const TileInfo ti = tile_info(g, w);
             const int hl = r / g.P, t = ti.t0 + r % g.P;
@@ -262,131 +266,259 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 mbar_arrive(bar(C_C_FREE + bf));
                 ++uses[bf];
             };
-            // one sweep over the row's scores: streamed tiles acquire and release every
-            // chunk of every pass, resident tiles acquire in pass 0 and release at the end
-            auto run_pass = [&](auto&& fn) -> bool {
-                if (!ti.resident || pass == 0) { sweep_base = gch; gch += ti.nch; }
-                for (int c = 0; c < ti.nch; ++c) {
-                    const int bf = (sweep_base + c) % kCtBufs;
-                    if ((!ti.resident || pass == 0) && !acquire(bf)) return false;
-                    const int ncol = min(kCtChunk, ti.bt - c * kCtChunk);
-                    for (int g32 = hf; g32 < (ncol + 31) / 32; g32 += 2) {
-                        uint32_t v[32];
-                        tmem_ld32(lane_addr + bf * kCtChunk + g32 * 32, v);
-                        tmem_wait_ld();
-                        fn(c * kCtChunk + g32 * 32, v, min(32, ncol - g32 * 32));
-                    }
-                    if (!ti.resident) release(bf);
-                }
-                ++pass;
-                return true;
-            };
-            // announce whether the scores are swept once more (streamed tiles only)
-            auto announce = [&](bool more) {
-                if (ti.resident) return;
-                if (r == 0 && hf == 0) {
-                    decision_sh = more ? 1 : 0;
-                    __threadfence_block();
-                    mbar_arrive(bar(C_DEC));
-                }
-            };
-            // ---- pass 0: row maximum
-            float m = -INFINITY;
-            if (!run_pass([&](int, const uint32_t* v, int nv) {
-                    for (int i = 0; i < 32; ++i)
-                        if (i < nv) m = fmaxf(m, __fmul_rn(__uint_as_float(v[i]), cx));
-                })) { ok = false; break; }
-            xs[hf][0][r] = m;
-            sync8();
-            m = fmaxf(xs[0][0][r], xs[1][0][r]);
-            EntmaxSolver sv;
-            sv.init(m, alpha);
-            float tau = INFINITY;
-            bool done = !valid;
-            // ---- Newton / exact-support passes until every row of the tile is final
-            while (true) {
-                sync8();                                   // the previous flag and sums have been read
-                if (r == 0 && hf == 0) unconverged_sh = 0;
-                sync8();
-                if (!done && hf == 0) atomicOr(&unconverged_sh, 1);
-                sync8();
-                const bool more = unconverged_sh != 0;
-                announce(true);                            // a Newton pass or the union pass follows
-                if (!more) break;
-                EntmaxPass ps;
-                ps.reset();
-                // z = (x - m) - u with x rounded exactly as in pass 0 (__fmul_rn is never fused
-                // into an FMA), so the maximum gives z = -u exactly
-                if (!run_pass([&](int, const uint32_t* v, int nv) {
-                        auto sweep = [&](auto mode) {
-                            constexpr int MODE = decltype(mode)::value;
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (i < nv) ps.add_t<MODE>((__fmul_rn(__uint_as_float(v[i]), cx) - sv.m) - sv.u, sv.e);
-                        };
-                        if (sv.mode == 1) sweep(std::integral_constant<int, 1>{});
-                        else if (sv.mode == 2) sweep(std::integral_constant<int, 2>{});
-                        else sweep(std::integral_constant<int, 0>{});
-                    })) { ok = false; break; }
-                xs[hf][0][r] = ps.z0; xs[hf][1][r] = ps.z1; xs[hf][2][r] = ps.z2;
-                xs[hf][3][r] = ps.fe; xs[hf][4][r] = ps.de; xs[hf][5][r] = ps.minz;
-                sync8();
-                // both threads of the row merge the halves in the same order
-                EntmaxPass tot;
-                tot.z0 = xs[0][0][r] + xs[1][0][r]; tot.z1 = xs[0][1][r] + xs[1][1][r];
-                tot.z2 = xs[0][2][r] + xs[1][2][r]; tot.fe = xs[0][3][r] + xs[1][3][r];
-                tot.de = xs[0][4][r] + xs[1][4][r]; tot.minz = fminf(xs[0][5][r], xs[1][5][r]);
-                if (!done) done = sv.update(tot, &tau, &no_conv);
-            }
-            if (!ok) break;
-            // ---- union pass: OR of x > tau over the rows, per block
             const int nw = (ti.bt + 31) / 32;
-            for (int i = warp * 32 + lane; i < nw; i += 256) bitmap[i] = 0u;
-            if (r == 0 && hf == 0) sel_sh = 0ull;
-            sync8();
+            float tau = INFINITY;
             float nsel = 0.f;
-            if (!run_pass([&](int j0, const uint32_t* v, int nv) {
+            if (ti.resident) {
+                // ---- every chunk stays in TMEM for the whole tile.  This thread's first four
+                // 32-column groups (chunks 0 and 1: blocks below 256) are read once into
+                // registers (-inf past bt); groups of chunks 2 and 3 are read from TMEM per pass.
+                sweep_base = gch;
+                gch += ti.nch;
+                bool got = true;
+                for (int c = 0; c < ti.nch && got; ++c) got = acquire((sweep_base + c) % kCtBufs);
+                if (!got) { ok = false; break; }
+                float xc[4][32];
+#pragma unroll
+                for (int kp = 0; kp < 2; ++kp) {               // two groups in flight at a time
+                    uint32_t v[2][32];
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk) {
+                        const int k = 2 * kp + kk, c = k >> 1, g32 = hf + 2 * (k & 1);
+                        if (c < ti.nch && c * kCtChunk + g32 * 32 < ti.bt)
+                            tmem_ld32(lane_addr + ((sweep_base + c) % kCtBufs) * kCtChunk + g32 * 32, v[kk]);
+                    }
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk) {
+                        const int k = 2 * kp + kk, c = k >> 1, g32 = hf + 2 * (k & 1);
+                        const int nv = ti.bt - (c * kCtChunk + g32 * 32);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            xc[k][i] = (c < ti.nch && i < nv) ? __fmul_rn(__uint_as_float(v[kk][i]), cx) : -INFINITY;
+                    }
+                }
+                // groups past the register cache (chunks 2 and 3), 16 columns per TMEM load
+                auto tail = [&](auto&& fn) {
+                    for (int c = 2; c < ti.nch; ++c) {
+                        const int ncol = min(kCtChunk, ti.bt - c * kCtChunk);
+                        for (int g32 = hf; g32 < (ncol + 31) / 32; g32 += 2)
+                            for (int h16 = 0; h16 < 2 && g32 * 32 + h16 * 16 < ncol; ++h16) {
+                                uint32_t v[16];
+                                tmem_ld16(lane_addr + ((sweep_base + c) % kCtBufs) * kCtChunk + g32 * 32 + h16 * 16, v);
+                                tmem_wait_ld();
+                                fn(c * kCtChunk + g32 * 32 + h16 * 16, v, min(16, ncol - g32 * 32 - h16 * 16));
+                            }
+                    }
+                };
+                float m = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) m = fmaxf(m, xc[k][i]);
+                tail([&](int, const uint32_t* v, int nv) {
+                    for (int i = 0; i < 16; ++i)
+                        if (i < nv) m = fmaxf(m, __fmul_rn(__uint_as_float(v[i]), cx));
+                });
+                xp[0][hf][0][r] = m;
+                sync_pair();
+                m = fmaxf(xp[0][0][0][r], xp[0][1][0][r]);
+                EntmaxSolver sv;
+                sv.init(m, alpha);
+                bool done = !valid;
+                // ---- Newton / exact-support passes; the pair of warps iterates until all of
+                // its 32 rows are final (both warps see the same flags), partial sums are
+                // exchanged through a buffer alternating with the pass parity
+                auto sweep = [&](auto mode) {
+                    constexpr int MODE = decltype(mode)::value;
+                    for (int pp = 1; __any_sync(0xffffffffu, !done); ++pp) {
+                        EntmaxPass ps;
+                        ps.reset();
+                        const float mm = sv.m, uu = sv.u;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) ps.add_t<MODE>((xc[k][i] - mm) - uu, sv.e);
+                        tail([&](int, const uint32_t* v, int nv) {
+                            for (int i = 0; i < 16; ++i)
+                                if (i < nv) ps.add_t<MODE>((__fmul_rn(__uint_as_float(v[i]), cx) - mm) - uu, sv.e);
+                        });
+                        float* xb = &xp[pp & 1][hf][0][0];
+                        xb[0 * kTileRows + r] = ps.z0; xb[1 * kTileRows + r] = ps.z1; xb[2 * kTileRows + r] = ps.z2;
+                        xb[3 * kTileRows + r] = ps.fe; xb[4 * kTileRows + r] = ps.de; xb[5 * kTileRows + r] = ps.minz;
+                        sync_pair();
+                        // both threads of the row merge the halves in the same order
+                        EntmaxPass tot;
+                        tot.z0 = xp[pp & 1][0][0][r] + xp[pp & 1][1][0][r]; tot.z1 = xp[pp & 1][0][1][r] + xp[pp & 1][1][1][r];
+                        tot.z2 = xp[pp & 1][0][2][r] + xp[pp & 1][1][2][r]; tot.fe = xp[pp & 1][0][3][r] + xp[pp & 1][1][3][r];
+                        tot.de = xp[pp & 1][0][4][r] + xp[pp & 1][1][4][r]; tot.minz = fminf(xp[pp & 1][0][5][r], xp[pp & 1][1][5][r]);
+                        if (!done) done = sv.update(tot, &tau, &no_conv);
+                    }
+                };
+                if (sv.mode == 1) sweep(std::integral_constant<int, 1>{});
+                else if (sv.mode == 2) sweep(std::integral_constant<int, 2>{});
+                else sweep(std::integral_constant<int, 0>{});
+                // ---- union pass: OR of x > tau over the rows, per block
+                for (int i = st; i < nw; i += 256) bitmap[i] = 0u;
+                if (st == 0) sel_sh = 0ull;
+                sync8();
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int c = k >> 1, g32 = hf + 2 * (k & 1);
+                    const int j0 = c * kCtChunk + g32 * 32;
+                    if (j0 < ti.bt) {                           // warp-uniform
+                        unsigned mask = 0u;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (valid && xc[k][i] > tau) mask |= 1u << i;
+                        nsel += (float)__popc(mask);
+                        const unsigned wm = __reduce_or_sync(0xffffffffu, mask);
+                        if (lane == 0 && wm) atomicOr(&bitmap[j0 >> 5], wm);
+                    }
+                }
+                tail([&](int j0, const uint32_t* v, int nv) {
                     unsigned mask = 0u;
-                    for (int i = 0; i < 32; ++i)
+                    for (int i = 0; i < 16; ++i)
                         if (i < nv && valid && __fmul_rn(__uint_as_float(v[i]), cx) > tau) mask |= 1u << i;
                     nsel += (float)__popc(mask);
                     const unsigned wm = __reduce_or_sync(0xffffffffu, mask);
-                    if (lane == 0 && wm) atomicOr(&bitmap[j0 >> 5], wm);
-                })) { ok = false; break; }
-            announce(false);
-            if (ti.resident)
+                    if (lane == 0 && wm) atomicOr(&bitmap[j0 >> 5], wm << (j0 & 31));
+                });
                 for (int c = 0; c < ti.nch; ++c) release((sweep_base + c) % kCtBufs);
+            } else {
+                // ---- streamed tile: score chunks are recomputed for every pass
+                auto run_pass = [&](auto&& fn) -> bool {
+                    sweep_base = gch;
+                    gch += ti.nch;
+                    for (int c = 0; c < ti.nch; ++c) {
+                        const int bf = (sweep_base + c) % kCtBufs;
+                        if (!acquire(bf)) return false;
+                        const int ncol = min(kCtChunk, ti.bt - c * kCtChunk);
+                        for (int g32 = hf; g32 < (ncol + 31) / 32; g32 += 2) {
+                            uint32_t v[32];
+                            tmem_ld32(lane_addr + bf * kCtChunk + g32 * 32, v);
+                            tmem_wait_ld();
+                            fn(c * kCtChunk + g32 * 32, v, min(32, ncol - g32 * 32));
+                        }
+                        release(bf);
+                    }
+                    ++pass;
+                    return true;
+                };
+                // tell the producer and the MMA issuer whether the scores are swept once more
+                auto announce = [&](bool more) {
+                    if (r == 0 && hf == 0) {
+                        decision_sh = more ? 1 : 0;
+                        __threadfence_block();
+                        mbar_arrive(bar(C_DEC));
+                    }
+                };
+                // ---- pass 0: row maximum
+                float m = -INFINITY;
+                if (!run_pass([&](int, const uint32_t* v, int nv) {
+                        for (int i = 0; i < 32; ++i)
+                            if (i < nv) m = fmaxf(m, __fmul_rn(__uint_as_float(v[i]), cx));
+                    })) { ok = false; break; }
+                xp[0][hf][0][r] = m;
+                sync8();
+                m = fmaxf(xp[0][0][0][r], xp[0][1][0][r]);
+                EntmaxSolver sv;
+                sv.init(m, alpha);
+                bool done = !valid;
+                // ---- Newton / exact-support passes until every row of the tile is final
+                while (true) {
+                    sync8();                                   // the previous flag and sums have been read
+                    if (r == 0 && hf == 0) unconverged_sh = 0;
+                    sync8();
+                    if (!done && hf == 0) atomicOr(&unconverged_sh, 1);
+                    sync8();
+                    const bool more = unconverged_sh != 0;
+                    announce(true);                            // a Newton pass or the union pass follows
+                    if (!more) break;
+                    EntmaxPass ps;
+                    ps.reset();
+                    // z = (x - m) - u with x rounded exactly as in pass 0 (__fmul_rn is never
+                    // fused into an FMA), so the maximum gives z = -u exactly
+                    if (!run_pass([&](int, const uint32_t* v, int nv) {
+                            auto acc = [&](auto mode) {
+                                constexpr int MODE = decltype(mode)::value;
+#pragma unroll
+                                for (int i = 0; i < 32; ++i)
+                                    if (i < nv) ps.add_t<MODE>((__fmul_rn(__uint_as_float(v[i]), cx) - sv.m) - sv.u, sv.e);
+                            };
+                            if (sv.mode == 1) acc(std::integral_constant<int, 1>{});
+                            else if (sv.mode == 2) acc(std::integral_constant<int, 2>{});
+                            else acc(std::integral_constant<int, 0>{});
+                        })) { ok = false; break; }
+                    xp[0][hf][0][r] = ps.z0; xp[0][hf][1][r] = ps.z1; xp[0][hf][2][r] = ps.z2;
+                    xp[0][hf][3][r] = ps.fe; xp[0][hf][4][r] = ps.de; xp[0][hf][5][r] = ps.minz;
+                    sync8();
+                    EntmaxPass tot;
+                    tot.z0 = xp[0][0][0][r] + xp[0][1][0][r]; tot.z1 = xp[0][0][1][r] + xp[0][1][1][r];
+                    tot.z2 = xp[0][0][2][r] + xp[0][1][2][r]; tot.fe = xp[0][0][3][r] + xp[0][1][3][r];
+                    tot.de = xp[0][0][4][r] + xp[0][1][4][r]; tot.minz = fminf(xp[0][0][5][r], xp[0][1][5][r]);
+                    if (!done) done = sv.update(tot, &tau, &no_conv);
+                }
+                if (!ok) break;
+                // ---- union pass: OR of x > tau over the rows, per block
+                for (int i = st; i < nw; i += 256) bitmap[i] = 0u;
+                if (st == 0) sel_sh = 0ull;
+                sync8();
+                if (!run_pass([&](int j0, const uint32_t* v, int nv) {
+                        unsigned mask = 0u;
+                        for (int i = 0; i < 32; ++i)
+                            if (i < nv && valid && __fmul_rn(__uint_as_float(v[i]), cx) > tau) mask |= 1u << i;
+                        nsel += (float)__popc(mask);
+                        const unsigned wm = __reduce_or_sync(0xffffffffu, mask);
+                        if (lane == 0 && wm) atomicOr(&bitmap[j0 >> 5], wm);
+                    })) { ok = false; break; }
+                announce(false);
+            }
             if (valid && hf == 0) tau_out[tau_idx] = tau;
             nsel = warp_sum(nsel);
             if (lane == 0) atomicAdd(&sel_sh, (unsigned long long)nsel);
             sync8();
-            if (warp == 0) {
-                int basei = 0;
-                int* dst = list + ti.tile_id * g.cap;
-                for (int w0 = 0; w0 < nw; w0 += 32) {
-                    const int wi = w0 + lane;
-                    unsigned word = wi < nw ? bitmap[wi] : 0u;
-                    const int pc = __popc(word);
-                    int incl = pc;
+            // ---- compaction: thread st owns bitmap words 2 st and 2 st + 1; a block-wide
+            // scan of their popcounts places them in the tile's ascending list
+            {
+                unsigned wv[2];
+                int pc = 0;
 #pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const int nn = __shfl_up_sync(0xffffffffu, incl, o);
-                        if (lane >= o) incl += nn;
-                    }
-                    int pos = basei + incl - pc;
+                for (int k = 0; k < 2; ++k) {
+                    const int wi = 2 * st + k;
+                    wv[k] = wi < nw ? bitmap[wi] : 0u;
+                    pc += __popc(wv[k]);
+                }
+                int incl = pc;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int nn = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += nn;
+                }
+                if (lane == 31) wtot_sh[warp] = incl;
+                sync8();
+                int basei = 0, total = 0;
+                for (int wv8 = 0; wv8 < 8; ++wv8) {
+                    if (wv8 < warp) basei += wtot_sh[wv8];
+                    total += wtot_sh[wv8];
+                }
+                int pos = basei + incl - pc;
+                int* dst = list + ti.tile_id * g.cap;
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    unsigned word = wv[k];
                     while (word) {
                         const int bit = __ffs(word) - 1;
-                        dst[pos++] = wi * 32 + bit;
+                        dst[pos++] = (2 * st + k) * 32 + bit;
                         word &= word - 1;
                     }
-                    basei += __shfl_sync(0xffffffffu, incl, 31);
                 }
-                if (lane == 0) {
-                    count[ti.tile_id] = basei;
+                if (st == 0) {
+                    count[ti.tile_id] = total;
                     const int rows_valid = g.G * min(g.P, g.T - ti.t0);
                     atomicAdd(&hdr->selected_pairs, sel_sh);
                     atomicAdd(&hdr->scored_pairs, (unsigned long long)rows_valid * ti.bt);
-                    atomicAdd(&hdr->union_blocks, (unsigned long long)basei);
+                    atomicAdd(&hdr->union_blocks, (unsigned long long)total);
                     atomicAdd(&hdr->tiles, 1ull);
                 }
             }
