@@ -485,7 +485,8 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="16k", choices=["16k", "32k", "96k"])
+    ap.add_argument("--workload", default="16k", choices=["16k", "32k", "96k", "16k-coherent"],
+                    help="16k-coherent is not a target workload: block-coherent query topics")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-only", action="store_true",

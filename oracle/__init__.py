@@ -50,6 +50,13 @@ def lib():
         L.oracle_entmax_tau.argtypes = [_ptr, _i64, _dbl, ctypes.c_int, _ptr]
         L.oracle_entmax.argtypes = [_ptr, _i64, _dbl, _ptr, _ptr]
         L.oracle_block_summary.argtypes = [_ptr, ctypes.c_int, _i64, _i64, _i64, _i64, _i64, _ptr]
+        L.oracle_block_summary_w.argtypes = [_ptr, ctypes.c_int, _ptr, _i64, _i64, _i64, _i64, _i64, _ptr]
+        L.oracle_select_rows_w.argtypes = ([_ptr, ctypes.c_int, _ptr, ctypes.c_int, _ptr]
+                                           + [_i64] * 6 + [_dbl, _dbl, _ptr, _i64]
+                                           + [_ptr] * 5 + [ctypes.c_int])
+        L.oracle_forward_rows_w.argtypes = ([_ptr, ctypes.c_int, _ptr, ctypes.c_int, _ptr, ctypes.c_int, _ptr]
+                                            + [_i64] * 6 + [_dbl, _dbl, _ptr, _i64]
+                                            + [_ptr] * 3 + [ctypes.c_int])
         L.oracle_select_rows.argtypes = ([_ptr, ctypes.c_int, _ptr, ctypes.c_int]
                                          + [_i64] * 6 + [_dbl, _dbl, _ptr, _i64]
                                          + [_ptr] * 5 + [ctypes.c_int])
@@ -60,6 +67,8 @@ def lib():
                                                + [_i64] * 6 + [_ptr, _i64, _ptr, _ptr, _ptr, ctypes.c_int])
         L.oracle_dense_causal_rows.argtypes = ([_ptr, ctypes.c_int, _ptr, ctypes.c_int, _ptr, ctypes.c_int]
                                                + [_i64] * 5 + [_ptr, _i64, _ptr, ctypes.c_int])
+        for f in (L.oracle_block_summary_w, L.oracle_select_rows_w, L.oracle_forward_rows_w):
+            f.restype = ctypes.c_int
         for f in (L.oracle_entmax_tau, L.oracle_entmax, L.oracle_block_summary, L.oracle_select_rows,
                   L.oracle_forward_rows, L.oracle_fine_rows_given_p, L.oracle_dense_causal_rows):
             f.restype = ctypes.c_int
@@ -111,13 +120,28 @@ def entmax(s, alpha):
     return p, float(tau[0])
 
 
-def block_summary(k, blk):
-    """Mean of each complete block of keys: k [B, Hkv, T, d] -> [B, Hkv, T // blk, d] fp64."""
+def block_summary(k, blk, w=None):
+    """Summary of each complete block of keys: k [B, Hkv, T, d] -> [B, Hkv, T // blk, d] fp64.
+
+    w=None: the mean.  w [Hkv, d]: the learned head, attention pooling of the block's keys
+    with softmax(w_g . k_i / sqrt(d)) weights ("DashAttention and the year sparse attention
+    became a field", section "What alpha-entmax changes", Stage 0)."""
     ka, kdt = _arr(k)
     B, Hkv, T, d = ka.shape
     out = np.zeros((B, Hkv, T // blk, d))
-    _check(lib().oracle_block_summary(_p(ka), kdt, B, Hkv, T, d, blk, _p(out)), "block_summary")
+    if w is None:
+        _check(lib().oracle_block_summary(_p(ka), kdt, B, Hkv, T, d, blk, _p(out)), "block_summary")
+    else:
+        wa = _wsum(w, Hkv, d)
+        _check(lib().oracle_block_summary_w(_p(ka), kdt, _p(wa), B, Hkv, T, d, blk, _p(out)), "block_summary_w")
     return out
+
+
+def _wsum(w, Hkv, d):
+    wa = np.ascontiguousarray(np.asarray(w, dtype=np.float64))
+    if wa.shape != (Hkv, d):
+        raise ValueError(f"summary head weights must be [Hkv, d] = [{Hkv}, {d}], got {wa.shape}")
+    return wa
 
 
 def _rows(rows):
@@ -125,8 +149,9 @@ def _rows(rows):
     return r, r.shape[0]
 
 
-def select_rows(q_rows, k, rows, Hq, blk, alpha, coarse_scale, nthreads=0):
+def select_rows(q_rows, k, rows, Hq, blk, alpha, coarse_scale, nthreads=0, w_summary=None):
     """Coarse stage for rows (b, h, t); q_rows [n, d] holds those rows' query vectors.
+    w_summary [Hkv, d]: learned summary head (None: mean pooling).
 
     Returns dict with x [n, nbs], p [n, nbs], tau [n], bt [n], nsel [n]."""
     qa, qdt = _arr(q_rows)
@@ -139,15 +164,18 @@ def select_rows(q_rows, k, rows, Hq, blk, alpha, coarse_scale, nthreads=0):
     tau = np.zeros(n)
     bt = np.zeros(n, dtype=np.int64)
     ns = np.zeros(n, dtype=np.int64)
-    _check(lib().oracle_select_rows(_p(qa), qdt, _p(ka), kdt, B, Hq, Hkv, Tk, d, blk,
-                                    float(alpha), float(coarse_scale), _p(r), n,
-                                    _p(x), _p(p), _p(tau), _p(bt), _p(ns), int(nthreads)),
+    wa = None if w_summary is None else _wsum(w_summary, Hkv, d)
+    _check(lib().oracle_select_rows_w(_p(qa), qdt, _p(ka), kdt, None if wa is None else _p(wa),
+                                      B, Hq, Hkv, Tk, d, blk,
+                                      float(alpha), float(coarse_scale), _p(r), n,
+                                      _p(x), _p(p), _p(tau), _p(bt), _p(ns), int(nthreads)),
            "select_rows")
     return {"x": x, "p": p, "tau": tau, "bt": bt, "nsel": ns}
 
 
-def forward_rows(q_rows, k, v, rows, Hq, blk, alpha, coarse_scale, nthreads=0):
-    """Full forward for rows (b, h, t): returns (out [n, d] fp64, tau [n], nsel [n])."""
+def forward_rows(q_rows, k, v, rows, Hq, blk, alpha, coarse_scale, nthreads=0, w_summary=None):
+    """Full forward for rows (b, h, t): returns (out [n, d] fp64, tau [n], nsel [n]).
+    w_summary [Hkv, d]: learned summary head (None: mean pooling)."""
     qa, qdt = _arr(q_rows)
     ka, kdt = _arr(k)
     va, vdt = _arr(v)
@@ -156,9 +184,11 @@ def forward_rows(q_rows, k, v, rows, Hq, blk, alpha, coarse_scale, nthreads=0):
     out = np.zeros((n, d))
     tau = np.zeros(n)
     ns = np.zeros(n, dtype=np.int64)
-    _check(lib().oracle_forward_rows(_p(qa), qdt, _p(ka), kdt, _p(va), vdt, B, Hq, Hkv, Tk, d, blk,
-                                     float(alpha), float(coarse_scale), _p(r), n,
-                                     _p(out), _p(tau), _p(ns), int(nthreads)),
+    wa = None if w_summary is None else _wsum(w_summary, Hkv, d)
+    _check(lib().oracle_forward_rows_w(_p(qa), qdt, _p(ka), kdt, _p(va), vdt, None if wa is None else _p(wa),
+                                       B, Hq, Hkv, Tk, d, blk,
+                                       float(alpha), float(coarse_scale), _p(r), n,
+                                       _p(out), _p(tau), _p(ns), int(nthreads)),
            "forward_rows")
     return out, tau, ns
 

@@ -22,6 +22,10 @@
  *
  * Readings where the pages are silent (stated once here, used everywhere below):
  *   - block summary = arithmetic mean of the block's keys (the zero-initialised head);
+ *     with a learned head ([P3] "What alpha-entmax changes": Stage 0 is a small attention
+ *     head initialised at zero), an attention pooling of the block's keys with one query
+ *     vector w_g per KV head: kbar_j = sum_i softmax_i(w_g . k_i / sqrt(d)) k_i, which is
+ *     the mean when w_g = 0;
  *   - only complete blocks strictly before the query's own block are scored;
  *   - coarse score s_j = coarse_scale * (q . kbar_j) / sqrt(d); fine logits use 1/sqrt(d);
  *   - the query's own block is always attended causally with prior weight 1 (log 0 prior);
@@ -238,6 +242,49 @@ int oracle_block_summary(const void* k, int kdtype, long long B, long long Hkv, 
     return ORC_OK;
 }
 
+/* Learned summary head: kbar[b,g,j,:] = sum_i a_i k_i over the blk keys of complete block j,
+ * a = softmax(w[g,:] . k_i / sqrt(d)).  w is fp64 [Hkv, d]; w = NULL gives the mean. */
+int oracle_block_summary_w(const void* k, int kdtype, const double* w, long long B, long long Hkv,
+                           long long Tk, long long d, long long blk, double* kbar) {
+    if (!w) return oracle_block_summary(k, kdtype, B, Hkv, Tk, d, blk, kbar);
+    if (!k || !kbar || B < 1 || Hkv < 1 || Tk < 0 || d < 1 || blk < 1) return ORC_ERR_ARG;
+    long long nbs = Tk / blk;
+    double isd = 1.0 / sqrt((double)d);
+    int fail = 0;
+    #pragma omp parallel
+    {
+        double* a = (double*)malloc((size_t)blk * sizeof(double));
+        if (!a) {
+            #pragma omp atomic write
+            fail = 1;
+        }
+        #pragma omp for collapse(2) schedule(static)
+        for (long long bg = 0; bg < B * Hkv; ++bg)
+            for (long long j = 0; j < nbs; ++j) {
+                if (!a) continue;
+                const double* wg = w + (bg % Hkv) * d;
+                double m = -INFINITY;
+                for (long long i = 0; i < blk; ++i) {
+                    long long base = (bg * Tk + j * blk + i) * d;
+                    double s = 0.0;
+                    for (long long c = 0; c < d; ++c) s += wg[c] * elem(k, kdtype, base + c);
+                    a[i] = s * isd;
+                    if (a[i] > m) m = a[i];
+                }
+                double den = 0.0;
+                for (long long i = 0; i < blk; ++i) { a[i] = exp(a[i] - m); den += a[i]; }
+                double* o = kbar + (bg * nbs + j) * d;
+                for (long long c = 0; c < d; ++c) o[c] = 0.0;
+                for (long long i = 0; i < blk; ++i) {
+                    long long base = (bg * Tk + j * blk + i) * d;
+                    for (long long c = 0; c < d; ++c) o[c] += (a[i] / den) * elem(k, kdtype, base + c);
+                }
+            }
+        free(a);
+    }
+    return fail ? ORC_ERR_NOMEM : ORC_OK;
+}
+
 /* ---------------------------------------------------------------- one row */
 
 typedef struct {
@@ -246,6 +293,7 @@ typedef struct {
     const void* v; int vdt;      /* [B, Hkv, Tk, d] */
     long long B, Hq, Hkv, Tk, d, blk;
     double alpha, cs;
+    const double* wsum;          /* learned summary head [Hkv, d], or NULL for the mean */
 } orc_problem;
 
 /* Coarse stage for one row: x_j = (alpha-1) * cs * (q . kbar_j) / sqrt(d) for j < bt,
@@ -311,7 +359,10 @@ static double* all_kbar(const orc_problem* P) {
     size_t cnt = (size_t)(P->B * P->Hkv * (nbs > 0 ? nbs : 1) * P->d);
     double* kb = (double*)malloc(cnt * sizeof(double));
     if (!kb) return NULL;
-    if (nbs > 0) oracle_block_summary(P->k, P->kdt, P->B, P->Hkv, P->Tk, P->d, P->blk, kb);
+    if (nbs > 0 && oracle_block_summary_w(P->k, P->kdt, P->wsum, P->B, P->Hkv, P->Tk, P->d, P->blk, kb)) {
+        free(kb);
+        return NULL;
+    }
     return kb;
 }
 
@@ -333,13 +384,13 @@ static int check_problem(const orc_problem* P, const long long* rows, long long 
  *   bt_out[r] = number of scored past blocks, nsel_out[r] = #{j : p_j > 0}.
  * Any output pointer may be NULL.
  */
-int oracle_select_rows(const void* q_rows, int qdt, const void* k, int kdt,
-                       long long B, long long Hq, long long Hkv, long long Tk, long long d,
-                       long long blk, double alpha, double coarse_scale,
-                       const long long* rows, long long nrows,
-                       double* x_out, double* p_out, double* tau_out,
-                       long long* bt_out, long long* nsel_out, int nthreads) {
-    orc_problem P = {q_rows, qdt, k, kdt, NULL, 0, B, Hq, Hkv, Tk, d, blk, alpha, coarse_scale};
+int oracle_select_rows_w(const void* q_rows, int qdt, const void* k, int kdt, const double* w_summary,
+                         long long B, long long Hq, long long Hkv, long long Tk, long long d,
+                         long long blk, double alpha, double coarse_scale,
+                         const long long* rows, long long nrows,
+                         double* x_out, double* p_out, double* tau_out,
+                         long long* bt_out, long long* nsel_out, int nthreads) {
+    orc_problem P = {q_rows, qdt, k, kdt, NULL, 0, B, Hq, Hkv, Tk, d, blk, alpha, coarse_scale, w_summary};
     int rc = check_problem(&P, rows, nrows);
     if (rc) return rc;
 #ifdef _OPENMP
@@ -384,12 +435,12 @@ int oracle_select_rows(const void* q_rows, int qdt, const void* k, int kdt,
  * out[r, :] (fp64), and optionally tau_out[r], nsel_out[r] (past blocks with p > 0).
  * For decode, pass the cache as k/v with Tk = Tmax and t = kv_len - 1.
  */
-int oracle_forward_rows(const void* q_rows, int qdt, const void* k, int kdt, const void* v, int vdt,
-                        long long B, long long Hq, long long Hkv, long long Tk, long long d,
-                        long long blk, double alpha, double coarse_scale,
-                        const long long* rows, long long nrows,
-                        double* out, double* tau_out, long long* nsel_out, int nthreads) {
-    orc_problem P = {q_rows, qdt, k, kdt, v, vdt, B, Hq, Hkv, Tk, d, blk, alpha, coarse_scale};
+int oracle_forward_rows_w(const void* q_rows, int qdt, const void* k, int kdt, const void* v, int vdt,
+                          const double* w_summary, long long B, long long Hq, long long Hkv, long long Tk,
+                          long long d, long long blk, double alpha, double coarse_scale,
+                          const long long* rows, long long nrows,
+                          double* out, double* tau_out, long long* nsel_out, int nthreads) {
+    orc_problem P = {q_rows, qdt, k, kdt, v, vdt, B, Hq, Hkv, Tk, d, blk, alpha, coarse_scale, w_summary};
     int rc = check_problem(&P, rows, nrows);
     if (rc || !v || !out) return rc ? rc : ORC_ERR_ARG;
 #ifdef _OPENMP
@@ -432,6 +483,25 @@ int oracle_forward_rows(const void* q_rows, int qdt, const void* k, int kdt, con
     return fail ? ORC_ERR_NOMEM : ORC_OK;
 }
 
+int oracle_select_rows(const void* q_rows, int qdt, const void* k, int kdt,
+                       long long B, long long Hq, long long Hkv, long long Tk, long long d,
+                       long long blk, double alpha, double coarse_scale,
+                       const long long* rows, long long nrows,
+                       double* x_out, double* p_out, double* tau_out,
+                       long long* bt_out, long long* nsel_out, int nthreads) {
+    return oracle_select_rows_w(q_rows, qdt, k, kdt, NULL, B, Hq, Hkv, Tk, d, blk, alpha, coarse_scale,
+                                rows, nrows, x_out, p_out, tau_out, bt_out, nsel_out, nthreads);
+}
+
+int oracle_forward_rows(const void* q_rows, int qdt, const void* k, int kdt, const void* v, int vdt,
+                        long long B, long long Hq, long long Hkv, long long Tk, long long d,
+                        long long blk, double alpha, double coarse_scale,
+                        const long long* rows, long long nrows,
+                        double* out, double* tau_out, long long* nsel_out, int nthreads) {
+    return oracle_forward_rows_w(q_rows, qdt, k, kdt, v, vdt, NULL, B, Hq, Hkv, Tk, d, blk, alpha,
+                                 coarse_scale, rows, nrows, out, tau_out, nsel_out, nthreads);
+}
+
 /*
  * Fine stage alone with caller-given weights: w_rows[r, j] for past blocks j < bt
  * (row-major with floor(Tk/blk) columns) and diagonal weight w_diag[r].
@@ -441,7 +511,7 @@ int oracle_fine_rows_given_p(const void* q_rows, int qdt, const void* k, int kdt
                              long long B, long long Hq, long long Hkv, long long Tk, long long d,
                              long long blk, const long long* rows, long long nrows,
                              const double* w_rows, const double* w_diag, double* out, int nthreads) {
-    orc_problem P = {q_rows, qdt, k, kdt, v, vdt, B, Hq, Hkv, Tk, d, blk, 1.5, 1.0};
+    orc_problem P = {q_rows, qdt, k, kdt, v, vdt, B, Hq, Hkv, Tk, d, blk, 1.5, 1.0, NULL};
     int rc = check_problem(&P, rows, nrows);
     if (rc || !v || !out || !w_rows || !w_diag) return rc ? rc : ORC_ERR_ARG;
 #ifdef _OPENMP
@@ -471,7 +541,7 @@ int oracle_fine_rows_given_p(const void* q_rows, int qdt, const void* k, int kdt
 int oracle_dense_causal_rows(const void* q_rows, int qdt, const void* k, int kdt, const void* v, int vdt,
                              long long B, long long Hq, long long Hkv, long long Tk, long long d,
                              const long long* rows, long long nrows, double* out, int nthreads) {
-    orc_problem P = {q_rows, qdt, k, kdt, v, vdt, B, Hq, Hkv, Tk, d, 1, 1.5, 1.0};
+    orc_problem P = {q_rows, qdt, k, kdt, v, vdt, B, Hq, Hkv, Tk, d, 1, 1.5, 1.0, NULL};
     int rc = check_problem(&P, rows, nrows);
     if (rc || !v || !out) return rc ? rc : ORC_ERR_ARG;
 #ifdef _OPENMP

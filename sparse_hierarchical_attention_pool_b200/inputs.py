@@ -39,6 +39,7 @@ class Workload:
     target_sparsity: float | None
     seed: int
     fp32_source: bool = False   # inputs drawn in fp32, rounded once to bf16
+    coherent: bool = False      # one query topic per (b, 64-position block), shared by all heads
 
 
 WORKLOADS = {
@@ -52,6 +53,11 @@ WORKLOADS = {
                     256, 0.9375, 0xDA5A + 3),
     "decode96k": Workload("96K decode, B=8, 93.75% block sparsity", "decode", 8, 32, 8, 98304, 128, 64,
                           1.5, 256, 0.9375, 0xDA5A + 4),
+    # not a target workload: query topics shared by the heads and positions of a 64-token
+    # block, so the rows of a tile select correlated block sets (little union inflation)
+    "16k-coherent": Workload("16K prefill, 75% block sparsity, block-coherent query topics (non-target)",
+                             "prefill", 1, 16, 2, 16384, 128, 64, 1.5, 64, 0.75, 0xDA5A + 5,
+                             coherent=True),
 }
 
 
@@ -61,10 +67,12 @@ def _gen(seed: int) -> torch.Generator:
     return g
 
 
-def topic_prefill(B, Hq, Hkv, T, d, block, n_topics, seed, fp32_source=False):
+def topic_prefill(B, Hq, Hkv, T, d, block, n_topics, seed, fp32_source=False, coherent=False):
     """q [B,Hq,T,d], k, v [B,Hkv,T,d] in bf16 (CPU) from the topic generator.
 
-    n_topics == 0 gives plain N(0, 1) q, k, v (drawn in fp32, rounded once to bf16)."""
+    n_topics == 0 gives plain N(0, 1) q, k, v (drawn in fp32, rounded once to bf16).
+    coherent: the query topic is drawn per (b, 64-position block) and shared by every head
+    and position of the block (noise stays per query vector)."""
     g = _gen(seed)
     if n_topics == 0:
         q = torch.randn(B, Hq, T, d, generator=g)
@@ -81,7 +89,11 @@ def topic_prefill(B, Hq, Hkv, T, d, block, n_topics, seed, fp32_source=False):
         for h in range(Hkv):
             k[b, h] = (base + torch.randn(T, d, generator=g)).bfloat16()
     q = torch.empty(B, Hq, T, d, dtype=torch.bfloat16)
-    q_topic = torch.randint(0, n_topics, (B, Hq, T), generator=g)
+    if coherent:
+        qb_topic = torch.randint(0, n_topics, (B, nb), generator=g)
+        q_topic = qb_topic.repeat_interleave(block, dim=1)[:, :T].unsqueeze(1).expand(B, Hq, T)
+    else:
+        q_topic = torch.randint(0, n_topics, (B, Hq, T), generator=g)
     for b in range(B):
         for h in range(Hq):
             q[b, h] = (2.0 * topics[q_topic[b, h]] + torch.randn(T, d, generator=g)).bfloat16()
@@ -135,7 +147,7 @@ def make(name_or_wl, **override):
     if wl.kind == "decode":
         return wl, topic_decode(wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.block, wl.n_topics, wl.seed)
     return wl, topic_prefill(wl.B, wl.Hq, wl.Hkv, wl.T, wl.d, wl.block, wl.n_topics, wl.seed,
-                             wl.fp32_source)
+                             wl.fp32_source, wl.coherent)
 
 
 def sample_rows(B, Hq, T, n, seed, t_fixed=(), t_lo=0):

@@ -323,3 +323,84 @@ def test_bf16_input_path_widens_exactly(orc):
     o2, t2, _ = orc.forward_rows(qr.float().numpy(), kb.float().numpy(), vb.float().numpy(),
                                  rows, 2, 64, 1.5, 2.0)
     assert np.array_equal(o1, o2) and np.array_equal(t1, t2, equal_nan=True)
+
+
+# ------------------------------------------------------------------ learned summary head
+# "DashAttention and the year sparse attention became a field", section "What alpha-entmax
+# changes": Stage 0 is a small attention head initialised at zero (mean pooling at zero).
+
+def _keys(B, Hkv, T, d, seed):
+    g = np.random.default_rng(seed)
+    return g.standard_normal((B, Hkv, T, d)).astype(np.float32)
+
+
+def test_learned_summary_zero_head_is_the_mean(orc):
+    k = _keys(2, 3, 256, 16, 1)
+    np.testing.assert_allclose(orc.block_summary(k, 64, w=np.zeros((3, 16))), orc.block_summary(k, 64),
+                               rtol=0, atol=1e-12)
+
+
+def test_learned_summary_two_valued_block_closed_form(orc):
+    # a block whose keys take two values a (first 24 keys) and b (40 keys): the pooling
+    # weights are proportional to n_a e^{s_a} and n_b e^{s_b}, s = w . key / sqrt(d)
+    d = 4
+    a = np.array([1.0, -2.0, 0.5, 3.0])
+    b = np.array([-1.0, 0.25, 2.0, 0.0])
+    w = np.array([[0.3, -0.7, 1.1, 0.2]])
+    k = np.zeros((1, 1, 64, d), dtype=np.float32)
+    k[0, 0, :24] = a
+    k[0, 0, 24:] = b
+    sa, sb = w[0] @ a / 2.0, w[0] @ b / 2.0
+    wa, wb = 24 * np.exp(sa), 40 * np.exp(sb)
+    want = (wa * a + wb * b) / (wa + wb)
+    np.testing.assert_allclose(orc.block_summary(k, 64, w=w)[0, 0, 0], want, rtol=0, atol=1e-12)
+
+
+def test_learned_summary_sharp_head_picks_the_top_key(orc):
+    k = _keys(1, 1, 128, 8, 2)
+    w = np.zeros((1, 8))
+    w[0, 3] = 4000.0
+    s = orc.block_summary(k, 64, w=w)
+    for j in range(2):
+        blk = k[0, 0, 64 * j:64 * (j + 1)].astype(np.float64)
+        np.testing.assert_allclose(s[0, 0, j], blk[np.argmax(blk[:, 3])], rtol=0, atol=1e-6)
+
+
+def test_learned_summary_permutation_and_orthogonal_shift(orc):
+    d = 16
+    k = _keys(1, 2, 192, d, 3)
+    w = np.random.default_rng(4).standard_normal((2, d))
+    base = orc.block_summary(k, 64, w=w)
+    perm = k.copy()
+    for j in range(3):
+        idx = np.random.default_rng(10 + j).permutation(64)
+        perm[:, :, 64 * j:64 * (j + 1)] = k[:, :, 64 * j + idx]
+    np.testing.assert_allclose(orc.block_summary(perm, 64, w=w), base, rtol=0, atol=1e-12)
+    # adding c with w_g . c = 0 to every key of head g leaves the weights, and moves kbar by c
+    shifted = k.astype(np.float64).copy()
+    for g_ in range(2):
+        c = np.random.default_rng(20 + g_).standard_normal(d)
+        c -= (c @ w[g_]) / (w[g_] @ w[g_]) * w[g_]
+        shifted[:, g_] += c
+        want = base[:, g_] + c
+        got = orc.block_summary(shifted.astype(np.float32), 64, w=w)[:, g_]
+        np.testing.assert_allclose(got, want, rtol=0, atol=2e-6)   # float32 inputs
+
+
+def test_forward_with_zero_head_equals_mean_forward(orc):
+    import torch
+    B, Hq, Hkv, T, d = 1, 4, 2, 512, 16
+    g = torch.Generator().manual_seed(5)
+    q = torch.randn(B, Hq, T, d, generator=g).bfloat16()
+    k = torch.randn(B, Hkv, T, d, generator=g).bfloat16()
+    v = torch.randn(B, Hkv, T, d, generator=g).bfloat16()
+    rows = [(0, h, t) for h in range(Hq) for t in (70, 200, 511)]
+    qr = orc.gather_q_rows(q, rows)
+    o0, t0, _ = orc.forward_rows(qr, k, v, rows, Hq, 64, 1.5, 2.0)
+    o1, t1, _ = orc.forward_rows(qr, k, v, rows, Hq, 64, 1.5, 2.0, w_summary=np.zeros((Hkv, d)))
+    np.testing.assert_allclose(o1, o0, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(t1, t0, rtol=0, atol=1e-12)
+    # a learned head changes the selection of some row (it is not silently ignored)
+    w = np.random.default_rng(6).standard_normal((Hkv, d)) * 3.0
+    o2, t2, _ = orc.forward_rows(qr, k, v, rows, Hq, 64, 1.5, 2.0, w_summary=w)
+    assert np.abs(t2 - t0).max() > 1e-6

@@ -144,7 +144,7 @@ def test_stats_count_selected_pairs():
 
 # ------------------------------------------------------------------ the workloads at full size
 
-@pytest.mark.parametrize("name", ["16k", "96k"])
+@pytest.mark.parametrize("name", ["16k", "96k", "16k-coherent"])
 def test_workload_sampled_rows(name):
     wl, (q, k, v) = inputs.make(name)
     cs = calibrated_scale(name)
