@@ -4,8 +4,10 @@
 // Differentiable with Adaptive Block Selection", section "Core Mechanism", Stage 2, and
 // section "Key Concepts", hierarchical prior): for every row of a 128-row work tile,
 // softmax over the tokens of its selected blocks (log p_j added to the logits) and of its
-// own block (causal, prior 1), times V.  x_j, hence p_j, comes from the row sums of the
-// Q K^T block the kernel computes anyway (q . kbar_j is the mean of q . k_i).
+// own block (causal, prior 1), times V.  x_j, hence p_j, comes from two extra columns of
+// the S product: block j's summary, split into bf16 hi and lo parts (kbar = hi + lo to
+// 16 significant bits, the operands of the coarse stage), is appended to the K tile as
+// rows 64 and 72, so S[:, 64] + S[:, 72] = q . kbar_j for any summary (mean or learned).
 //
 // One CTA per tile.  The tile's listed blocks (steps s = 0 .. n-1, own block last) are
 // dealt alternately to two softmax groups (group s & 1), each with its own TMEM S buffer,
@@ -14,8 +16,10 @@
 // serial chain (load S, row stats, weights, exponentials, P), so two groups keep two chains
 // in flight while sharing the Q tile and every K/V load.  Warps:
 //   8 SPLIT            TMA producer (one lane): the Q tile once (one 64-column box per head
-//                      and half of d), then K and V of every listed block, 4-stage ring;
-//   8 SPLIT + 1        S issuer (one lane): S_s = Q K_s^T (M=128, N=64) into the S buffer of
+//                      and half of d), then K, the summary rows and V of every listed
+//                      block, 4-stage ring;
+//   8 SPLIT + 1        S issuer (one lane): S_s = Q [K_s | kbar_hi | kbar_lo]^T (M=128, N=80
+//                      with the summary atoms at columns 64 and 72) into the S buffer of
 //                      group s & 1 as soon as block s is loaded and that group has read
 //                      S_{s-2}, so S_{s+2} is computed while the group works on step s;
 //   8 SPLIT + 2        PV issuer (one lane): O_g += P_s V_s (M=128, N=d) and L_g += P_s 1
@@ -49,9 +53,12 @@ template <int D>
 struct TcLayout {
     static constexpr uint32_t kQHalf = 128 * 128;               // 128 rows x 64 bf16
     static constexpr uint32_t kQ = (D / 64) * kQHalf;
-    static constexpr uint32_t kKVHalf = 64 * 128;               // 64 keys x 64 bf16
-    static constexpr uint32_t kKV = (D / 64) * kKVHalf;
-    static constexpr uint32_t kStage = 2 * kKV;                 // K then V
+    static constexpr uint32_t kKRows = 80;                      // 64 keys, kbar hi atom, kbar lo atom
+    static constexpr uint32_t kKHalf = kKRows * 128;            // 80 rows x 64 bf16
+    static constexpr uint32_t kK = (D / 64) * kKHalf;
+    static constexpr uint32_t kVHalf = 64 * 128;                // 64 keys x 64 bf16
+    static constexpr uint32_t kV = (D / 64) * kVHalf;
+    static constexpr uint32_t kStage = kK + kV;                 // K (+ summary rows) then V
     static constexpr uint32_t kP = 128 * 128;                   // 128 rows x 64 keys bf16
     static constexpr uint32_t off_q = 0;
     static constexpr uint32_t off_kv = kQ;
@@ -59,8 +66,9 @@ struct TcLayout {
     static constexpr uint32_t off_ones = off_p + 2 * kP;        // 16 x 64 bf16 ones (B of the row sum)
     static constexpr uint32_t bytes = off_ones + 2048 + 1024;   // + alignment slack
     // TMEM columns: S of group 0 and 1, O of group 0 and 1, row sums of group 0 and 1
-    static constexpr uint32_t colO = 128;
-    static constexpr uint32_t colL = 128 + 2 * D;
+    static constexpr uint32_t colS = 96;                        // S buffer of group g at g * 96 (80 used)
+    static constexpr uint32_t colO = 192;
+    static constexpr uint32_t colL = 192 + 2 * D;
 };
 constexpr uint32_t kTmemCols = 512;
 
@@ -72,9 +80,10 @@ enum : int { B_Q = 0, B_KV_FULL = 1, B_KV_EMPTY = 1 + kTcStages, B_S_FULL = 1 + 
 template <int D, int SPLIT>
 __global__ void __launch_bounds__((8 * SPLIT + 3) * 32, 1)
 fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_hi,
+               const __grid_constant__ CUtensorMap tm_lo, __nv_bfloat16* __restrict__ out,
                const float* __restrict__ tau, const int* __restrict__ list, const int* __restrict__ count,
-               WsHeader* __restrict__ hdr, PrefillGeom g, float cxm, float e_pow, float sm2) {
+               WsHeader* __restrict__ hdr, PrefillGeom g, float cx, float e_pow, float sm2) {
     using L = TcLayout<D>;
     using namespace sm100;
     constexpr int kGroupThreads = 128 * SPLIT;  // softmax threads per group
@@ -157,6 +166,8 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
+            prefetch_tmap(&tm_hi);
+            prefetch_tmap(&tm_lo);
             mbar_arrive_expect_tx(bar(B_Q), (uint32_t)(g.M * D * 2));
             for (int hl = 0; hl < g.G; ++hl) {
                 const int row = (b * g.Hq + kvh * g.G + hl) * g.T + t0;
@@ -170,10 +181,15 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (s >= kTcStages && !mbar_wait(bar(B_KV_EMPTY + st), ((s / kTcStages) - 1) & 1, abort_flag)) break;
                 const int j = s < U ? lst[s] : bt;
                 const int row = bg * g.T + j * kBlock;
-                mbar_arrive_expect_tx(bar(B_KV_FULL + st), (uint32_t)(2 * kBlock * D * 2));
+                // the summary atoms: 8 rows of kbar hi / lo starting at block j (the own block,
+                // whose x is not used, reads a neighbour; rows past the array read zeros)
+                const int srow = g.nbs > 0 ? bg * g.nbs + min(j, g.nbs - 1) : 0;
+                mbar_arrive_expect_tx(bar(B_KV_FULL + st), (uint32_t)((2 * kBlock + 16) * D * 2));
                 for (int h = 0; h < D / 64; ++h) {
-                    tma_load_2d(kv_addr(st) + h * L::kKVHalf, &tm_k, h * 64, row, bar(B_KV_FULL + st));
-                    tma_load_2d(kv_addr(st) + L::kKV + h * L::kKVHalf, &tm_v, h * 64, row, bar(B_KV_FULL + st));
+                    tma_load_2d(kv_addr(st) + h * L::kKHalf, &tm_k, h * 64, row, bar(B_KV_FULL + st));
+                    tma_load_2d(kv_addr(st) + h * L::kKHalf + 64 * 128, &tm_hi, h * 64, srow, bar(B_KV_FULL + st));
+                    tma_load_2d(kv_addr(st) + h * L::kKHalf + 72 * 128, &tm_lo, h * 64, srow, bar(B_KV_FULL + st));
+                    tma_load_2d(kv_addr(st) + L::kK + h * L::kVHalf, &tm_v, h * 64, row, bar(B_KV_FULL + st));
                 }
                 last_armed[st] = s;
             }
@@ -190,7 +206,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // S_s = Q K_s^T into the S buffer of group s & 1, as soon as block s is loaded and the
         // group has read S_{s-2}: it runs ahead of the softmax by up to one step per group.
         if (lane == 0) {
-            const uint32_t idesc_s = idesc_bf16(128, 64, false);
+            const uint32_t idesc_s = idesc_bf16(128, L::kKRows, false);
             bool ok = mbar_wait(bar(B_Q), 0, abort_flag);
             for (int s = 0; ok && s < n; ++s) {
                 const int st = s % kTcStages, sb = s & 1;
@@ -201,8 +217,8 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const int h = kk >> 2, wk = kk & 3;
                     const uint64_t a = smem_desc_sw128(base + L::off_q + h * L::kQHalf + wk * 32, 16, 1024);
-                    const uint64_t bk = smem_desc_sw128(kv_addr(st) + h * L::kKVHalf + wk * 32, 16, 1024);
-                    mma_bf16_ss(tmem + sb * 64, a, bk, idesc_s, kk > 0 ? 1u : 0u);
+                    const uint64_t bk = smem_desc_sw128(kv_addr(st) + h * L::kKHalf + wk * 32, 16, 1024);
+                    mma_bf16_ss(tmem + sb * L::colS, a, bk, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar(B_S_FULL + sb));
             }
@@ -229,7 +245,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint64_t a = smem_desc_sw128(base + L::off_p + bp * L::kP + kk * 32, 16, 1024);
-                    const uint64_t bv = smem_desc_sw128(kv_addr(stp) + L::kKV + kk * 2048, L::kKVHalf, 1024);
+                    const uint64_t bv = smem_desc_sw128(kv_addr(stp) + L::kK + kk * 2048, L::kVHalf, 1024);
                     mma_bf16_ss(tmem + L::colO + bp * D, a, bv, idesc_pv, (acc || kk > 0) ? 1u : 0u);
                 }
 #pragma unroll
@@ -258,7 +274,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int tpos = valid ? t : -1;
         const float tau_r = (valid && bt > 0) ? tau[(size_t)(b * g.Hq + kvh * g.G + hl) * g.T + t] : INFINITY;
         const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
-        const uint32_t s_col = grp * 64 + sp * KEYS;        // this thread's keys in its group's S buffer
+        const uint32_t s_col = grp * L::colS + sp * KEYS;   // this thread's keys in its group's S buffer
         const uint32_t o_col = L::colO + grp * D + sp * RCOLS;   // O columns it rescales
         const uint32_t l_col = L::colL + grp * 32;
         uint8_t* const prow = base_ptr + L::off_p + grp * L::kP + (r >> 3) * 1024 + (r & 7) * 128;
@@ -286,19 +302,14 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (okw) {
                 tc_fence_after();
                 tmem_ld<KEYS>(lane_addr + s_col, sr);
+                // q . kbar_j = q . kbar_hi + q . kbar_lo: the summary columns of the S buffer
+                const uint32_t qhi = tmem_ld1(lane_addr + grp * L::colS + 64);
+                const uint32_t qlo = tmem_ld1(lane_addr + grp * L::colS + 72);
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(bar(B_S_FREE + grp));
-                // partial row sum (for x_j): packed pairwise adds
-                uint64_t a2[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) a2[i] = f2_pack(sr[2 * i], sr[2 * i + 1]);
-#pragma unroll
-                for (int i = 4; i < KEYS / 2; ++i) a2[i & 3] = f2_add(a2[i & 3], f2_pack(sr[2 * i], sr[2 * i + 1]));
-                float s0, s1, s2, s3;
-                f2_unpack(f2_add(a2[0], a2[1]), s0, s1);
-                f2_unpack(f2_add(a2[2], a2[3]), s2, s3);
-                ps_own = (s0 + s1) + (s2 + s3);
+                // counted once per row when SPLIT threads share it
+                ps_own = sp == 0 ? __uint_as_float(qhi) + __uint_as_float(qlo) : 0.f;
                 // own block: keys after the query position are masked
                 if (diag) {
                     const int key0 = j * kBlock + sp * KEYS;
@@ -331,7 +342,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
             }
             if (!okw) { ok = false; continue; }
-            const float x = rs * cxm;
+            const float x = __fmul_rn(rs, cx);
             const float lp2 = diag ? (tpos >= 0 ? 0.f : -INFINITY)
                                    : (x > tau_r ? e_pow * __log2f(x - tau_r) : -INFINITY);
             const bool active = lp2 > -INFINITY;
@@ -485,14 +496,18 @@ bool fine_tc_supported(const PrefillGeom& g) { return g.P >= 8 && (g.d == 64 || 
 
 cudaError_t launch_fine_tc(const void* q, const void* k, const void* v, void* out, const PrefillGeom& g,
                            char* ws, float alpha, float coarse_scale, cudaStream_t stream) {
-    const float cxm = (alpha - 1.0f) * coarse_scale / sqrtf((float)g.d) / (float)kBlock;
+    const float cx = (alpha - 1.0f) * coarse_scale / sqrtf((float)g.d);
     const float e_pow = 1.0f / (alpha - 1.0f);
     const float sm2 = 1.4426950408889634f / sqrtf((float)g.d);
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, thi, tlo;
     const unsigned long long qrows = (unsigned long long)g.B * g.Hq * g.T;
     const unsigned long long kvrows = (unsigned long long)g.B * g.Hkv * g.T;
+    // block summaries as bf16 hi / lo [B * Hkv * nbs, d] (at least one row: with no complete
+    // block every tile has only its own block and the summary columns are never read)
+    const unsigned long long srows = (unsigned long long)g.B * g.Hkv * (g.nbs > 0 ? g.nbs : 1);
     if (!make_map(&tq, q, qrows, g.d, g.P) || !make_map(&tk, k, kvrows, g.d, kBlock) ||
-        !make_map(&tv, v, kvrows, g.d, kBlock))
+        !make_map(&tv, v, kvrows, g.d, kBlock) || !make_map(&thi, ws + g.off_khi, srows, g.d, 8) ||
+        !make_map(&tlo, ws + g.off_klo, srows, g.d, 8))
         return cudaErrorInvalidValue;
     const float* tau = reinterpret_cast<const float*>(ws + g.off_tau);
     const int* list = reinterpret_cast<const int*>(ws + g.off_list);
@@ -504,12 +519,12 @@ cudaError_t launch_fine_tc(const void* q, const void* k, const void* v, void* ou
         const int sm = (int)TcLayout<128>::bytes;
         cudaError_t e = cudaFuncSetAttribute(fine_tc_kernel<128, kFineSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
         if (e != cudaSuccess) return e;
-        fine_tc_kernel<128, kFineSplit><<<g.ntiles, threads, sm, stream>>>(tq, tk, tv, ob, tau, list, count, hdr, g, cxm, e_pow, sm2);
+        fine_tc_kernel<128, kFineSplit><<<g.ntiles, threads, sm, stream>>>(tq, tk, tv, thi, tlo, ob, tau, list, count, hdr, g, cx, e_pow, sm2);
     } else {
         const int sm = (int)TcLayout<64>::bytes;
         cudaError_t e = cudaFuncSetAttribute(fine_tc_kernel<64, kFineSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
         if (e != cudaSuccess) return e;
-        fine_tc_kernel<64, kFineSplit><<<g.ntiles, threads, sm, stream>>>(tq, tk, tv, ob, tau, list, count, hdr, g, cxm, e_pow, sm2);
+        fine_tc_kernel<64, kFineSplit><<<g.ntiles, threads, sm, stream>>>(tq, tk, tv, thi, tlo, ob, tau, list, count, hdr, g, cx, e_pow, sm2);
     }
     return cudaGetLastError();
 }
