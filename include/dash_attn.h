@@ -80,6 +80,21 @@ DASH_API int dash_version(void);
 DASH_API int dash_block_summary(const void* k, float* ksum, int B, int Hkv, int T, int d, int block,
                        dash_stream_t stream);
 
+/*
+ * Stage 0 with a learned summary head ("DashAttention and the year sparse attention became
+ * a field", section "What alpha-entmax changes": the chunk summary is a small attention
+ * head, initialised at zero so that training starts from mean pooling).  Attention pooling
+ * with one query vector per KV head:
+ *   ksum[b, g, j, :] = sum_i a_i k[b, g, j*block + i, :],  a = softmax_i(w[g] . k_i / sqrt(d))
+ * over the block's keys; w = 0 gives the mean of dash_block_summary (up to rounding).
+ *   k     device bf16 [B, Hkv, T, d]
+ *   w     device fp32 [Hkv, d], 16-byte aligned (must not be NULL)
+ *   ksum  device fp32 [B, Hkv, T / block, d]
+ * Use it to keep the summaries of a decode cache for a model with a learned head.
+ */
+DASH_API int dash_block_summary_w(const void* k, const float* w, float* ksum, int B, int Hkv, int T,
+                                  int d, int block, dash_stream_t stream);
+
 /* Bytes of workspace dash_prefill needs (0 when the shape is unsupported). */
 DASH_API size_t dash_prefill_workspace_size(int B, int Hq, int Hkv, int T, int d, int block);
 
@@ -97,6 +112,17 @@ DASH_API int dash_prefill(const void* q, const void* k, const void* v, void* out
                  int B, int Hq, int Hkv, int T, int d, int block,
                  float alpha, float coarse_scale,
                  void* workspace, size_t ws_bytes, dash_stream_t stream);
+
+/*
+ * dash_prefill with the learned summary head of dash_block_summary_w for Stage 0.
+ *   w_summary  device fp32 [Hkv, d], 16-byte aligned; NULL is dash_prefill (mean pooling).
+ * Returns DASH_ERR_UNSUPPORTED for a non-NULL head when a tile holds fewer than 8
+ * positions (more than 16 query heads per KV head): that path's fine kernel recovers
+ * q . kbar from the mean of the block's scores, which only the mean summary satisfies.
+ */
+DASH_API int dash_prefill_w(const void* q, const void* k, const void* v, const float* w_summary, void* out,
+                            int B, int Hq, int Hkv, int T, int d, int block, float alpha,
+                            float coarse_scale, void* workspace, size_t ws_bytes, dash_stream_t stream);
 
 /*
  * dash_prefill with HOST inputs and output: copies q, k, v from host memory into the

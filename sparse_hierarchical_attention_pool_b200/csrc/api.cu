@@ -64,6 +64,15 @@ int dash_block_summary(const void* k, float* ksum, int B, int Hkv, int T, int d,
     return launch_block_summary(k, ksum, B, Hkv, T, d, S(stream)) == cudaSuccess ? DASH_OK : DASH_ERR_CUDA;
 }
 
+int dash_block_summary_w(const void* k, const float* w, float* ksum, int B, int Hkv, int T, int d,
+                         int block, dash_stream_t stream) {
+    if (!k || !w || !ksum || !al16(k) || !al16(w) || !al16(ksum)) return DASH_ERR_ARG;
+    if (block != kBlock || (d != 64 && d != 128) || B < 1 || Hkv < 1 || T < 1 || T > kMaxT)
+        return DASH_ERR_SHAPE;
+    return launch_block_summary(k, ksum, B, Hkv, T, d, S(stream), nullptr, nullptr, w) == cudaSuccess
+               ? DASH_OK : DASH_ERR_CUDA;
+}
+
 size_t dash_prefill_workspace_size(int B, int Hq, int Hkv, int T, int d, int block) {
     PrefillGeom g;
     if (block != kBlock || !make_prefill_geom(B, Hq, Hkv, T, d, &g)) return 0;
@@ -72,11 +81,16 @@ size_t dash_prefill_workspace_size(int B, int Hq, int Hkv, int T, int d, int blo
 
 static int prefill_impl(const void* q, const void* k, const void* v, void* out, int B, int Hq,
                         int Hkv, int T, int d, int block, float alpha, float coarse_scale,
-                        void* workspace, size_t ws_bytes, dash_stream_t stream, void* const* events) {
+                        void* workspace, size_t ws_bytes, dash_stream_t stream, void* const* events,
+                        const float* wsum = nullptr) {
     if (!q || !k || !v || !out || !al16(q) || !al16(k) || !al16(v) || !al16(out)) return DASH_ERR_ARG;
+    if (wsum && !al16(wsum)) return DASH_ERR_ARG;
     if (!good_params(alpha, coarse_scale)) return DASH_ERR_ARG;
     PrefillGeom g;
     if (block != kBlock || !make_prefill_geom(B, Hq, Hkv, T, d, &g)) return DASH_ERR_SHAPE;
+    // the CUDA-core fine kernel recovers q . kbar from the mean of the block's scores, which
+    // only a mean summary satisfies
+    if (wsum && !fine_tc_supported(g)) return DASH_ERR_UNSUPPORTED;
     if (!workspace || !al256(workspace) || ws_bytes < g.total) return DASH_ERR_WORKSPACE;
     char* ws = static_cast<char*>(workspace);
     cudaStream_t s = S(stream);
@@ -86,7 +100,7 @@ static int prefill_impl(const void* q, const void* k, const void* v, void* out, 
     if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), s) != cudaSuccess) return DASH_ERR_CUDA;
     if (!mark(0)) return DASH_ERR_CUDA;
     if (g.nbs > 0 && launch_block_summary(k, reinterpret_cast<float*>(ws + g.off_ksum), B, Hkv, T, d, s,
-                                          ws + g.off_khi, ws + g.off_klo) != cudaSuccess)
+                                          ws + g.off_khi, ws + g.off_klo, wsum) != cudaSuccess)
         return DASH_ERR_CUDA;
     if (!mark(1)) return DASH_ERR_CUDA;
     const cudaError_t ce = g.tc ? (coarse_tc_supported(g) ? launch_coarse_tc(q, g, ws, alpha, coarse_scale, s)
@@ -104,6 +118,13 @@ int dash_prefill(const void* q, const void* k, const void* v, void* out, int B, 
                  size_t ws_bytes, dash_stream_t stream) {
     return prefill_impl(q, k, v, out, B, Hq, Hkv, T, d, block, alpha, coarse_scale, workspace,
                         ws_bytes, stream, nullptr);
+}
+
+int dash_prefill_w(const void* q, const void* k, const void* v, const float* w_summary, void* out, int B,
+                   int Hq, int Hkv, int T, int d, int block, float alpha, float coarse_scale, void* workspace,
+                   size_t ws_bytes, dash_stream_t stream) {
+    return prefill_impl(q, k, v, out, B, Hq, Hkv, T, d, block, alpha, coarse_scale, workspace,
+                        ws_bytes, stream, nullptr, w_summary);
 }
 
 int dash_prefill_profiled(const void* q, const void* k, const void* v, void* out, int B, int Hq,

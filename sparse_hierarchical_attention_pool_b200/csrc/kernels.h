@@ -7,9 +7,11 @@
 
 namespace dash {
 
-// kbar in fp32, and optionally split into bf16 hi + lo parts for the tensor-core scores
+// kbar in fp32, and optionally split into bf16 hi + lo parts for the tensor-core scores;
+// w (fp32 [Hkv, d], device) selects the learned attention-pooling head, nullptr the mean
 cudaError_t launch_block_summary(const void* k, float* ksum, int B, int Hkv, int T, int d,
-                                 cudaStream_t stream, void* khi = nullptr, void* klo = nullptr);
+                                 cudaStream_t stream, void* khi = nullptr, void* klo = nullptr,
+                                 const float* w = nullptr);
 
 // Stage 1 for prefill: scores of every work tile against the block summaries, per-row
 // thresholds and the per-tile union of selected blocks.

@@ -27,7 +27,7 @@ EXPORTS = ("dash_status_string", "dash_version", "dash_block_summary", "dash_pre
            "dash_prefill", "dash_prefill_host", "dash_prefill_stats", "dash_decode_stats",
            "dash_prefill_tau", "dash_select_dump", "dash_decode_workspace_size", "dash_decode",
            "dash_get_device_status", "dash_prefill_profiled", "dash_decode_profiled",
-           "dash_decode_noalloc")
+           "dash_decode_noalloc", "dash_block_summary_w", "dash_prefill_w")
 
 
 class DashError(RuntimeError):
@@ -62,6 +62,8 @@ def lib():
     L.dash_status_string.argtypes = [_i]
     L.dash_version.restype = _i
     L.dash_block_summary.argtypes = [_p, _p, _i, _i, _i, _i, _i, _p]
+    L.dash_block_summary_w.argtypes = [_p, _p, _p, _i, _i, _i, _i, _i, _p]
+    L.dash_prefill_w.argtypes = [_p] * 5 + [_i] * 6 + [_f, _f, _p, _sz, _p]
     L.dash_prefill_workspace_size.argtypes = [_i] * 6
     L.dash_prefill_workspace_size.restype = _sz
     L.dash_prefill.argtypes = [_p] * 4 + [_i] * 6 + [_f, _f, _p, _sz, _p]
@@ -118,6 +120,19 @@ def dash_block_summary(k, ksum=None, block=64, stream=None):
     return ksum
 
 
+def dash_block_summary_w(k, w, ksum=None, block=64, stream=None):
+    """Learned-head summaries: k [B, Hkv, T, d], w fp32 [Hkv, d] -> ksum fp32 [B, Hkv, T // 64, d]."""
+    B, Hkv, T, d = k.shape
+    if tuple(w.shape) != (Hkv, d):
+        raise ValueError("w must be [Hkv, d]")
+    if ksum is None:
+        ksum = torch.empty(B, Hkv, max(T // block, 1), d, device=k.device, dtype=torch.float32)
+    _check("dash_block_summary_w", lib().dash_block_summary_w(
+        _dev(k, torch.bfloat16, "k"), _dev(w, torch.float32, "w"), _dev(ksum, torch.float32, "ksum"),
+        B, Hkv, T, d, block, _stream(stream)))
+    return ksum
+
+
 def prefill_workspace_size(B, Hq, Hkv, T, d, block=64) -> int:
     n = lib().dash_prefill_workspace_size(B, Hq, Hkv, T, d, block)
     if n == 0:
@@ -155,6 +170,29 @@ def dash_prefill(q, k, v, out=None, alpha=1.5, coarse_scale=1.0, workspace=None,
                             B, Hq, Hkv, T, d, block, float(alpha), float(coarse_scale),
                             ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream))
     _check("dash_prefill", rc)
+    return out, workspace
+
+
+def dash_prefill_w(q, k, v, w_summary, out=None, alpha=1.5, coarse_scale=1.0, workspace=None, block=64,
+                   stream=None):
+    """dash_prefill with a learned summary head w_summary fp32 [Hkv, d] (None: mean pooling)."""
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, T, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Hkv, T, d] matching q")
+    if w_summary is not None and tuple(w_summary.shape) != (Hkv, d):
+        raise ValueError("w_summary must be [Hkv, d]")
+    if out is None:
+        out = torch.empty_like(q)
+    need = prefill_workspace_size(B, Hq, Hkv, T, d, block)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    wp = None if w_summary is None else _dev(w_summary, torch.float32, "w_summary")
+    rc = lib().dash_prefill_w(_dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"),
+                              _dev(v, torch.bfloat16, "v"), wp, _dev(out, torch.bfloat16, "out"),
+                              B, Hq, Hkv, T, d, block, float(alpha), float(coarse_scale),
+                              ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream))
+    _check("dash_prefill_w", rc)
     return out, workspace
 
 
