@@ -342,6 +342,17 @@ def bench_decode(args, ws, rank, local):
     torch.cuda.synchronize()
     st_ms = [mean([e[i].elapsed_time(e[i + 1]) for e in evs]) for i in range(3)]
     eager = mean([e[0].elapsed_time(e[3]) for e in evs])
+    # the threshold solve started at the histogram edge instead of u = -1, for comparison
+    os.environ["DASH_ENTMAX_INIT"] = "histogram"
+    evn = []
+    for _ in range(steps):
+        flush()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        da.dash_decode_profiled(qd, kcd, vcd, ksum, lens, out, wl.alpha, cs, wsb, e)
+        evn.append(e)
+    torch.cuda.synchronize()
+    del os.environ["DASH_ENTMAX_INIT"]
+    coarse_hist_ms = mean([e[0].elapsed_time(e[1]) for e in evn])
     # the step as a serving loop runs it: one CUDA graph replay (header reset + 2 kernels)
     graph = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream()
@@ -399,6 +410,8 @@ def bench_decode(args, ws, rank, local):
         "timing": "CUDA graph replay of the step; stage_ms from an eager profiled run",
         "eager_ms_per_step": eager,
         "stage_ms": dict(zip(["coarse_select", "attention", "merge"], st_ms)),
+        "tau_start": {"newton_from_minus_one_coarse_select_ms": st_ms[0],
+                      "histogram_edge_coarse_select_ms": coarse_hist_ms},
         "sparsity": 1.0 - st["selected_pairs"] / max(1, st["scored_pairs"]),
         "union_blocks_per_group": st["union_blocks"] / (B * Hkv),
         "roofline": {"bound": "hbm", "kernel": "decode_attn_tc_kernel", "achieved": round(attn_gbs, 1),

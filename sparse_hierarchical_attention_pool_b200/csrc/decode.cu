@@ -19,6 +19,9 @@
 //   4. decode_combine: merging those partials of each (b, h) into bf16.
 // The HBM traffic that matters is step 3: (union blocks + 1) * 64 * d * 2 bytes * 2 per
 // (b, kv head).
+#include <cstdlib>
+#include <cstring>
+
 #include "common.cuh"
 #include "entmax.cuh"
 #include "kernels.h"
@@ -251,11 +254,77 @@ struct WarpRow {
     }
 };
 
-// Threshold of one row held by a warp (every lane returns it); MODE as in EntmaxPass::add_t.
+constexpr int kHistBins = 64;       // bins of the histogram start over y = x - m in [-1, 0)
+
+// Histogram start of the threshold solve (the idea of AdaSplash-2, "a coarse histogram of
+// the scores in on-chip memory gives a close initial threshold", as summarised in "DashAttention
+// and the year sparse attention became a field"; the construction here is this library's):
+// the values y = x - m in [-1, 0) go to bin k = floor((y + 1) * 64) with their count, sum and
+// sum of squares, accumulated as integers (y and y^2 in 2^-24 fixed point), so the sums and
+// the start do not depend on the order of the shared-memory atomics.  At a bin's lower edge
+// e every value of the bins above lies above e, so f(e) = sum_{y > e} (y - e)^(1/(alpha-1))
+// is exact there for alpha = 1.5 (S2 - 2 e S1 + e^2 S0) and alpha = 2 (S1 - e S0).  f is
+// decreasing, so the highest edge with f >= 1 lies just below the root: Newton starts there
+// instead of at -1.
+// bins: this warp's shared area (kHistBins counts, then kHistBins sums, kHistBins sums of
+// squares).  Every lane returns the start.
+struct HistBins {
+    unsigned int c[kHistBins];
+    unsigned long long s1[kHistBins], s2[kHistBins];
+};
+
 template <int MODE>
-__device__ __forceinline__ float warp_row_tau(const WarpRow& xr, float m, float alpha, int* no_conv) {
+__device__ __forceinline__ float hist_start(const WarpRow& xr, float m, HistBins* hb) {
+    const int lane = threadIdx.x & 31;
+    constexpr float kFix = 16777216.0f;                 // 2^24
+    for (int i = lane; i < kHistBins; i += 32) { hb->c[i] = 0u; hb->s1[i] = 0ull; hb->s2[i] = 0ull; }
+    __syncwarp();
+    xr.each([&](int, float v) {
+        const float y = v - m;
+        if (y > -1.0f) {
+            const int k = min(kHistBins - 1, (int)((y + 1.0f) * (float)kHistBins));
+            atomicAdd(&hb->c[k], 1u);
+            atomicAdd(&hb->s1[k], (unsigned long long)__float2ll_rn(y * kFix));
+            atomicAdd(&hb->s2[k], (unsigned long long)__float2ll_rn(y * y * kFix));
+        }
+    });
+    __syncwarp();
+    // lane l holds bins 2l, 2l + 1; exact suffix sums over the bins at and above each edge
+    long long c0 = hb->c[2 * lane], c1 = hb->c[2 * lane + 1];
+    long long p0 = (long long)hb->s1[2 * lane], p1 = (long long)hb->s1[2 * lane + 1];
+    long long q0 = (long long)hb->s2[2 * lane], q1 = (long long)hb->s2[2 * lane + 1];
+    long long ac = c0 + c1, a1 = p0 + p1, a2 = q0 + q1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long nc = __shfl_down_sync(0xffffffffu, ac, o);
+        const long long n1 = __shfl_down_sync(0xffffffffu, a1, o);
+        const long long n2 = __shfl_down_sync(0xffffffffu, a2, o);
+        if (lane + o < 32) { ac += nc; a1 += n1; a2 += n2; }
+    }
+    auto f_at = [&](int k, long long S0, long long S1q, long long S2q) {
+        const double e = -1.0 + (double)k / kHistBins;
+        const double S1 = (double)S1q / kFix, S2 = (double)S2q / kFix;
+        return MODE == 1 ? S2 - 2.0 * e * S1 + e * e * (double)S0 : S1 - e * (double)S0;
+    };
+    const unsigned ok_odd = __ballot_sync(0xffffffffu, f_at(2 * lane + 1, ac - c0, a1 - p0, a2 - q0) >= 1.0);
+    const unsigned ok_even = __ballot_sync(0xffffffffu, f_at(2 * lane, ac, a1, a2) >= 1.0);
+    const int k_odd = ok_odd ? 2 * (31 - __clz((int)ok_odd)) + 1 : -1;
+    const int k_even = ok_even ? 2 * (31 - __clz((int)ok_even)) : 0;
+    __syncwarp();
+    return -1.0f + (float)max(k_odd, k_even) / (float)kHistBins;
+}
+
+// Threshold of one row held by a warp (every lane returns it); MODE as in EntmaxPass::add_t.
+// bins != nullptr: start from the histogram edge (alpha = 1.5 and 2), else from u = -1.
+template <int MODE>
+__device__ __forceinline__ float warp_row_tau(const WarpRow& xr, float m, float alpha, int* no_conv,
+                                              HistBins* bins) {
+    float u0 = -1.0f;
+    if constexpr (MODE != 0) {
+        if (bins) u0 = hist_start<MODE>(xr, m, bins);
+    }
     EntmaxSolver sv;
-    sv.init(m, alpha);
+    sv.init(m, alpha, u0);
     float t = m;
     while (true) {
         EntmaxPass ps;
@@ -333,8 +402,9 @@ decode_select_kernel(const int* __restrict__ kv_len, const float* __restrict__ x
                      float* __restrict__ tau, int* __restrict__ list, int* __restrict__ count,
                      int* __restrict__ done, int* __restrict__ offs, int* __restrict__ plan,
                      __nv_bfloat16* __restrict__ out, WsHeader* __restrict__ hdr, DecodeGeom g,
-                     float alpha, int nctas) {
+                     float alpha, int nctas, int hist_init) {
     constexpr int kWords = kMaxT / kBlock / 32;
+    __shared__ HistBins hist[kSelThreads / 32];
     constexpr int kWpt = kWords / kSelThreads;        // bitmap words per thread
     __shared__ unsigned bitmap[kWords];
     __shared__ int wtot[kSelThreads / 32];
@@ -365,9 +435,10 @@ decode_select_kernel(const int* __restrict__ kv_len, const float* __restrict__ x
             float m = -INFINITY;
             xr.each([&](int, float v) { m = fmaxf(m, v); });
             m = warp_max(m);
-            t = alpha == 1.5f ? warp_row_tau<1>(xr, m, alpha, &no_conv)
-              : alpha == 2.0f ? warp_row_tau<2>(xr, m, alpha, &no_conv)
-                              : warp_row_tau<0>(xr, m, alpha, &no_conv);
+            HistBins* bins = hist_init ? &hist[warp] : nullptr;
+            t = alpha == 1.5f ? warp_row_tau<1>(xr, m, alpha, &no_conv, bins)
+              : alpha == 2.0f ? warp_row_tau<2>(xr, m, alpha, &no_conv, bins)
+                              : warp_row_tau<0>(xr, m, alpha, &no_conv, bins);
         }
         if (lane == 0) tau[row] = t;
         float nsel = 0.f;
@@ -624,8 +695,13 @@ cudaError_t launch_decode(const void* q, const void* kc, const void* vc, const f
     if (!mark(0)) return cudaErrorUnknown;
     if (g.d == 128) launch_scores<128>(qb, ksum, kv_len, xs, g, cx, stream);
     else launch_scores<64>(qb, ksum, kv_len, xs, g, cx, stream);
+    // DASH_ENTMAX_INIT=histogram starts each threshold solve at the histogram edge; the
+    // default, Newton from u = -1, is faster on the rows measured here (the binning pass
+    // costs more than the passes it saves)
+    const char* init = getenv("DASH_ENTMAX_INIT");
+    const int hist_init = (init && strcmp(init, "histogram") == 0) ? 1 : 0;
     decode_select_kernel<<<BH, kSelThreads, 0, stream>>>(kv_len, xs, tau, list, count, done, offs, plan, ob, hdr, g,
-                                                         alpha, nctas);
+                                                         alpha, nctas, hist_init);
     if (!mark(1)) return cudaErrorUnknown;
     if (fused) {
         e = launch_decode_attn_tc(q, kc, vc, kv_len, out, g, ws, e_pow, sm2, nctas, stream);

@@ -17,6 +17,9 @@
 // support and u* is exact; otherwise a Newton step is taken.  Other alpha: safeguarded
 // Newton (bisection when a step leaves the bracket) until the step is below 2.5e-7.
 //
+// Any start u0 in [-1, 0) works: from below (f(u0) >= 1) Newton climbs monotonically; from
+// above, the first step of a convex decreasing f lands at or below the root.
+//
 // The iteration is written as a per-pass accumulator (EntmaxPass) and an update
 // (EntmaxSolver::update) so that callers can stream a row's values through any memory:
 // the single-thread and warp solves below, and the tensor-memory coarse kernel.
@@ -80,9 +83,9 @@ struct EntmaxPass {
 struct EntmaxSolver {
     float m, u, lo, hi, e;
     int mode, it;
-    __device__ __forceinline__ void init(float row_max, float alpha) {
+    __device__ __forceinline__ void init(float row_max, float alpha, float u0 = -1.0f) {
         m = row_max;
-        u = -1.0f; lo = -1.0f; hi = 0.0f;
+        u = u0; lo = -1.0f; hi = 0.0f;
         e = 1.0f / (alpha - 1.0f);
         mode = alpha == 2.0f ? 2 : (alpha == 1.5f ? 1 : 0);
         it = 0;

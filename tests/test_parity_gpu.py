@@ -219,3 +219,27 @@ def test_decode_96k_workload_all_rows():
     (mx, mean), _, ws = check_decode(q, kc, vc, kv_len.tolist(), wl.alpha, calibrated_scale("decode96k"), "decode96k")
     st = da.dash_decode_stats(ws)
     print("decode96k", mx, mean, st, "sparsity", 1 - st["selected_pairs"] / st["scored_pairs"])
+
+
+def test_decode_threshold_start_does_not_change_the_result():
+    """The histogram start and the start at u = -1 reach the same thresholds and lists."""
+    import os
+    wl, (q, kc, vc, kv_len) = inputs.make("decode96k", B=2)
+    cs = calibrated_scale("decode96k")
+    qd, kcd, vcd, lens = q.cuda(), kc.cuda(), vc.cuda(), kv_len.cuda()
+    ksum = da.dash_block_summary(kcd)
+    outs, stats = [], []
+    for mode in ("newton", "histogram"):
+        if mode == "histogram":
+            os.environ["DASH_ENTMAX_INIT"] = "histogram"
+        try:
+            out, ws = da.dash_decode(qd, kcd, vcd, ksum, lens, alpha=wl.alpha, coarse_scale=cs)
+            torch.cuda.synchronize()
+            assert da.dash_get_device_status(ws) == 0
+            outs.append(out.float().cpu())
+            stats.append(da.dash_decode_stats(ws))
+        finally:
+            os.environ.pop("DASH_ENTMAX_INIT", None)
+    assert stats[0]["selected_pairs"] == stats[1]["selected_pairs"]
+    assert stats[0]["union_blocks"] == stats[1]["union_blocks"]
+    assert (outs[0] - outs[1]).abs().max().item() <= 2e-3
