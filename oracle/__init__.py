@@ -67,7 +67,11 @@ def lib():
                                                + [_i64] * 6 + [_ptr, _i64, _ptr, _ptr, _ptr, ctypes.c_int])
         L.oracle_dense_causal_rows.argtypes = ([_ptr, ctypes.c_int, _ptr, ctypes.c_int, _ptr, ctypes.c_int]
                                                + [_i64] * 5 + [_ptr, _i64, _ptr, ctypes.c_int])
-        for f in (L.oracle_block_summary_w, L.oracle_select_rows_w, L.oracle_forward_rows_w):
+        L.oracle_forward_rows_agg.argtypes = ([_ptr, ctypes.c_int, _ptr, ctypes.c_int, _ptr, ctypes.c_int, _ptr]
+                                              + [_i64] * 6 + [_dbl, _dbl, _ptr, _i64]
+                                              + [_ptr] * 2 + [ctypes.c_int])
+        for f in (L.oracle_block_summary_w, L.oracle_select_rows_w, L.oracle_forward_rows_w,
+                  L.oracle_forward_rows_agg):
             f.restype = ctypes.c_int
         for f in (L.oracle_entmax_tau, L.oracle_entmax, L.oracle_block_summary, L.oracle_select_rows,
                   L.oracle_forward_rows, L.oracle_fine_rows_given_p, L.oracle_dense_causal_rows):
@@ -191,6 +195,33 @@ def forward_rows(q_rows, k, v, rows, Hq, blk, alpha, coarse_scale, nthreads=0, w
                                        _p(out), _p(tau), _p(ns), int(nthreads)),
            "forward_rows")
     return out, tau, ns
+
+
+def forward_rows_agg(q, k, v, rows, blk, alpha, coarse_scale, nthreads=0, w_summary=None):
+    """Head-aggregated forward ("DashAttention and the year sparse attention became a field",
+    section "Non-dispersive attention at long context": entmax head aggregation) for rows
+    (b, h, t): the KV group's heads average their block distributions and share that prior.
+    q is the full [B, Hq, T, d] query tensor (every head of a row's group is needed).
+    Returns (out [n, d] fp64, nsel [n] = size of the shared support)."""
+    import torch
+    B, Hq, T, d = q.shape
+    ka, kdt = _arr(k)
+    va, vdt = _arr(v)
+    Hkv, Tk = ka.shape[1], ka.shape[2]
+    G = Hq // Hkv
+    r, n = _rows(rows)
+    rt = torch.as_tensor(r)
+    heads = (rt[:, 1] // G * G).unsqueeze(1) + torch.arange(G).unsqueeze(0)          # [n, G]
+    qg = q[rt[:, 0].unsqueeze(1), heads, rt[:, 2].unsqueeze(1)]                      # [n, G, d]
+    qa, qdt = _arr(qg.contiguous())
+    out = np.zeros((n, d))
+    ns = np.zeros(n, dtype=np.int64)
+    wa = None if w_summary is None else _wsum(w_summary, Hkv, d)
+    _check(lib().oracle_forward_rows_agg(_p(qa), qdt, _p(ka), kdt, _p(va), vdt, None if wa is None else _p(wa),
+                                         B, Hq, Hkv, Tk, d, blk, float(alpha), float(coarse_scale),
+                                         _p(r), n, _p(out), _p(ns), int(nthreads)),
+           "forward_rows_agg")
+    return out, ns
 
 
 def fine_rows_given_p(q_rows, k, v, rows, Hq, blk, w_rows, w_diag, nthreads=0):

@@ -30,7 +30,9 @@
  *   - coarse score s_j = coarse_scale * (q . kbar_j) / sqrt(d); fine logits use 1/sqrt(d);
  *   - the query's own block is always attended causally with prior weight 1 (log 0 prior);
  *   - query head h reads KV head floor(h / (Hq/Hkv));
- *   - a block whose x_j equals tau exactly gets weight 0 (strict ">").
+ *   - a block whose x_j equals tau exactly gets weight 0 (strict ">");
+ *   - head aggregation (the optional variant): the heads of a KV group average their block
+ *     distributions and share the result as their prior (oracle_forward_rows_agg).
  *
  * Parity pins (tests/test_oracle_pins.py): exact tau is checked against 200-step
  * bisection, brute force over supports and scipy's constrained optimiser on the
@@ -478,6 +480,65 @@ int oracle_forward_rows_w(const void* q_rows, int qdt, const void* k, int kdt, c
             if (nsel_out) nsel_out[r] = ns;
         }
         free(x); free(p); free(lp); free(lbuf);
+    }
+    free(kb);
+    return fail ? ORC_ERR_NOMEM : ORC_OK;
+}
+
+/*
+ * Head-aggregated selection ("DashAttention and the year sparse attention became a field",
+ * section "Non-dispersive attention at long context": entmax head aggregation).  Reading:
+ * the G query heads of a KV group share one block distribution at each position,
+ *   pbar_j = (1/G) sum_{h in group} p_{h,j}
+ * (support: the union of the heads' supports), and every head of the group uses log pbar_j
+ * as its prior in the fine stage; the own block keeps prior 1.
+ * q_group [nrows, G, d]: the query vectors of all G heads of row r's KV group at the row's
+ * position, in head order; row (b, h, t) uses its own head h % G for the fine logits.
+ * nsel_out[r] = #{j : pbar_j > 0}.
+ */
+int oracle_forward_rows_agg(const void* q_group, int qdt, const void* k, int kdt, const void* v, int vdt,
+                            const double* w_summary, long long B, long long Hq, long long Hkv, long long Tk,
+                            long long d, long long blk, double alpha, double coarse_scale,
+                            const long long* rows, long long nrows,
+                            double* out, long long* nsel_out, int nthreads) {
+    orc_problem P = {q_group, qdt, k, kdt, v, vdt, B, Hq, Hkv, Tk, d, blk, alpha, coarse_scale, w_summary};
+    int rc = check_problem(&P, rows, nrows);
+    if (rc || !v || !out) return rc ? rc : ORC_ERR_ARG;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+    double* kb = all_kbar(&P);
+    if (!kb) return ORC_ERR_NOMEM;
+    long long nbs = Tk / blk, G = Hq / Hkv;
+    int fail = 0;
+    #pragma omp parallel
+    {
+        double* x = (double*)malloc((size_t)(nbs + 1) * sizeof(double));
+        double* p = (double*)malloc((size_t)(nbs + 1) * sizeof(double));
+        double* pbar = (double*)malloc((size_t)(nbs + 1) * sizeof(double));
+        double* lbuf = (double*)malloc((size_t)Tk * sizeof(double));
+        if (!x || !p || !pbar || !lbuf) {
+            #pragma omp atomic write
+            fail = 1;
+        }
+        #pragma omp for schedule(dynamic, 1)
+        for (long long r = 0; r < nrows; ++r) {
+            if (!x || !p || !pbar || !lbuf) continue;
+            long long b = rows[3 * r], h = rows[3 * r + 1], t = rows[3 * r + 2];
+            long long g = h / G, bt = t / blk;
+            for (long long j = 0; j < bt; ++j) pbar[j] = 0.0;
+            for (long long hh = 0; hh < G; ++hh) {
+                double tau;
+                /* row index r * G + hh addresses query vector hh of row r's group */
+                row_select(&P, r * G + hh, t, kb + (b * Hkv + g) * nbs * d, x, p, &tau);
+                for (long long j = 0; j < bt; ++j) pbar[j] += p[j] / (double)G;
+            }
+            long long ns = 0;
+            for (long long j = 0; j < bt; ++j) ns += pbar[j] > 0.0;
+            row_fine(&P, r * G + h % G, b, g, t, pbar, NULL, 1.0, lbuf, out + r * d);
+            if (nsel_out) nsel_out[r] = ns;
+        }
+        free(x); free(p); free(pbar); free(lbuf);
     }
     free(kb);
     return fail ? ORC_ERR_NOMEM : ORC_OK;

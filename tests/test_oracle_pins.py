@@ -404,3 +404,81 @@ def test_forward_with_zero_head_equals_mean_forward(orc):
     w = np.random.default_rng(6).standard_normal((Hkv, d)) * 3.0
     o2, t2, _ = orc.forward_rows(qr, k, v, rows, Hq, 64, 1.5, 2.0, w_summary=w)
     assert np.abs(t2 - t0).max() > 1e-6
+
+
+# ------------------------------------------------------------------ head aggregation
+# "DashAttention and the year sparse attention became a field", section "Non-dispersive
+# attention at long context" (entmax head aggregation): the heads of a KV group average their
+# block distributions and share that prior.
+
+def _agg_inputs(Hq, Hkv, T, d, seed, same_heads=False):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(1, Hq, T, d, generator=g) * 1.5
+    if same_heads:
+        G = Hq // Hkv
+        q = q[:, ::G].repeat_interleave(G, dim=1)
+    k = torch.randn(1, Hkv, T, d, generator=g)
+    v = torch.randn(1, Hkv, T, d, generator=g)
+    return q.bfloat16(), k.bfloat16(), v.bfloat16()
+
+
+def _agg_rows(Hq, T):
+    return [(0, h, t) for h in range(Hq) for t in (0, 63, 64, 200, 450, T - 1)]
+
+
+def test_aggregation_of_one_head_is_the_per_head_forward(orc):
+    q, k, v = _agg_inputs(3, 3, 512, 16, 1)
+    rows = _agg_rows(3, 512)
+    a, ns_a = orc.forward_rows_agg(q, k, v, rows, 64, 1.5, 3.0)
+    b, _, ns_b = orc.forward_rows(orc.gather_q_rows(q, rows), k, v, rows, 3, 64, 1.5, 3.0)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+    assert np.array_equal(ns_a, ns_b)
+
+
+def test_aggregation_of_identical_heads_is_the_per_head_forward(orc):
+    q, k, v = _agg_inputs(8, 2, 512, 16, 2, same_heads=True)
+    rows = _agg_rows(8, 512)
+    a, _ = orc.forward_rows_agg(q, k, v, rows, 64, 1.5, 3.0)
+    b, _, _ = orc.forward_rows(orc.gather_q_rows(q, rows), k, v, rows, 8, 64, 1.5, 3.0)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+def test_aggregated_prior_is_the_mean_distribution_and_its_support_the_union(orc):
+    Hq, Hkv, T, d, G = 8, 2, 512, 16, 4
+    q, k, v = _agg_inputs(Hq, Hkv, T, d, 3)
+    rows = [(0, h, t) for h in range(Hq) for t in (130, 300, 511)]
+    out, ns = orc.forward_rows_agg(q, k, v, rows, 64, 1.5, 3.0)
+    # the same rows through two other routes: every head's selection, then the fine stage
+    # with the averaged weights injected
+    wts, unions = [], []
+    for (b, h, t) in rows:
+        grp = [(b, (h // G) * G + i, t) for i in range(G)]
+        sel = orc.select_rows(orc.gather_q_rows(q, grp), k, grp, Hq, 64, 1.5, 3.0)
+        wts.append(sel["p"].mean(0))
+        unions.append(int((sel["p"] > 0).any(0).sum()))
+    wts = np.array(wts)
+    assert np.allclose(wts.sum(1), 1.0, atol=1e-12)
+    assert np.array_equal(ns, np.array(unions))
+    ref = orc.fine_rows_given_p(orc.gather_q_rows(q, rows), k, v, rows, Hq, 64, wts, np.ones(len(rows)))
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+
+
+def test_aggregated_attention_ignores_blocks_outside_the_shared_support(orc):
+    # the values of a past block that no head of the group selects never reach the output
+    Hq, Hkv, T, d, G = 4, 1, 640, 16, 4
+    q, k, v = _agg_inputs(Hq, Hkv, T, d, 4)
+    t = 639
+    grp = [(0, h, t) for h in range(G)]
+    p = orc.select_rows(orc.gather_q_rows(q, grp), k, grp, Hq, 64, 2.0, 6.0)["p"]
+    bt = t // 64                           # the own block is always attended
+    unused = np.where(~(p[:, :bt] > 0).any(0))[0]
+    used = np.where((p[:, :bt] > 0).any(0))[0]
+    assert len(unused) > 0 and len(used) > 0
+    base, _ = orc.forward_rows_agg(q, k, v, grp, 64, 2.0, 6.0)
+    v2 = v.clone()
+    for j in unused:
+        v2[0, 0, 64 * j:64 * (j + 1)] = (torch.randn(64, d) * 100).bfloat16()
+    np.testing.assert_allclose(orc.forward_rows_agg(q, k, v2, grp, 64, 2.0, 6.0)[0], base, rtol=0, atol=1e-12)
+    v3 = v.clone()
+    v3[0, 0, 64 * used[0]:64 * (used[0] + 1)] += 1.0
+    assert np.abs(orc.forward_rows_agg(q, k, v3, grp, 64, 2.0, 6.0)[0] - base).max() > 1e-6
