@@ -124,6 +124,27 @@ DASH_API int dash_prefill_w(const void* q, const void* k, const void* v, const f
                             int B, int Hq, int Hkv, int T, int d, int block, float alpha,
                             float coarse_scale, void* workspace, size_t ws_bytes, dash_stream_t stream);
 
+/* Flags of dash_prefill_ex / dash_decode_ex. */
+#define DASH_HEAD_AGGREGATION 1u
+
+/*
+ * dash_prefill with options.
+ *   w_summary  learned summary head as in dash_prefill_w (NULL: mean pooling).
+ *   flags      0 or DASH_HEAD_AGGREGATION: entmax head aggregation ("DashAttention and the
+ *              year sparse attention became a field", section "Non-dispersive attention at
+ *              long context").  The G heads of a KV group average their alpha-entmax block
+ *              weights at each position, pbar_j = (1/G) sum_h p_hj, and every head of the
+ *              group takes log pbar_j as its fine-stage prior (the own block keeps prior 1);
+ *              the thresholds and block lists stay per head.
+ * Unknown flag bits return DASH_ERR_ARG.  A learned head or head aggregation returns
+ * DASH_ERR_UNSUPPORTED when a tile holds fewer than 8 positions (more than 16 query heads
+ * per KV head).
+ */
+DASH_API int dash_prefill_ex(const void* q, const void* k, const void* v, const float* w_summary, void* out,
+                             int B, int Hq, int Hkv, int T, int d, int block, float alpha,
+                             float coarse_scale, unsigned flags, void* workspace, size_t ws_bytes,
+                             dash_stream_t stream);
+
 /*
  * dash_prefill with HOST inputs and output: copies q, k, v from host memory into the
  * caller's device buffers, runs dash_prefill, copies out back to host memory, all
@@ -205,6 +226,15 @@ DASH_API int dash_decode(const void* q, const void* k_cache, const void* v_cache
                 const int* kv_len, void* out, int B, int Hq, int Hkv, int Tmax, int d, int block,
                 float alpha, float coarse_scale, void* workspace, size_t ws_bytes,
                 dash_stream_t stream);
+
+/*
+ * dash_decode with options: flags 0 or DASH_HEAD_AGGREGATION (as in dash_prefill_ex).  Head
+ * aggregation returns DASH_ERR_UNSUPPORTED for more than 8 query heads per KV head.
+ */
+DASH_API int dash_decode_ex(const void* q, const void* k_cache, const void* v_cache, const float* ksum,
+                            const int* kv_len, void* out, int B, int Hq, int Hkv, int Tmax, int d, int block,
+                            float alpha, float coarse_scale, unsigned flags, void* workspace,
+                            size_t ws_bytes, dash_stream_t stream);
 
 /*
  * dash_decode that also records four caller-created CUDA events on `stream`: events[0]

@@ -82,15 +82,18 @@ size_t dash_prefill_workspace_size(int B, int Hq, int Hkv, int T, int d, int blo
 static int prefill_impl(const void* q, const void* k, const void* v, void* out, int B, int Hq,
                         int Hkv, int T, int d, int block, float alpha, float coarse_scale,
                         void* workspace, size_t ws_bytes, dash_stream_t stream, void* const* events,
-                        const float* wsum = nullptr) {
+                        const float* wsum = nullptr, unsigned flags = 0) {
     if (!q || !k || !v || !out || !al16(q) || !al16(k) || !al16(v) || !al16(out)) return DASH_ERR_ARG;
     if (wsum && !al16(wsum)) return DASH_ERR_ARG;
     if (!good_params(alpha, coarse_scale)) return DASH_ERR_ARG;
     PrefillGeom g;
     if (block != kBlock || !make_prefill_geom(B, Hq, Hkv, T, d, &g)) return DASH_ERR_SHAPE;
+    if (flags & ~(unsigned)DASH_HEAD_AGGREGATION) return DASH_ERR_ARG;
+    const int agg = (flags & DASH_HEAD_AGGREGATION) ? 1 : 0;
     // the CUDA-core fine kernel recovers q . kbar from the mean of the block's scores, which
-    // only a mean summary satisfies
-    if (wsum && !fine_tc_supported(g)) return DASH_ERR_UNSUPPORTED;
+    // only a mean summary satisfies, and keeps per-head priors only
+    const bool need_tc = wsum != nullptr || agg;
+    if (need_tc && !fine_tc_supported(g)) return DASH_ERR_UNSUPPORTED;
     if (!workspace || !al256(workspace) || ws_bytes < g.total) return DASH_ERR_WORKSPACE;
     char* ws = static_cast<char*>(workspace);
     cudaStream_t s = S(stream);
@@ -108,7 +111,7 @@ static int prefill_impl(const void* q, const void* k, const void* v, void* out, 
                                 : launch_coarse(q, g, ws, alpha, coarse_scale, s);
     if (ce != cudaSuccess) return DASH_ERR_CUDA;
     if (!mark(2)) return DASH_ERR_CUDA;
-    if (launch_fine(q, k, v, out, g, ws, alpha, coarse_scale, s) != cudaSuccess) return DASH_ERR_CUDA;
+    if (launch_fine(q, k, v, out, g, ws, alpha, coarse_scale, s, agg, need_tc) != cudaSuccess) return DASH_ERR_CUDA;
     if (!mark(3)) return DASH_ERR_CUDA;
     return DASH_OK;
 }
@@ -125,6 +128,13 @@ int dash_prefill_w(const void* q, const void* k, const void* v, const float* w_s
                    size_t ws_bytes, dash_stream_t stream) {
     return prefill_impl(q, k, v, out, B, Hq, Hkv, T, d, block, alpha, coarse_scale, workspace,
                         ws_bytes, stream, nullptr, w_summary);
+}
+
+int dash_prefill_ex(const void* q, const void* k, const void* v, const float* w_summary, void* out, int B,
+                    int Hq, int Hkv, int T, int d, int block, float alpha, float coarse_scale,
+                    unsigned flags, void* workspace, size_t ws_bytes, dash_stream_t stream) {
+    return prefill_impl(q, k, v, out, B, Hq, Hkv, T, d, block, alpha, coarse_scale, workspace,
+                        ws_bytes, stream, nullptr, w_summary, flags);
 }
 
 int dash_prefill_profiled(const void* q, const void* k, const void* v, void* out, int B, int Hq,
@@ -197,18 +207,21 @@ size_t dash_decode_workspace_size(int B, int Hq, int Hkv, int Tmax, int d, int b
 static int decode_impl(const void* q, const void* k_cache, const void* v_cache, const float* ksum,
                        const int* kv_len, void* out, int B, int Hq, int Hkv, int Tmax, int d, int block,
                        float alpha, float coarse_scale, void* workspace, size_t ws_bytes,
-                       dash_stream_t stream, void* const* events) {
+                       dash_stream_t stream, void* const* events, unsigned flags = 0) {
     if (!q || !k_cache || !v_cache || !ksum || !kv_len || !out) return DASH_ERR_ARG;
     if (!al16(q) || !al16(k_cache) || !al16(v_cache) || !al16(ksum) || !al16(out)) return DASH_ERR_ARG;
     if (!good_params(alpha, coarse_scale)) return DASH_ERR_ARG;
     DecodeGeom g;
     if (block != kBlock || !make_decode_geom(B, Hq, Hkv, Tmax, d, &g)) return DASH_ERR_SHAPE;
+    if (flags & ~(unsigned)DASH_HEAD_AGGREGATION) return DASH_ERR_ARG;
+    const int agg = (flags & DASH_HEAD_AGGREGATION) ? 1 : 0;
+    if (agg && !decode_tc_supported(g)) return DASH_ERR_UNSUPPORTED;
     if (!workspace || !al256(workspace) || ws_bytes < g.total) return DASH_ERR_WORKSPACE;
     char* ws = static_cast<char*>(workspace);
     cudaStream_t s = S(stream);
     if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), s) != cudaSuccess) return DASH_ERR_CUDA;
     return launch_decode(q, k_cache, v_cache, ksum, kv_len, out, g, ws, alpha, coarse_scale, s,
-                         reinterpret_cast<cudaEvent_t const*>(events)) == cudaSuccess
+                         reinterpret_cast<cudaEvent_t const*>(events), agg) == cudaSuccess
                ? DASH_OK : DASH_ERR_CUDA;
 }
 
@@ -217,6 +230,14 @@ int dash_decode(const void* q, const void* k_cache, const void* v_cache, const f
                 float alpha, float coarse_scale, void* workspace, size_t ws_bytes, dash_stream_t stream) {
     return decode_impl(q, k_cache, v_cache, ksum, kv_len, out, B, Hq, Hkv, Tmax, d, block, alpha,
                        coarse_scale, workspace, ws_bytes, stream, nullptr);
+}
+
+int dash_decode_ex(const void* q, const void* k_cache, const void* v_cache, const float* ksum,
+                   const int* kv_len, void* out, int B, int Hq, int Hkv, int Tmax, int d, int block,
+                   float alpha, float coarse_scale, unsigned flags, void* workspace, size_t ws_bytes,
+                   dash_stream_t stream) {
+    return decode_impl(q, k_cache, v_cache, ksum, kv_len, out, B, Hq, Hkv, Tmax, d, block, alpha,
+                       coarse_scale, workspace, ws_bytes, stream, nullptr, flags);
 }
 
 int dash_decode_profiled(const void* q, const void* k_cache, const void* v_cache, const float* ksum,

@@ -668,7 +668,7 @@ decode_combine_kernel(const int* __restrict__ count, const float* __restrict__ p
 cudaError_t launch_decode(const void* q, const void* kc, const void* vc, const float* ksum,
                           const int* kv_len, void* out, const DecodeGeom& g, char* ws,
                           float alpha, float coarse_scale, cudaStream_t stream,
-                          const cudaEvent_t* events) {
+                          const cudaEvent_t* events, int agg) {
     auto mark = [&](int i) {
         return !events || cudaEventRecord(events[i], stream) == cudaSuccess;
     };
@@ -704,11 +704,12 @@ cudaError_t launch_decode(const void* q, const void* kc, const void* vc, const f
                                                          alpha, nctas, hist_init);
     if (!mark(1)) return cudaErrorUnknown;
     if (fused) {
-        e = launch_decode_attn_tc(q, kc, vc, kv_len, out, g, ws, e_pow, sm2, nctas, stream);
+        e = launch_decode_attn_tc(q, kc, vc, kv_len, out, g, ws, e_pow, sm2, nctas, stream, agg);
         if (e != cudaSuccess) return e;
         if (!mark(2) || !mark(3)) return cudaErrorUnknown;   // no separate merge pass
         return cudaGetLastError();
     }
+    if (agg) return cudaErrorNotSupported;              // the CUDA-core path has per-head priors only
     const size_t sm_attn = (size_t)4 * kBlock * g.d * sizeof(__nv_bfloat16)
                          + (size_t)(2 * g.G * g.d + g.G * kBlock + 4 * 32) * sizeof(float);
     e = g.d == 128

@@ -79,7 +79,7 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                       const int* __restrict__ list, const int* __restrict__ offs,
                       const int* __restrict__ plan, float* __restrict__ part, int* __restrict__ done,
                       __nv_bfloat16* __restrict__ out, WsHeader* __restrict__ hdr, DecodeGeom g,
-                      float e_pow, float sm2) {
+                      float e_pow, float sm2, int agg) {
     using L = DtLayout<D>;
     using namespace sm100;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -203,19 +203,31 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
             for (int idx = tid; idx < nsub * kDtMaxG; idx += 128) {
                 const int i = idx / kDtMaxG, hl = idx % kDtMaxG;
                 const int j = list[(size_t)bg * cap + i0 + i];
-                float v2 = -INFINITY;
+                float v2 = agg ? 0.f : -INFINITY;
                 if (hl < g.G) {
                     if (j == bt) v2 = 0.f;
                     else {
                         const float x = xs[(qrow0 + hl) * cap + j];
                         const float tu = tau[qrow0 + hl];
-                        if (x > tu) v2 = e_pow * __log2f(x - tu);
+                        // head aggregation keeps the weight itself for the average below
+                        if (x > tu) v2 = agg ? exp2f(e_pow * __log2f(x - tu)) : e_pow * __log2f(x - tu);
                     }
                 }
                 lptab[idx] = v2;
                 if (hl == 0) jtab[i] = j;
             }
             cons_sync();
+            if (agg) {
+                // the group's heads share log2 of their mean weight (own block: prior 1)
+                for (int i = tid; i < nsub; i += 128) {
+                    float pbar = 0.f;
+                    for (int hl = 0; hl < g.G; ++hl) pbar += lptab[i * kDtMaxG + hl];
+                    pbar *= 1.0f / (float)g.G;
+                    const float v2 = jtab[i] == bt ? 0.f : (pbar > 0.f ? __log2f(pbar) : -INFINITY);
+                    for (int hl = 0; hl < kDtMaxG; ++hl) lptab[i * kDtMaxG + hl] = hl < g.G ? v2 : -INFINITY;
+                }
+                cons_sync();
+            }
             for (int i = 0; i < nsub; ++i) {
                 if ((int)(cnt & 3) != warp && (int)((cnt + 1) & 3) != warp) { cnt += 2; continue; }
                 const int j = jtab[i];
@@ -445,7 +457,7 @@ int decode_tc_ctas() {
 
 cudaError_t launch_decode_attn_tc(const void* q, const void* kc, const void* vc, const int* kv_len,
                                   void* out, const DecodeGeom& g, char* ws, float e_pow, float sm2,
-                                  int nctas, cudaStream_t stream) {
+                                  int nctas, cudaStream_t stream, int agg) {
     if (nctas < 1 || nctas > kDecodeMaxCtas) return cudaErrorInvalidValue;
     CUtensorMap tk, tv;
     const unsigned long long rows = (unsigned long long)g.B * g.Hkv * g.Tmax;
@@ -464,12 +476,12 @@ cudaError_t launch_decode_attn_tc(const void* q, const void* kc, const void* vc,
         const int sm = (int)DtLayout<128>::bytes;
         cudaError_t e = cudaFuncSetAttribute(decode_attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
         if (e != cudaSuccess) return e;
-        decode_attn_tc_kernel<128><<<nctas, 160, sm, stream>>>(tk, tv, qb, kv_len, xs, tau, list, offs, plan, part, done, ob, hdr, g, e_pow, sm2);
+        decode_attn_tc_kernel<128><<<nctas, 160, sm, stream>>>(tk, tv, qb, kv_len, xs, tau, list, offs, plan, part, done, ob, hdr, g, e_pow, sm2, agg);
     } else {
         const int sm = (int)DtLayout<64>::bytes;
         cudaError_t e = cudaFuncSetAttribute(decode_attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
         if (e != cudaSuccess) return e;
-        decode_attn_tc_kernel<64><<<nctas, 160, sm, stream>>>(tk, tv, qb, kv_len, xs, tau, list, offs, plan, part, done, ob, hdr, g, e_pow, sm2);
+        decode_attn_tc_kernel<64><<<nctas, 160, sm, stream>>>(tk, tv, qb, kv_len, xs, tau, list, offs, plan, part, done, ob, hdr, g, e_pow, sm2, agg);
     }
     return cudaGetLastError();
 }

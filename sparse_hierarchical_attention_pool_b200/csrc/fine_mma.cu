@@ -241,9 +241,10 @@ static bool use_mma_kernel() {
 
 cudaError_t launch_fine(const void* q, const void* k, const void* v, void* out,
                         const PrefillGeom& g, char* ws, float alpha, float coarse_scale,
-                        cudaStream_t stream) {
-    if (!use_mma_kernel() && fine_tc_supported(g))
-        return launch_fine_tc(q, k, v, out, g, ws, alpha, coarse_scale, stream);
+                        cudaStream_t stream, int agg, bool need_tc) {
+    if ((need_tc || !use_mma_kernel()) && fine_tc_supported(g))
+        return launch_fine_tc(q, k, v, out, g, ws, alpha, coarse_scale, stream, agg);
+    if (need_tc) return cudaErrorNotSupported;
     const float cxm = (alpha - 1.0f) * coarse_scale / sqrtf((float)g.d) / (float)kBlock;
     const float e_pow = 1.0f / (alpha - 1.0f);
     const float sm2 = 1.4426950408889634f / sqrtf((float)g.d);

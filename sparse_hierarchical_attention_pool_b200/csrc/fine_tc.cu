@@ -33,6 +33,8 @@
 //                      and exchange partial row sums and maxima through shared memory behind
 //                      a named barrier).  Online softmax in the log2 domain; O_g is rescaled
 //                      in TMEM only when the running max grows by more than 2^8.
+// Head aggregation (optional): the rows of a position average their block weights
+// through shared memory (one group barrier per step) and share log of the mean as prior.
 // Operands: Q, K, P K-major and V MN-major, all 128-byte swizzled (TMA writes that layout).
 // Every wait is bounded (~2 s); a CTA that gives up sets a status bit and exits cleanly.
 #include <cudaTypedefs.h>
@@ -83,7 +85,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_hi,
                const __grid_constant__ CUtensorMap tm_lo, __nv_bfloat16* __restrict__ out,
                const float* __restrict__ tau, const int* __restrict__ list, const int* __restrict__ count,
-               WsHeader* __restrict__ hdr, PrefillGeom g, float cx, float e_pow, float sm2) {
+               WsHeader* __restrict__ hdr, PrefillGeom g, float cx, float e_pow, float sm2, int agg) {
     using L = TcLayout<D>;
     using namespace sm100;
     constexpr int kGroupThreads = 128 * SPLIT;  // softmax threads per group
@@ -98,6 +100,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
     __shared__ float2 xch[2][2][SPLIT][kTileRows]; // [step parity][group][split][row]: partial (sum, max)
+    __shared__ float pagg[2][2][kTileRows];     // [step parity][group][row]: weights for head aggregation
     __shared__ float m_sh[2][kTileRows];        // running max of each group, for the merge
 
     const uint32_t raw = smem_u32(smem_raw);
@@ -341,10 +344,24 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     smax = fmaxf(smax, e.y);
                 }
             }
-            if (!okw) { ok = false; continue; }
             const float x = __fmul_rn(rs, cx);
-            const float lp2 = diag ? (tpos >= 0 ? 0.f : -INFINITY)
-                                   : (x > tau_r ? e_pow * __log2f(x - tau_r) : -INFINITY);
+            float lp2;
+            if (agg) {
+                // head aggregation: the rows of one position (r = hl P + pl for every head hl)
+                // average their weights p = (x - tau)^(1/(alpha-1)); every warp of the group
+                // passes this barrier once per step, failed step or not
+                const float pown = (okw && !diag && x > tau_r) ? exp2f(e_pow * __log2f(x - tau_r)) : 0.f;
+                if (sp == 0) pagg[i2 & 1][grp][r] = pown;
+                asm volatile("bar.sync %0, %1;" :: "r"(10 + grp), "n"(kGroupThreads) : "memory");
+                float pbar = 0.f;
+                for (int h2 = 0; h2 < g.G; ++h2) pbar += pagg[i2 & 1][grp][h2 * g.P + (r % g.P)];
+                pbar *= 1.0f / (float)g.G;
+                lp2 = diag ? (tpos >= 0 ? 0.f : -INFINITY) : (pbar > 0.f && valid ? __log2f(pbar) : -INFINITY);
+            } else {
+                lp2 = diag ? (tpos >= 0 ? 0.f : -INFINITY)
+                           : (x > tau_r ? e_pow * __log2f(x - tau_r) : -INFINITY);
+            }
+            if (!okw) { ok = false; continue; }
             const bool active = lp2 > -INFINITY;
             const float mx = active ? fmaf(smax, sm2, lp2) : -INFINITY;
             float factor = 1.f;
@@ -495,7 +512,7 @@ bool make_map(CUtensorMap* m, const void* ptr, unsigned long long rows, int d, i
 bool fine_tc_supported(const PrefillGeom& g) { return g.P >= 8 && (g.d == 64 || g.d == 128); }
 
 cudaError_t launch_fine_tc(const void* q, const void* k, const void* v, void* out, const PrefillGeom& g,
-                           char* ws, float alpha, float coarse_scale, cudaStream_t stream) {
+                           char* ws, float alpha, float coarse_scale, cudaStream_t stream, int agg) {
     const float cx = (alpha - 1.0f) * coarse_scale / sqrtf((float)g.d);
     const float e_pow = 1.0f / (alpha - 1.0f);
     const float sm2 = 1.4426950408889634f / sqrtf((float)g.d);
@@ -519,12 +536,12 @@ cudaError_t launch_fine_tc(const void* q, const void* k, const void* v, void* ou
         const int sm = (int)TcLayout<128>::bytes;
         cudaError_t e = cudaFuncSetAttribute(fine_tc_kernel<128, kFineSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
         if (e != cudaSuccess) return e;
-        fine_tc_kernel<128, kFineSplit><<<g.ntiles, threads, sm, stream>>>(tq, tk, tv, thi, tlo, ob, tau, list, count, hdr, g, cx, e_pow, sm2);
+        fine_tc_kernel<128, kFineSplit><<<g.ntiles, threads, sm, stream>>>(tq, tk, tv, thi, tlo, ob, tau, list, count, hdr, g, cx, e_pow, sm2, agg);
     } else {
         const int sm = (int)TcLayout<64>::bytes;
         cudaError_t e = cudaFuncSetAttribute(fine_tc_kernel<64, kFineSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
         if (e != cudaSuccess) return e;
-        fine_tc_kernel<64, kFineSplit><<<g.ntiles, threads, sm, stream>>>(tq, tk, tv, thi, tlo, ob, tau, list, count, hdr, g, cx, e_pow, sm2);
+        fine_tc_kernel<64, kFineSplit><<<g.ntiles, threads, sm, stream>>>(tq, tk, tv, thi, tlo, ob, tau, list, count, hdr, g, cx, e_pow, sm2, agg);
     }
     return cudaGetLastError();
 }

@@ -24,15 +24,17 @@ cudaError_t launch_coarse_tc(const void* q, const PrefillGeom& g, char* ws, floa
                              float coarse_scale, cudaStream_t stream);
 
 // Stage 2 for prefill: prior-weighted softmax attention over each tile's listed blocks.
+// agg: head-aggregated prior; need_tc: the tensor-core kernel is required (head aggregation
+// or a learned summary head), whatever DASH_FINE_KERNEL says.
 cudaError_t launch_fine(const void* q, const void* k, const void* v, void* out,
                         const PrefillGeom& g, char* ws, float alpha, float coarse_scale,
-                        cudaStream_t stream);
+                        cudaStream_t stream, int agg = 0, bool need_tc = false);
 
 // tcgen05 variant of launch_fine (needs P >= 8, i.e. at most 16 query heads per KV head)
 bool fine_tc_supported(const PrefillGeom& g);
 cudaError_t launch_fine_tc(const void* q, const void* k, const void* v, void* out,
                            const PrefillGeom& g, char* ws, float alpha, float coarse_scale,
-                           cudaStream_t stream);
+                           cudaStream_t stream, int agg = 0);
 
 cudaError_t launch_select_dump(const void* q, const float* ksum, const long long* rows, int nrows,
                                int max_sel, int* out_idx, float* out_p, int* out_count,
@@ -45,10 +47,11 @@ bool decode_tc_supported(const DecodeGeom& g);
 int decode_tc_ctas();
 cudaError_t launch_decode_attn_tc(const void* q, const void* kc, const void* vc, const int* kv_len,
                                   void* out, const DecodeGeom& g, char* ws, float e_pow, float sm2,
-                                  int nctas, cudaStream_t stream);
+                                  int nctas, cudaStream_t stream, int agg = 0);
+// agg: head-aggregated prior (needs decode_tc_supported)
 cudaError_t launch_decode(const void* q, const void* kc, const void* vc, const float* ksum,
                           const int* kv_len, void* out, const DecodeGeom& g, char* ws,
                           float alpha, float coarse_scale, cudaStream_t stream,
-                          const cudaEvent_t* events);
+                          const cudaEvent_t* events, int agg = 0);
 
 }  // namespace dash

@@ -27,7 +27,10 @@ EXPORTS = ("dash_status_string", "dash_version", "dash_block_summary", "dash_pre
            "dash_prefill", "dash_prefill_host", "dash_prefill_stats", "dash_decode_stats",
            "dash_prefill_tau", "dash_select_dump", "dash_decode_workspace_size", "dash_decode",
            "dash_get_device_status", "dash_prefill_profiled", "dash_decode_profiled",
-           "dash_decode_noalloc", "dash_block_summary_w", "dash_prefill_w")
+           "dash_decode_noalloc", "dash_block_summary_w", "dash_prefill_w", "dash_prefill_ex",
+           "dash_decode_ex")
+
+HEAD_AGGREGATION = 1       # flag of dash_prefill_ex / dash_decode_ex
 
 
 class DashError(RuntimeError):
@@ -64,6 +67,8 @@ def lib():
     L.dash_block_summary.argtypes = [_p, _p, _i, _i, _i, _i, _i, _p]
     L.dash_block_summary_w.argtypes = [_p, _p, _p, _i, _i, _i, _i, _i, _p]
     L.dash_prefill_w.argtypes = [_p] * 5 + [_i] * 6 + [_f, _f, _p, _sz, _p]
+    L.dash_prefill_ex.argtypes = [_p] * 5 + [_i] * 6 + [_f, _f, ctypes.c_uint, _p, _sz, _p]
+    L.dash_decode_ex.argtypes = [_p] * 6 + [_i] * 6 + [_f, _f, ctypes.c_uint, _p, _sz, _p]
     L.dash_prefill_workspace_size.argtypes = [_i] * 6
     L.dash_prefill_workspace_size.restype = _sz
     L.dash_prefill.argtypes = [_p] * 4 + [_i] * 6 + [_f, _f, _p, _sz, _p]
@@ -193,6 +198,45 @@ def dash_prefill_w(q, k, v, w_summary, out=None, alpha=1.5, coarse_scale=1.0, wo
                               B, Hq, Hkv, T, d, block, float(alpha), float(coarse_scale),
                               ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream))
     _check("dash_prefill_w", rc)
+    return out, workspace
+
+
+def dash_prefill_ex(q, k, v, w_summary=None, flags=0, out=None, alpha=1.5, coarse_scale=1.0, workspace=None,
+                    block=64, stream=None):
+    """dash_prefill with options: learned summary head w_summary [Hkv, d] (None: mean) and
+    flags (HEAD_AGGREGATION)."""
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, T, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Hkv, T, d] matching q")
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(prefill_workspace_size(B, Hq, Hkv, T, d, block), q.device)
+    wp = None if w_summary is None else _dev(w_summary, torch.float32, "w_summary")
+    rc = lib().dash_prefill_ex(_dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"),
+                               _dev(v, torch.bfloat16, "v"), wp, _dev(out, torch.bfloat16, "out"),
+                               B, Hq, Hkv, T, d, block, float(alpha), float(coarse_scale), int(flags),
+                               ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream))
+    _check("dash_prefill_ex", rc)
+    return out, workspace
+
+
+def dash_decode_ex(q, k_cache, v_cache, ksum, kv_len, flags=0, out=None, alpha=1.5, coarse_scale=1.0,
+                   workspace=None, block=64, stream=None):
+    """dash_decode with flags (HEAD_AGGREGATION)."""
+    B, Hq, d = q.shape
+    Hkv, Tmax = k_cache.shape[1], k_cache.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(decode_workspace_size(B, Hq, Hkv, Tmax, d, block), q.device)
+    rc = lib().dash_decode_ex(_dev(q, torch.bfloat16, "q"), _dev(k_cache, torch.bfloat16, "k_cache"),
+                              _dev(v_cache, torch.bfloat16, "v_cache"), _dev(ksum, torch.float32, "ksum"),
+                              _dev(kv_len, torch.int32, "kv_len"), _dev(out, torch.bfloat16, "out"),
+                              B, Hq, Hkv, Tmax, d, block, float(alpha), float(coarse_scale), int(flags),
+                              ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream))
+    _check("dash_decode_ex", rc)
     return out, workspace
 
 
