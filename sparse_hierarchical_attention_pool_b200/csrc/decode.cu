@@ -256,9 +256,10 @@ struct WarpRow {
 
 constexpr int kHistBins = 64;       // bins of the histogram start over y = x - m in [-1, 0)
 
-// Histogram start of the threshold solve (the idea of AdaSplash-2, "a coarse histogram of
-// the scores in on-chip memory gives a close initial threshold", as summarised in "DashAttention
-// and the year sparse attention became a field"; the construction here is this library's):
+// Histogram start of the threshold solve (the idea of AdaSplash-2, whose abstract appears on
+// the listing page "DashAttention: Differentiable and Adaptive Sparse Hierarchical Attention":
+// a coarse histogram of the scores kept in on-chip memory gives a close initial threshold;
+// the construction here is this library's):
 // the values y = x - m in [-1, 0) go to bin k = floor((y + 1) * 64) with their count, sum and
 // sum of squares, accumulated as integers (y and y^2 in 2^-24 fixed point), so the sums and
 // the start do not depend on the order of the shared-memory atomics.  At a bin's lower edge

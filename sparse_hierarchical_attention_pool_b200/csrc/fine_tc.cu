@@ -79,13 +79,13 @@ enum : int { B_Q = 0, B_KV_FULL = 1, B_KV_EMPTY = 1 + kTcStages, B_S_FULL = 1 + 
              B_S_FREE = B_S_FULL + 2, B_P_FULL = B_S_FREE + 2, B_PV_DONE = B_P_FULL + 2,
              B_DRAIN = B_PV_DONE + 2, B_DRAIN2 = B_DRAIN + 1, B_COUNT = B_DRAIN2 + 1 };
 
-template <int D, int SPLIT>
+template <int D, int SPLIT, bool AGG>
 __global__ void __launch_bounds__((8 * SPLIT + 3) * 32, 1)
 fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_hi,
                const __grid_constant__ CUtensorMap tm_lo, __nv_bfloat16* __restrict__ out,
                const float* __restrict__ tau, const int* __restrict__ list, const int* __restrict__ count,
-               WsHeader* __restrict__ hdr, PrefillGeom g, float cx, float e_pow, float sm2, int agg) {
+               WsHeader* __restrict__ hdr, PrefillGeom g, float cx, float e_pow, float sm2) {
     using L = TcLayout<D>;
     using namespace sm100;
     constexpr int kGroupThreads = 128 * SPLIT;  // softmax threads per group
@@ -100,7 +100,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
     __shared__ float2 xch[2][2][SPLIT][kTileRows]; // [step parity][group][split][row]: partial (sum, max)
-    __shared__ float pagg[2][2][kTileRows];     // [step parity][group][row]: weights for head aggregation
+    __shared__ float pagg[AGG ? 2 : 1][2][kTileRows];   // [step parity][group][row]: weights for head aggregation
     __shared__ float m_sh[2][kTileRows];        // running max of each group, for the merge
 
     const uint32_t raw = smem_u32(smem_raw);
@@ -344,12 +344,12 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     smax = fmaxf(smax, e.y);
                 }
             }
-            const float x = __fmul_rn(rs, cx);
             float lp2;
-            if (agg) {
+            if constexpr (AGG) {
                 // head aggregation: the rows of one position (r = hl P + pl for every head hl)
                 // average their weights p = (x - tau)^(1/(alpha-1)); every warp of the group
                 // passes this barrier once per step, failed step or not
+                const float x = __fmul_rn(rs, cx);
                 const float pown = (okw && !diag && x > tau_r) ? exp2f(e_pow * __log2f(x - tau_r)) : 0.f;
                 if (sp == 0) pagg[i2 & 1][grp][r] = pown;
                 asm volatile("bar.sync %0, %1;" :: "r"(10 + grp), "n"(kGroupThreads) : "memory");
@@ -357,11 +357,13 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 for (int h2 = 0; h2 < g.G; ++h2) pbar += pagg[i2 & 1][grp][h2 * g.P + (r % g.P)];
                 pbar *= 1.0f / (float)g.G;
                 lp2 = diag ? (tpos >= 0 ? 0.f : -INFINITY) : (pbar > 0.f && valid ? __log2f(pbar) : -INFINITY);
+                if (!okw) { ok = false; continue; }
             } else {
+                if (!okw) { ok = false; continue; }
+                const float x = __fmul_rn(rs, cx);
                 lp2 = diag ? (tpos >= 0 ? 0.f : -INFINITY)
                            : (x > tau_r ? e_pow * __log2f(x - tau_r) : -INFINITY);
             }
-            if (!okw) { ok = false; continue; }
             const bool active = lp2 > -INFINITY;
             const float mx = active ? fmaf(smax, sm2, lp2) : -INFINITY;
             float factor = 1.f;
@@ -532,17 +534,21 @@ cudaError_t launch_fine_tc(const void* q, const void* k, const void* v, void* ou
     WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
     auto* ob = static_cast<__nv_bfloat16*>(out);
     constexpr int threads = (8 * kFineSplit + 3) * 32;
+    auto go = [&](auto kernel, int sm) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+        if (e != cudaSuccess) return e;
+        kernel<<<g.ntiles, threads, sm, stream>>>(tq, tk, tv, thi, tlo, ob, tau, list, count, hdr, g, cx, e_pow, sm2);
+        return cudaSuccess;
+    };
+    cudaError_t e;
     if (g.d == 128) {
         const int sm = (int)TcLayout<128>::bytes;
-        cudaError_t e = cudaFuncSetAttribute(fine_tc_kernel<128, kFineSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-        if (e != cudaSuccess) return e;
-        fine_tc_kernel<128, kFineSplit><<<g.ntiles, threads, sm, stream>>>(tq, tk, tv, thi, tlo, ob, tau, list, count, hdr, g, cx, e_pow, sm2, agg);
+        e = agg ? go(fine_tc_kernel<128, kFineSplit, true>, sm) : go(fine_tc_kernel<128, kFineSplit, false>, sm);
     } else {
         const int sm = (int)TcLayout<64>::bytes;
-        cudaError_t e = cudaFuncSetAttribute(fine_tc_kernel<64, kFineSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-        if (e != cudaSuccess) return e;
-        fine_tc_kernel<64, kFineSplit><<<g.ntiles, threads, sm, stream>>>(tq, tk, tv, thi, tlo, ob, tau, list, count, hdr, g, cx, e_pow, sm2, agg);
+        e = agg ? go(fine_tc_kernel<64, kFineSplit, true>, sm) : go(fine_tc_kernel<64, kFineSplit, false>, sm);
     }
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
