@@ -147,10 +147,15 @@ DASH_API int dash_prefill_ex(const void* q, const void* k, const void* v, const 
 
 /*
  * dash_prefill with HOST inputs and output: copies q, k, v from host memory into the
- * caller's device buffers, runs dash_prefill, copies out back to host memory, all
- * asynchronously on `stream` (host buffers should be pinned for the copies to overlap).
+ * caller's device buffers, runs the prefill, copies out back to host memory, asynchronously
+ * with respect to the host and ordered after the work already on `stream`; `stream` waits
+ * for the last copy (host buffers should be pinned for the copies to overlap).
  * Host pointers: q_host, k_host, v_host (read), out_host (written).  Device pointers:
  * q_dev, k_dev, v_dev, out_dev (same shapes as dash_prefill) and the workspace.
+ * The (b, kv head) groups are independent, so with B * Hkv > 1 the call pipelines them:
+ * the copies of one group overlap the kernels of the previous one (two short-lived helper
+ * streams).  The workspace then holds the state of the last group only (its statistics and
+ * thresholds are those of a prefill with B = 1, Hq = Hq / Hkv, Hkv = 1).
  */
 DASH_API int dash_prefill_host(const void* q_host, const void* k_host, const void* v_host, void* out_host,
                       void* q_dev, void* k_dev, void* v_dev, void* out_dev,

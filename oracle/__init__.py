@@ -70,8 +70,9 @@ def lib():
         L.oracle_forward_rows_agg.argtypes = ([_ptr, ctypes.c_int, _ptr, ctypes.c_int, _ptr, ctypes.c_int, _ptr]
                                               + [_i64] * 6 + [_dbl, _dbl, _ptr, _i64]
                                               + [_ptr] * 2 + [ctypes.c_int])
+        L.oracle_backward.argtypes = ([_ptr, ctypes.c_int] * 4 + [_i64] * 6 + [_dbl, _dbl] + [_ptr] * 3)
         for f in (L.oracle_block_summary_w, L.oracle_select_rows_w, L.oracle_forward_rows_w,
-                  L.oracle_forward_rows_agg):
+                  L.oracle_forward_rows_agg, L.oracle_backward):
             f.restype = ctypes.c_int
         for f in (L.oracle_entmax_tau, L.oracle_entmax, L.oracle_block_summary, L.oracle_select_rows,
                   L.oracle_forward_rows, L.oracle_fine_rows_given_p, L.oracle_dense_causal_rows):
@@ -81,19 +82,22 @@ def lib():
 
 
 def _arr(a):
-    """numpy view of an element array: (contiguous array, dtype code 0=f32 / 1=bf16 bits)."""
+    """numpy view of an element array: (contiguous array, dtype code 0=f32 / 1=bf16 bits /
+    2=f64).  float64 inputs stay float64 (finite-difference checks need them)."""
     try:
         import torch
         if isinstance(a, torch.Tensor):
             a = a.detach().cpu().contiguous()
             if a.dtype == torch.bfloat16:
                 return a.view(torch.int16).numpy().view(np.uint16), 1
-            a = a.float().numpy()
+            a = a.numpy() if a.dtype == torch.float64 else a.float().numpy()
     except ImportError:  # pragma: no cover
         pass
     a = np.ascontiguousarray(a)
     if a.dtype == np.uint16:
         return a, 1
+    if a.dtype == np.float64:
+        return a, 2
     return np.ascontiguousarray(a, dtype=np.float32), 0
 
 
@@ -222,6 +226,24 @@ def forward_rows_agg(q, k, v, rows, blk, alpha, coarse_scale, nthreads=0, w_summ
                                          _p(r), n, _p(out), _p(ns), int(nthreads)),
            "forward_rows_agg")
     return out, ns
+
+
+def backward(q, k, v, dout, blk, alpha, coarse_scale):
+    """Gradients (dq, dk, dv) in fp64 of a scalar loss with d loss / d out = dout, through
+    the whole forward: fine softmax, log prior, alpha-entmax (its Jacobian on the support),
+    coarse scores and mean summaries.  Every row of the [B, Hq, T, d] problem."""
+    qa, qdt = _arr(q)
+    ka, kdt = _arr(k)
+    va, vdt = _arr(v)
+    ga, gdt = _arr(dout)
+    B, Hq, T, d = qa.shape
+    Hkv = ka.shape[1]
+    dq = np.zeros((B, Hq, T, d))
+    dk = np.zeros((B, Hkv, T, d))
+    dv = np.zeros((B, Hkv, T, d))
+    _check(lib().oracle_backward(_p(qa), qdt, _p(ka), kdt, _p(va), vdt, _p(ga), gdt, B, Hq, Hkv, T, d, blk,
+                                 float(alpha), float(coarse_scale), _p(dq), _p(dk), _p(dv)), "backward")
+    return dq, dk, dv
 
 
 def fine_rows_given_p(q_rows, k, v, rows, Hq, blk, w_rows, w_diag, nthreads=0):

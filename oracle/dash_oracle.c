@@ -40,8 +40,8 @@
  * equal prior and T <= 2 blocks against dense causal attention (torch SDPA);
  * non-dispersiveness; a hand-derived worked example.
  *
- * Inputs: element arrays are either float32 (dtype 0) or bf16 bit patterns
- * (dtype 1, uint16); both are widened exactly to double.  Every routine is fp64.
+ * Inputs: element arrays are float32 (dtype 0), bf16 bit patterns (dtype 1, uint16) or
+ * float64 (dtype 2); all are widened exactly to double.  Every routine is fp64.
  * Threads: OpenMP over independent rows.
  */
 #include <math.h>
@@ -60,6 +60,7 @@
 
 static double elem(const void* base, int dtype, long long i) {
     if (dtype == 0) return (double)((const float*)base)[i];
+    if (dtype == 2) return ((const double*)base)[i];
     uint32_t u = ((uint32_t)((const uint16_t*)base)[i]) << 16;
     float f;
     memcpy(&f, &u, sizeof f);
@@ -542,6 +543,128 @@ int oracle_forward_rows_agg(const void* q_group, int qdt, const void* k, int kdt
     }
     free(kb);
     return fail ? ORC_ERR_NOMEM : ORC_OK;
+}
+
+/*
+ * Backward of the full causal forward (mean summaries), for every row (b, h, t):
+ * given dout [B, Hq, T, d] (the gradient of a scalar loss with respect to out), returns
+ * dq [B, Hq, T, d], dk, dv [B, Hkv, T, d] in fp64 (zeroed here).  The chain, per row:
+ *   fine stage  l_i = q . k_i / sqrt(d) + log p_j(i) over the row's tokens, P = softmax(l),
+ *               o = sum P_i v_i:  dP_i = dout . v_i, dl_i = P_i (dP_i - dout . o),
+ *               dv_i += P_i dout, dq += dl_i k_i / sqrt(d), dk_i += dl_i q / sqrt(d),
+ *               d log p_j = sum of dl_i over the tokens of past block j;
+ *   entmax      p = alpha-entmax(s) has the Jacobian diag(g) - g g^T / sum(g) with
+ *               g_j = p_j^(2 - alpha) on the support (0 elsewhere), so with dp_j = d log p_j / p_j:
+ *               ds_j = g_j dp_j - g_j (sum_k g_k dp_k) / sum_k g_k;
+ *   scores      s_j = cs (q . kbar_j) / sqrt(d):  dq += ds_j cs kbar_j / sqrt(d),
+ *               dkbar_j += ds_j cs q / sqrt(d);
+ *   summaries   kbar_j = mean of block j's keys:  dk_i += dkbar_j / blk.
+ * The own block has prior 1 (no gradient into the coarse stage).  Serial over rows.
+ */
+int oracle_backward(const void* q, int qdt, const void* k, int kdt, const void* v, int vdt,
+                    const void* dout, int ddt, long long B, long long Hq, long long Hkv, long long Tk,
+                    long long d, long long blk, double alpha, double coarse_scale,
+                    double* dq, double* dk, double* dv) {
+    if (!q || !k || !v || !dout || !dq || !dk || !dv) return ORC_ERR_ARG;
+    if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || d < 1 || blk < 1 || Tk < 1 || !(alpha > 1.0)) return ORC_ERR_ARG;
+    orc_problem P = {q, qdt, k, kdt, v, vdt, B, Hq, Hkv, Tk, d, blk, alpha, coarse_scale, NULL};
+    double* kb = all_kbar(&P);
+    if (!kb) return ORC_ERR_NOMEM;
+    long long nbs = Tk / blk, G = Hq / Hkv;
+    double isd = 1.0 / sqrt((double)d);
+    memset(dq, 0, (size_t)(B * Hq * Tk * d) * sizeof(double));
+    memset(dk, 0, (size_t)(B * Hkv * Tk * d) * sizeof(double));
+    memset(dv, 0, (size_t)(B * Hkv * Tk * d) * sizeof(double));
+    double* dkbar = (double*)calloc((size_t)(B * Hkv * (nbs > 0 ? nbs : 1) * d), sizeof(double));
+    double* x = (double*)malloc((size_t)(nbs + 1) * sizeof(double));
+    double* p = (double*)malloc((size_t)(nbs + 1) * sizeof(double));
+    double* lp = (double*)malloc((size_t)(nbs + 1) * sizeof(double));
+    double* dlp = (double*)malloc((size_t)(nbs + 1) * sizeof(double));
+    double* lbuf = (double*)malloc((size_t)Tk * sizeof(double));
+    double* o = (double*)malloc((size_t)d * sizeof(double));
+    double* qv = (double*)malloc((size_t)d * sizeof(double));
+    double* gv = (double*)malloc((size_t)d * sizeof(double));
+    int rc = ORC_OK;
+    if (!dkbar || !x || !p || !lp || !dlp || !lbuf || !o || !qv || !gv) rc = ORC_ERR_NOMEM;
+    for (long long b = 0; rc == ORC_OK && b < B; ++b)
+        for (long long h = 0; h < Hq; ++h)
+            for (long long t = 0; t < Tk; ++t) {
+                long long g = h / G, bt = t / blk, row = (b * Hq + h) * Tk + t;
+                long long kvbase = (b * Hkv + g) * Tk;
+                const double* kbg = kb + (b * Hkv + g) * nbs * d;
+                for (long long c = 0; c < d; ++c) {
+                    qv[c] = elem(q, qdt, row * d + c);
+                    gv[c] = elem(dout, ddt, row * d + c);
+                }
+                /* coarse stage (row_select reads q row r = row) */
+                double tau = NAN;
+                row_select(&P, row, t, kbg, x, p, &tau);
+                for (long long j = 0; j < bt; ++j) lp[j] = p[j] > 0.0 ? log(x[j] - tau) / (alpha - 1.0) : -INFINITY;
+                /* fine forward: logits, max, softmax, output */
+                double m = -INFINITY;
+                for (long long i = 0; i <= t; ++i) {
+                    long long j = i / blk;
+                    double lw = j == bt ? 0.0 : lp[j];
+                    if (lw == -INFINITY) { lbuf[i] = -INFINITY; continue; }
+                    double dot = 0.0;
+                    for (long long c = 0; c < d; ++c) dot += qv[c] * elem(k, kdt, (kvbase + i) * d + c);
+                    lbuf[i] = dot * isd + lw;
+                    if (lbuf[i] > m) m = lbuf[i];
+                }
+                double den = 0.0;
+                for (long long c = 0; c < d; ++c) o[c] = 0.0;
+                for (long long i = 0; i <= t; ++i) {
+                    if (lbuf[i] == -INFINITY) continue;
+                    double a = exp(lbuf[i] - m);
+                    den += a;
+                    for (long long c = 0; c < d; ++c) o[c] += a * elem(v, vdt, (kvbase + i) * d + c);
+                }
+                for (long long c = 0; c < d; ++c) o[c] /= den;
+                double Drow = 0.0;
+                for (long long c = 0; c < d; ++c) Drow += gv[c] * o[c];
+                /* fine backward */
+                for (long long j = 0; j < bt; ++j) dlp[j] = 0.0;
+                for (long long i = 0; i <= t; ++i) {
+                    if (lbuf[i] == -INFINITY) continue;
+                    double Pi = exp(lbuf[i] - m) / den;
+                    double dPi = 0.0;
+                    for (long long c = 0; c < d; ++c) dPi += gv[c] * elem(v, vdt, (kvbase + i) * d + c);
+                    double dl = Pi * (dPi - Drow);
+                    for (long long c = 0; c < d; ++c) {
+                        dv[(kvbase + i) * d + c] += Pi * gv[c];
+                        dq[row * d + c] += dl * elem(k, kdt, (kvbase + i) * d + c) * isd;
+                        dk[(kvbase + i) * d + c] += dl * qv[c] * isd;
+                    }
+                    long long j = i / blk;
+                    if (j < bt) dlp[j] += dl;
+                }
+                /* entmax backward on the support, then the coarse scores */
+                double sg = 0.0, sgdp = 0.0;
+                for (long long j = 0; j < bt; ++j) {
+                    if (!(p[j] > 0.0)) continue;
+                    double gj = pow(p[j], 2.0 - alpha);
+                    sg += gj;
+                    sgdp += gj * (dlp[j] / p[j]);
+                }
+                for (long long j = 0; j < bt; ++j) {
+                    if (!(p[j] > 0.0)) continue;
+                    double gj = pow(p[j], 2.0 - alpha);
+                    double ds = gj * (dlp[j] / p[j]) - gj * sgdp / sg;
+                    double f = ds * coarse_scale * isd;
+                    for (long long c = 0; c < d; ++c) {
+                        dq[row * d + c] += f * kbg[j * d + c];
+                        dkbar[((b * Hkv + g) * nbs + j) * d + c] += f * qv[c];
+                    }
+                }
+            }
+    /* summaries: every key of complete block j receives dkbar_j / blk */
+    for (long long bg = 0; rc == ORC_OK && bg < B * Hkv; ++bg)
+        for (long long j = 0; j < nbs; ++j)
+            for (long long i = 0; i < blk; ++i)
+                for (long long c = 0; c < d; ++c)
+                    dk[(bg * Tk + j * blk + i) * d + c] += dkbar[(bg * nbs + j) * d + c] / (double)blk;
+    free(dkbar); free(x); free(p); free(lp); free(dlp); free(lbuf); free(o); free(qv); free(gv); free(kb);
+    return rc;
 }
 
 int oracle_select_rows(const void* q_rows, int qdt, const void* k, int kdt,

@@ -3,6 +3,8 @@
 // Argument checks happen here, before any launch; kernels live in summary.cu, coarse.cu,
 // fine_mma.cu, decode.cu and dump.cu.  Nothing here allocates memory.
 #include <math.h>
+
+#include <new>
 #include <stdint.h>
 #include <string.h>
 
@@ -153,16 +155,71 @@ int dash_prefill_host(const void* q_host, const void* k_host, const void* v_host
     PrefillGeom g;
     if (block != kBlock || !make_prefill_geom(B, Hq, Hkv, T, d, &g)) return DASH_ERR_SHAPE;
     if (!q_dev || !k_dev || !v_dev || !out_dev) return DASH_ERR_ARG;
-    const size_t qb = (size_t)B * Hq * T * d * 2, kb = (size_t)B * Hkv * T * d * 2;
+    if (!good_params(alpha, coarse_scale)) return DASH_ERR_ARG;
+    if (!workspace || !al256(workspace) || ws_bytes < g.total) return DASH_ERR_WORKSPACE;
     cudaStream_t s = S(stream);
-    if (cudaMemcpyAsync(q_dev, q_host, qb, cudaMemcpyHostToDevice, s) != cudaSuccess) return DASH_ERR_CUDA;
-    if (cudaMemcpyAsync(k_dev, k_host, kb, cudaMemcpyHostToDevice, s) != cudaSuccess) return DASH_ERR_CUDA;
-    if (cudaMemcpyAsync(v_dev, v_host, kb, cudaMemcpyHostToDevice, s) != cudaSuccess) return DASH_ERR_CUDA;
-    int rc = dash_prefill(q_dev, k_dev, v_dev, out_dev, B, Hq, Hkv, T, d, block, alpha, coarse_scale,
-                          workspace, ws_bytes, stream);
-    if (rc != DASH_OK) return rc;
-    if (cudaMemcpyAsync(out_host, out_dev, qb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return DASH_ERR_CUDA;
-    return DASH_OK;
+    // The (b, kv head) groups are independent prefills on contiguous slices of q, k, v and
+    // out, so the copies of one group overlap the kernels of another: copies in on one
+    // helper stream, the groups' kernels in order on `stream` (sharing the workspace),
+    // copies out on a second helper stream; `stream` finally waits for the last copy out.
+    const int ng = B * Hkv, G = Hq / Hkv;
+    const size_t qg = (size_t)G * T * d * 2, kg = (size_t)T * d * 2;    // bytes per group
+    auto cp = [](void* dst, const void* src, size_t n, cudaMemcpyKind kind, cudaStream_t st) {
+        return cudaMemcpyAsync(dst, src, n, kind, st) == cudaSuccess;
+    };
+    auto at = [](const void* p, size_t off) { return static_cast<const char*>(p) + off; };
+    auto atw = [](void* p, size_t off) { return static_cast<char*>(p) + off; };
+    if (ng == 1) {
+        if (!cp(k_dev, k_host, kg, cudaMemcpyHostToDevice, s) || !cp(v_dev, v_host, kg, cudaMemcpyHostToDevice, s) ||
+            !cp(q_dev, q_host, qg, cudaMemcpyHostToDevice, s))
+            return DASH_ERR_CUDA;
+        int rc = dash_prefill(q_dev, k_dev, v_dev, out_dev, B, Hq, Hkv, T, d, block, alpha, coarse_scale,
+                              workspace, ws_bytes, stream);
+        if (rc != DASH_OK) return rc;
+        return cp(out_host, out_dev, qg, cudaMemcpyDeviceToHost, s) ? DASH_OK : DASH_ERR_CUDA;
+    }
+    cudaStream_t sin = nullptr, sout = nullptr;
+    cudaEvent_t start = nullptr, fin = nullptr;
+    cudaEvent_t* ev = new (std::nothrow) cudaEvent_t[2 * (size_t)ng]();
+    int rc = DASH_OK;
+    auto mkev = [](cudaEvent_t* e) { return cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess; };
+    if (!ev || cudaStreamCreateWithFlags(&sin, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&sout, cudaStreamNonBlocking) != cudaSuccess || !mkev(&start) || !mkev(&fin))
+        rc = DASH_ERR_CUDA;
+    for (int i = 0; rc == DASH_OK && i < 2 * ng; ++i)
+        if (!mkev(&ev[i])) rc = DASH_ERR_CUDA;
+    // the helper streams start after the work already queued on `stream`
+    if (rc == DASH_OK && (cudaEventRecord(start, s) != cudaSuccess || cudaStreamWaitEvent(sin, start, 0) != cudaSuccess ||
+                          cudaStreamWaitEvent(sout, start, 0) != cudaSuccess))
+        rc = DASH_ERR_CUDA;
+    for (int gi = 0; rc == DASH_OK && gi < ng; ++gi) {
+        const size_t oq = (size_t)gi * qg, ok = (size_t)gi * kg;
+        if (!cp(atw(k_dev, ok), at(k_host, ok), kg, cudaMemcpyHostToDevice, sin) ||
+            !cp(atw(v_dev, ok), at(v_host, ok), kg, cudaMemcpyHostToDevice, sin) ||
+            !cp(atw(q_dev, oq), at(q_host, oq), qg, cudaMemcpyHostToDevice, sin) ||
+            cudaEventRecord(ev[2 * gi], sin) != cudaSuccess || cudaStreamWaitEvent(s, ev[2 * gi], 0) != cudaSuccess) {
+            rc = DASH_ERR_CUDA;
+            break;
+        }
+        rc = dash_prefill(atw(q_dev, oq), atw(k_dev, ok), atw(v_dev, ok), atw(out_dev, oq), 1, G, 1, T, d, block,
+                          alpha, coarse_scale, workspace, ws_bytes, stream);
+        if (rc != DASH_OK) break;
+        if (cudaEventRecord(ev[2 * gi + 1], s) != cudaSuccess || cudaStreamWaitEvent(sout, ev[2 * gi + 1], 0) != cudaSuccess ||
+            !cp(atw(out_host, oq), at(out_dev, oq), qg, cudaMemcpyDeviceToHost, sout))
+            rc = DASH_ERR_CUDA;
+    }
+    // `stream` waits for everything issued on the helper streams, also after an error
+    if (sout && fin && cudaEventRecord(fin, sout) == cudaSuccess) cudaStreamWaitEvent(s, fin, 0);
+    if (sin && start && cudaEventRecord(start, sin) == cudaSuccess) cudaStreamWaitEvent(s, start, 0);
+    // destroying a stream or event with work pending releases it once the work completes
+    for (int i = 0; ev && i < 2 * ng; ++i)
+        if (ev[i]) cudaEventDestroy(ev[i]);
+    delete[] ev;
+    if (start) cudaEventDestroy(start);
+    if (fin) cudaEventDestroy(fin);
+    if (sin) cudaStreamDestroy(sin);
+    if (sout) cudaStreamDestroy(sout);
+    return rc;
 }
 
 int dash_prefill_stats(const void* workspace, size_t ws_bytes, dash_stats* out, dash_stream_t stream) {

@@ -482,3 +482,57 @@ def test_aggregated_attention_ignores_blocks_outside_the_shared_support(orc):
     v3 = v.clone()
     v3[0, 0, 64 * used[0]:64 * (used[0] + 1)] += 1.0
     assert np.abs(orc.forward_rows_agg(q, k, v3, grp, 64, 2.0, 6.0)[0] - base).max() > 1e-6
+
+
+# ------------------------------------------------------------------ backward
+# Differentiability is the method's central claim ("DashAttention: Making Sparse Attention Fully
+# Differentiable with Adaptive Block Selection", section "Key Concepts"): the oracle backward
+# (fine softmax, log prior, alpha-entmax Jacobian, coarse scores, mean summaries) is pinned
+# by central finite differences of the fp64 forward.
+
+@pytest.mark.parametrize("alpha,cs,Hq,Hkv,T", [(1.5, 2.0, 2, 1, 448), (2.0, 3.0, 4, 2, 384),
+                                               (1.25, 4.0, 2, 2, 320), (3.0, 1.5, 2, 1, 448)])
+def test_backward_matches_finite_differences(orc, alpha, cs, Hq, Hkv, T):
+    d, B = 8, 1
+    rng = np.random.default_rng(int(alpha * 100) + T)
+    q = rng.standard_normal((B, Hq, T, d)) * 1.5
+    k = rng.standard_normal((B, Hkv, T, d))
+    v = rng.standard_normal((B, Hkv, T, d))
+    G = rng.standard_normal((B, Hq, T, d))
+    rows = [(0, h, t) for h in range(Hq) for t in range(T)]
+
+    def loss(q_, k_, v_):
+        out, _, _ = orc.forward_rows(q_.reshape(-1, d), k_, v_, rows, Hq, 64, alpha, cs)
+        return float((out * G.reshape(-1, d)).sum())
+
+    dq, dk, dv = orc.backward(q, k, v, G, 64, alpha, cs)
+    # the coarse stage is exercised: some rows have a sparse, non-trivial support
+    sel = orc.select_rows(q.reshape(-1, d), k, rows, Hq, 64, alpha, cs)
+    assert np.any((sel["nsel"] < sel["bt"]) & (sel["nsel"] >= 2))
+    h = 1e-6
+    for name, arr, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for _ in range(6):
+            idx = tuple(int(rng.integers(0, s)) for s in arr.shape)
+            args = {"q": q, "k": k, "v": v}
+            a = arr.copy(); a[idx] += h; args[name] = a; lp = loss(args["q"], args["k"], args["v"])
+            a = arr.copy(); a[idx] -= h; args[name] = a; lm = loss(args["q"], args["k"], args["v"])
+            fd = (lp - lm) / (2 * h)
+            assert abs(fd - grad[idx]) <= 1e-6 * max(1.0, abs(fd)), (name, idx, fd, grad[idx])
+
+
+def test_backward_of_dense_rows_is_softmax_attention_backward(orc):
+    # T <= 2 blocks: one past block (p = 1, no gradient into the coarse stage) -- plain causal
+    # attention, whose gradients torch.autograd gives independently
+    B, Hq, Hkv, T, d = 1, 2, 1, 128, 8
+    g = torch.Generator().manual_seed(3)
+    q = torch.randn(B, Hq, T, d, generator=g, dtype=torch.float64, requires_grad=True)
+    k = torch.randn(B, Hkv, T, d, generator=g, dtype=torch.float64, requires_grad=True)
+    v = torch.randn(B, Hkv, T, d, generator=g, dtype=torch.float64, requires_grad=True)
+    G = torch.randn(B, Hq, T, d, generator=g, dtype=torch.float64)
+    kk, vv = k.repeat_interleave(Hq // Hkv, 1), v.repeat_interleave(Hq // Hkv, 1)
+    out = F.scaled_dot_product_attention(q, kk, vv, is_causal=True)
+    (out * G).sum().backward()
+    dq, dk, dv = orc.backward(q.detach(), k.detach(), v.detach(), G, 64, 1.5, 2.0)
+    np.testing.assert_allclose(dq, q.grad.numpy(), rtol=0, atol=1e-10)
+    np.testing.assert_allclose(dk, k.grad.numpy(), rtol=0, atol=1e-10)
+    np.testing.assert_allclose(dv, v.grad.numpy(), rtol=0, atol=1e-10)
