@@ -44,6 +44,7 @@ namespace dash {
 constexpr int kCtStages = 2;
 constexpr int kCtChunk = 128;        // blocks per score chunk (MMA N)
 constexpr int kCtBufs = 4;           // TMEM chunk buffers (4 x 128 columns)
+constexpr int kTopK = 4;             // largest scores per half-row kept for the threshold start
 
 template <int D>
 struct CtLayout {
@@ -99,6 +100,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __shared__ unsigned bitmap[kMaxT / kBlock / 32];
     __shared__ unsigned long long sel_sh;
     __shared__ float xp[2][2][6][kTileRows];     // [pass parity][half][sum][row]: partial pass sums
+    __shared__ float topv[2][kTopK][kTileRows];  // [half][rank][row]: each half-row's largest scores
     __shared__ int wtot_sh[8];
 
     const uint32_t raw = smem_u32(smem_raw);
@@ -323,14 +325,16 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 xp[0][hf][0][r] = m;
                 sync_pair();
                 m = fmaxf(xp[0][0][0][r], xp[0][1][0][r]);
+                // Newton from u = -1: with the scores in registers a pass is cheap, and the
+                // subset start of the streamed tiles costs more here than the passes it saves
                 EntmaxSolver sv;
-                sv.init(m, alpha);
                 bool done = !valid;
                 // ---- Newton / exact-support passes; the pair of warps iterates until all of
                 // its 32 rows are final (both warps see the same flags), partial sums are
                 // exchanged through a buffer alternating with the pass parity
                 auto sweep = [&](auto mode) {
                     constexpr int MODE = decltype(mode)::value;
+                    sv.init(m, alpha);
                     for (int pp = 1; __any_sync(0xffffffffu, !done); ++pp) {
                         EntmaxPass ps;
                         ps.reset();
@@ -355,8 +359,8 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         if (!done) done = sv.update(tot, &tau, &no_conv);
                     }
                 };
-                if (sv.mode == 1) sweep(std::integral_constant<int, 1>{});
-                else if (sv.mode == 2) sweep(std::integral_constant<int, 2>{});
+                if (alpha == 1.5f) sweep(std::integral_constant<int, 1>{});
+                else if (alpha == 2.0f) sweep(std::integral_constant<int, 2>{});
                 else sweep(std::integral_constant<int, 0>{});
                 // ---- union pass: OR of x > tau over the rows, per block
                 for (int i = st; i < nw; i += 256) bitmap[i] = 0u;
@@ -413,17 +417,34 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         mbar_arrive(bar(C_DEC));
                     }
                 };
-                // ---- pass 0: row maximum
+                // ---- pass 0: row maximum and each half-row's largest scores (every further
+                // pass recomputes the scores, so a start close to the root saves whole GEMMs)
                 float m = -INFINITY;
+                float tk[kTopK];
+#pragma unroll
+                for (int i = 0; i < kTopK; ++i) tk[i] = -INFINITY;
                 if (!run_pass([&](int, const uint32_t* v, int nv) {
                         for (int i = 0; i < 32; ++i)
-                            if (i < nv) m = fmaxf(m, __fmul_rn(__uint_as_float(v[i]), cx));
+                            if (i < nv) {
+                                const float x = __fmul_rn(__uint_as_float(v[i]), cx);
+                                m = fmaxf(m, x);
+                                topk_insert(tk, x);
+                            }
                     })) { ok = false; break; }
                 xp[0][hf][0][r] = m;
+#pragma unroll
+                for (int i = 0; i < kTopK; ++i) topv[hf][i][r] = tk[i];
                 sync8();
                 m = fmaxf(xp[0][0][0][r], xp[0][1][0][r]);
+                // the pooled values are read from shared memory on every subset pass (they
+                // would otherwise take registers from the whole kernel)
+                auto ysub = [&](int i) { return topv[i / kTopK][i % kTopK][r] - m; };
+                const float u0 = !valid ? -1.0f
+                               : alpha == 1.5f ? subset_start<2 * kTopK, 1>(ysub, alpha)
+                               : alpha == 2.0f ? subset_start<2 * kTopK, 2>(ysub, alpha)
+                                               : subset_start<2 * kTopK, 0>(ysub, alpha);
                 EntmaxSolver sv;
-                sv.init(m, alpha);
+                sv.init(m, alpha, u0);
                 bool done = !valid;
                 // ---- Newton / exact-support passes until every row of the tile is final
                 while (true) {
@@ -589,17 +610,21 @@ cudaError_t launch_coarse_tc(const void* q, const PrefillGeom& g, char* ws, floa
     int* list = reinterpret_cast<int*>(ws + g.off_list);
     int* count = reinterpret_cast<int*>(ws + g.off_count);
     const int grid = g.ntiles < sm_count() ? g.ntiles : sm_count();
+    auto go = [&](auto kernel, int sm) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+        if (e != cudaSuccess) return e;
+        kernel<<<grid, 320, sm, stream>>>(tq, thi, tlo, tau, list, count, hdr, g, alpha, cx);
+        return cudaSuccess;
+    };
+    cudaError_t e;
     if (g.d == 128) {
         const int sm = (int)CtLayout<128>::bytes;
-        cudaError_t e = cudaFuncSetAttribute(coarse_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-        if (e != cudaSuccess) return e;
-        coarse_tc_kernel<128><<<grid, 320, sm, stream>>>(tq, thi, tlo, tau, list, count, hdr, g, alpha, cx);
+        e = go(coarse_tc_kernel<128>, sm);
     } else {
         const int sm = (int)CtLayout<64>::bytes;
-        cudaError_t e = cudaFuncSetAttribute(coarse_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
-        if (e != cudaSuccess) return e;
-        coarse_tc_kernel<64><<<grid, 320, sm, stream>>>(tq, thi, tlo, tau, list, count, hdr, g, alpha, cx);
+        e = go(coarse_tc_kernel<64>, sm);
     }
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -111,6 +111,40 @@ struct EntmaxSolver {
     }
 };
 
+// Start from a subset.  For any subset S of the row, sum_S [y - u]_+^e <= f(u), so the root
+// u_S of the subset's equation lies at or below the row's root: Newton may start there.  With
+// S the row's largest values the start is close (typically one or two passes remain instead
+// of the five to ten from u = -1).
+
+// Keep the K largest values seen, in descending order (registers, static indexing).
+template <int K>
+__device__ __forceinline__ void topk_insert(float (&tk)[K], float v) {
+    if (v > tk[K - 1]) {
+#pragma unroll
+        for (int i = K - 1; i > 0; --i) tk[i] = v > tk[i - 1] ? tk[i - 1] : (v > tk[i] ? v : tk[i]);
+        tk[0] = fmaxf(tk[0], v);
+    }
+}
+
+// Root u_S in shifted units of the subset y(0..N) (values x - m <= 0, -inf ignored; y is an
+// accessor), one thread; MODE as in EntmaxPass::add_t.  Returns a start in [-1, 0) at or
+// below u_S.
+template <int N, int MODE, class Y>
+__device__ __forceinline__ float subset_start(const Y& y, float alpha) {
+    EntmaxSolver sv;
+    sv.init(0.0f, alpha);
+    float t = -1.0f;
+    int nc = 0;
+    for (int it = 0; it < 24; ++it) {
+        EntmaxPass ps;
+        ps.reset();
+#pragma unroll
+        for (int i = 0; i < N; ++i) ps.add_t<MODE>(y(i) - sv.u, sv.e);
+        if (sv.update(ps, &t, &nc)) return (nc || !(t >= -1.0f)) ? sv.lo : fminf(t, -1e-30f);
+    }
+    return sv.lo;
+}
+
 // Whole-row solve through an accessor x(j), j in [0, n): on one thread (WARP = false) or
 // on a whole warp (lanes take j = lane, lane + 32, ...; every lane returns the same value).
 template <bool WARP, class Acc>
