@@ -110,10 +110,11 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     auto kv_addr = [&](int st) { return base + L::off_kv + (uint32_t)st * L::kStage; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int BH = g.B * g.Hkv;
+    // group-major order (longest tiles of a group first): the CTAs in flight share one KV
+    // group, whose K and V stay in L2 while its tiles re-read them
     const int w = blockIdx.x;
-    const int it = g.ntile_bg - 1 - w / BH;
-    const int bg = w % BH;
+    const int bg = w / g.ntile_bg;
+    const int it = g.ntile_bg - 1 - w % g.ntile_bg;
     const int b = bg / g.Hkv, kvh = bg % g.Hkv;
     const int t0 = it * g.P;
     const int bt = t0 / kBlock;
