@@ -86,7 +86,7 @@ struct DecodeGeom {
 };
 
 constexpr int kDecodeChunk = 16;     // list entries (key blocks) per split-KV work item
-constexpr int kDecodeMaxCtas = 256;  // CTAs of the balanced split-KV attention pass
+constexpr int kDecodeMaxCtas = 512;  // CTAs of the balanced split-KV attention pass
 
 inline bool make_decode_geom(int B, int Hq, int Hkv, int Tmax, int d, DecodeGeom* g) {
     if (B < 1 || Hq < 1 || Hkv < 1 || Tmax < 1 || Tmax > kMaxT || (Hq % Hkv) != 0) return false;

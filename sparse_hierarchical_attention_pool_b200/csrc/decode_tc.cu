@@ -19,9 +19,9 @@
 // starts in.
 //
 // Inside a CTA, warp 4 (one lane) streams 32-key halves of the listed blocks (K and V,
-// 128-byte swizzled TMA boxes) into a 12-stage ring; consumer warp w (0-3) takes every 4th
-// half and owns stages w, w + 4 and w + 8, so a stage always returns to the warp that used it
-// before.  A consumer computes the scores transposed, S^T = K Q^T, with mma.sync m16n8k16
+// 128-byte swizzled TMA boxes) into a 4-stage ring; consumer warp w (0-3) takes every 4th
+// half and owns stage w.  Two CTAs share an SM, so one streams while the other sets up or
+// merges.  A consumer computes the scores transposed, S^T = K Q^T, with mma.sync m16n8k16
 // (the 32 keys are the M rows, the G <= 8 heads of the group the N columns), turns them into
 // bf16 weights P^T, transposes those in registers (movmatrix) into the B operand of
 // O^T += V^T P^T, and keeps its own online-softmax state; the four states are merged in
@@ -38,7 +38,7 @@
 
 namespace dash {
 
-constexpr int kDtStages = 12;        // 32-key halves in flight (3 per consumer warp)
+constexpr int kDtStages = 4;         // 32-key halves in flight per CTA (one per consumer warp)
 constexpr int kDtMaxG = 8;           // query heads per KV group handled here (one n8 tile)
 constexpr int kDtKeys = 32;          // keys per pipeline unit
 constexpr int kDtTab = 64;           // list entries staged per table fill
@@ -52,7 +52,7 @@ struct DtLayout {
     static constexpr uint32_t off_kv = 0;
     static constexpr uint32_t off_q = kDtStages * kStage;
     static constexpr uint32_t off_merge = off_q + (D / 64) * kQHalf;
-    // per-warp states [warp][head][2 + D]; reused by the final merge for 2 x 256 x 8 floats
+    // per-warp states [warp][head][2 + D]; reused by the final merge for 2 x kDecodeMaxCtas x 8 floats
     static constexpr uint32_t merge_floats = 4 * kDtMaxG * (D + 2) > 2 * kDecodeMaxCtas * kDtMaxG
                                                  ? 4 * kDtMaxG * (D + 2) : 2 * kDecodeMaxCtas * kDtMaxG;
     static constexpr uint32_t off_tab = off_merge + merge_floats * 4;
@@ -72,7 +72,7 @@ __device__ __forceinline__ int dt_cta_of(long long pos, long long U, int n) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__(160, 2)
 decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const __nv_bfloat16* __restrict__ q, const int* __restrict__ kv_len,
                       const float* __restrict__ xs, const float* __restrict__ tau,
@@ -452,6 +452,7 @@ int decode_tc_ctas() {
     int dev = 0, n = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     if (n < 1) n = 148;
+    n *= 2;                                       // two CTAs per SM (4-stage rings, ~87 KB each)
     return n < kDecodeMaxCtas ? n : kDecodeMaxCtas;
 }
 
