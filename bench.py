@@ -149,35 +149,24 @@ def _num(s):
 
 # ------------------------------------------------------------------ distributed plumbing
 
+_REPLICAS = None
+
+
 def dist_setup(n_gpus):
-    import torch
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if ws > 1:
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
-    elif torch.cuda.is_available():
-        torch.cuda.set_device(0)
-    return ws, rank, local
+    """One process per GPU (independent replicas, see replicas.py): (world, rank, local)."""
+    global _REPLICAS
+    from sparse_hierarchical_attention_pool_b200.replicas import Replicas
+    _REPLICAS = Replicas(timeout_s=300.0)
+    return _REPLICAS.world, _REPLICAS.rank, _REPLICAS.local
 
 
 def barrier(ws):
-    if ws > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    if _REPLICAS is not None:
+        _REPLICAS.barrier()
 
 
 def max_over_ranks(ws, x):
-    if ws == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return x if _REPLICAS is None else _REPLICAS.max(x)
 
 
 # ------------------------------------------------------------------ GPU arms
@@ -523,9 +512,8 @@ def main():
         if rank == 0:
             print(json.dumps(dec), flush=True)
         if ws > 1:
-            import torch.distributed as dist
             barrier(ws)
-            dist.destroy_process_group()
+            _REPLICAS.close()
         return
     pre = bench_prefill(args, ws, rank, local)
     dec = None if args.no_decode else bench_decode(args, ws, rank, local)
@@ -557,9 +545,8 @@ def main():
         }
         print(json.dumps(line), flush=True)
     if ws > 1:
-        import torch.distributed as dist
         barrier(ws)
-        dist.destroy_process_group()
+        _REPLICAS.close()
 
 
 if __name__ == "__main__":
