@@ -124,6 +124,30 @@ DASH_API int dash_prefill_w(const void* q, const void* k, const void* v, const f
                             int B, int Hq, int Hkv, int T, int d, int block, float alpha,
                             float coarse_scale, void* workspace, size_t ws_bytes, dash_stream_t stream);
 
+/* Bytes of workspace dash_prefill_backward needs (0 when the shape is unsupported). */
+DASH_API size_t dash_prefill_backward_workspace_size(int B, int Hq, int Hkv, int T, int d, int block);
+
+/*
+ * Gradients of dash_prefill ("DashAttention: Making Sparse Attention Fully Differentiable
+ * with Adaptive Block Selection", sections "Core Mechanism" and "Key Concepts": the block
+ * selection is differentiable, so gradients flow through the fine softmax, the log prior,
+ * the alpha-entmax Jacobian on the support, the coarse scores and the mean summaries).
+ *   q, k, v    the forward's inputs (device bf16, layouts as dash_prefill);
+ *   out        dash_prefill's output for them (device bf16 [B,Hq,T,d]);
+ *   dout       d loss / d out (device bf16 [B,Hq,T,d]);
+ *   dq         written: d loss / d q  (device bf16 [B,Hq,T,d]);
+ *   dk, dv     written: d loss / d k, d loss / d v (device bf16 [B,Hkv,T,d]), including the
+ *              summary path into every key of a complete block.
+ *   workspace  device, 256-byte aligned, >= dash_prefill_backward_workspace_size(...) bytes;
+ *              the call recomputes the summaries, thresholds and tile lists into it.
+ * Mean-pooled summaries and per-head priors only (the dash_prefill configuration).  The
+ * output is deterministic: no atomics, every gradient element has one writer.
+ */
+DASH_API int dash_prefill_backward(const void* q, const void* k, const void* v, const void* out,
+                                   const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv,
+                                   int T, int d, int block, float alpha, float coarse_scale,
+                                   void* workspace, size_t ws_bytes, dash_stream_t stream);
+
 /* Flags of dash_prefill_ex / dash_decode_ex. */
 #define DASH_HEAD_AGGREGATION 1u
 

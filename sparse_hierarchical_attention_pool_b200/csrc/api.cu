@@ -1,7 +1,8 @@
 // api.cu -- the extern "C" entry points declared in include/dash_attn.h.
 //
 // Argument checks happen here, before any launch; kernels live in summary.cu, coarse.cu,
-// fine_mma.cu, decode.cu and dump.cu.  Nothing here allocates memory.
+// coarse_tc.cu, fine_mma.cu, fine_tc.cu, backward.cu, decode.cu, decode_tc.cu and dump.cu.
+// Nothing here allocates memory.
 #include <math.h>
 
 #include <new>
@@ -137,6 +138,41 @@ int dash_prefill_ex(const void* q, const void* k, const void* v, const float* w_
                     unsigned flags, void* workspace, size_t ws_bytes, dash_stream_t stream) {
     return prefill_impl(q, k, v, out, B, Hq, Hkv, T, d, block, alpha, coarse_scale, workspace,
                         ws_bytes, stream, nullptr, w_summary, flags);
+}
+
+size_t dash_prefill_backward_workspace_size(int B, int Hq, int Hkv, int T, int d, int block) {
+    PrefillGeom g;
+    if (block != kBlock || !make_prefill_geom(B, Hq, Hkv, T, d, &g)) return 0;
+    BwdGeom bw;
+    make_bwd_geom(g, &bw);
+    return bw.total;
+}
+
+int dash_prefill_backward(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                          void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int T, int d, int block,
+                          float alpha, float coarse_scale, void* workspace, size_t ws_bytes,
+                          dash_stream_t stream) {
+    if (!q || !k || !v || !out || !dout || !dq || !dk || !dv) return DASH_ERR_ARG;
+    if (!al16(q) || !al16(k) || !al16(v) || !al16(out) || !al16(dout) || !al16(dq) || !al16(dk) || !al16(dv))
+        return DASH_ERR_ARG;
+    if (!good_params(alpha, coarse_scale)) return DASH_ERR_ARG;
+    PrefillGeom g;
+    if (block != kBlock || !make_prefill_geom(B, Hq, Hkv, T, d, &g)) return DASH_ERR_SHAPE;
+    BwdGeom bw;
+    make_bwd_geom(g, &bw);
+    if (!workspace || !al256(workspace) || ws_bytes < bw.total) return DASH_ERR_WORKSPACE;
+    char* ws = static_cast<char*>(workspace);
+    cudaStream_t s = S(stream);
+    // the forward's Stage 0 and Stage 1 again: summaries, thresholds and tile lists
+    if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), s) != cudaSuccess) return DASH_ERR_CUDA;
+    if (g.nbs > 0 && launch_block_summary(k, reinterpret_cast<float*>(ws + g.off_ksum), B, Hkv, T, d, s,
+                                          ws + g.off_khi, ws + g.off_klo) != cudaSuccess)
+        return DASH_ERR_CUDA;
+    const cudaError_t ce = (g.tc && coarse_tc_supported(g)) ? launch_coarse_tc(q, g, ws, alpha, coarse_scale, s)
+                                                            : launch_coarse(q, g, ws, alpha, coarse_scale, s);
+    if (ce != cudaSuccess) return DASH_ERR_CUDA;
+    return launch_backward(q, k, v, out, dout, dq, dk, dv, g, bw, ws, alpha, coarse_scale, s) == cudaSuccess
+               ? DASH_OK : DASH_ERR_CUDA;
 }
 
 int dash_prefill_profiled(const void* q, const void* k, const void* v, void* out, int B, int Hq,

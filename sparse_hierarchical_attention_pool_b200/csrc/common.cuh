@@ -79,6 +79,21 @@ inline bool make_prefill_geom(int B, int Hq, int Hkv, int T, int d, PrefillGeom*
     return true;
 }
 
+// Workspace of a backward call: the prefill workspace, then per row D = dout . out, the
+// log2-domain log-sum-exp of the fine logits and r = sum_j H_j / sum_j g_j (fp32 each).
+struct BwdGeom {
+    size_t off_drow, off_lse, off_r, total;
+};
+
+inline void make_bwd_geom(const PrefillGeom& g, BwdGeom* bw) {
+    const size_t rows = (size_t)g.B * g.Hq * g.T * sizeof(float);
+    size_t off = g.total;
+    bw->off_drow = off; off = align256(off + rows);
+    bw->off_lse = off;  off = align256(off + rows);
+    bw->off_r = off;    off = align256(off + rows);
+    bw->total = off;
+}
+
 // Geometry of a decode call.
 struct DecodeGeom {
     int B, Hq, Hkv, Tmax, d, G, nbs, chunk, maxchunks;

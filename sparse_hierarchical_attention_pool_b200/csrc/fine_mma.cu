@@ -25,10 +25,6 @@
 
 namespace dash {
 
-// element offset of (row, 16-byte chunk c) in a [rows][D] bf16 tile, chunks XOR-swizzled
-template <int D>
-__device__ __forceinline__ int swz(int row, int c) { return row * D + ((c ^ (row & 7)) << 3); }
-
 template <int D>
 __global__ void __launch_bounds__(256, 1)
 fine_mma_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,

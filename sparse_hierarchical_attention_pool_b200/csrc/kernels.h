@@ -36,6 +36,12 @@ cudaError_t launch_fine_tc(const void* q, const void* k, const void* v, void* ou
                            const PrefillGeom& g, char* ws, float alpha, float coarse_scale,
                            cudaStream_t stream, int agg = 0);
 
+// Gradients of the prefill (dq, dk, dv) after the coarse stage has filled the workspace
+cudaError_t launch_backward(const void* q, const void* k, const void* v, const void* out,
+                            const void* dout, void* dq, void* dk, void* dv, const PrefillGeom& g,
+                            const BwdGeom& bw, char* ws, float alpha, float coarse_scale,
+                            cudaStream_t stream);
+
 cudaError_t launch_select_dump(const void* q, const float* ksum, const long long* rows, int nrows,
                                int max_sel, int* out_idx, float* out_p, int* out_count,
                                float* out_tau, int B, int Hq, int Hkv, int T, int d, float alpha,

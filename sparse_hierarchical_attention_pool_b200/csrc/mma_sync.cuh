@@ -23,6 +23,11 @@ __device__ __forceinline__ void mma_bf16(float* c, const uint32_t* a, uint32_t b
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+// element offset of (row, 16-byte chunk c) in a [rows][D] bf16 tile, chunks XOR-swizzled
+// so that ldmatrix row addresses of one 8x8 matrix fall in distinct bank groups
+template <int D>
+__device__ __forceinline__ int swz(int row, int c) { return row * D + ((c ^ (row & 7)) << 3); }
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);

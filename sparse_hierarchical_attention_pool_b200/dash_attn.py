@@ -28,7 +28,7 @@ EXPORTS = ("dash_status_string", "dash_version", "dash_block_summary", "dash_pre
            "dash_prefill_tau", "dash_select_dump", "dash_decode_workspace_size", "dash_decode",
            "dash_get_device_status", "dash_prefill_profiled", "dash_decode_profiled",
            "dash_decode_noalloc", "dash_block_summary_w", "dash_prefill_w", "dash_prefill_ex",
-           "dash_decode_ex")
+           "dash_decode_ex", "dash_prefill_backward_workspace_size", "dash_prefill_backward")
 
 HEAD_AGGREGATION = 1       # flag of dash_prefill_ex / dash_decode_ex
 
@@ -71,6 +71,9 @@ def lib():
     L.dash_decode_ex.argtypes = [_p] * 6 + [_i] * 6 + [_f, _f, ctypes.c_uint, _p, _sz, _p]
     L.dash_prefill_workspace_size.argtypes = [_i] * 6
     L.dash_prefill_workspace_size.restype = _sz
+    L.dash_prefill_backward_workspace_size.argtypes = [_i] * 6
+    L.dash_prefill_backward_workspace_size.restype = _sz
+    L.dash_prefill_backward.argtypes = [_p] * 8 + [_i] * 6 + [_f, _f, _p, _sz, _p]
     L.dash_prefill.argtypes = [_p] * 4 + [_i] * 6 + [_f, _f, _p, _sz, _p]
     L.dash_prefill_host.argtypes = [_p] * 8 + [_i] * 6 + [_f, _f, _p, _sz, _p]
     L.dash_prefill_stats.argtypes = [_p, _sz, ctypes.POINTER(dash_stats), _p]
@@ -85,7 +88,8 @@ def lib():
     L.dash_decode_profiled.argtypes = [_p] * 6 + [_i] * 6 + [_f, _f, _p, _sz, _p, _p]
     L.dash_decode_noalloc.argtypes = [_p] * 6 + [_i] * 6 + [_f, _f, _p]
     for name in EXPORTS:
-        if name not in ("dash_status_string", "dash_prefill_workspace_size", "dash_decode_workspace_size"):
+        if name not in ("dash_status_string", "dash_prefill_workspace_size", "dash_decode_workspace_size",
+                        "dash_prefill_backward_workspace_size"):
             getattr(L, name).restype = _i
     _lib = L
     return L
@@ -142,6 +146,13 @@ def prefill_workspace_size(B, Hq, Hkv, T, d, block=64) -> int:
     n = lib().dash_prefill_workspace_size(B, Hq, Hkv, T, d, block)
     if n == 0:
         raise DashError("dash_prefill_workspace_size", -2)
+    return n
+
+
+def prefill_backward_workspace_size(B, Hq, Hkv, T, d, block=64) -> int:
+    n = lib().dash_prefill_backward_workspace_size(B, Hq, Hkv, T, d, block)
+    if n == 0:
+        raise DashError("dash_prefill_backward_workspace_size", -2)
     return n
 
 
@@ -373,3 +384,29 @@ def dash_decode_noalloc(q, k_cache, v_cache, ksum, kv_len, out=None, alpha=1.5, 
 
 def dash_get_device_status(workspace, stream=None) -> int:
     return lib().dash_get_device_status(ctypes.c_void_p(workspace.data_ptr()), _stream(stream))
+
+
+def dash_prefill_backward(q, k, v, out, dout, alpha=1.5, coarse_scale=1.0, dq=None, dk=None, dv=None,
+                          workspace=None, block=64, stream=None):
+    """Gradients of dash_prefill: (dq, dk, dv) for d loss / d out = dout.  `out` is the
+    forward's output for (q, k, v, alpha, coarse_scale)."""
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, T, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Hkv, T, d] matching q")
+    if out.shape != q.shape or dout.shape != q.shape:
+        raise ValueError("out and dout must be [B, Hq, T, d]")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = prefill_backward_workspace_size(B, Hq, Hkv, T, d, block)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    rc = lib().dash_prefill_backward(
+        _dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"), _dev(v, torch.bfloat16, "v"),
+        _dev(out, torch.bfloat16, "out"), _dev(dout, torch.bfloat16, "dout"), _dev(dq, torch.bfloat16, "dq"),
+        _dev(dk, torch.bfloat16, "dk"), _dev(dv, torch.bfloat16, "dv"), B, Hq, Hkv, T, d, block,
+        float(alpha), float(coarse_scale), ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
+        _stream(stream))
+    _check("dash_prefill_backward", rc)
+    return dq, dk, dv

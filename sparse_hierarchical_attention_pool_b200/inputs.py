@@ -104,6 +104,11 @@ def topic_prefill(B, Hq, Hkv, T, d, block, n_topics, seed, fp32_source=False, co
     return q, k, v
 
 
+def out_grad(B, Hq, T, d, seed):
+    """Upstream gradient d loss / d out [B, Hq, T, d]: N(0, 1) drawn in fp32, rounded to bf16."""
+    return torch.randn(B, Hq, T, d, generator=_gen(seed)).bfloat16()
+
+
 def topic_decode(B, Hq, Hkv, Tmax, d, block, n_topics, seed):
     """Decode step inputs: q [B,Hq,d], caches k, v [B,Hkv,Tmax,d] (bf16, CPU), kv_len [B].
 
