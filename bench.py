@@ -295,8 +295,59 @@ def bench_prefill(args, ws, rank, local):
     res["e2e"] = {"value": ws * B * T / (e2e_step * 1e-3), "unit": "tok/s",
                   "h2d_bytes_per_step": q.numel() * 2 + k.numel() * 2 + v.numel() * 2,
                   "d2h_bytes_per_step": q.numel() * 2, "ms_per_step": e2e_step}
+    if not args.no_backward:
+        res["backward"] = bench_backward(args, ws, qd, kd, vd, out, wl, cs, st, fine_alg, fine_exec, flush)
     del flush, wsb
     return res
+
+
+def bench_backward(args, ws, qd, kd, vd, out, wl, cs, st, fine_alg, fine_exec, flush):
+    """Gradients of the same prefill (dash_prefill_backward: coarse stage again, then the
+    D, query-major and key-major kernels) for an N(0, 1) upstream gradient."""
+    import torch
+    from sparse_hierarchical_attention_pool_b200 import dash_attn as da
+    from sparse_hierarchical_attention_pool_b200 import inputs
+    B, Hq, Hkv, T, d = wl.B, wl.Hq, wl.Hkv, wl.T, wl.d
+    da.dash_prefill(qd, kd, vd, out, wl.alpha, cs)
+    dout = inputs.out_grad(B, Hq, T, d, seed=wl.seed + 1).cuda()
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    bws = da.alloc_workspace(da.prefill_backward_workspace_size(B, Hq, Hkv, T, d))
+    for _ in range(args.warmup):
+        flush()
+        da.dash_prefill_backward(qd, kd, vd, out, dout, wl.alpha, cs, dq, dk, dv, bws)
+    torch.cuda.synchronize()
+    barrier(ws)
+    n = max(3, min(args.steps, 10))
+    evs = []
+    for _ in range(n):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        da.dash_prefill_backward(qd, kd, vd, out, dout, wl.alpha, cs, dq, dk, dv, bws)
+        e1.record()
+        evs.append((e0, e1))
+    torch.cuda.synchronize()
+    ms = max_over_ranks(ws, sum(a.elapsed_time(b) for a, b in evs) / n)
+    if da.dash_get_device_status(bws) != 0 or not all(bool(torch.isfinite(t).all()) for t in (dq, dk, dv)):
+        raise RuntimeError("backward: device status not clean or non-finite gradients")
+    pk, pk_kind = peaks()
+    # five products per (row, key) at minimum (S again, dP, dV, dK, dQ): 2.5x the forward's
+    # four-flop-per-d count; the kernels execute eight 2 d products per (row, key) of the
+    # tiles' unions (S twice and dP in the query-major kernel, S and dP again in the
+    # key-major one, plus dQ, dV, dK)
+    alg = 2.5 * fine_alg
+    exe = 4.0 * fine_exec
+    ach = alg / (ms * 1e-3) / 1e12
+    return {"ms": round(ms, 4), "tok_s": ws * B * T / (ms * 1e-3), "steps": n,
+            "kernels": ["block_summary_kernel", "coarse_tc_kernel", "bwd_rowdot_kernel", "bwd_dq_kernel",
+                        "bwd_dkv_kernel"],
+            "roofline": {"bound": "tensor", "achieved": round(ach, 2), "peak": pk["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": round(ach / pk["bf16_tflops"], 4),
+                         "peak_source": f"{pk_kind} bf16_tflops (burst)",
+                         "algorithmic_flops": alg, "executed_flops": exe,
+                         "executed_tflops": round(exe / (ms * 1e-3) / 1e12, 2),
+                         "note": "mma.sync m16n8k16 kernels (legacy tensor path)"},
+            "l2": "flushed before every timed call"}
 
 
 def bench_decode(args, ws, rank, local):
@@ -490,6 +541,7 @@ def main():
     ap.add_argument("--workload", default="16k", choices=["16k", "32k", "96k", "16k-coherent"],
                     help="16k-coherent is not a target workload: block-coherent query topics")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-backward", action="store_true", help="skip the prefill backward measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the decode step and print its object (for profiling runs)")
@@ -541,6 +593,7 @@ def main():
             "summary_roofline": pre["summary_roofline"],
             "context": pre["context"],
             "prefill_stats": pre["stats"],
+            "backward": pre.get("backward"),
             "decode": dec,
         }
         print(json.dumps(line), flush=True)

@@ -423,11 +423,17 @@ bwd_dkv_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
     int* mtp = reinterpret_cast<int*>(mr + 2 * kTileRows);           // [2][128]
     float* xs = reinterpret_cast<float*>(mtp + 2 * kTileRows);       // [4][128] partial row sums
     float* cl = xs + 4 * kTileRows;                                  // [4][128]
-    int* tl = reinterpret_cast<int*>(cl + 4 * kTileRows);            // [kBwdChunk]
+    float* lps = cl + 4 * kTileRows;                                 // [128] log2 prior - lse
+    float* xms = lps + kTileRows;                                    // [128] x_j - tau
+    float* fs = xms + kTileRows;                                     // [128] cs ds_j / 64
+    int* tl = reinterpret_cast<int*>(fs + kTileRows);                // [kBwdChunk]
     int* wtot = tl + kBwdChunk;                                      // [8]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int kw = warp & 3, rb = (warp >> 2) * 64;   // this warp: keys 16 kw.., rows rb..rb+63
+    const int th = tid & 127;                         // thread index within the row half
+    // the four warps of one row half (warps 4 (rb / 64) .. +3) synchronise on barrier 1 + rb / 64
+    auto half_bar = [&]() { asm volatile("bar.sync %0, 128;" :: "r"(1 + (rb >> 6)) : "memory"); };
     const int g4 = lane >> 2, t4 = lane & 3;
     const int BH = g.B * g.Hkv;
     const int j = blockIdx.x / BH;                    // low blocks (most listing tiles) first
@@ -570,38 +576,39 @@ bwd_dkv_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
                     mma_bf16(st[2 * np + 1], a, b2, b3);
                 }
             }
-            if (!diag) {
-                col_partial(st, xs);
-                __syncthreads();
-            }
-            // log2 prior of every row this thread touches (rows rb + 8n + 2t4 + e)
-            float lp2[8][2];
-#pragma unroll
-            for (int n = 0; n < 8; ++n)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int row = rb + n * 8 + 2 * t4 + e;
-                    const int tp = tp_s[row];
-                    if (diag) {
-                        lp2[n][e] = tp >= 0 ? 0.f : -INFINITY;
-                    } else {
-                        const float x = (xs[row] + xs[kTileRows + row] + xs[2 * kTileRows + row] +
-                                         xs[3 * kTileRows + row]) * C.cxm;
-                        const float xm = x - mtau[stage * kTileRows + row];
-                        lp2[n][e] = (tp >= 0 && xm > 0.f) ? C.e_pow * __log2f(xm) : -INFINITY;
-                    }
+            // per-row values, once per row: the 64 threads th < 64 of each row half own
+            // rows rb + th; the half's four warps meet at a named barrier of 128 threads
+            if (!diag) col_partial(st, xs);
+            half_bar();
+            if (th < 64) {
+                const int row = rb + th;
+                const int tp = tp_s[row];
+                float lp = tp >= 0 ? 0.f : -INFINITY, xm = 1.f;
+                if (!diag) {
+                    const float x = (xs[row] + xs[kTileRows + row] + xs[2 * kTileRows + row] +
+                                     xs[3 * kTileRows + row]) * C.cxm;
+                    xm = x - mtau[stage * kTileRows + row];
+                    lp = (tp >= 0 && xm > 0.f) ? C.e_pow * __log2f(xm) : -INFINITY;
                 }
+                lps[row] = lp - mlse[stage * kTileRows + row];
+                xms[row] = xm;
+            }
+            half_bar();
             // P^T in st
             const int key0 = j * kBlock + kw * 16 + g4;
 #pragma unroll
             for (int n = 0; n < 8; ++n)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int e = c & 1;
+                for (int e = 0; e < 2; ++e) {
                     const int row = rb + n * 8 + 2 * t4 + e;
-                    float l2 = fmaf(st[n][c], C.sm2, lp2[n][e]);
-                    if (diag && key0 + (c >> 1) * 8 > tp_s[row]) l2 = -INFINITY;
-                    st[n][c] = exp2f(l2 - mlse[stage * kTileRows + row]);
+                    const float lp = lps[row];
+                    const int tp = diag ? tp_s[row] : 0x7fffffff;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float l2 = fmaf(st[n][e + 2 * hh], C.sm2, lp);
+                        if (key0 + hh * 8 > tp) l2 = -INFINITY;
+                        st[n][e + 2 * hh] = exp2f(l2);
+                    }
                 }
             // dV += P^T dout
 #pragma unroll
@@ -643,29 +650,33 @@ bwd_dkv_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
 #pragma unroll
             for (int n = 0; n < 8; ++n)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int row = rb + n * 8 + 2 * t4 + (c & 1);
-                    dpt[n][c] = st[n][c] * (dpt[n][c] - mdrow[stage * kTileRows + row]);
+                for (int e = 0; e < 2; ++e) {
+                    const float dr = mdrow[stage * kTileRows + rb + n * 8 + 2 * t4 + e];
+                    dpt[n][e] = st[n][e] * (dpt[n][e] - dr);
+                    dpt[n][e + 2] = st[n][e + 2] * (dpt[n][e + 2] - dr);
                 }
             if (!diag) {
                 // c_j per row over all 64 keys, then the folded cs ds_j / 64
                 col_partial(dpt, cl);
-                __syncthreads();
+                half_bar();
+                if (th < 64) {
+                    const int row = rb + th;
+                    float f = 0.f;
+                    if (lps[row] > -INFINITY) {
+                        const float xm = xms[row];
+                        const float c = cl[row] + cl[kTileRows + row] + cl[2 * kTileRows + row] +
+                                        cl[3 * kTileRows + row];
+                        const float gj = exp2f(C.gpow * __log2f(xm));
+                        f = C.cs64 * (c / xm - mr[stage * kTileRows + row] * gj);
+                    }
+                    fs[row] = f;
+                }
+                half_bar();
 #pragma unroll
                 for (int n = 0; n < 8; ++n)
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int row = rb + n * 8 + 2 * t4 + e;
-                        float f = 0.f;
-                        if (lp2[n][e] > -INFINITY) {
-                            const float x = (xs[row] + xs[kTileRows + row] + xs[2 * kTileRows + row] +
-                                             xs[3 * kTileRows + row]) * C.cxm;
-                            const float xm = x - mtau[stage * kTileRows + row];
-                            const float c = cl[row] + cl[kTileRows + row] + cl[2 * kTileRows + row] +
-                                            cl[3 * kTileRows + row];
-                            const float gj = exp2f(C.gpow * __log2f(xm));
-                            f = C.cs64 * (c / xm - mr[stage * kTileRows + row] * gj);
-                        }
+                        const float f = fs[rb + n * 8 + 2 * t4 + e];
                         dpt[n][e] += f;
                         dpt[n][2 + e] += f;
                     }
@@ -735,9 +746,10 @@ bwd_dkv_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
 static size_t bwd_dq_smem(int d) {
     return (size_t)(2 * kTileRows + 4 * kBlock) * d * 2 + (size_t)kTileRows * d * 4; }
 // K, V of the block and two stages of Q and dout tiles (bf16); per-row data of two stages
-// (log-sum-exp, D, tau, r, position) and the two cross-warp row-sum buffers; the tile list
+// (log-sum-exp, D, tau, r, position), the two cross-warp row-sum buffers, three per-row
+// values of the current tile and the tile list
 static size_t bwd_dkv_smem(int d) {
-    return (size_t)(2 * kBlock + 4 * kTileRows) * d * 2 + (size_t)(5 * 2 + 2 * 4) * kTileRows * 4 +
+    return (size_t)(2 * kBlock + 4 * kTileRows) * d * 2 + (size_t)(5 * 2 + 2 * 4 + 3) * kTileRows * 4 +
            (size_t)(kBwdChunk + 8) * 4;
 }
 
