@@ -252,7 +252,7 @@ def bench_prefill(args, ws, rank, local):
     G = Hq // Hkv
     fine_kernel = "fine_tc_kernel" if G <= 16 else "fine_mma_kernel"
     traffic = (recorded_traffic("fine_tc_kernel", source_sha("fine_tc.cu", "sm100.cuh", "common.cuh"))
-               if G <= 16 else recorded_traffic("fine_mma_kernel", source_sha("fine_mma.cu", "common.cuh")))
+               if G <= 16 else recorded_traffic("fine_mma_kernel", source_sha("fine_mma.cu", "mma_sync.cuh", "common.cuh")))
     res = {
         "step_ms": step_ms,
         "tok_s": ws * B * T / (step_ms * 1e-3),
@@ -299,6 +299,26 @@ def bench_prefill(args, ws, rank, local):
         res["backward"] = bench_backward(args, ws, qd, kd, vd, out, wl, cs, st, fine_alg, fine_exec, flush)
     del flush, wsb
     return res
+
+
+def backward_only(args, ws):
+    """The backward measurement alone on the prefill workload (for profiling runs)."""
+    import torch
+    from sparse_hierarchical_attention_pool_b200 import dash_attn as da
+    from sparse_hierarchical_attention_pool_b200 import inputs
+    wl, (q, k, v) = inputs.make(args.workload)
+    cs = calibrated(args.workload)["coarse_scale"]
+    B, Hq, Hkv, T, d = wl.B, wl.Hq, wl.Hkv, wl.T, wl.d
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    out = torch.empty_like(qd)
+    wsb = da.alloc_workspace(da.prefill_workspace_size(B, Hq, Hkv, T, d))
+    da.dash_prefill(qd, kd, vd, out, wl.alpha, cs, wsb)
+    st = da.dash_prefill_stats(wsb)
+    diag_tokens = sum((t % 64) + 1 for t in range(T)) * B * Hq
+    fine_alg = 4.0 * d * (64.0 * st["selected_pairs"] + diag_tokens)
+    P = min(64, 1 << (max(1, 128 // (Hq // Hkv)).bit_length() - 1))
+    fine_exec = 4.0 * d * 64.0 * 128.0 * (st["union_blocks"] + B * Hkv * ((T + P - 1) // P))
+    return bench_backward(args, ws, qd, kd, vd, out, wl, cs, st, fine_alg, fine_exec, L2Flush())
 
 
 def bench_backward(args, ws, qd, kd, vd, out, wl, cs, st, fine_alg, fine_exec, flush):
@@ -427,7 +447,8 @@ def bench_decode(args, ws, rank, local):
     pk, pk_kind = peaks()
     attn_gbs = gathered / (st_ms[1] * 1e-3) / 1e9
     step_gbs = (gathered + other) / (tot * 1e-3) / 1e9
-    traffic = recorded_traffic("decode_attn_tc_kernel", source_sha("decode_tc.cu", "common.cuh"))
+    traffic = recorded_traffic("decode_attn_tc_kernel",
+                               source_sha("decode_tc.cu", "mma_sync.cuh", "sm100.cuh", "common.cuh"))
     # end to end: the new query goes up, the graph runs, the output comes back (the cache
     # stays resident)
     qh, oh = q.pin_memory(), torch.empty_like(q).pin_memory()
@@ -542,6 +563,8 @@ def main():
                     help="16k-coherent is not a target workload: block-coherent query topics")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the prefill backward measurement")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only the prefill backward and print its object (for profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the decode step and print its object (for profiling runs)")
@@ -559,6 +582,14 @@ def main():
     if rank == 0:
         _b.build()
     barrier(ws)
+    if args.backward_only:
+        bwd = backward_only(args, ws)
+        if rank == 0:
+            print(json.dumps(bwd), flush=True)
+        if ws > 1:
+            barrier(ws)
+            _REPLICAS.close()
+        return
     if args.decode_only:
         dec = bench_decode(args, ws, rank, local)
         if rank == 0:
