@@ -36,6 +36,8 @@
 // with fp32 accumulators; K/V (query-major) or Q/dout (key-major) tiles stream through a
 // two-stage cp.async ring in XOR-swizzled shared memory.
 #include <math.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -756,7 +758,8 @@ static size_t bwd_dkv_smem(int d) {
 template <int D>
 static cudaError_t launch_bwd_d(const void* q, const void* k, const void* v, const void* out,
                                 const void* dout, void* dq, void* dk, void* dv, const PrefillGeom& g,
-                                const BwdGeom& bw, char* ws, const BwdConsts& C, cudaStream_t stream) {
+                                const BwdGeom& bw, char* ws, const BwdConsts& C, bool tc, float alpha,
+                                float coarse_scale, cudaStream_t stream) {
     const auto* qb = static_cast<const __nv_bfloat16*>(q);
     const auto* kb = static_cast<const __nv_bfloat16*>(k);
     const auto* vb = static_cast<const __nv_bfloat16*>(v);
@@ -775,12 +778,16 @@ static cudaError_t launch_bwd_d(const void* q, const void* k, const void* v, con
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
-    const size_t sm1 = bwd_dq_smem(D);
-    e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
-    if (e != cudaSuccess) return e;
-    bwd_dq_kernel<D><<<g.ntiles, 256, sm1, stream>>>(qb, kb, vb, gb, drow, tau, list, count, ksum,
-                                                     static_cast<__nv_bfloat16*>(dq), lse, rr, g, C);
-    e = cudaGetLastError();
+    if (tc) {
+        e = launch_bwd_dq_tc(q, k, v, dout, dq, g, bw, ws, alpha, coarse_scale, stream);
+    } else {
+        const size_t sm1 = bwd_dq_smem(D);
+        e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
+        if (e != cudaSuccess) return e;
+        bwd_dq_kernel<D><<<g.ntiles, 256, sm1, stream>>>(qb, kb, vb, gb, drow, tau, list, count, ksum,
+                                                         static_cast<__nv_bfloat16*>(dq), lse, rr, g, C);
+        e = cudaGetLastError();
+    }
     if (e != cudaSuccess) return e;
 
     const size_t sm2 = bwd_dkv_smem(D);
@@ -791,6 +798,17 @@ static cudaError_t launch_bwd_d(const void* q, const void* k, const void* v, con
         qb, kb, vb, gb, drow, tau, lse, rr, list, count, static_cast<__nv_bfloat16*>(dk),
         static_cast<__nv_bfloat16*>(dv), g, C);
     return cudaGetLastError();
+}
+
+// Which query-major kernel runs: the tcgen05 pair (backward_tc.cu) wherever the tile holds
+// at least 8 positions, unless DASH_BWD_KERNEL=mma selects the mma.sync kernel above (kept
+// for comparison and for more than 16 query heads per KV head).
+static bool use_mma_backward() {
+    static const int choice = [] {
+        const char* e = getenv("DASH_BWD_KERNEL");
+        return (e && strcmp(e, "mma") == 0) ? 1 : 0;
+    }();
+    return choice == 1;
 }
 
 cudaError_t launch_backward(const void* q, const void* k, const void* v, const void* out,
@@ -806,8 +824,9 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
     C.cs64 = coarse_scale / (float)kBlock;
     C.cs = coarse_scale;
     C.isd = 1.0f / sd;
-    return g.d == 128 ? launch_bwd_d<128>(q, k, v, out, dout, dq, dk, dv, g, bw, ws, C, stream)
-                      : launch_bwd_d<64>(q, k, v, out, dout, dq, dk, dv, g, bw, ws, C, stream);
+    const bool tc = fine_tc_supported(g) && !use_mma_backward();
+    return g.d == 128 ? launch_bwd_d<128>(q, k, v, out, dout, dq, dk, dv, g, bw, ws, C, tc, alpha, coarse_scale, stream)
+                      : launch_bwd_d<64>(q, k, v, out, dout, dq, dk, dv, g, bw, ws, C, tc, alpha, coarse_scale, stream);
 }
 
 }  // namespace dash

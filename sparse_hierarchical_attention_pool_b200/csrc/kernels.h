@@ -42,6 +42,11 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
                             const BwdGeom& bw, char* ws, float alpha, float coarse_scale,
                             cudaStream_t stream);
 
+// tcgen05 variant of the backward's query-major half (statistics, then dq); needs P >= 8
+cudaError_t launch_bwd_dq_tc(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                             const PrefillGeom& g, const BwdGeom& bw, char* ws, float alpha, float coarse_scale,
+                             cudaStream_t stream);
+
 cudaError_t launch_select_dump(const void* q, const float* ksum, const long long* rows, int nrows,
                                int max_sel, int* out_idx, float* out_p, int* out_count,
                                float* out_tau, int B, int Hq, int Hkv, int T, int d, float alpha,
