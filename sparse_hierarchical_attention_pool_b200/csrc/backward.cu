@@ -790,6 +790,7 @@ static cudaError_t launch_bwd_d(const void* q, const void* k, const void* v, con
     }
     if (e != cudaSuccess) return e;
 
+    if (tc) return launch_bwd_dkv_tc(q, k, v, dout, dk, dv, g, bw, ws, alpha, coarse_scale, stream);
     const size_t sm2 = bwd_dkv_smem(D);
     e = cudaFuncSetAttribute(bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
     if (e != cudaSuccess) return e;
@@ -800,9 +801,9 @@ static cudaError_t launch_bwd_d(const void* q, const void* k, const void* v, con
     return cudaGetLastError();
 }
 
-// Which query-major kernel runs: the tcgen05 pair (backward_tc.cu) wherever the tile holds
-// at least 8 positions, unless DASH_BWD_KERNEL=mma selects the mma.sync kernel above (kept
-// for comparison and for more than 16 query heads per KV head).
+// Which kernels run: the tcgen05 ones (backward_tc.cu: statistics, dq, then dk/dv) wherever
+// the tile holds at least 8 positions, unless DASH_BWD_KERNEL=mma selects the mma.sync
+// kernels above (kept for comparison and for more than 16 query heads per KV head).
 static bool use_mma_backward() {
     static const int choice = [] {
         const char* e = getenv("DASH_BWD_KERNEL");

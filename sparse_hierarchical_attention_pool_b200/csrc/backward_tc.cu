@@ -421,6 +421,410 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (tid == 0 && abort_sh) atomicOr(&hdr->status, kStWaitTimeout);
 }
 
+// ------------------------------------------------------------------ key-major: dk, dv
+//
+// One CTA per (b, KV head, pair of key blocks j0 = 2 jp, j1 = 2 jp + 1): the 128 keys of
+// the pair are the M dimension of the dk and dv products.  The steps are the work tiles
+// whose own block is j0 or j1 or whose list holds j0 or j1, ascending; each carries, per
+// block, whether the block is the tile's own block (causal), a listed past block, or
+// neither (nothing to add).  Per step:
+//   S  = Q [K_j0; K_j1]^T    (M = 128 rows, N = 128 keys)   rows in TMEM lanes, so the
+//   dP = dout [V_j0; V_j1]^T                                 per-row block sums (x_j from
+//                                                            S, c_j from dS) stay in-thread
+//   dV += P^T dout, dK += (dS + cs ds_j / 64)^T Q  (M = 128 keys, N = d, K = 128 rows):
+//        P and dS are written row-major ([row][key], bf16) and read as MN-major A.
+// Warps: 8 producer (the pair's K and V once; per step the Q and dout tiles into a
+// two-stage ring; it also finds the steps: each lane tests one candidate tile -- own block,
+// or a binary search of the tile's sorted list -- and a warp ballot keeps them in order;
+// a sentinel step ends the loop), 9 S/dP issuer, 10 dK/dV issuer, 0-7 softmax (thread =
+// (row, block of the pair): warp w serves TMEM lanes 32 (w % 4).. and block w / 4).
+// P and dS share one buffer: dS is written once dV has read P.
+template <int D>
+struct BkLayout {
+    static constexpr uint32_t kHalf = 128 * 128;                // 128 rows x 64 bf16 (one swizzle column)
+    static constexpr uint32_t kT = (D / 64) * kHalf;            // a 128-row [rows][D] tile
+    static constexpr uint32_t off_k = 0;                        // K of the pair [128 keys][D]
+    static constexpr uint32_t off_v = kT;
+    static constexpr uint32_t off_ring = 2 * kT;                // stage: Q tile, dout tile
+    static constexpr uint32_t kStage = 2 * kT;
+    static constexpr uint32_t off_buf = off_ring + 2 * kStage;  // P / dS [2 key halves][128 rows][64]
+    static constexpr uint32_t bytes = off_buf + 2 * kHalf + 1024;
+    static constexpr uint32_t colS = 0, colDP = 128, colDV = 256, colDK = 256 + D;
+};
+
+enum : int { BK_KV = 0, BK_QF = 1, BK_QE = 3, BK_S_FULL = 5, BK_S_FREE = 6, BK_P_FULL = 7, BK_DV_DONE = 8,
+             BK_DS_FULL = 9, BK_DK_DONE = 10, BK_DRAIN = 11, BK_DRAIN2 = 12, BK_COUNT = 13 };
+enum : int { kModeNone = 0, kModePast = 1, kModeDiag = 2 };
+
+// kind::f16 instruction descriptor with either operand MN-major (bit 15: A, bit 16: B)
+__host__ __device__ constexpr uint32_t idesc_bf16_ab(int M, int N, bool a_mn, bool b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16)
+         | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+struct BkConsts {
+    float cxm;     // (alpha-1) cs / sqrt(d) / 64: row sum of S over a block -> x_j
+    float e_pow, gpow, sm2, cs64, isd;
+};
+
+template <int D>
+__global__ void __launch_bounds__(352, 1)
+bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv,
+                  const float* __restrict__ lse, const float* __restrict__ rrow, const float* __restrict__ drow,
+                  const float* __restrict__ tau, const int* __restrict__ list, const int* __restrict__ count,
+                  WsHeader* __restrict__ hdr, PrefillGeom g, BkConsts C) {
+    using L = BkLayout<D>;
+    using namespace sm100;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t bars[BK_COUNT];
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+    __shared__ int info_sh[2];                 // per ring stage: tile | mode0 << 24 | mode1 << 26, or -1
+
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* const base_ptr = smem_raw + (base - raw);
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
+    auto q_addr = [&](int st) { return base + L::off_ring + (uint32_t)st * L::kStage; };
+    auto do_addr = [&](int st) { return base + L::off_ring + (uint32_t)st * L::kStage + L::kT; };
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int BH = g.B * g.Hkv;
+    const int jp = blockIdx.x / BH;            // low pairs (listed by the most tiles) first
+    const int bg = blockIdx.x % BH;
+    const int b = bg / g.Hkv, kvh = bg % g.Hkv;
+    const int nb = (g.T + kBlock - 1) / kBlock;
+    const int j0 = 2 * jp, j1 = 2 * jp + 1;
+    const bool has1 = j1 < nb;
+
+    if (tid == 0) {
+        abort_sh = 0;
+        mbar_init(bar(BK_KV), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar(BK_QF + i), 1);
+            mbar_init(bar(BK_QE + i), 1);
+        }
+        mbar_init(bar(BK_S_FULL), 1);
+        mbar_init(bar(BK_S_FREE), 256);
+        mbar_init(bar(BK_P_FULL), 256);
+        mbar_init(bar(BK_DV_DONE), 1);
+        mbar_init(bar(BK_DS_FULL), 256);
+        mbar_init(bar(BK_DK_DONE), 1);
+        mbar_init(bar(BK_DRAIN), 1);
+        mbar_init(bar(BK_DRAIN2), 1);
+        fence_mbar_init();
+    }
+    // rows of the Q and dout tiles beyond G * P are never loaded: zero them in both stages
+    if (g.M < kTileRows && tid < kTileRows && tid >= g.M) {
+        for (int st = 0; st < 2; ++st)
+            for (int h = 0; h < 2 * (D / 64); ++h) {
+                uint4* p = reinterpret_cast<uint4*>(base_ptr + L::off_ring + st * L::kStage + h * L::kHalf + tid * 128);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) p[c] = make_uint4(0u, 0u, 0u, 0u);
+            }
+    }
+    fence_proxy_async_smem();
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&tmem_base_sh), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+    volatile int* abort_flag = &abort_sh;
+
+    if (warp == 8) {
+        // ------------------------------------------------------------ producer and step finder
+        if (lane == 0) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_do);
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+            // K and V of the pair; a missing second block reads rows that are never used
+            // (finite data of the next rows, or zeros past the end of the tensor)
+            mbar_arrive_expect_tx(bar(BK_KV), (uint32_t)(4 * kBlock * D * 2));
+            for (int h = 0; h < D / 64; ++h)
+                for (int jb = 0; jb < 2; ++jb) {
+                    const int row = bg * g.T + (j0 + jb) * kBlock;
+                    tma_load_2d(base + L::off_k + h * L::kHalf + jb * 64 * 128, &tm_k, h * 64, row, bar(BK_KV));
+                    tma_load_2d(base + L::off_v + h * L::kHalf + jb * 64 * 128, &tm_v, h * 64, row, bar(BK_KV));
+                }
+        }
+        const int it_first = j0 * kBlock / g.P;
+        int s = 0;
+        bool ok = true;
+        int armed[2] = {-1, -1};
+        for (int c0 = it_first; ok && c0 < g.ntile_bg; c0 += 32) {
+            const int it = c0 + lane;
+            int info = -1;
+            if (it < g.ntile_bg) {
+                const int bt = it * g.P / kBlock;
+                int m0 = bt == j0 ? kModeDiag : kModeNone;
+                int m1 = (has1 && bt == j1) ? kModeDiag : kModeNone;
+                if (bt > j0) {
+                    const size_t tile = (size_t)bg * g.ntile_bg + it;
+                    const int* Lst = list + tile * g.cap;
+                    const int cnt = count[tile];
+                    int lo = 0, hi = cnt;              // first entry >= j0
+                    while (lo < hi) {
+                        const int mid = (lo + hi) >> 1;
+                        if (Lst[mid] < j0) lo = mid + 1; else hi = mid;
+                    }
+                    if (lo < cnt && Lst[lo] == j0) { m0 = kModePast; ++lo; }
+                    if (has1 && bt > j1 && lo < cnt && Lst[lo] == j1) m1 = kModePast;
+                }
+                if (m0 != kModeNone || m1 != kModeNone) info = it | (m0 << 24) | (m1 << 26);
+            }
+            unsigned keep = __ballot_sync(0xffffffffu, info >= 0);
+            while (keep) {
+                const int src = __ffs(keep) - 1;
+                keep &= keep - 1;
+                const int inf = __shfl_sync(0xffffffffu, info, src);
+                if (lane == 0) {
+                    const int st = s & 1;
+                    if (s >= 2 && !mbar_wait(bar(BK_QE + st), ((s >> 1) - 1) & 1, abort_flag)) ok = false;
+                    if (ok) {
+                        const int t0 = (inf & 0xFFFFFF) * g.P;
+                        info_sh[st] = inf;
+                        mbar_arrive_expect_tx(bar(BK_QF + st), (uint32_t)(2 * g.M * D * 2));
+                        for (int hl = 0; hl < g.G; ++hl) {
+                            const int row = (b * g.Hq + kvh * g.G + hl) * g.T + t0;
+                            for (int h = 0; h < D / 64; ++h) {
+                                tma_load_2d(q_addr(st) + h * L::kHalf + hl * g.P * 128, &tm_q, h * 64, row, bar(BK_QF + st));
+                                tma_load_2d(do_addr(st) + h * L::kHalf + hl * g.P * 128, &tm_do, h * 64, row, bar(BK_QF + st));
+                            }
+                        }
+                        armed[st] = s;
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                ++s;
+                if (!ok) break;
+            }
+        }
+        if (lane == 0) {
+            // the sentinel step: consumers see -1 and leave their loops
+            const int st = s & 1;
+            if (ok && s >= 2 && !mbar_wait(bar(BK_QE + st), ((s >> 1) - 1) & 1, abort_flag)) ok = false;
+            if (ok) {
+                info_sh[st] = -1;
+                mbar_arrive(bar(BK_QF + st));
+            } else {
+                *abort_flag = 1;
+                volatile int dummy = 0;
+                mbar_wait(bar(BK_KV), 0, &dummy);
+                for (int st2 = 0; st2 < 2; ++st2)
+                    if (armed[st2] >= 0) { dummy = 0; mbar_wait(bar(BK_QF + st2), (armed[st2] >> 1) & 1, &dummy); }
+            }
+        }
+    } else if (warp == 9) {
+        // ------------------------------------------------------------ S and dP issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_ab(128, 128, false, false);
+            bool ok = mbar_wait(bar(BK_KV), 0, abort_flag);
+            for (int s = 0; ok; ++s) {
+                const int st = s & 1;
+                if (!mbar_wait(bar(BK_QF + st), (s >> 1) & 1, abort_flag)) { ok = false; break; }
+                if (info_sh[st] < 0) break;
+                if (s >= 1 && !mbar_wait(bar(BK_S_FREE), (s - 1) & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int h = kk >> 2, wk = kk & 3;
+                    const uint64_t a = smem_desc_sw128(q_addr(st) + h * L::kHalf + wk * 32, 16, 1024);
+                    const uint64_t bk = smem_desc_sw128(base + L::off_k + h * L::kHalf + wk * 32, 16, 1024);
+                    mma_bf16_ss(tmem + L::colS, a, bk, idesc, kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int h = kk >> 2, wk = kk & 3;
+                    const uint64_t a = smem_desc_sw128(do_addr(st) + h * L::kHalf + wk * 32, 16, 1024);
+                    const uint64_t bv = smem_desc_sw128(base + L::off_v + h * L::kHalf + wk * 32, 16, 1024);
+                    mma_bf16_ss(tmem + L::colDP, a, bv, idesc, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar(BK_S_FULL));
+            }
+            if (!ok) {
+                mma_commit(bar(BK_DRAIN));
+                volatile int dummy = 0;
+                mbar_wait(bar(BK_DRAIN), 0, &dummy);
+            }
+        }
+    } else if (warp == 10) {
+        // ------------------------------------------------------------ dV and dK issuer
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_ab(128, D, true, true);
+            bool ok = true;
+            for (int s = 0; ok; ++s) {
+                const int st = s & 1;
+                if (!mbar_wait(bar(BK_QF + st), (s >> 1) & 1, abort_flag)) { ok = false; break; }
+                if (info_sh[st] < 0) break;
+                if (!mbar_wait(bar(BK_P_FULL), s & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t a = smem_desc_sw128(base + L::off_buf + kk * 2048, L::kHalf, 1024);
+                    const uint64_t bo = smem_desc_sw128(do_addr(st) + kk * 2048, L::kHalf, 1024);
+                    mma_bf16_ss(tmem + L::colDV, a, bo, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(bar(BK_DV_DONE));
+                if (!mbar_wait(bar(BK_DS_FULL), s & 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t a = smem_desc_sw128(base + L::off_buf + kk * 2048, L::kHalf, 1024);
+                    const uint64_t bq = smem_desc_sw128(q_addr(st) + kk * 2048, L::kHalf, 1024);
+                    mma_bf16_ss(tmem + L::colDK, a, bq, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(bar(BK_DK_DONE));
+                mma_commit(bar(BK_QE + st));
+            }
+            if (!ok) {
+                mma_commit(bar(BK_DRAIN2));
+                volatile int dummy = 0;
+                mbar_wait(bar(BK_DRAIN2), 0, &dummy);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ softmax: (row, block)
+        const int quarter = warp & 3, kb = warp >> 2;
+        const int r = quarter * 32 + lane;
+        const int jb = j0 + kb;
+        const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
+        uint8_t* const brow = base_ptr + L::off_buf + kb * L::kHalf + (r >> 3) * 1024 + (r & 7) * 128;
+        const int hl = r / g.P;
+        bool ok = true;
+        int nsteps = 0;
+        auto wwait = [&](uint32_t bar_addr, uint32_t parity) -> bool {
+            const bool got = mbar_wait(bar_addr, parity, abort_flag);
+            return __all_sync(0xffffffffu, got);
+        };
+        for (int s = 0;; ++s) {
+            const int st = s & 1;
+            if (!wwait(bar(BK_QF + st), (s >> 1) & 1)) { ok = false; break; }
+            const int inf = info_sh[st];
+            if (inf < 0) break;
+            const int it = inf & 0xFFFFFF;
+            const int mode = (inf >> (24 + 2 * kb)) & 3;
+            const int t0 = it * g.P;
+            const int t = t0 + r % g.P;
+            const bool valid = r < g.M && t < g.T;
+            const int tpos = valid ? t : -1;
+            const size_t rowid = valid ? (size_t)(b * g.Hq + kvh * g.G + hl) * g.T + t : 0;
+            const float lse_r = valid ? lse[rowid] : 0.f;
+            const float d_r = valid ? drow[rowid] : 0.f;
+            const float rr = valid ? rrow[rowid] : 0.f;
+            const float tau_r = (valid && mode == kModePast) ? tau[rowid] : INFINITY;
+            if (!wwait(bar(BK_S_FULL), s & 1)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t sr[64];
+            tmem_ld<64>(lane_addr + L::colS + kb * 64, sr);
+            tmem_wait_ld();
+            float lp2 = -INFINITY, xm = 1.f;
+            if (mode == kModeDiag) {
+                lp2 = tpos >= 0 ? 0.f : -INFINITY;
+#pragma unroll
+                for (int i = 0; i < 64; ++i)
+                    if (jb * kBlock + i > tpos) sr[i] = __float_as_uint(-INFINITY);
+            } else if (mode == kModePast) {
+                float rs = 0.f;
+#pragma unroll
+                for (int i = 0; i < 64; ++i) rs += __uint_as_float(sr[i]);
+                xm = rs * C.cxm - tau_r;
+                if (tpos >= 0 && xm > 0.f) lp2 = C.e_pow * __log2f(xm);
+            }
+            const bool sel = mode == kModePast && lp2 > -INFINITY;
+            const float c0 = lp2 - lse_r;
+            uint32_t pk[32];
+            float cj = 0.f;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t dp[32];
+                tmem_ld<32>(lane_addr + L::colDP + kb * 64 + hh * 32, dp);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    const float p0 = exp2f(fmaf(__uint_as_float(sr[hh * 32 + i]), C.sm2, c0));
+                    const float p1 = exp2f(fmaf(__uint_as_float(sr[hh * 32 + i + 1]), C.sm2, c0));
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                    pk[(hh * 32 + i) >> 1] = *reinterpret_cast<uint32_t*>(&h2);
+                    const float d0 = p0 * (__uint_as_float(dp[i]) - d_r);
+                    const float d1 = p1 * (__uint_as_float(dp[i + 1]) - d_r);
+                    sr[hh * 32 + i] = __float_as_uint(d0);
+                    sr[hh * 32 + i + 1] = __float_as_uint(d1);
+                    cj += d0 + d1;
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar(BK_S_FREE));
+            const float f = sel ? C.cs64 * (cj / xm - rr * exp2f(C.gpow * __log2f(xm))) : 0.f;
+            // the buffer was last read by the previous step's dK product
+            if (s >= 1 && !wwait(bar(BK_DK_DONE), (s - 1) & 1)) { ok = false; break; }
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4*>(brow + ((c ^ (r & 7)) << 4)) =
+                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar(BK_P_FULL));
+            if (!wwait(bar(BK_DV_DONE), s & 1)) { ok = false; break; }
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int q2 = 0; q2 < 4; ++q2) {
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(sr[c * 8 + 2 * q2]) + f,
+                                                              __uint_as_float(sr[c * 8 + 2 * q2 + 1]) + f);
+                    w4[q2] = *reinterpret_cast<uint32_t*>(&h2);
+                }
+                *reinterpret_cast<uint4*>(brow + ((c ^ (r & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar(BK_DS_FULL));
+            nsteps = s + 1;
+        }
+        // ---- epilogue: warps 0-3 store dV, warps 4-7 dK of key lane 32 (warp % 4) + lane
+        if (ok && nsteps > 0 && wwait(bar(BK_DK_DONE), (nsteps - 1) & 1)) {
+            tc_fence_after();
+            const int key = quarter * 32 + lane;           // 0..127 over the pair
+            const int tok = (j0 + (key >> 6)) * kBlock + (key & 63);
+            const bool kval = tok < g.T;
+            const uint32_t col = kb == 0 ? L::colDV : L::colDK;
+            const float scale = kb == 0 ? 1.f : C.isd;
+            __nv_bfloat16* dst = kval ? (kb == 0 ? dv : dk) + ((size_t)bg * g.T + tok) * D : nullptr;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld<32>(lane_addr + col + c * 32, o);
+                tmem_wait_ld();
+                if (kval) {
+                    uint32_t w4[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(o[2 * i]) * scale,
+                                                                  __uint_as_float(o[2 * i + 1]) * scale);
+                        w4[i] = *reinterpret_cast<uint32_t*>(&h2);
+                    }
+                    uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w4[4 * i], w4[4 * i + 1], w4[4 * i + 2], w4[4 * i + 3]);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+    if (tid == 0 && abort_sh) atomicOr(&hdr->status, kStWaitTimeout);
+}
+
 // ------------------------------------------------------------------ host side
 
 namespace {
@@ -495,6 +899,44 @@ cudaError_t launch_bwd_dq_tc(const void* q, const void* k, const void* v, const 
         if (e == cudaSuccess) e = go(bwd_tc_kernel<64, 1>, (int)BtLayout<64, 1>::bytes);
     }
     return e;
+}
+
+cudaError_t launch_bwd_dkv_tc(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv,
+                              const PrefillGeom& g, const BwdGeom& bw, char* ws, float alpha, float coarse_scale,
+                              cudaStream_t stream) {
+    BkConsts C;
+    const float sd = sqrtf((float)g.d);
+    C.cxm = (alpha - 1.0f) * coarse_scale / sd / (float)kBlock;
+    C.e_pow = 1.0f / (alpha - 1.0f);
+    C.gpow = (2.0f - alpha) / (alpha - 1.0f);
+    C.sm2 = 1.4426950408889634f / sd;
+    C.cs64 = coarse_scale / (float)kBlock;
+    C.isd = 1.0f / sd;
+    CUtensorMap tq, tdo, tk, tv;
+    const unsigned long long qrows = (unsigned long long)g.B * g.Hq * g.T;
+    const unsigned long long kvrows = (unsigned long long)g.B * g.Hkv * g.T;
+    if (!make_map_bt(&tq, q, qrows, g.d, g.P) || !make_map_bt(&tdo, dout, qrows, g.d, g.P) ||
+        !make_map_bt(&tk, k, kvrows, g.d, kBlock) || !make_map_bt(&tv, v, kvrows, g.d, kBlock))
+        return cudaErrorInvalidValue;
+    const float* lse = reinterpret_cast<const float*>(ws + bw.off_lse);
+    const float* rr = reinterpret_cast<const float*>(ws + bw.off_r);
+    const float* drow = reinterpret_cast<const float*>(ws + bw.off_drow);
+    const float* tau = reinterpret_cast<const float*>(ws + g.off_tau);
+    const int* list = reinterpret_cast<const int*>(ws + g.off_list);
+    const int* count = reinterpret_cast<const int*>(ws + g.off_count);
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
+    const int nb = (g.T + kBlock - 1) / kBlock;
+    const int grid = g.B * g.Hkv * ((nb + 1) / 2);
+    auto* dkb = static_cast<__nv_bfloat16*>(dk);
+    auto* dvb = static_cast<__nv_bfloat16*>(dv);
+    auto go = [&](auto kernel, int sm) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+        if (e != cudaSuccess) return e;
+        kernel<<<grid, 352, sm, stream>>>(tq, tdo, tk, tv, dkb, dvb, lse, rr, drow, tau, list, count, hdr, g, C);
+        return cudaGetLastError();
+    };
+    return g.d == 128 ? go(bwd_dkv_tc_kernel<128>, (int)BkLayout<128>::bytes)
+                      : go(bwd_dkv_tc_kernel<64>, (int)BkLayout<64>::bytes);
 }
 
 }  // namespace dash

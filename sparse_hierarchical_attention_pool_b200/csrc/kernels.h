@@ -47,6 +47,11 @@ cudaError_t launch_bwd_dq_tc(const void* q, const void* k, const void* v, const 
                              const PrefillGeom& g, const BwdGeom& bw, char* ws, float alpha, float coarse_scale,
                              cudaStream_t stream);
 
+// tcgen05 variant of the backward's key-major half (dk, dv over pairs of key blocks)
+cudaError_t launch_bwd_dkv_tc(const void* q, const void* k, const void* v, const void* dout, void* dk, void* dv,
+                              const PrefillGeom& g, const BwdGeom& bw, char* ws, float alpha, float coarse_scale,
+                              cudaStream_t stream);
+
 cudaError_t launch_select_dump(const void* q, const float* ksum, const long long* rows, int nrows,
                                int max_sel, int* out_idx, float* out_p, int* out_count,
                                float* out_tau, int B, int Hq, int Hkv, int T, int d, float alpha,
