@@ -352,21 +352,23 @@ def bench_backward(args, ws, qd, kd, vd, out, wl, cs, st, fine_alg, fine_exec, f
         raise RuntimeError("backward: device status not clean or non-finite gradients")
     pk, pk_kind = peaks()
     # five products per (row, key) at minimum (S again, dP, dV, dK, dQ): 2.5x the forward's
-    # four-flop-per-d count; the kernels execute eight 2 d products per (row, key) of the
-    # tiles' unions (S twice and dP in the query-major kernel, S and dP again in the
-    # key-major one, plus dQ, dV, dK)
+    # four-flop-per-d count.  The tcgen05 kernels execute nine 2 d products per (row, key)
+    # of the tiles' unions (S and dP in the statistics pass, S, dP and dQ in the dq pass,
+    # S, dP, dV and dK in the key-major pass), 4.5x the forward's executed count; the
+    # summary columns of S and the blocks a key-block pair carries for its partner are
+    # not counted
     alg = 2.5 * fine_alg
-    exe = 4.0 * fine_exec
+    exe = 4.5 * fine_exec
     ach = alg / (ms * 1e-3) / 1e12
     return {"ms": round(ms, 4), "tok_s": ws * B * T / (ms * 1e-3), "steps": n,
-            "kernels": ["block_summary_kernel", "coarse_tc_kernel", "bwd_rowdot_kernel", "bwd_dq_kernel",
-                        "bwd_dkv_kernel"],
+            "kernels": ["block_summary_kernel", "coarse_tc_kernel", "bwd_rowdot_kernel",
+                        "bwd_tc_kernel<statistics>", "bwd_tc_kernel<dq>", "bwd_dkv_tc_kernel"],
             "roofline": {"bound": "tensor", "achieved": round(ach, 2), "peak": pk["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": round(ach / pk["bf16_tflops"], 4),
                          "peak_source": f"{pk_kind} bf16_tflops (burst)",
                          "algorithmic_flops": alg, "executed_flops": exe,
                          "executed_tflops": round(exe / (ms * 1e-3) / 1e12, 2),
-                         "note": "mma.sync m16n8k16 kernels (legacy tensor path)"},
+                         "note": "tcgen05 kernels (TMEM accumulators, TMA rings)"},
             "l2": "flushed before every timed call"}
 
 

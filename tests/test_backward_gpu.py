@@ -155,3 +155,28 @@ def test_backward_argument_errors():
         da.dash_prefill_backward(q, k, k, q, q, alpha=1.0)
     with pytest.raises(ValueError):
         da.dash_prefill_backward(q, k, k, q[:, :1], q)
+
+
+def test_mma_sync_backward_matches_oracle():
+    """The mma.sync kernels (forced with DASH_BWD_KERNEL=mma, read once per process, hence
+    the child process) give the same gradients as the tcgen05 ones, within the tolerance."""
+    import json
+    import subprocess
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = (
+        "import sys, json, numpy as np\n"
+        f"sys.path.insert(0, {root!r}); sys.path.insert(0, {os.path.join(root, 'tests')!r})\n"
+        "import oracle\n"
+        "from sparse_hierarchical_attention_pool_b200 import dash_attn as da, inputs\n"
+        "_, (q, k, v) = inputs.make('16k', B=1, Hq=8, Hkv=2, T=900, d=128, n_topics=8, seed=17)\n"
+        "dout = inputs.out_grad(1, 8, 900, 128, seed=18)\n"
+        "out, _ = da.dash_prefill(q.cuda(), k.cuda(), v.cuda(), alpha=1.5, coarse_scale=0.3)\n"
+        "g = da.dash_prefill_backward(q.cuda(), k.cuda(), v.cuda(), out, dout.cuda(), alpha=1.5, coarse_scale=0.3)\n"
+        "ref = oracle.backward(q, k, v, dout, 64, 1.5, 0.3)\n"
+        "print(json.dumps([float(np.linalg.norm(a.double().cpu().numpy() - r) / np.linalg.norm(r))\n"
+        "                  for a, r in zip(g, ref)]))\n")
+    env = dict(os.environ, DASH_BWD_KERNEL="mma")
+    res = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
+    assert res.returncode == 0, res.stderr[-2000:]
+    errs = json.loads(res.stdout.strip().splitlines()[-1])
+    assert max(errs) <= REL_NORM, errs
