@@ -118,11 +118,13 @@ def test_coarse_path_carries_gradient():
         assert err <= REL_NORM, (name, err)
 
 
-@pytest.mark.parametrize("Hq,Hkv,T,d", [(4, 2, 128, 128), (8, 1, 100, 64)])
+@pytest.mark.parametrize("Hq,Hkv,T,d", [(4, 2, 128, 128), (8, 1, 100, 64), (4, 2, 17, 128), (8, 2, 64, 128),
+                                         (2, 1, 65, 64)])
 def test_two_blocks_is_dense_causal_backward(Hq, Hkv, T, d):
     """With T <= 128 every row has at most one past block: its entmax weight is 1, the
     prior is log 1 = 0 and a one-element entmax has a zero Jacobian, so the gradients are
-    those of dense causal softmax attention (torch autograd in fp64 on the CPU)."""
+    those of dense causal softmax attention (torch autograd in fp64 on the CPU).  Includes
+    T < 64 (no complete block), exactly one block, and one block plus a token."""
     B = 1
     _, (q, k, v) = inputs.make("16k", B=B, Hq=Hq, Hkv=Hkv, T=T, d=d, n_topics=8, seed=90 + T)
     dout = inputs.out_grad(B, Hq, T, d, seed=91)
