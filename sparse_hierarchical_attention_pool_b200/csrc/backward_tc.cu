@@ -30,10 +30,6 @@
 // Operands: Q, dout, K, V (for S and dP) and dS K-major; K (for dq) MN-major; 128-byte
 // swizzle everywhere (TMA writes it).  Every wait is bounded (~2 s); a CTA that gives up
 // sets a status bit, lets its copies and products finish, frees TMEM and exits.
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -827,36 +823,6 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
 // ------------------------------------------------------------------ host side
 
-namespace {
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn_bt() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-// 2-D map over a [rows, d] bf16 matrix, boxes of 64 columns x box_rows rows, 128-byte swizzle
-bool make_map_bt(CUtensorMap* m, const void* ptr, unsigned long long rows, int d, int box_rows) {
-    auto fn = encode_fn_bt();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1u, 1u};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-}  // namespace
-
 cudaError_t launch_bwd_dq_tc(const void* q, const void* k, const void* v, const void* dout, void* dq,
                              const PrefillGeom& g, const BwdGeom& bw, char* ws, float alpha, float coarse_scale,
                              cudaStream_t stream) {
@@ -872,9 +838,9 @@ cudaError_t launch_bwd_dq_tc(const void* q, const void* k, const void* v, const 
     const unsigned long long qrows = (unsigned long long)g.B * g.Hq * g.T;
     const unsigned long long kvrows = (unsigned long long)g.B * g.Hkv * g.T;
     const unsigned long long srows = (unsigned long long)g.B * g.Hkv * (g.nbs > 0 ? g.nbs : 1);
-    if (!make_map_bt(&tq, q, qrows, g.d, g.P) || !make_map_bt(&tdo, dout, qrows, g.d, g.P) ||
-        !make_map_bt(&tk, k, kvrows, g.d, kBlock) || !make_map_bt(&tv, v, kvrows, g.d, kBlock) ||
-        !make_map_bt(&thi, ws + g.off_khi, srows, g.d, 8) || !make_map_bt(&tlo, ws + g.off_klo, srows, g.d, 8))
+    if (!make_tmap_bf16(&tq, q, qrows, g.d, g.P) || !make_tmap_bf16(&tdo, dout, qrows, g.d, g.P) ||
+        !make_tmap_bf16(&tk, k, kvrows, g.d, kBlock) || !make_tmap_bf16(&tv, v, kvrows, g.d, kBlock) ||
+        !make_tmap_bf16(&thi, ws + g.off_khi, srows, g.d, 8) || !make_tmap_bf16(&tlo, ws + g.off_klo, srows, g.d, 8))
         return cudaErrorInvalidValue;
     float* lse = reinterpret_cast<float*>(ws + bw.off_lse);
     float* rr = reinterpret_cast<float*>(ws + bw.off_r);
@@ -915,8 +881,8 @@ cudaError_t launch_bwd_dkv_tc(const void* q, const void* k, const void* v, const
     CUtensorMap tq, tdo, tk, tv;
     const unsigned long long qrows = (unsigned long long)g.B * g.Hq * g.T;
     const unsigned long long kvrows = (unsigned long long)g.B * g.Hkv * g.T;
-    if (!make_map_bt(&tq, q, qrows, g.d, g.P) || !make_map_bt(&tdo, dout, qrows, g.d, g.P) ||
-        !make_map_bt(&tk, k, kvrows, g.d, kBlock) || !make_map_bt(&tv, v, kvrows, g.d, kBlock))
+    if (!make_tmap_bf16(&tq, q, qrows, g.d, g.P) || !make_tmap_bf16(&tdo, dout, qrows, g.d, g.P) ||
+        !make_tmap_bf16(&tk, k, kvrows, g.d, kBlock) || !make_tmap_bf16(&tv, v, kvrows, g.d, kBlock))
         return cudaErrorInvalidValue;
     const float* lse = reinterpret_cast<const float*>(ws + bw.off_lse);
     const float* rr = reinterpret_cast<const float*>(ws + bw.off_r);

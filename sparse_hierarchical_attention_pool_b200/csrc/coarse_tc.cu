@@ -29,9 +29,6 @@
 // reads TMEM.  Longer tiles recompute their score chunks for every pass; the threshold
 // warps tell the producer and the MMA issuer after each pass whether another is needed.
 // Every wait is bounded (~2 s); a CTA that gives up sets a status bit and exits cleanly.
-#include <cudaTypedefs.h>
-
-#include <mutex>
 #include <type_traits>
 
 #include "common.cuh"
@@ -560,31 +557,6 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
 namespace {
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn_ct() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-bool make_map_ct(CUtensorMap* m, const void* ptr, unsigned long long rows, int d, int box_rows) {
-    auto fn = encode_fn_ct();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1u, 1u};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 int sm_count() {
     int dev = 0, n = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -601,9 +573,9 @@ cudaError_t launch_coarse_tc(const void* q, const PrefillGeom& g, char* ws, floa
     CUtensorMap tq, thi, tlo;
     const unsigned long long qrows = (unsigned long long)g.B * g.Hq * g.T;
     const unsigned long long krows = (unsigned long long)g.B * g.Hkv * g.nbs;
-    if (!make_map_ct(&tq, q, qrows, g.d, g.P) ||
-        !make_map_ct(&thi, ws + g.off_khi, krows, g.d, kCtChunk) ||
-        !make_map_ct(&tlo, ws + g.off_klo, krows, g.d, kCtChunk))
+    if (!make_tmap_bf16(&tq, q, qrows, g.d, g.P) ||
+        !make_tmap_bf16(&thi, ws + g.off_khi, krows, g.d, kCtChunk) ||
+        !make_tmap_bf16(&tlo, ws + g.off_klo, krows, g.d, kCtChunk))
         return cudaErrorInvalidValue;
     WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
     float* tau = reinterpret_cast<float*>(ws + g.off_tau);

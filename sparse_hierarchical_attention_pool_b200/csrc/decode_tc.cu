@@ -27,10 +27,6 @@
 // O^T += V^T P^T, and keeps its own online-softmax state; the four states are merged in
 // shared memory at the end of every segment.  Block indices and log-priors of the segment
 // are staged in shared memory 64 entries at a time.
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
 #include "common.cuh"
 #include "kernels.h"
 #include "mma_sync.cuh"
@@ -417,35 +413,6 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
     if (tid == 0 && *abort_flag) atomicOr(&hdr->status, kStWaitTimeout);
 }
 
-namespace {
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn_dt() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult qr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
-            qr == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-bool make_map_dt(CUtensorMap* m, const void* ptr, unsigned long long rows, int d) {
-    auto fn = encode_fn_dt();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    cuuint32_t box[2] = {64u, (cuuint32_t)kDtKeys};
-    cuuint32_t estr[2] = {1u, 1u};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-}  // namespace
-
 bool decode_tc_supported(const DecodeGeom& g) { return g.G <= kDtMaxG && (g.d == 64 || g.d == 128); }
 
 int decode_tc_ctas() {
@@ -462,7 +429,7 @@ cudaError_t launch_decode_attn_tc(const void* q, const void* kc, const void* vc,
     if (nctas < 1 || nctas > kDecodeMaxCtas) return cudaErrorInvalidValue;
     CUtensorMap tk, tv;
     const unsigned long long rows = (unsigned long long)g.B * g.Hkv * g.Tmax;
-    if (!make_map_dt(&tk, kc, rows, g.d) || !make_map_dt(&tv, vc, rows, g.d)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16(&tk, kc, rows, g.d, kDtKeys) || !make_tmap_bf16(&tv, vc, rows, g.d, kDtKeys)) return cudaErrorInvalidValue;
     const float* xs = reinterpret_cast<const float*>(ws + g.off_x);
     const float* tau = reinterpret_cast<const float*>(ws + g.off_tau);
     const int* list = reinterpret_cast<const int*>(ws + g.off_list);

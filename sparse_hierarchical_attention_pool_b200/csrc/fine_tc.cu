@@ -37,10 +37,6 @@
 // through shared memory (one group barrier per step) and share log of the mean as prior.
 // Operands: Q, K, P K-major and V MN-major, all 128-byte swizzled (TMA writes that layout).
 // Every wait is bounded (~2 s); a CTA that gives up sets a status bit and exits cleanly.
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -482,36 +478,6 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
 // ------------------------------------------------------------------ host side
 
-namespace {
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-// 2-D map over a [rows, d] bf16 matrix, boxes of 64 columns x box_rows rows, 128-byte swizzle
-bool make_map(CUtensorMap* m, const void* ptr, unsigned long long rows, int d, int box_rows) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1u, 1u};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-}  // namespace
-
 bool fine_tc_supported(const PrefillGeom& g) { return g.P >= 8 && (g.d == 64 || g.d == 128); }
 
 cudaError_t launch_fine_tc(const void* q, const void* k, const void* v, void* out, const PrefillGeom& g,
@@ -525,9 +491,9 @@ cudaError_t launch_fine_tc(const void* q, const void* k, const void* v, void* ou
     // block summaries as bf16 hi / lo [B * Hkv * nbs, d] (at least one row: with no complete
     // block every tile has only its own block and the summary columns are never read)
     const unsigned long long srows = (unsigned long long)g.B * g.Hkv * (g.nbs > 0 ? g.nbs : 1);
-    if (!make_map(&tq, q, qrows, g.d, g.P) || !make_map(&tk, k, kvrows, g.d, kBlock) ||
-        !make_map(&tv, v, kvrows, g.d, kBlock) || !make_map(&thi, ws + g.off_khi, srows, g.d, 8) ||
-        !make_map(&tlo, ws + g.off_klo, srows, g.d, 8))
+    if (!make_tmap_bf16(&tq, q, qrows, g.d, g.P) || !make_tmap_bf16(&tk, k, kvrows, g.d, kBlock) ||
+        !make_tmap_bf16(&tv, v, kvrows, g.d, kBlock) || !make_tmap_bf16(&thi, ws + g.off_khi, srows, g.d, 8) ||
+        !make_tmap_bf16(&tlo, ws + g.off_klo, srows, g.d, 8))
         return cudaErrorInvalidValue;
     const float* tau = reinterpret_cast<const float*>(ws + g.off_tau);
     const int* list = reinterpret_cast<const int*>(ws + g.off_list);

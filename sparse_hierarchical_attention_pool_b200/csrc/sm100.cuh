@@ -18,6 +18,12 @@
 #include "common.cuh"
 
 namespace dash {
+
+// Host: 2-D TMA map over a row-major [rows, d] bf16 matrix, boxes of 64 columns x box_rows
+// rows, 128-byte swizzle, zero fill out of bounds (tmap.cu).  False if the encoder is missing
+// or rejects the arguments (base 16-byte aligned, d * 2 a multiple of 16).
+bool make_tmap_bf16(CUtensorMap* m, const void* ptr, unsigned long long rows, int d, int box_rows);
+
 namespace sm100 {
 
 // ------------------------------------------------------------------ mbarriers
