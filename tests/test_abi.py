@@ -102,3 +102,32 @@ def test_product_never_imports_the_oracle():
                 src = open(os.path.join(dirpath, fn)).read()
                 assert "import oracle" not in src and "from oracle" not in src, fn
                 assert "dash_oracle" not in src, fn
+
+
+def test_backward_workspace_and_argument_errors(L):
+    from sparse_hierarchical_attention_pool_b200 import dash_attn as da
+    B, Hq, Hkv, T, d = 1, 16, 2, 16384, 128
+    fwd = da.prefill_workspace_size(B, Hq, Hkv, T, d)
+    bwd = da.prefill_backward_workspace_size(B, Hq, Hkv, T, d)
+    # the forward's workspace plus three fp32 values per row (D, log-sum-exp, r)
+    assert bwd >= fwd + 3 * B * Hq * T * 4
+    assert L.dash_prefill_backward_workspace_size(1, 16, 3, 16384, 128, 64) == 0
+    assert L.dash_prefill_backward_workspace_size(1, 16, 2, 16384, 128, 32) == 0
+    f = ctypes.c_void_p
+    fake = f(1 << 20)
+    big = 1 << 30
+    args = [fake] * 8 + [1, 2, 1, 256, 64, 64, 1.5, 1.0, fake, big, None]
+
+    def call(**over):
+        a = list(args)
+        for i, v in over.items():
+            a[int(i[1:])] = v
+        return L.dash_prefill_backward(*a)
+
+    assert call(a4=None) == -1                        # dout null
+    assert call(a7=f((1 << 20) + 8)) == -1            # dv misaligned
+    assert call(a14=1.0) == -1                        # alpha <= 1
+    assert call(a9=3, a10=2) == -2                    # Hq % Hkv
+    assert call(a13=32) == -2                         # block
+    assert call(a16=None) == -5                       # workspace null
+    assert call(a17=16) == -5                         # workspace too small
