@@ -83,7 +83,7 @@ DASH_API int dash_block_summary(const void* k, float* ksum, int B, int Hkv, int 
 /*
  * Stage 0 with a learned summary head ("DashAttention and the year sparse attention became
  * a field", section "What alpha-entmax changes": the chunk summary is a small attention
- * head, initialised at zero so that training starts from mean pooling).  Attention pooling
+ * head whose zero initialisation makes it the block mean).  Attention pooling
  * with one query vector per KV head:
  *   ksum[b, g, j, :] = sum_i a_i k[b, g, j*block + i, :],  a = softmax_i(w[g] . k_i / sqrt(d))
  * over the block's keys; w = 0 gives the mean of dash_block_summary (up to rounding).

@@ -8,7 +8,7 @@
  * What it computes, and where the pages define it:
  *   [P1] "DashAttention: Making Sparse Attention Fully Differentiable with Adaptive
  *        Block Selection" (alanhou.org), section "Core Mechanism" (the two-stage
- *        diagram: divide K,V into blocks; coarse scores Q * block_summary; alpha-entmax
+ *        diagram: keys and values cut into fixed blocks; coarse scores Q * block_summary; alpha-entmax
  *        gives sparse block weights p; fine logits Q * K_block plus log(p); softmax;
  *        weighted sum of V) and section "Key Concepts" (alpha-entmax; alpha=1 is
  *        softmax, alpha=2 is sparsemax; higher alpha is sparser; hierarchical prior).
