@@ -311,7 +311,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const float e = exp2f(__uint_as_float(sr[hh * 32 + i]) - m_use);
+                        const float e = fast_exp2(__uint_as_float(sr[hh * 32 + i]) - m_use);
                         ls += e;
                         ch = fmaf(e, __uint_as_float(dp[i]) - drow_r, ch);
                     }
@@ -333,7 +333,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const float p = exp2f(fmaf(__uint_as_float(sr[hh * 32 + i]), C.sm2, c0));
+                        const float p = fast_exp2(fmaf(__uint_as_float(sr[hh * 32 + i]), C.sm2, c0));
                         const float ds = p * (__uint_as_float(dp[i]) - drow_r);
                         sr[hh * 32 + i] = __float_as_uint(ds);
                         cj += ds;
@@ -743,8 +743,8 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
-                    const float p0 = exp2f(fmaf(__uint_as_float(sr[hh * 32 + i]), C.sm2, c0));
-                    const float p1 = exp2f(fmaf(__uint_as_float(sr[hh * 32 + i + 1]), C.sm2, c0));
+                    const float p0 = fast_exp2(fmaf(__uint_as_float(sr[hh * 32 + i]), C.sm2, c0));
+                    const float p1 = fast_exp2(fmaf(__uint_as_float(sr[hh * 32 + i + 1]), C.sm2, c0));
                     __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
                     pk[(hh * 32 + i) >> 1] = *reinterpret_cast<uint32_t*>(&h2);
                     const float d0 = p0 * (__uint_as_float(dp[i]) - d_r);
