@@ -59,14 +59,15 @@ def source_sha(*names):
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel, sha):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel is unchanged since."""
+def recorded_traffic(kernel, sha, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on this workload
+    and the kernel is unchanged since."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f).get(kernel)
-    if not d or d.get("source_sha256_16") != sha:
+    if not d or d.get("source_sha256_16") != sha or d.get("workload_key") != workload:
         return None
     return d.get("traffic_bytes_per_launch")
 
@@ -251,8 +252,9 @@ def bench_prefill(args, ws, rank, local):
                "note": "library dense attention on the same inputs, for context only"}
     G = Hq // Hkv
     fine_kernel = "fine_tc_kernel" if G <= 16 else "fine_mma_kernel"
-    traffic = (recorded_traffic("fine_tc_kernel", source_sha("fine_tc.cu", "sm100.cuh", "common.cuh"))
-               if G <= 16 else recorded_traffic("fine_mma_kernel", source_sha("fine_mma.cu", "mma_sync.cuh", "common.cuh")))
+    traffic = (recorded_traffic("fine_tc_kernel", source_sha("fine_tc.cu", "sm100.cuh", "common.cuh"), args.workload)
+               if G <= 16 else recorded_traffic("fine_mma_kernel", source_sha("fine_mma.cu", "mma_sync.cuh", "common.cuh"),
+                                                args.workload))
     res = {
         "step_ms": step_ms,
         "tok_s": ws * B * T / (step_ms * 1e-3),
@@ -450,7 +452,8 @@ def bench_decode(args, ws, rank, local):
     attn_gbs = gathered / (st_ms[1] * 1e-3) / 1e9
     step_gbs = (gathered + other) / (tot * 1e-3) / 1e9
     traffic = recorded_traffic("decode_attn_tc_kernel",
-                               source_sha("decode_tc.cu", "mma_sync.cuh", "sm100.cuh", "common.cuh"))
+                               source_sha("decode_tc.cu", "mma_sync.cuh", "sm100.cuh", "common.cuh"),
+                               f"decode96k-b{B}")
     # end to end: the new query goes up, the graph runs, the output comes back (the cache
     # stays resident)
     qh, oh = q.pin_memory(), torch.empty_like(q).pin_memory()
