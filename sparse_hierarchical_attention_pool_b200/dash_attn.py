@@ -410,3 +410,31 @@ def dash_prefill_backward(q, k, v, out, dout, alpha=1.5, coarse_scale=1.0, dq=No
         _stream(stream))
     _check("dash_prefill_backward", rc)
     return dq, dk, dv
+
+
+class DashAttentionFunction(torch.autograd.Function):
+    """torch.autograd binding of dash_prefill / dash_prefill_backward (mean summaries, per-head
+    priors).  The forward saves q, k, v and the output; the backward recomputes the coarse
+    stage and the statistics inside dash_prefill_backward."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, alpha, coarse_scale):
+        out, _ = dash_prefill(q, k, v, alpha=alpha, coarse_scale=coarse_scale)
+        ctx.save_for_backward(q, k, v, out)
+        ctx.alpha, ctx.coarse_scale = float(alpha), float(coarse_scale)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, out = ctx.saved_tensors
+        dq, dk, dv = dash_prefill_backward(q, k, v, out, dout.to(torch.bfloat16).contiguous(),
+                                           alpha=ctx.alpha, coarse_scale=ctx.coarse_scale)
+        return dq, dk, dv, None, None
+
+
+def dash_attention(q, k, v, alpha=1.5, coarse_scale=1.0):
+    """Differentiable causal DashAttention prefill: out [B, Hq, T, d] from bf16 q [B, Hq, T, d]
+    and k, v [B, Hkv, T, d]; gradients reach q, k and v through the fine softmax, the log
+    prior, the alpha-entmax selection and the block summaries."""
+    return DashAttentionFunction.apply(q, k, v, alpha, coarse_scale)
+

@@ -182,3 +182,17 @@ def test_mma_sync_backward_matches_oracle():
     assert res.returncode == 0, res.stderr[-2000:]
     errs = json.loads(res.stdout.strip().splitlines()[-1])
     assert max(errs) <= REL_NORM, errs
+
+
+def test_autograd_function_matches_oracle():
+    """dash_attention under torch.autograd: a loss of the output back-propagates to q, k, v
+    through the library's backward, matching the oracle's gradients."""
+    B, Hq, Hkv, T, d, alpha, cs = 1, 8, 2, 640, 128, 1.5, 0.3
+    _, (q, k, v) = inputs.make("16k", B=B, Hq=Hq, Hkv=Hkv, T=T, d=d, n_topics=8, seed=23)
+    G = inputs.out_grad(B, Hq, T, d, seed=24)
+    qd, kd, vd = (t.cuda().requires_grad_(True) for t in (q, k, v))
+    out = da.dash_attention(qd, kd, vd, alpha=alpha, coarse_scale=cs)
+    (out.float() * G.cuda().float()).sum().backward()
+    got = [t.grad.double().cpu().numpy() for t in (qd, kd, vd)]
+    ref = oracle.backward(q, k, v, G, 64, alpha, cs)
+    _compare(got, ref, "autograd")
