@@ -19,7 +19,10 @@
 // dS^T Q into the dk update.  The own block has prior 1 and no coarse term.
 //
 // Kernels, after the coarse stage of the forward (summaries, thresholds, tile lists):
-//   bwd_rowdot_kernel  D per row.
+//   bwd_rowdot_kernel  D per row (every path).
+// then, where a work tile holds at least 8 positions, the tcgen05 kernels of
+// backward_tc.cu (statistics, dq, dk/dv); otherwise (more than 16 query heads per KV head,
+// or DASH_BWD_KERNEL=mma) the two mma.sync kernels below:
 //   bwd_dq_kernel      one CTA per work tile (query-major).  Pass 1 over the tile's steps
 //                      (listed blocks, then the own block) gives each row's log-sum-exp,
 //                      sum_j g_j and sum_j g_j kbar_j; pass 2 gives P, dS, c_j and H_j and
