@@ -71,8 +71,10 @@ def lib():
                                               + [_i64] * 6 + [_dbl, _dbl, _ptr, _i64]
                                               + [_ptr] * 2 + [ctypes.c_int])
         L.oracle_backward.argtypes = ([_ptr, ctypes.c_int] * 4 + [_i64] * 6 + [_dbl, _dbl] + [_ptr] * 3)
+        L.oracle_backward_dq_rows.argtypes = ([_ptr, ctypes.c_int] * 4 + [_i64] * 6 + [_dbl, _dbl]
+                                              + [_ptr, _i64, _ptr, ctypes.c_int])
         for f in (L.oracle_block_summary_w, L.oracle_select_rows_w, L.oracle_forward_rows_w,
-                  L.oracle_forward_rows_agg, L.oracle_backward):
+                  L.oracle_forward_rows_agg, L.oracle_backward, L.oracle_backward_dq_rows):
             f.restype = ctypes.c_int
         for f in (L.oracle_entmax_tau, L.oracle_entmax, L.oracle_block_summary, L.oracle_select_rows,
                   L.oracle_forward_rows, L.oracle_fine_rows_given_p, L.oracle_dense_causal_rows):
@@ -244,6 +246,23 @@ def backward(q, k, v, dout, blk, alpha, coarse_scale):
     _check(lib().oracle_backward(_p(qa), qdt, _p(ka), kdt, _p(va), vdt, _p(ga), gdt, B, Hq, Hkv, T, d, blk,
                                  float(alpha), float(coarse_scale), _p(dq), _p(dk), _p(dv)), "backward")
     return dq, dk, dv
+
+
+def backward_dq_rows(q, k, v, dout, rows, blk, alpha, coarse_scale, nthreads=0):
+    """dq (fp64 [n, d]) of the listed rows (b, h, t) alone: each row's dq depends only on its
+    own forward, so full-size problems can be checked on a sample.  q, dout: [B, Hq, T, d]."""
+    qa, qdt = _arr(q)
+    ka, kdt = _arr(k)
+    va, vdt = _arr(v)
+    ga, gdt = _arr(dout)
+    B, Hq, T, d = qa.shape
+    Hkv = ka.shape[1]
+    r, n = _rows(rows)
+    out = np.zeros((n, d))
+    _check(lib().oracle_backward_dq_rows(_p(qa), qdt, _p(ka), kdt, _p(va), vdt, _p(ga), gdt, B, Hq, Hkv, T, d, blk,
+                                         float(alpha), float(coarse_scale), _p(r), n, _p(out), int(nthreads)),
+           "backward_dq_rows")
+    return out
 
 
 def fine_rows_given_p(q_rows, k, v, rows, Hq, blk, w_rows, w_diag, nthreads=0):

@@ -561,6 +561,108 @@ int oracle_forward_rows_agg(const void* q_group, int qdt, const void* k, int kdt
  *   summaries   kbar_j = mean of block j's keys:  dk_i += dkbar_j / blk.
  * The own block has prior 1 (no gradient into the coarse stage).  Serial over rows.
  */
+/* Scratch of one row's backward: x, p, log p, d log p over the past blocks, the logits over
+ * the row's tokens, and d-vectors o, q, dout. */
+typedef struct {
+    double *x, *p, *lp, *dlp, *lbuf, *o, *qv, *gv;
+} bwd_scratch;
+
+static int bwd_scratch_alloc(bwd_scratch* S, long long nbs, long long Tk, long long d) {
+    S->x = (double*)malloc((size_t)(nbs + 1) * sizeof(double));
+    S->p = (double*)malloc((size_t)(nbs + 1) * sizeof(double));
+    S->lp = (double*)malloc((size_t)(nbs + 1) * sizeof(double));
+    S->dlp = (double*)malloc((size_t)(nbs + 1) * sizeof(double));
+    S->lbuf = (double*)malloc((size_t)Tk * sizeof(double));
+    S->o = (double*)malloc((size_t)d * sizeof(double));
+    S->qv = (double*)malloc((size_t)d * sizeof(double));
+    S->gv = (double*)malloc((size_t)d * sizeof(double));
+    return S->x && S->p && S->lp && S->dlp && S->lbuf && S->o && S->qv && S->gv;
+}
+
+static void bwd_scratch_free(bwd_scratch* S) {
+    free(S->x); free(S->p); free(S->lp); free(S->dlp); free(S->lbuf); free(S->o); free(S->qv); free(S->gv);
+}
+
+/* The chain above for row (b, h, t): adds the row's dq into dq_row; when dk is not NULL also
+ * its shares of dk, dv and dkbar (the summary term reaches dk later, from dkbar). */
+static void backward_row(const orc_problem* P, const double* kb, const void* dout, int ddt,
+                         long long b, long long h, long long t, bwd_scratch* S,
+                         double* dq_row, double* dk, double* dv, double* dkbar) {
+    const void* k = P->k; const void* v = P->v;
+    const int kdt = P->kdt, vdt = P->vdt;
+    const long long G = P->Hq / P->Hkv, d = P->d, blk = P->blk, nbs = P->Tk / P->blk;
+    const long long g = h / G, bt = t / blk, row = (b * P->Hq + h) * P->Tk + t;
+    const long long kvbase = (b * P->Hkv + g) * P->Tk;
+    const double isd = 1.0 / sqrt((double)d), alpha = P->alpha;
+    const double* kbg = kb + (b * P->Hkv + g) * nbs * d;
+    for (long long c = 0; c < d; ++c) {
+        S->qv[c] = elem(P->q, P->qdt, row * d + c);
+        S->gv[c] = elem(dout, ddt, row * d + c);
+    }
+    /* coarse stage (row_select reads q row r = row) */
+    double tau = NAN;
+    row_select(P, row, t, kbg, S->x, S->p, &tau);
+    for (long long j = 0; j < bt; ++j) S->lp[j] = S->p[j] > 0.0 ? log(S->x[j] - tau) / (alpha - 1.0) : -INFINITY;
+    /* fine forward: logits, max, softmax, output */
+    double m = -INFINITY;
+    for (long long i = 0; i <= t; ++i) {
+        const long long j = i / blk;
+        const double lw = j == bt ? 0.0 : S->lp[j];
+        if (lw == -INFINITY) { S->lbuf[i] = -INFINITY; continue; }
+        double dot = 0.0;
+        for (long long c = 0; c < d; ++c) dot += S->qv[c] * elem(k, kdt, (kvbase + i) * d + c);
+        S->lbuf[i] = dot * isd + lw;
+        if (S->lbuf[i] > m) m = S->lbuf[i];
+    }
+    double den = 0.0;
+    for (long long c = 0; c < d; ++c) S->o[c] = 0.0;
+    for (long long i = 0; i <= t; ++i) {
+        if (S->lbuf[i] == -INFINITY) continue;
+        const double a = exp(S->lbuf[i] - m);
+        den += a;
+        for (long long c = 0; c < d; ++c) S->o[c] += a * elem(v, vdt, (kvbase + i) * d + c);
+    }
+    for (long long c = 0; c < d; ++c) S->o[c] /= den;
+    double Drow = 0.0;
+    for (long long c = 0; c < d; ++c) Drow += S->gv[c] * S->o[c];
+    /* fine backward */
+    for (long long j = 0; j < bt; ++j) S->dlp[j] = 0.0;
+    for (long long i = 0; i <= t; ++i) {
+        if (S->lbuf[i] == -INFINITY) continue;
+        const double Pi = exp(S->lbuf[i] - m) / den;
+        double dPi = 0.0;
+        for (long long c = 0; c < d; ++c) dPi += S->gv[c] * elem(v, vdt, (kvbase + i) * d + c);
+        const double dl = Pi * (dPi - Drow);
+        for (long long c = 0; c < d; ++c) {
+            dq_row[c] += dl * elem(k, kdt, (kvbase + i) * d + c) * isd;
+            if (dk) {
+                dv[(kvbase + i) * d + c] += Pi * S->gv[c];
+                dk[(kvbase + i) * d + c] += dl * S->qv[c] * isd;
+            }
+        }
+        const long long j = i / blk;
+        if (j < bt) S->dlp[j] += dl;
+    }
+    /* entmax backward on the support, then the coarse scores */
+    double sg = 0.0, sgdp = 0.0;
+    for (long long j = 0; j < bt; ++j) {
+        if (!(S->p[j] > 0.0)) continue;
+        const double gj = pow(S->p[j], 2.0 - alpha);
+        sg += gj;
+        sgdp += gj * (S->dlp[j] / S->p[j]);
+    }
+    for (long long j = 0; j < bt; ++j) {
+        if (!(S->p[j] > 0.0)) continue;
+        const double gj = pow(S->p[j], 2.0 - alpha);
+        const double ds = gj * (S->dlp[j] / S->p[j]) - gj * sgdp / sg;
+        const double f = ds * P->cs * isd;
+        for (long long c = 0; c < d; ++c) {
+            dq_row[c] += f * kbg[j * d + c];
+            if (dkbar) dkbar[((b * P->Hkv + g) * nbs + j) * d + c] += f * S->qv[c];
+        }
+    }
+}
+
 int oracle_backward(const void* q, int qdt, const void* k, int kdt, const void* v, int vdt,
                     const void* dout, int ddt, long long B, long long Hq, long long Hkv, long long Tk,
                     long long d, long long blk, double alpha, double coarse_scale,
@@ -570,101 +672,64 @@ int oracle_backward(const void* q, int qdt, const void* k, int kdt, const void* 
     orc_problem P = {q, qdt, k, kdt, v, vdt, B, Hq, Hkv, Tk, d, blk, alpha, coarse_scale, NULL};
     double* kb = all_kbar(&P);
     if (!kb) return ORC_ERR_NOMEM;
-    long long nbs = Tk / blk, G = Hq / Hkv;
-    double isd = 1.0 / sqrt((double)d);
+    const long long nbs = Tk / blk;
     memset(dq, 0, (size_t)(B * Hq * Tk * d) * sizeof(double));
     memset(dk, 0, (size_t)(B * Hkv * Tk * d) * sizeof(double));
     memset(dv, 0, (size_t)(B * Hkv * Tk * d) * sizeof(double));
     double* dkbar = (double*)calloc((size_t)(B * Hkv * (nbs > 0 ? nbs : 1) * d), sizeof(double));
-    double* x = (double*)malloc((size_t)(nbs + 1) * sizeof(double));
-    double* p = (double*)malloc((size_t)(nbs + 1) * sizeof(double));
-    double* lp = (double*)malloc((size_t)(nbs + 1) * sizeof(double));
-    double* dlp = (double*)malloc((size_t)(nbs + 1) * sizeof(double));
-    double* lbuf = (double*)malloc((size_t)Tk * sizeof(double));
-    double* o = (double*)malloc((size_t)d * sizeof(double));
-    double* qv = (double*)malloc((size_t)d * sizeof(double));
-    double* gv = (double*)malloc((size_t)d * sizeof(double));
+    bwd_scratch S = {NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL};
     int rc = ORC_OK;
-    if (!dkbar || !x || !p || !lp || !dlp || !lbuf || !o || !qv || !gv) rc = ORC_ERR_NOMEM;
+    if (!dkbar || !bwd_scratch_alloc(&S, nbs, Tk, d)) rc = ORC_ERR_NOMEM;
     for (long long b = 0; rc == ORC_OK && b < B; ++b)
         for (long long h = 0; h < Hq; ++h)
-            for (long long t = 0; t < Tk; ++t) {
-                long long g = h / G, bt = t / blk, row = (b * Hq + h) * Tk + t;
-                long long kvbase = (b * Hkv + g) * Tk;
-                const double* kbg = kb + (b * Hkv + g) * nbs * d;
-                for (long long c = 0; c < d; ++c) {
-                    qv[c] = elem(q, qdt, row * d + c);
-                    gv[c] = elem(dout, ddt, row * d + c);
-                }
-                /* coarse stage (row_select reads q row r = row) */
-                double tau = NAN;
-                row_select(&P, row, t, kbg, x, p, &tau);
-                for (long long j = 0; j < bt; ++j) lp[j] = p[j] > 0.0 ? log(x[j] - tau) / (alpha - 1.0) : -INFINITY;
-                /* fine forward: logits, max, softmax, output */
-                double m = -INFINITY;
-                for (long long i = 0; i <= t; ++i) {
-                    long long j = i / blk;
-                    double lw = j == bt ? 0.0 : lp[j];
-                    if (lw == -INFINITY) { lbuf[i] = -INFINITY; continue; }
-                    double dot = 0.0;
-                    for (long long c = 0; c < d; ++c) dot += qv[c] * elem(k, kdt, (kvbase + i) * d + c);
-                    lbuf[i] = dot * isd + lw;
-                    if (lbuf[i] > m) m = lbuf[i];
-                }
-                double den = 0.0;
-                for (long long c = 0; c < d; ++c) o[c] = 0.0;
-                for (long long i = 0; i <= t; ++i) {
-                    if (lbuf[i] == -INFINITY) continue;
-                    double a = exp(lbuf[i] - m);
-                    den += a;
-                    for (long long c = 0; c < d; ++c) o[c] += a * elem(v, vdt, (kvbase + i) * d + c);
-                }
-                for (long long c = 0; c < d; ++c) o[c] /= den;
-                double Drow = 0.0;
-                for (long long c = 0; c < d; ++c) Drow += gv[c] * o[c];
-                /* fine backward */
-                for (long long j = 0; j < bt; ++j) dlp[j] = 0.0;
-                for (long long i = 0; i <= t; ++i) {
-                    if (lbuf[i] == -INFINITY) continue;
-                    double Pi = exp(lbuf[i] - m) / den;
-                    double dPi = 0.0;
-                    for (long long c = 0; c < d; ++c) dPi += gv[c] * elem(v, vdt, (kvbase + i) * d + c);
-                    double dl = Pi * (dPi - Drow);
-                    for (long long c = 0; c < d; ++c) {
-                        dv[(kvbase + i) * d + c] += Pi * gv[c];
-                        dq[row * d + c] += dl * elem(k, kdt, (kvbase + i) * d + c) * isd;
-                        dk[(kvbase + i) * d + c] += dl * qv[c] * isd;
-                    }
-                    long long j = i / blk;
-                    if (j < bt) dlp[j] += dl;
-                }
-                /* entmax backward on the support, then the coarse scores */
-                double sg = 0.0, sgdp = 0.0;
-                for (long long j = 0; j < bt; ++j) {
-                    if (!(p[j] > 0.0)) continue;
-                    double gj = pow(p[j], 2.0 - alpha);
-                    sg += gj;
-                    sgdp += gj * (dlp[j] / p[j]);
-                }
-                for (long long j = 0; j < bt; ++j) {
-                    if (!(p[j] > 0.0)) continue;
-                    double gj = pow(p[j], 2.0 - alpha);
-                    double ds = gj * (dlp[j] / p[j]) - gj * sgdp / sg;
-                    double f = ds * coarse_scale * isd;
-                    for (long long c = 0; c < d; ++c) {
-                        dq[row * d + c] += f * kbg[j * d + c];
-                        dkbar[((b * Hkv + g) * nbs + j) * d + c] += f * qv[c];
-                    }
-                }
-            }
+            for (long long t = 0; t < Tk; ++t)
+                backward_row(&P, kb, dout, ddt, b, h, t, &S, dq + ((b * Hq + h) * Tk + t) * d, dk, dv, dkbar);
     /* summaries: every key of complete block j receives dkbar_j / blk */
     for (long long bg = 0; rc == ORC_OK && bg < B * Hkv; ++bg)
         for (long long j = 0; j < nbs; ++j)
             for (long long i = 0; i < blk; ++i)
                 for (long long c = 0; c < d; ++c)
                     dk[(bg * Tk + j * blk + i) * d + c] += dkbar[(bg * nbs + j) * d + c] / (double)blk;
-    free(dkbar); free(x); free(p); free(lp); free(dlp); free(lbuf); free(o); free(qv); free(gv); free(kb);
+    bwd_scratch_free(&S);
+    free(dkbar); free(kb);
     return rc;
+}
+
+/*
+ * dq of the listed rows (b, h, t) only -- the same per-row chain as oracle_backward, whose dq
+ * rows do not depend on any other row.  q and dout are the full [B, Hq, T, d] tensors;
+ * dq_out [nrows, d].  OpenMP over rows when nthreads != 1.
+ */
+int oracle_backward_dq_rows(const void* q, int qdt, const void* k, int kdt, const void* v, int vdt,
+                            const void* dout, int ddt, long long B, long long Hq, long long Hkv,
+                            long long Tk, long long d, long long blk, double alpha, double coarse_scale,
+                            const long long* rows, long long nrows, double* dq_out, int nthreads) {
+    if (!q || !k || !v || !dout || (nrows > 0 && (!rows || !dq_out))) return ORC_ERR_ARG;
+    if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || d < 1 || blk < 1 || Tk < 1 || !(alpha > 1.0)) return ORC_ERR_ARG;
+    orc_problem P = {q, qdt, k, kdt, v, vdt, B, Hq, Hkv, Tk, d, blk, alpha, coarse_scale, NULL};
+    if (check_problem(&P, rows, nrows) != ORC_OK) return ORC_ERR_ARG;
+    double* kb = all_kbar(&P);
+    if (!kb) return ORC_ERR_NOMEM;
+    const long long nbs = Tk / blk;
+    int fail = 0;
+#pragma omp parallel num_threads(nthreads > 0 ? nthreads : omp_get_max_threads()) if (nthreads != 1)
+    {
+        bwd_scratch S;
+        if (!bwd_scratch_alloc(&S, nbs, Tk, d)) {
+#pragma omp atomic write
+            fail = 1;
+        } else {
+#pragma omp for schedule(dynamic, 4)
+            for (long long r = 0; r < nrows; ++r) {
+                double* out = dq_out + r * d;
+                for (long long c = 0; c < d; ++c) out[c] = 0.0;
+                backward_row(&P, kb, dout, ddt, rows[3 * r], rows[3 * r + 1], rows[3 * r + 2], &S, out, NULL, NULL, NULL);
+            }
+        }
+        bwd_scratch_free(&S);
+    }
+    free(kb);
+    return fail ? ORC_ERR_NOMEM : ORC_OK;
 }
 
 int oracle_select_rows(const void* q_rows, int qdt, const void* k, int kdt,

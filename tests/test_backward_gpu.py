@@ -196,3 +196,34 @@ def test_autograd_function_matches_oracle():
     got = [t.grad.double().cpu().numpy() for t in (qd, kd, vd)]
     ref = oracle.backward(q, k, v, G, 64, alpha, cs)
     _compare(got, ref, "autograd")
+
+
+def test_full_size_backward_sampled_rows_and_identities():
+    """The 16K workload at the bench's shapes and calibrated scale: dq of stratified rows
+    against the oracle's per-row backward (a row's dq depends on its own forward only), and
+    dk, dv of the whole problem through two exact identities: per KV group the dv rows sum to
+    the sum of dout over the group's query rows, and the dk rows sum to zero."""
+    from gpu_helpers import calibrated_scale
+    wl, (q, k, v) = inputs.make("16k")
+    cs = calibrated_scale("16k")
+    B, Hq, Hkv, T, d = wl.B, wl.Hq, wl.Hkv, wl.T, wl.d
+    dout = inputs.out_grad(B, Hq, T, d, seed=wl.seed + 1)
+    qd, kd, vd, gd = q.cuda(), k.cuda(), v.cuda(), dout.cuda()
+    out, _ = da.dash_prefill(qd, kd, vd, alpha=wl.alpha, coarse_scale=cs)
+    dq, dk, dv = da.dash_prefill_backward(qd, kd, vd, out, gd, alpha=wl.alpha, coarse_scale=cs)
+    torch.cuda.synchronize()
+    rows = [(0, h, t) for h in (0, 7, 8, 15) for t in (0, 63, 64, 1000, 4096, 8191, 12345, T - 1)]
+    ref = oracle.backward_dq_rows(q, k, v, dout, rows, 64, wl.alpha, cs)
+    got = np.stack([dq[b, h, t].double().cpu().numpy() for b, h, t in rows])
+    assert np.all(np.isfinite(got))
+    err = np.abs(got - ref)
+    assert err.max() <= REL_MAX * np.abs(ref).max(), err.max()
+    assert np.linalg.norm(got - ref) <= REL_NORM * np.linalg.norm(ref), np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    G = Hq // Hkv
+    want = gd.double().reshape(B, Hkv, G, T, d).sum(dim=(2, 3))
+    have = dv.double().sum(dim=2)
+    assert torch.isfinite(have).all()
+    assert (have - want).norm() <= 1e-2 * want.norm(), ((have - want).norm() / want.norm()).item()
+    s_dk = dk.double().sum(dim=2)
+    scale = dk.double().abs().sum(dim=2)
+    assert s_dk.norm() <= 1e-2 * scale.norm(), (s_dk.norm() / scale.norm()).item()

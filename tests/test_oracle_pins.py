@@ -536,3 +536,28 @@ def test_backward_of_dense_rows_is_softmax_attention_backward(orc):
     np.testing.assert_allclose(dq, q.grad.numpy(), rtol=0, atol=1e-10)
     np.testing.assert_allclose(dk, k.grad.numpy(), rtol=0, atol=1e-10)
     np.testing.assert_allclose(dv, v.grad.numpy(), rtol=0, atol=1e-10)
+
+
+def test_backward_identities_and_row_dq(orc):
+    """Exact identities of the backward, any size: per KV group the dv rows sum to the sum of
+    dout over the group's query rows (each row's softmax weights sum to one), and the dk rows
+    sum to zero (each row's dS sums to zero over its tokens, and its entmax terms ds_j sum to
+    zero over its support).  The rows-only dq equals the full backward's rows."""
+    B, Hq, Hkv, T, d, alpha, cs = 1, 4, 2, 384, 8, 1.5, 2.0
+    rng = np.random.default_rng(41)
+    q = rng.standard_normal((B, Hq, T, d)) * 1.5
+    k = rng.standard_normal((B, Hkv, T, d))
+    v = rng.standard_normal((B, Hkv, T, d))
+    G = rng.standard_normal((B, Hq, T, d))
+    dq, dk, dv = orc.backward(q, k, v, G, 64, alpha, cs)
+    grp = G.reshape(B, Hkv, Hq // Hkv, T, d).sum(axis=(2, 3))
+    np.testing.assert_allclose(dv.sum(axis=2), grp, rtol=0, atol=1e-10 * np.abs(G).sum())
+    assert np.abs(dk.sum(axis=2)).max() <= 1e-10 * np.abs(dk).sum()
+    # the coarse path is active in this case (sparse, non-trivial supports)
+    rows = [(0, h, t) for h in range(Hq) for t in range(T)]
+    sel = orc.select_rows(q.reshape(-1, d), k, rows, Hq, 64, alpha, cs)
+    assert np.any((sel["nsel"] < sel["bt"]) & (sel["nsel"] >= 2))
+    pick = [(0, 1, 383), (0, 3, 200), (0, 0, 64), (0, 2, 5)]
+    got = orc.backward_dq_rows(q, k, v, G, pick, 64, alpha, cs)
+    ref = np.stack([dq[b, h, t] for b, h, t in pick])
+    np.testing.assert_array_equal(got, ref)
