@@ -1,4 +1,4 @@
-"""fp64 CPU oracle for the DashAttention forward pass -- TEST INFRASTRUCTURE ONLY.
+"""fp64 CPU oracle for the DashAttention forward pass and its backward -- TEST INFRASTRUCTURE ONLY.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference legs of
 ``bench.py`` may import this package.  The product path (the CUDA library and its

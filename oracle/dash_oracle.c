@@ -1,5 +1,6 @@
 /*
- * dash_oracle.c -- plain, slow, fp64 CPU oracle for the DashAttention forward pass.
+ * dash_oracle.c -- plain, slow, fp64 CPU oracle for the DashAttention forward pass and
+ * its backward.
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing in the product path links, loads or calls this
  * file: only the tests, the smoke check and the CPU-baseline leg of the benchmark do.
@@ -32,13 +33,19 @@
  *   - query head h reads KV head floor(h / (Hq/Hkv));
  *   - a block whose x_j equals tau exactly gets weight 0 (strict ">");
  *   - head aggregation (the optional variant): the heads of a KV group average their block
- *     distributions and share the result as their prior (oracle_forward_rows_agg).
+ *     distributions and share the result as their prior (oracle_forward_rows_agg);
+ *   - backward (oracle_backward, oracle_backward_dq_rows): the exact gradient of the
+ *     forward above ([P1] "Core Mechanism" / "Key Concepts": the selection is
+ *     differentiable) through the fine softmax, log p, the alpha-entmax Jacobian on the
+ *     support, the coarse scores and the mean summaries; the own block has no coarse term.
  *
  * Parity pins (tests/test_oracle_pins.py): exact tau is checked against 200-step
  * bisection, brute force over supports and scipy's constrained optimiser on the
  * variational definition; alpha=2 against sparsemax; alpha->1 against softmax;
  * equal prior and T <= 2 blocks against dense causal attention (torch SDPA);
- * non-dispersiveness; a hand-derived worked example.
+ * non-dispersiveness; a hand-derived worked example; the backward against central finite
+ * differences of the fp64 forward, against torch autograd of dense attention, and through
+ * two exact identities (dv rows sum to the group's dout, dk rows to zero).
  *
  * Inputs: element arrays are float32 (dtype 0), bf16 bit patterns (dtype 1, uint16) or
  * float64 (dtype 2); all are widened exactly to double.  Every routine is fp64.
