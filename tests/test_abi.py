@@ -131,3 +131,18 @@ def test_backward_workspace_and_argument_errors(L):
     assert call(a13=32) == -2                         # block
     assert call(a16=None) == -5                       # workspace null
     assert call(a17=16) == -5                         # workspace too small
+
+
+def test_backward_binding_rejects_bad_shapes_before_any_call():
+    import torch
+    from sparse_hierarchical_attention_pool_b200 import dash_attn as da
+    q = torch.zeros(1, 2, 128, 64, dtype=torch.bfloat16)
+    k = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        da.dash_prefill_backward(q, k, k[:, :, :64], q, q)          # v shape
+    with pytest.raises(ValueError):
+        da.dash_prefill_backward(q, k, k, q[:, :1], q)              # out shape
+    with pytest.raises(ValueError):
+        da.dash_prefill_backward(q, k, k, q, q[..., :32])           # dout shape
+    with pytest.raises(ValueError):                                 # CPU tensors: no CPU path
+        da.dash_prefill_backward(q, k, k, q, q, workspace=torch.zeros(1 << 20, dtype=torch.uint8))
