@@ -27,7 +27,10 @@
  *   - Supported: d in {64, 128}; block == 64; Hq % Hkv == 0 and Hq / Hkv <= 128;
  *     1 <= T <= 1048576; alpha > 1 and finite; coarse_scale finite.
  *   - Device-side conditions (a threshold solve that hit its iteration cap) set a status
- *     word inside the workspace; dash_get_device_status reads it.
+ *     word inside the workspace; dash_get_device_status reads it.  The environment
+ *     variable DASH_DEBUG_SOLVE_CAP=n (1 <= n < 64), read at each call, lowers that cap to
+ *     n iterations so that the status path can be exercised with a normal launch; rows
+ *     whose solve is cut short get an inexact threshold.
  *   - No C++ exception crosses this interface.
  */
 #ifndef DASH_ATTN_H
@@ -59,8 +62,11 @@ typedef enum {
     DASH_ERR_NO_CONVERGE = -7,   /* device status: a tau solve hit its iteration cap */
     DASH_ERR_SCRATCH_LIMIT = -8, /* dash_decode_noalloc: the step needs more scratch than
                                     the library's fixed array holds */
-    DASH_ERR_DEVICE_TIMEOUT = -9 /* device status: a kernel's bounded wait gave up (about 2 s);
+    DASH_ERR_DEVICE_TIMEOUT = -9,/* device status: a kernel's bounded wait gave up (about 2 s);
                                     the outputs of that call are invalid */
+    DASH_ERR_SETUP_IN_CAPTURE = -10 /* dash_decode_noalloc: its once-per-device set-up (a symbol
+                                    lookup) was due while `stream` was being captured; make
+                                    one call outside capture first */
 } dash_status;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -221,7 +227,33 @@ DASH_API int dash_prefill_tau(const void* workspace, size_t ws_bytes, float* tau
                      int B, int Hq, int Hkv, int T, int d, int block, dash_stream_t stream);
 
 /*
- * Block-weight dump (parity hook for Stage 1).  For each listed row (b, h, t):
+ * dash_prefill that also reports, for caller-chosen rows, the block weights the fine stage
+ * (Stage 2) actually applied: the parity hook of the selection on the prefill's own path
+ * ("DashAttention: Making Sparse Attention Fully Differentiable with Adaptive Block
+ * Selection", section "Core Mechanism": Stage 1 hands its sparse block weights to Stage 2
+ * as a log prior).  Outputs and workspace contents are those of dash_prefill_ex with the
+ * same arguments; the kernels run in a variant that also writes the dump.
+ *   w_summary, flags  as in dash_prefill_ex.
+ *   row_slot  device int32 [B, Hq, T]: slot s in [0, nslots) of each reported row, -1 for
+ *             rows not reported (two rows must not share a slot).
+ *   x_out     device fp32 [nslots, T / block]: for every block j in the row's work-tile
+ *             list, x_j = (alpha - 1) s_j as Stage 2 recomputed it; NaN for blocks not
+ *             listed (those get no weight).
+ *   p_out     device fp32 [nslots, T / block]: the row's own alpha-entmax weight of block j
+ *             that Stage 2 applied, [x_j - tau]_+^(1/(alpha-1)); 0 for unlisted blocks.
+ *   The threshold tau of each row is read afterwards with dash_prefill_tau.
+ * Returns DASH_ERR_UNSUPPORTED when a tile holds fewer than 8 positions (more than 16
+ * query heads per KV head: the CUDA-core fine kernel has no dump variant).
+ */
+DASH_API int dash_prefill_dump(const void* q, const void* k, const void* v, const float* w_summary, void* out,
+                               int B, int Hq, int Hkv, int T, int d, int block, float alpha,
+                               float coarse_scale, unsigned flags, const int* row_slot, int nslots,
+                               float* x_out, float* p_out, void* workspace, size_t ws_bytes,
+                               dash_stream_t stream);
+
+/*
+ * Block-weight recomputation for listed rows (an independent fp32 path, for analysis).
+ * For each listed row (b, h, t):
  *   rows      device int64 [nrows, 3]
  *   ksum      device fp32 [B, Hkv, T / block, d]  (from dash_block_summary)
  *   out_idx   device int32 [nrows, max_sel]  selected past blocks, ascending
@@ -229,7 +261,11 @@ DASH_API int dash_prefill_tau(const void* workspace, size_t ws_bytes, float* tau
  *   out_count device int32 [nrows]           full support size (may exceed max_sel;
  *                                            only the first max_sel entries are written)
  *   out_tau   device fp32  [nrows]           threshold (NaN when t < block)
- * Uses the same score arithmetic and threshold solver as dash_prefill.
+ * Scores are serial fp32 dot products of q with the fp32 summaries and the threshold comes
+ * from a one-thread solve.  This is NOT dash_prefill's arithmetic (tensor-core products
+ * with the summaries split into bf16 hi + lo parts, per-row passes shared by two threads):
+ * the two agree to fp32 rounding of the scores.  dash_prefill_dump reports the weights the
+ * prefill itself applies.
  */
 DASH_API int dash_select_dump(const void* q, const float* ksum, const long long* rows, int nrows, int max_sel,
                      int* out_idx, float* out_p, int* out_count, float* out_tau,
@@ -266,6 +302,22 @@ DASH_API int dash_decode_ex(const void* q, const void* k_cache, const void* v_ca
                             size_t ws_bytes, dash_stream_t stream);
 
 /*
+ * dash_decode that also reports the block weights its attention kernel applied (the decode
+ * step's selection parity hook; see dash_prefill_dump).  Outputs are those of
+ * dash_decode_ex with the same arguments.
+ *   x_out    device fp32 [B, Hq, Tmax / block]: for every past block j in the (b, KV head)
+ *            union list, x_j = (alpha - 1) s_j of head h; NaN for blocks not listed.
+ *   p_out    device fp32 [B, Hq, Tmax / block]: head h's own alpha-entmax weight of block j
+ *            as applied, [x_j - tau]_+^(1/(alpha-1)); 0 for unlisted blocks.
+ *   tau_out  device fp32 [B, Hq]: the thresholds (NaN for rows without past blocks).
+ * Returns DASH_ERR_UNSUPPORTED for more than 8 query heads per KV head.
+ */
+DASH_API int dash_decode_dump(const void* q, const void* k_cache, const void* v_cache, const float* ksum,
+                              const int* kv_len, void* out, int B, int Hq, int Hkv, int Tmax, int d, int block,
+                              float alpha, float coarse_scale, unsigned flags, float* x_out, float* p_out,
+                              float* tau_out, void* workspace, size_t ws_bytes, dash_stream_t stream);
+
+/*
  * dash_decode that also records four caller-created CUDA events on `stream`: events[0]
  * before the coarse kernels (scores, then thresholds and block lists), events[1] before the
  * attention kernel, events[2] after it (before the partial merge kernel, which only the
@@ -278,11 +330,11 @@ DASH_API int dash_decode_profiled(const void* q, const void* k_cache, const void
 
 /*
  * dash_decode without a workspace argument, for callers that cannot allocate device memory
- * where they decode: code running while a CUDA graph is captured (cudaMalloc cannot be
- * captured), real-time loops that must not take the device-wide synchronisation
- * cudaMalloc / cudaFree can cause, and hosts whose device memory belongs to an allocator
- * this library cannot call.  The pages describe no such entry point; it has no
- * counterpart in the paper.
+ * where they decode: real-time serving loops that must not take the device-wide
+ * synchronisation cudaMalloc / cudaFree can cause, hosts whose device memory belongs to an
+ * allocator this library cannot call, and plug-in code that is handed only its input and
+ * output buffers.  The pages describe no such entry point; it has no counterpart in the
+ * paper.
  *   Arguments, layouts and results are those of dash_decode; the caller still owns and
  *   passes every input and output buffer.
  *   Scratch is one 32 MiB array in device memory that the library declares statically:
@@ -290,17 +342,27 @@ DASH_API int dash_decode_profiled(const void* q, const void* k_cache, const void
  *   whose scratch (dash_decode_workspace_size) exceeds 32 MiB is rejected with
  *   DASH_ERR_SCRATCH_LIMIT before anything is launched (the 96K workload, B=8, Hq=32,
  *   Hkv=8, d=128, needs about 15 MiB).
- *   The first call on a device looks the array's device address up (cudaGetSymbolAddress)
- *   and caches it; make that first call before any stream capture begins.
+ *   Set-up: the first call on a device looks the array's device address up
+ *   (cudaGetSymbolAddress, with that device current) and caches it with the identity of
+ *   the device's context; a call on a context created since (after cudaDeviceReset, for
+ *   instance) repeats the lookup.  Make that first call before any stream capture begins:
+ *   a set-up that falls due while `stream` is being captured returns
+ *   DASH_ERR_SETUP_IN_CAPTURE and launches nothing.
  *   No memory is allocated or freed.  Every call, on every stream, shares the one array
  *   and leaves its contents behind; the counters that must start at zero are cleared at
  *   the start of each call.  Calls whose executions overlap on the GPU (other streams,
  *   other host threads) race on the array and give wrong results: serialise them.
- *   dash_decode_stats / dash_get_device_status do not see this array.
+ *   The device status of the last call (a threshold solve that hit its cap, a bounded wait
+ *   that gave up) lives in the array; dash_decode_noalloc_status reads it.
  */
 DASH_API int dash_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, const float* ksum,
                                  const int* kv_len, void* out, int B, int Hq, int Hkv, int Tmax, int d,
                                  int block, float alpha, float coarse_scale, dash_stream_t stream);
+
+/* Synchronises `stream`, then returns the device status the last dash_decode_noalloc on the
+ * current device left in the static scratch array: DASH_OK, DASH_ERR_DEVICE_TIMEOUT,
+ * DASH_ERR_NO_CONVERGE (as dash_get_device_status), or DASH_ERR_CUDA. */
+DASH_API int dash_decode_noalloc_status(dash_stream_t stream);
 
 /* Synchronises `stream` and returns DASH_OK, DASH_ERR_DEVICE_TIMEOUT when a kernel that used
  * `workspace` gave up a bounded wait, DASH_ERR_NO_CONVERGE when one recorded a failed

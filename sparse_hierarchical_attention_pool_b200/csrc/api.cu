@@ -53,6 +53,9 @@ const char* dash_status_string(int status) {
         case DASH_ERR_NO_CONVERGE: return "DASH_ERR_NO_CONVERGE: a threshold solve hit its iteration cap";
         case DASH_ERR_DEVICE_TIMEOUT: return "DASH_ERR_DEVICE_TIMEOUT: a device-side wait gave up; outputs invalid";
         case DASH_ERR_SCRATCH_LIMIT: return "DASH_ERR_SCRATCH_LIMIT: the decode step needs more than the 32 MiB static scratch";
+        case DASH_ERR_SETUP_IN_CAPTURE:
+            return "DASH_ERR_SETUP_IN_CAPTURE: dash_decode_noalloc's once-per-device set-up fell due while the stream "
+                   "was being captured; make one call outside capture first";
         default: return "unknown dash status";
     }
 }
@@ -85,7 +88,8 @@ size_t dash_prefill_workspace_size(int B, int Hq, int Hkv, int T, int d, int blo
 static int prefill_impl(const void* q, const void* k, const void* v, void* out, int B, int Hq,
                         int Hkv, int T, int d, int block, float alpha, float coarse_scale,
                         void* workspace, size_t ws_bytes, dash_stream_t stream, void* const* events,
-                        const float* wsum = nullptr, unsigned flags = 0) {
+                        const float* wsum = nullptr, unsigned flags = 0, const FineDump* dump = nullptr,
+                        size_t dump_entries = 0) {
     if (!q || !k || !v || !out || !al16(q) || !al16(k) || !al16(v) || !al16(out)) return DASH_ERR_ARG;
     if (wsum && !al16(wsum)) return DASH_ERR_ARG;
     if (!good_params(alpha, coarse_scale)) return DASH_ERR_ARG;
@@ -95,7 +99,7 @@ static int prefill_impl(const void* q, const void* k, const void* v, void* out, 
     const int agg = (flags & DASH_HEAD_AGGREGATION) ? 1 : 0;
     // the CUDA-core fine kernel recovers q . kbar from the mean of the block's scores, which
     // only a mean summary satisfies, and keeps per-head priors only
-    const bool need_tc = wsum != nullptr || agg;
+    const bool need_tc = wsum != nullptr || agg || dump != nullptr;
     if (need_tc && !fine_tc_supported(g)) return DASH_ERR_UNSUPPORTED;
     if (!workspace || !al256(workspace) || ws_bytes < g.total) return DASH_ERR_WORKSPACE;
     char* ws = static_cast<char*>(workspace);
@@ -114,7 +118,13 @@ static int prefill_impl(const void* q, const void* k, const void* v, void* out, 
                                 : launch_coarse(q, g, ws, alpha, coarse_scale, s);
     if (ce != cudaSuccess) return DASH_ERR_CUDA;
     if (!mark(2)) return DASH_ERR_CUDA;
-    if (launch_fine(q, k, v, out, g, ws, alpha, coarse_scale, s, agg, need_tc) != cudaSuccess) return DASH_ERR_CUDA;
+    if (dump) {
+        if (launch_dump_fill(dump->x, dump->p, dump_entries, s) != cudaSuccess ||
+            launch_fine_tc(q, k, v, out, g, ws, alpha, coarse_scale, s, agg, dump) != cudaSuccess)
+            return DASH_ERR_CUDA;
+    } else if (launch_fine(q, k, v, out, g, ws, alpha, coarse_scale, s, agg, need_tc) != cudaSuccess) {
+        return DASH_ERR_CUDA;
+    }
     if (!mark(3)) return DASH_ERR_CUDA;
     return DASH_OK;
 }
@@ -138,6 +148,18 @@ int dash_prefill_ex(const void* q, const void* k, const void* v, const float* w_
                     unsigned flags, void* workspace, size_t ws_bytes, dash_stream_t stream) {
     return prefill_impl(q, k, v, out, B, Hq, Hkv, T, d, block, alpha, coarse_scale, workspace,
                         ws_bytes, stream, nullptr, w_summary, flags);
+}
+
+int dash_prefill_dump(const void* q, const void* k, const void* v, const float* w_summary, void* out, int B,
+                      int Hq, int Hkv, int T, int d, int block, float alpha, float coarse_scale, unsigned flags,
+                      const int* row_slot, int nslots, float* x_out, float* p_out, void* workspace,
+                      size_t ws_bytes, dash_stream_t stream) {
+    if (nslots < 0) return DASH_ERR_ARG;
+    if (!row_slot || (nslots > 0 && (!x_out || !p_out))) return DASH_ERR_ARG;
+    if (block != kBlock || T < 1) return DASH_ERR_SHAPE;
+    FineDump dump{row_slot, x_out, p_out};
+    return prefill_impl(q, k, v, out, B, Hq, Hkv, T, d, block, alpha, coarse_scale, workspace, ws_bytes,
+                        stream, nullptr, w_summary, flags, &dump, (size_t)nslots * (size_t)(T / kBlock));
 }
 
 size_t dash_prefill_backward_workspace_size(int B, int Hq, int Hkv, int T, int d, int block) {
@@ -300,7 +322,8 @@ size_t dash_decode_workspace_size(int B, int Hq, int Hkv, int Tmax, int d, int b
 static int decode_impl(const void* q, const void* k_cache, const void* v_cache, const float* ksum,
                        const int* kv_len, void* out, int B, int Hq, int Hkv, int Tmax, int d, int block,
                        float alpha, float coarse_scale, void* workspace, size_t ws_bytes,
-                       dash_stream_t stream, void* const* events, unsigned flags = 0) {
+                       dash_stream_t stream, void* const* events, unsigned flags = 0,
+                       float* x_dump = nullptr, float* p_dump = nullptr, float* tau_dump = nullptr) {
     if (!q || !k_cache || !v_cache || !ksum || !kv_len || !out) return DASH_ERR_ARG;
     if (!al16(q) || !al16(k_cache) || !al16(v_cache) || !al16(ksum) || !al16(out)) return DASH_ERR_ARG;
     if (!good_params(alpha, coarse_scale)) return DASH_ERR_ARG;
@@ -308,14 +331,19 @@ static int decode_impl(const void* q, const void* k_cache, const void* v_cache, 
     if (block != kBlock || !make_decode_geom(B, Hq, Hkv, Tmax, d, &g)) return DASH_ERR_SHAPE;
     if (flags & ~(unsigned)DASH_HEAD_AGGREGATION) return DASH_ERR_ARG;
     const int agg = (flags & DASH_HEAD_AGGREGATION) ? 1 : 0;
-    if (agg && !decode_tc_supported(g)) return DASH_ERR_UNSUPPORTED;
+    if ((agg || x_dump) && !decode_tc_supported(g)) return DASH_ERR_UNSUPPORTED;
     if (!workspace || !al256(workspace) || ws_bytes < g.total) return DASH_ERR_WORKSPACE;
     char* ws = static_cast<char*>(workspace);
     cudaStream_t s = S(stream);
     if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), s) != cudaSuccess) return DASH_ERR_CUDA;
-    return launch_decode(q, k_cache, v_cache, ksum, kv_len, out, g, ws, alpha, coarse_scale, s,
-                         reinterpret_cast<cudaEvent_t const*>(events), agg) == cudaSuccess
-               ? DASH_OK : DASH_ERR_CUDA;
+    if (x_dump && launch_dump_fill(x_dump, p_dump, (size_t)B * Hq * g.nbs, s) != cudaSuccess) return DASH_ERR_CUDA;
+    if (launch_decode(q, k_cache, v_cache, ksum, kv_len, out, g, ws, alpha, coarse_scale, s,
+                      reinterpret_cast<cudaEvent_t const*>(events), agg, x_dump, p_dump) != cudaSuccess)
+        return DASH_ERR_CUDA;
+    if (tau_dump && cudaMemcpyAsync(tau_dump, ws + g.off_tau, (size_t)B * Hq * sizeof(float),
+                                    cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return DASH_ERR_CUDA;
+    return DASH_OK;
 }
 
 int dash_decode(const void* q, const void* k_cache, const void* v_cache, const float* ksum,
@@ -331,6 +359,15 @@ int dash_decode_ex(const void* q, const void* k_cache, const void* v_cache, cons
                    dash_stream_t stream) {
     return decode_impl(q, k_cache, v_cache, ksum, kv_len, out, B, Hq, Hkv, Tmax, d, block, alpha,
                        coarse_scale, workspace, ws_bytes, stream, nullptr, flags);
+}
+
+int dash_decode_dump(const void* q, const void* k_cache, const void* v_cache, const float* ksum,
+                     const int* kv_len, void* out, int B, int Hq, int Hkv, int Tmax, int d, int block,
+                     float alpha, float coarse_scale, unsigned flags, float* x_out, float* p_out, float* tau_out,
+                     void* workspace, size_t ws_bytes, dash_stream_t stream) {
+    if (!x_out || !p_out || !tau_out) return DASH_ERR_ARG;
+    return decode_impl(q, k_cache, v_cache, ksum, kv_len, out, B, Hq, Hkv, Tmax, d, block, alpha,
+                       coarse_scale, workspace, ws_bytes, stream, nullptr, flags, x_out, p_out, tau_out);
 }
 
 int dash_decode_profiled(const void* q, const void* k_cache, const void* v_cache, const float* ksum,

@@ -129,7 +129,7 @@ coarse_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ ksu
             const int r = tid, hl = r / g.P, t = t0 + r % g.P;
             const bool valid = r < g.M && t < g.T;
             float tau = INFINITY;
-            if (valid) tau = entmax_threshold<false>(SlabCol{slab + r}, bt, alpha, &no_conv);
+            if (valid) tau = entmax_threshold<false>(SlabCol{slab + r}, bt, alpha, &no_conv, g.maxit);
             if (valid) tau_out[((size_t)(b * g.Hq + kvh * g.G + hl)) * g.T + t] = tau;
             unsigned nsel = 0;
             for (int j = 0; j < bt; ++j) {

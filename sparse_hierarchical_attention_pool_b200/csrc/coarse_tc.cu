@@ -331,7 +331,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 // exchanged through a buffer alternating with the pass parity
                 auto sweep = [&](auto mode) {
                     constexpr int MODE = decltype(mode)::value;
-                    sv.init(m, alpha);
+                    sv.init(m, alpha, -1.0f, g.maxit);
                     for (int pp = 1; __any_sync(0xffffffffu, !done); ++pp) {
                         EntmaxPass ps;
                         ps.reset();
@@ -441,7 +441,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                : alpha == 2.0f ? subset_start<2 * kTopK, 2>(ysub, alpha)
                                                : subset_start<2 * kTopK, 0>(ysub, alpha);
                 EntmaxSolver sv;
-                sv.init(m, alpha, u0);
+                sv.init(m, alpha, u0, g.maxit);
                 bool done = !valid;
                 // ---- Newton / exact-support passes until every row of the tile is final
                 while (true) {

@@ -4,6 +4,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 namespace dash {
 
@@ -30,6 +31,16 @@ static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Iteration cap of the threshold solves of a call: kSolveMaxIt, or the smaller value of the
+// environment variable DASH_DEBUG_SOLVE_CAP (1 .. kSolveMaxIt), which exists to exercise the
+// no-convergence status path with a normal, terminating launch.
+inline int solve_cap_from_env() {
+    const char* e = getenv("DASH_DEBUG_SOLVE_CAP");
+    if (!e || !*e) return kSolveMaxIt;
+    const long v = strtol(e, nullptr, 10);
+    return (v >= 1 && v < kSolveMaxIt) ? (int)v : kSolveMaxIt;
+}
+
 // Geometry of a prefill call.  Work tiles are P consecutive positions (inside one key
 // block) x the G query heads of one KV head: rows r = head_local * P + pos_local.
 struct PrefillGeom {
@@ -39,6 +50,7 @@ struct PrefillGeom {
     int nbs;                         // complete blocks = T / 64
     int cap;                         // list capacity per tile = max(1, nbs)
     bool tc;                         // tensor-core Stage 1/2 kernels (needs P >= 8)
+    int maxit;                       // iteration cap of the threshold solves
     size_t off_ksum, off_khi, off_klo, off_tau, off_list, off_count, off_scratch, total;
 };
 
@@ -64,6 +76,7 @@ inline bool make_prefill_geom(int B, int Hq, int Hkv, int T, int d, PrefillGeom*
     g->nbs = T / kBlock;
     g->cap = g->nbs > 0 ? g->nbs : 1;
     g->tc = P >= 8;
+    g->maxit = solve_cap_from_env();
     const size_t nsum = (size_t)B * Hkv * (g->nbs > 0 ? g->nbs : 1) * d;
     size_t off = align256(sizeof(WsHeader));
     g->off_ksum = off;    off = align256(off + nsum * sizeof(float));
@@ -97,6 +110,7 @@ inline void make_bwd_geom(const PrefillGeom& g, BwdGeom* bw) {
 // Geometry of a decode call.
 struct DecodeGeom {
     int B, Hq, Hkv, Tmax, d, G, nbs, chunk, maxchunks;
+    int maxit;                       // iteration cap of the threshold solves
     size_t off_x, off_tau, off_list, off_count, off_done, off_offs, off_plan, off_part, total;
 };
 
@@ -112,6 +126,7 @@ inline bool make_decode_geom(int B, int Hq, int Hkv, int Tmax, int d, DecodeGeom
     g->nbs = Tmax / kBlock;
     g->chunk = kDecodeChunk;
     g->maxchunks = (g->nbs + 1 + kDecodeChunk - 1) / kDecodeChunk;
+    g->maxit = solve_cap_from_env();
     int cap = g->nbs + 1;
     size_t off = align256(sizeof(WsHeader));
     g->off_x = off;     off = align256(off + (size_t)B * Hq * cap * sizeof(float));

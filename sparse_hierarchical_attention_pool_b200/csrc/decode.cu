@@ -319,13 +319,13 @@ __device__ __forceinline__ float hist_start(const WarpRow& xr, float m, HistBins
 // bins != nullptr: start from the histogram edge (alpha = 1.5 and 2), else from u = -1.
 template <int MODE>
 __device__ __forceinline__ float warp_row_tau(const WarpRow& xr, float m, float alpha, int* no_conv,
-                                              HistBins* bins) {
+                                              HistBins* bins, int cap) {
     float u0 = -1.0f;
     if constexpr (MODE != 0) {
         if (bins) u0 = hist_start<MODE>(xr, m, bins);
     }
     EntmaxSolver sv;
-    sv.init(m, alpha, u0);
+    sv.init(m, alpha, u0, cap);
     float t = m;
     while (true) {
         EntmaxPass ps;
@@ -437,9 +437,9 @@ decode_select_kernel(const int* __restrict__ kv_len, const float* __restrict__ x
             xr.each([&](int, float v) { m = fmaxf(m, v); });
             m = warp_max(m);
             HistBins* bins = hist_init ? &hist[warp] : nullptr;
-            t = alpha == 1.5f ? warp_row_tau<1>(xr, m, alpha, &no_conv, bins)
-              : alpha == 2.0f ? warp_row_tau<2>(xr, m, alpha, &no_conv, bins)
-                              : warp_row_tau<0>(xr, m, alpha, &no_conv, bins);
+            t = alpha == 1.5f ? warp_row_tau<1>(xr, m, alpha, &no_conv, bins, g.maxit)
+              : alpha == 2.0f ? warp_row_tau<2>(xr, m, alpha, &no_conv, bins, g.maxit)
+                              : warp_row_tau<0>(xr, m, alpha, &no_conv, bins, g.maxit);
         }
         if (lane == 0) tau[row] = t;
         float nsel = 0.f;
@@ -669,7 +669,7 @@ decode_combine_kernel(const int* __restrict__ count, const float* __restrict__ p
 cudaError_t launch_decode(const void* q, const void* kc, const void* vc, const float* ksum,
                           const int* kv_len, void* out, const DecodeGeom& g, char* ws,
                           float alpha, float coarse_scale, cudaStream_t stream,
-                          const cudaEvent_t* events, int agg) {
+                          const cudaEvent_t* events, int agg, float* x_dump, float* p_dump) {
     auto mark = [&](int i) {
         return !events || cudaEventRecord(events[i], stream) == cudaSuccess;
     };
@@ -705,12 +705,13 @@ cudaError_t launch_decode(const void* q, const void* kc, const void* vc, const f
                                                          alpha, nctas, hist_init);
     if (!mark(1)) return cudaErrorUnknown;
     if (fused) {
-        e = launch_decode_attn_tc(q, kc, vc, kv_len, out, g, ws, e_pow, sm2, nctas, stream, agg);
+        e = launch_decode_attn_tc(q, kc, vc, kv_len, out, g, ws, e_pow, sm2, nctas, stream, agg, x_dump, p_dump);
         if (e != cudaSuccess) return e;
         if (!mark(2) || !mark(3)) return cudaErrorUnknown;   // no separate merge pass
         return cudaGetLastError();
     }
-    if (agg) return cudaErrorNotSupported;              // the CUDA-core path has per-head priors only
+    // the CUDA-core path has per-head priors only and no parity dump
+    if (agg || x_dump) return cudaErrorNotSupported;
     const size_t sm_attn = (size_t)4 * kBlock * g.d * sizeof(__nv_bfloat16)
                          + (size_t)(2 * g.G * g.d + g.G * kBlock + 4 * 32) * sizeof(float);
     e = g.d == 128

@@ -27,6 +27,9 @@
 // O^T += V^T P^T, and keeps its own online-softmax state; the four states are merged in
 // shared memory at the end of every segment.  Block indices and log-priors of the segment
 // are staged in shared memory 64 entries at a time.
+// Parity dump (x_dump != nullptr, checks only): while staging, every listed past block's
+// x_j and the weight p_j the prior applies (0 when x_j <= tau) are written per head to
+// x_dump / p_dump [B Hq, Tmax / 64]; each (group, list entry) is staged by one CTA only.
 #include "common.cuh"
 #include "kernels.h"
 #include "mma_sync.cuh"
@@ -75,7 +78,7 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                       const int* __restrict__ list, const int* __restrict__ offs,
                       const int* __restrict__ plan, float* __restrict__ part, int* __restrict__ done,
                       __nv_bfloat16* __restrict__ out, WsHeader* __restrict__ hdr, DecodeGeom g,
-                      float e_pow, float sm2, int agg) {
+                      float e_pow, float sm2, int agg, float* __restrict__ x_dump, float* __restrict__ p_dump) {
     using L = DtLayout<D>;
     using namespace sm100;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -207,6 +210,10 @@ decode_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_con
                         const float tu = tau[qrow0 + hl];
                         // head aggregation keeps the weight itself for the average below
                         if (x > tu) v2 = agg ? exp2f(e_pow * __log2f(x - tu)) : e_pow * __log2f(x - tu);
+                        if (x_dump) {
+                            x_dump[(qrow0 + hl) * g.nbs + j] = x;
+                            p_dump[(qrow0 + hl) * g.nbs + j] = x > tu ? exp2f(e_pow * __log2f(x - tu)) : 0.f;
+                        }
                     }
                 }
                 lptab[idx] = v2;
@@ -425,7 +432,7 @@ int decode_tc_ctas() {
 
 cudaError_t launch_decode_attn_tc(const void* q, const void* kc, const void* vc, const int* kv_len,
                                   void* out, const DecodeGeom& g, char* ws, float e_pow, float sm2,
-                                  int nctas, cudaStream_t stream, int agg) {
+                                  int nctas, cudaStream_t stream, int agg, float* x_dump, float* p_dump) {
     if (nctas < 1 || nctas > kDecodeMaxCtas) return cudaErrorInvalidValue;
     CUtensorMap tk, tv;
     const unsigned long long rows = (unsigned long long)g.B * g.Hkv * g.Tmax;
@@ -444,12 +451,12 @@ cudaError_t launch_decode_attn_tc(const void* q, const void* kc, const void* vc,
         const int sm = (int)DtLayout<128>::bytes;
         cudaError_t e = cudaFuncSetAttribute(decode_attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
         if (e != cudaSuccess) return e;
-        decode_attn_tc_kernel<128><<<nctas, 160, sm, stream>>>(tk, tv, qb, kv_len, xs, tau, list, offs, plan, part, done, ob, hdr, g, e_pow, sm2, agg);
+        decode_attn_tc_kernel<128><<<nctas, 160, sm, stream>>>(tk, tv, qb, kv_len, xs, tau, list, offs, plan, part, done, ob, hdr, g, e_pow, sm2, agg, x_dump, p_dump);
     } else {
         const int sm = (int)DtLayout<64>::bytes;
         cudaError_t e = cudaFuncSetAttribute(decode_attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
         if (e != cudaSuccess) return e;
-        decode_attn_tc_kernel<64><<<nctas, 160, sm, stream>>>(tk, tv, qb, kv_len, xs, tau, list, offs, plan, part, done, ob, hdr, g, e_pow, sm2, agg);
+        decode_attn_tc_kernel<64><<<nctas, 160, sm, stream>>>(tk, tv, qb, kv_len, xs, tau, list, offs, plan, part, done, ob, hdr, g, e_pow, sm2, agg, x_dump, p_dump);
     }
     return cudaGetLastError();
 }

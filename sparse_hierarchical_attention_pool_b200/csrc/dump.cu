@@ -1,9 +1,12 @@
-// dump.cu -- block weights of listed rows (Stage 1 only), for parity checks and analysis.
+// dump.cu -- block weights of listed rows (Stage 1 only), an independent fp32 recomputation
+// for analysis, and the fill kernel of the prefill / decode parity dumps.
 //
-// Same arithmetic as the prefill coarse kernel: x_j accumulated with one fp32 fma chain
-// over the head dimension in order, times (alpha - 1) cs / sqrt(d); tau from the same
-// single-thread solve (entmax.cuh); p_j = (x_j - tau)^(1/(alpha-1)) for x_j > tau.
-// One CTA per listed row.
+// select_dump_kernel: x_j accumulated with one fp32 fma chain over the head dimension in
+// order against the fp32 summaries, times (alpha - 1) cs / sqrt(d); tau from the
+// single-thread solve of entmax.cuh; p_j = (x_j - tau)^(1/(alpha-1)) for x_j > tau.  One CTA
+// per listed row.  This is not the prefill's own arithmetic (its scores are tensor-core
+// products with the summaries split into bf16 hi + lo parts): the weights the prefill
+// applies come from the dump variant of the fine kernel (fine_tc.cu).
 #include "common.cuh"
 #include "entmax.cuh"
 #include "kernels.h"
@@ -65,6 +68,20 @@ select_dump_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict_
         out_count[r] = c;
         out_tau[r] = tau;
     }
+}
+
+__global__ void dump_fill_kernel(float* __restrict__ x, float* __restrict__ p, size_t n) {
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+        x[i] = __int_as_float(0x7fc00000);
+        p[i] = 0.f;
+    }
+}
+
+cudaError_t launch_dump_fill(float* x, float* p, size_t n, cudaStream_t stream) {
+    if (n == 0) return cudaSuccess;
+    const size_t blocks = (n + 255) / 256;
+    dump_fill_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, stream>>>(x, p, n);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_select_dump(const void* q, const float* ksum, const long long* rows, int nrows,

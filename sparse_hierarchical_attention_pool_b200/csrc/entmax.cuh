@@ -82,13 +82,14 @@ struct EntmaxPass {
 
 struct EntmaxSolver {
     float m, u, lo, hi, e;
-    int mode, it;
-    __device__ __forceinline__ void init(float row_max, float alpha, float u0 = -1.0f) {
+    int mode, it, maxit;
+    __device__ __forceinline__ void init(float row_max, float alpha, float u0 = -1.0f, int cap = kSolveMaxIt) {
         m = row_max;
         u = u0; lo = -1.0f; hi = 0.0f;
         e = 1.0f / (alpha - 1.0f);
         mode = alpha == 2.0f ? 2 : (alpha == 1.5f ? 1 : 0);
         it = 0;
+        maxit = cap;
     }
     // One iteration from the pass sums.  Returns true when tau (in x space) is final.
     __device__ __forceinline__ bool update(EntmaxPass p, float* tau, int* no_converge) {
@@ -106,7 +107,7 @@ struct EntmaxSolver {
         float un = u + step;
         if (!(un > lo && un < hi)) un = 0.5f * (lo + hi);
         u = un;
-        if (++it >= kSolveMaxIt) { *no_converge = 1; *tau = m + u; return true; }
+        if (++it >= maxit) { *no_converge = 1; *tau = m + u; return true; }
         return false;
     }
 };
@@ -148,14 +149,14 @@ __device__ __forceinline__ float subset_start(const Y& y, float alpha) {
 // Whole-row solve through an accessor x(j), j in [0, n): on one thread (WARP = false) or
 // on a whole warp (lanes take j = lane, lane + 32, ...; every lane returns the same value).
 template <bool WARP, class Acc>
-__device__ float entmax_threshold(const Acc& x, int n, float alpha, int* no_converge) {
+__device__ float entmax_threshold(const Acc& x, int n, float alpha, int* no_converge, int cap = kSolveMaxIt) {
     const int j0 = WARP ? (threadIdx.x & 31) : 0;
     const int js = WARP ? 32 : 1;
     float m = -INFINITY;
     for (int j = j0; j < n; j += js) m = fmaxf(m, x(j));
     if (WARP) m = warp_max(m);
     EntmaxSolver sv;
-    sv.init(m, alpha);
+    sv.init(m, alpha, -1.0f, cap);
     float tau = m - 1.0f;
     while (true) {
         EntmaxPass ps;

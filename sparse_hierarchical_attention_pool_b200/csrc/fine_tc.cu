@@ -37,6 +37,11 @@
 // through shared memory (one group barrier per step) and share log of the mean as prior.
 // Operands: Q, K, P K-major and V MN-major, all 128-byte swizzled (TMA writes that layout).
 // Every wait is bounded (~2 s); a CTA that gives up sets a status bit and exits cleanly.
+// Dump variant (DUMP = true, parity checks only): for rows with a slot in dump.slot, every
+// listed block's x_j (as recomputed here from the summary columns) and the weight p_j the
+// prior applies (0 when x_j <= tau) are written to dump.x / dump.p [slot, T / 64].
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -75,13 +80,14 @@ enum : int { B_Q = 0, B_KV_FULL = 1, B_KV_EMPTY = 1 + kTcStages, B_S_FULL = 1 + 
              B_S_FREE = B_S_FULL + 2, B_P_FULL = B_S_FREE + 2, B_PV_DONE = B_P_FULL + 2,
              B_DRAIN = B_PV_DONE + 2, B_DRAIN2 = B_DRAIN + 1, B_COUNT = B_DRAIN2 + 1 };
 
-template <int D, int SPLIT, bool AGG>
+template <int D, int SPLIT, bool AGG, bool DUMP>
 __global__ void __launch_bounds__((8 * SPLIT + 3) * 32, 1)
 fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_hi,
                const __grid_constant__ CUtensorMap tm_lo, __nv_bfloat16* __restrict__ out,
                const float* __restrict__ tau, const int* __restrict__ list, const int* __restrict__ count,
-               WsHeader* __restrict__ hdr, PrefillGeom g, float cx, float e_pow, float sm2) {
+               WsHeader* __restrict__ hdr, PrefillGeom g, float cx, float e_pow, float sm2,
+               FineDump dump) {
     using L = TcLayout<D>;
     using namespace sm100;
     constexpr int kGroupThreads = 128 * SPLIT;  // softmax threads per group
@@ -273,6 +279,16 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const bool valid = r < g.M && t < g.T;
         const int tpos = valid ? t : -1;
         const float tau_r = (valid && bt > 0) ? tau[(size_t)(b * g.Hq + kvh * g.G + hl) * g.T + t] : INFINITY;
+        const int slot = (DUMP && valid) ? dump.slot[(size_t)(b * g.Hq + kvh * g.G + hl) * g.T + t] : -1;
+        // parity dump of one listed past block: x_j and the weight the prior applies
+        auto dump_block = [&](int j, float x) {
+            if constexpr (DUMP) {
+                if (slot >= 0 && sp == 0) {
+                    dump.x[(size_t)slot * g.nbs + j] = x;
+                    dump.p[(size_t)slot * g.nbs + j] = x > tau_r ? exp2f(e_pow * __log2f(x - tau_r)) : 0.f;
+                }
+            }
+        };
         const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
         const uint32_t s_col = grp * L::colS + sp * KEYS;   // this thread's keys in its group's S buffer
         const uint32_t o_col = L::colO + grp * D + sp * RCOLS;   // O columns it rescales
@@ -348,6 +364,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 // passes this barrier once per step, failed step or not
                 const float x = __fmul_rn(rs, cx);
                 const float pown = (okw && !diag && x > tau_r) ? exp2f(e_pow * __log2f(x - tau_r)) : 0.f;
+                if (okw && !diag) dump_block(j, x);
                 if (sp == 0) pagg[i2 & 1][grp][r] = pown;
                 asm volatile("bar.sync %0, %1;" :: "r"(10 + grp), "n"(kGroupThreads) : "memory");
                 float pbar = 0.f;
@@ -360,6 +377,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const float x = __fmul_rn(rs, cx);
                 lp2 = diag ? (tpos >= 0 ? 0.f : -INFINITY)
                            : (x > tau_r ? e_pow * __log2f(x - tau_r) : -INFINITY);
+                if (!diag) dump_block(j, x);
             }
             const bool active = lp2 > -INFINITY;
             const float mx = active ? fmaf(smax, sm2, lp2) : -INFINITY;
@@ -481,7 +499,8 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 bool fine_tc_supported(const PrefillGeom& g) { return g.P >= 8 && (g.d == 64 || g.d == 128); }
 
 cudaError_t launch_fine_tc(const void* q, const void* k, const void* v, void* out, const PrefillGeom& g,
-                           char* ws, float alpha, float coarse_scale, cudaStream_t stream, int agg) {
+                           char* ws, float alpha, float coarse_scale, cudaStream_t stream, int agg,
+                           const FineDump* dump) {
     const float cx = (alpha - 1.0f) * coarse_scale / sqrtf((float)g.d);
     const float e_pow = 1.0f / (alpha - 1.0f);
     const float sm2 = 1.4426950408889634f / sqrtf((float)g.d);
@@ -501,20 +520,22 @@ cudaError_t launch_fine_tc(const void* q, const void* k, const void* v, void* ou
     WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
     auto* ob = static_cast<__nv_bfloat16*>(out);
     constexpr int threads = (8 * kFineSplit + 3) * 32;
+    const FineDump dv = dump ? *dump : FineDump{nullptr, nullptr, nullptr};
     auto go = [&](auto kernel, int sm) -> cudaError_t {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
         if (e != cudaSuccess) return e;
-        kernel<<<g.ntiles, threads, sm, stream>>>(tq, tk, tv, thi, tlo, ob, tau, list, count, hdr, g, cx, e_pow, sm2);
+        kernel<<<g.ntiles, threads, sm, stream>>>(tq, tk, tv, thi, tlo, ob, tau, list, count, hdr, g, cx, e_pow, sm2, dv);
         return cudaSuccess;
     };
-    cudaError_t e;
-    if (g.d == 128) {
-        const int sm = (int)TcLayout<128>::bytes;
-        e = agg ? go(fine_tc_kernel<128, kFineSplit, true>, sm) : go(fine_tc_kernel<128, kFineSplit, false>, sm);
-    } else {
-        const int sm = (int)TcLayout<64>::bytes;
-        e = agg ? go(fine_tc_kernel<64, kFineSplit, true>, sm) : go(fine_tc_kernel<64, kFineSplit, false>, sm);
-    }
+    auto pick = [&](auto dcon) -> cudaError_t {
+        constexpr int DD = decltype(dcon)::value;
+        const int sm = (int)TcLayout<DD>::bytes;
+        if (dump) return agg ? go(fine_tc_kernel<DD, kFineSplit, true, true>, sm)
+                             : go(fine_tc_kernel<DD, kFineSplit, false, true>, sm);
+        return agg ? go(fine_tc_kernel<DD, kFineSplit, true, false>, sm)
+                   : go(fine_tc_kernel<DD, kFineSplit, false, false>, sm);
+    };
+    cudaError_t e = g.d == 128 ? pick(std::integral_constant<int, 128>{}) : pick(std::integral_constant<int, 64>{});
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

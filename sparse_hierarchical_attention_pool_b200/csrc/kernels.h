@@ -23,6 +23,15 @@ bool coarse_tc_supported(const PrefillGeom& g);
 cudaError_t launch_coarse_tc(const void* q, const PrefillGeom& g, char* ws, float alpha,
                              float coarse_scale, cudaStream_t stream);
 
+// Parity dump of the tensor-core fine kernel: rows with slot[row] >= 0 (row = (b Hq + h) T + t)
+// get x_j and the applied weight p_j of every listed past block j at x[slot nbs + j],
+// p[slot nbs + j].
+struct FineDump {
+    const int* slot;
+    float* x;
+    float* p;
+};
+
 // Stage 2 for prefill: prior-weighted softmax attention over each tile's listed blocks.
 // agg: head-aggregated prior; need_tc: the tensor-core kernel is required (head aggregation
 // or a learned summary head), whatever DASH_FINE_KERNEL says.
@@ -30,11 +39,15 @@ cudaError_t launch_fine(const void* q, const void* k, const void* v, void* out,
                         const PrefillGeom& g, char* ws, float alpha, float coarse_scale,
                         cudaStream_t stream, int agg = 0, bool need_tc = false);
 
-// tcgen05 variant of launch_fine (needs P >= 8, i.e. at most 16 query heads per KV head)
+// tcgen05 variant of launch_fine (needs P >= 8, i.e. at most 16 query heads per KV head);
+// dump != nullptr selects the dump variant
 bool fine_tc_supported(const PrefillGeom& g);
 cudaError_t launch_fine_tc(const void* q, const void* k, const void* v, void* out,
                            const PrefillGeom& g, char* ws, float alpha, float coarse_scale,
-                           cudaStream_t stream, int agg = 0);
+                           cudaStream_t stream, int agg = 0, const FineDump* dump = nullptr);
+
+// x = NaN and p = 0 for n entries (the "not listed" marks of the parity dumps)
+cudaError_t launch_dump_fill(float* x, float* p, size_t n, cudaStream_t stream);
 
 // Gradients of the prefill (dq, dk, dv) after the coarse stage has filled the workspace
 cudaError_t launch_backward(const void* q, const void* k, const void* v, const void* out,
@@ -61,13 +74,18 @@ cudaError_t launch_select_dump(const void* q, const float* ksum, const long long
 // heads per group); decode_tc_ctas() is the grid it is launched with
 bool decode_tc_supported(const DecodeGeom& g);
 int decode_tc_ctas();
+// x_dump / p_dump (both or neither, fp32 [B Hq, Tmax / 64]): the parity dump of each head's
+// listed blocks
 cudaError_t launch_decode_attn_tc(const void* q, const void* kc, const void* vc, const int* kv_len,
                                   void* out, const DecodeGeom& g, char* ws, float e_pow, float sm2,
-                                  int nctas, cudaStream_t stream, int agg = 0);
-// agg: head-aggregated prior (needs decode_tc_supported)
+                                  int nctas, cudaStream_t stream, int agg = 0, float* x_dump = nullptr,
+                                  float* p_dump = nullptr);
+// agg: head-aggregated prior (needs decode_tc_supported); x_dump / p_dump as above (needs
+// decode_tc_supported)
 cudaError_t launch_decode(const void* q, const void* kc, const void* vc, const float* ksum,
                           const int* kv_len, void* out, const DecodeGeom& g, char* ws,
                           float alpha, float coarse_scale, cudaStream_t stream,
-                          const cudaEvent_t* events, int agg = 0);
+                          const cudaEvent_t* events, int agg = 0, float* x_dump = nullptr,
+                          float* p_dump = nullptr);
 
 }  // namespace dash

@@ -21,14 +21,15 @@ DASH_OK = 0
 STATUS = {0: "DASH_OK", -1: "DASH_ERR_ARG", -2: "DASH_ERR_SHAPE", -3: "DASH_ERR_DTYPE",
           -4: "DASH_ERR_UNSUPPORTED", -5: "DASH_ERR_WORKSPACE", -6: "DASH_ERR_CUDA",
           -7: "DASH_ERR_NO_CONVERGE", -8: "DASH_ERR_SCRATCH_LIMIT",
-          -9: "DASH_ERR_DEVICE_TIMEOUT"}
+          -9: "DASH_ERR_DEVICE_TIMEOUT", -10: "DASH_ERR_SETUP_IN_CAPTURE"}
 
 EXPORTS = ("dash_status_string", "dash_version", "dash_block_summary", "dash_prefill_workspace_size",
            "dash_prefill", "dash_prefill_host", "dash_prefill_stats", "dash_decode_stats",
            "dash_prefill_tau", "dash_select_dump", "dash_decode_workspace_size", "dash_decode",
            "dash_get_device_status", "dash_prefill_profiled", "dash_decode_profiled",
-           "dash_decode_noalloc", "dash_block_summary_w", "dash_prefill_w", "dash_prefill_ex",
-           "dash_decode_ex", "dash_prefill_backward_workspace_size", "dash_prefill_backward")
+           "dash_decode_noalloc", "dash_decode_noalloc_status", "dash_block_summary_w", "dash_prefill_w", "dash_prefill_ex",
+           "dash_decode_ex", "dash_prefill_backward_workspace_size", "dash_prefill_backward",
+           "dash_prefill_dump", "dash_decode_dump")
 
 HEAD_AGGREGATION = 1       # flag of dash_prefill_ex / dash_decode_ex
 
@@ -87,6 +88,9 @@ def lib():
     L.dash_prefill_profiled.argtypes = [_p] * 4 + [_i] * 6 + [_f, _f, _p, _sz, _p, _p]
     L.dash_decode_profiled.argtypes = [_p] * 6 + [_i] * 6 + [_f, _f, _p, _sz, _p, _p]
     L.dash_decode_noalloc.argtypes = [_p] * 6 + [_i] * 6 + [_f, _f, _p]
+    L.dash_decode_noalloc_status.argtypes = [_p]
+    L.dash_prefill_dump.argtypes = [_p] * 5 + [_i] * 6 + [_f, _f, ctypes.c_uint, _p, _i, _p, _p, _p, _sz, _p]
+    L.dash_decode_dump.argtypes = [_p] * 6 + [_i] * 6 + [_f, _f, ctypes.c_uint, _p, _p, _p, _p, _sz, _p]
     for name in EXPORTS:
         if name not in ("dash_status_string", "dash_prefill_workspace_size", "dash_decode_workspace_size",
                         "dash_prefill_backward_workspace_size"):
@@ -368,8 +372,10 @@ def dash_decode(q, k_cache, v_cache, ksum, kv_len, out=None, alpha=1.5, coarse_s
 def dash_decode_noalloc(q, k_cache, v_cache, ksum, kv_len, out=None, alpha=1.5, coarse_scale=1.0,
                         block=64, stream=None):
     """dash_decode on the library's fixed 32 MiB device scratch array, for callers that cannot
-    allocate device memory where they decode (graph capture, real-time loops, foreign
-    allocators).  No workspace; calls that overlap on the GPU race on the shared array."""
+    allocate device memory where they decode (real-time loops that must not synchronise the
+    device through cudaMalloc / cudaFree, memory owned by a foreign allocator).  No
+    workspace; calls that overlap on the GPU race on the shared array.  The device status
+    of the call is read with dash_decode_noalloc_status."""
     B, Hq, d = q.shape
     Hkv, Tmax = k_cache.shape[1], k_cache.shape[2]
     if out is None:
@@ -380,6 +386,68 @@ def dash_decode_noalloc(q, k_cache, v_cache, ksum, kv_len, out=None, alpha=1.5, 
                                    B, Hq, Hkv, Tmax, d, block, float(alpha), float(coarse_scale), _stream(stream))
     _check("dash_decode_noalloc", rc)
     return out
+
+
+def dash_prefill_dump(q, k, v, rows, alpha=1.5, coarse_scale=1.0, w_summary=None, flags=0, out=None,
+                      workspace=None, block=64, stream=None):
+    """dash_prefill plus the weights its fine stage applied to the listed rows.
+
+    rows: sequence of (b, h, t).  Returns (out, workspace, x, p) with x, p fp32
+    [len(rows), T // 64]: x_j of every block in the row's tile list (NaN when not listed)
+    and the applied weight p_j (0 when not selected or not listed)."""
+    B, Hq, T, d = q.shape
+    Hkv = k.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(prefill_workspace_size(B, Hq, Hkv, T, d, block), q.device)
+    slot = torch.full((B, Hq, T), -1, dtype=torch.int32)
+    r = torch.as_tensor([list(x) for x in rows], dtype=torch.long).reshape(-1, 3)
+    slot[r[:, 0], r[:, 1], r[:, 2]] = torch.arange(len(r), dtype=torch.int32)
+    slot = slot.to(q.device)
+    nbs = T // block
+    x = torch.empty(max(len(r), 1), max(nbs, 1), dtype=torch.float32, device=q.device)
+    p = torch.empty_like(x)
+    wp = _dev(w_summary, torch.float32, "w_summary") if w_summary is not None else None
+    rc = lib().dash_prefill_dump(_dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"),
+                                 _dev(v, torch.bfloat16, "v"), wp, _dev(out, torch.bfloat16, "out"),
+                                 B, Hq, Hkv, T, d, block, float(alpha), float(coarse_scale), int(flags),
+                                 _dev(slot, torch.int32, "row_slot"), len(r), _dev(x, torch.float32, "x"),
+                                 _dev(p, torch.float32, "p"), ctypes.c_void_p(workspace.data_ptr()),
+                                 workspace.numel(), _stream(stream))
+    _check("dash_prefill_dump", rc)
+    return out, workspace, x[:len(r), :nbs], p[:len(r), :nbs]
+
+
+def dash_decode_dump(q, k_cache, v_cache, ksum, kv_len, alpha=1.5, coarse_scale=1.0, flags=0, out=None,
+                     workspace=None, block=64, stream=None):
+    """dash_decode plus the weights its attention kernel applied.  Returns (out, workspace,
+    x, p, tau): x, p fp32 [B, Hq, Tmax // 64] (NaN / 0 for blocks outside the group's list),
+    tau fp32 [B, Hq]."""
+    B, Hq, d = q.shape
+    Hkv, Tmax = k_cache.shape[1], k_cache.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(decode_workspace_size(B, Hq, Hkv, Tmax, d, block), q.device)
+    nbs = Tmax // block
+    x = torch.empty(B, Hq, max(nbs, 1), dtype=torch.float32, device=q.device)
+    p = torch.empty_like(x)
+    tau = torch.empty(B, Hq, dtype=torch.float32, device=q.device)
+    rc = lib().dash_decode_dump(_dev(q, torch.bfloat16, "q"), _dev(k_cache, torch.bfloat16, "k_cache"),
+                                _dev(v_cache, torch.bfloat16, "v_cache"), _dev(ksum, torch.float32, "ksum"),
+                                _dev(kv_len, torch.int32, "kv_len"), _dev(out, torch.bfloat16, "out"),
+                                B, Hq, Hkv, Tmax, d, block, float(alpha), float(coarse_scale), int(flags),
+                                _dev(x, torch.float32, "x"), _dev(p, torch.float32, "p"),
+                                _dev(tau, torch.float32, "tau"), ctypes.c_void_p(workspace.data_ptr()),
+                                workspace.numel(), _stream(stream))
+    _check("dash_decode_dump", rc)
+    return out, workspace, x[:, :, :nbs], p[:, :, :nbs], tau
+
+
+def dash_decode_noalloc_status(stream=None) -> int:
+    """Device status of the last dash_decode_noalloc on the current device (syncs the stream)."""
+    return lib().dash_decode_noalloc_status(_stream(stream))
 
 
 def dash_get_device_status(workspace, stream=None) -> int:

@@ -30,10 +30,16 @@ def _built():
 @pytest.mark.parametrize("d,T", [(64, 512), (128, 1000), (128, 63)])
 def test_block_summary_vs_oracle(d, T):
     _, (q, k, v) = inputs.make("16k", T=T, d=d, Hq=4, Hkv=2, B=2)
+    if T < 64:
+        # no complete block: nothing is written (a NaN-filled buffer stays NaN)
+        ks = torch.full((2, 2, 1, d), float("nan"), device="cuda")
+        da.dash_block_summary(k.cuda(), ks)
+        torch.cuda.synchronize()
+        assert ks.isnan().all()
+        assert oracle.block_summary(k, 64).shape[2] == 0
+        return
     ks = da.dash_block_summary(k.cuda()).cpu().double().numpy()
     ref = oracle.block_summary(k, 64)
-    if T < 64:
-        return
     assert ks.shape == ref.shape
     assert np.abs(ks - ref).max() <= 1e-6 * max(1.0, np.abs(ref).max())
 
@@ -49,7 +55,9 @@ def test_tiny_config_all_rows():
 @pytest.mark.parametrize("cs", [0.0, 8.0, 32.0, 1e4])
 def test_tiny_scales(cs):
     wl, (q, k, v) = inputs.make("tiny")
-    check_prefill(q, k, v, 1.5, cs, all_rows(1, 1, wl.T), f"tiny cs={cs}")
+    # at cs = 1e4 the scores' bf16 hi + lo rounding (A) exceeds 1e-4: band widened by 2 A
+    res, _, _ = check_prefill(q, k, v, 1.5, cs, all_rows(1, 1, wl.T), f"tiny cs={cs}", strict_band=cs < 1e3)
+    print(cs, res)
 
 
 @pytest.mark.parametrize("alpha", [1.25, 2.0, 3.0])
@@ -157,7 +165,7 @@ def test_workload_sampled_rows(name):
 @pytest.mark.parametrize("alpha", [1.25, 1.5, 2.0])
 def test_32k_alpha_sweep_sampled_rows(alpha):
     wl, (q, k, v) = inputs.make("32k")
-    rows = stratified_rows(wl.B, wl.Hq, wl.T, 1024, seed=wl.seed + int(alpha * 100))
+    rows = stratified_rows(wl.B, wl.Hq, wl.T, 2048 - 17 * wl.Hq, seed=wl.seed + int(alpha * 100))
     res, _, _ = check_prefill(q, k, v, alpha, calibrated_scale("32k"), rows, f"32k alpha={alpha}")
     print(alpha, res)
 
@@ -169,7 +177,9 @@ def test_decode_small_ragged_lengths():
     _, (q4, k, v) = inputs.make("16k", B=B, Hq=Hq, Hkv=Hkv, T=Tmax, d=d, n_topics=16, seed=123)
     lens = [700, 333, 64, 1]
     q = torch.stack([q4[b, :, lens[b] - 1] for b in range(B)])
-    check_decode(q, k, v, lens, 1.5, 0.05, "decode small")
+    res, _, _ = check_decode(q, k, v, lens, 1.5, 0.05, "decode small")
+    assert res[1] is not None
+    print(res)
 
 
 def test_decode_equals_last_prefill_row():
@@ -209,16 +219,17 @@ def test_decode_invalid_lengths_write_zeros():
 ])
 def test_decode_group_sizes(B, Hq, Hkv, Tmax, d, lens):
     _, (q, kc, vc, _) = inputs.make("decode96k", B=B, Hq=Hq, Hkv=Hkv, T=Tmax, d=d, seed=77 + Hq)
-    (mx, mean), _, ws = check_decode(q, kc, vc, lens, 1.5, calibrated_scale("decode96k"),
-                                     f"decode G={Hq // Hkv} d={d}")
-    print("decode groups", Hq // Hkv, d, mx, mean)
+    res, _, ws = check_decode(q, kc, vc, lens, 1.5, calibrated_scale("decode96k"),
+                              f"decode G={Hq // Hkv} d={d}")
+    print("decode groups", Hq // Hkv, d, res)
 
 
 def test_decode_96k_workload_all_rows():
     wl, (q, kc, vc, kv_len) = inputs.make("decode96k")
-    (mx, mean), _, ws = check_decode(q, kc, vc, kv_len.tolist(), wl.alpha, calibrated_scale("decode96k"), "decode96k")
+    res, _, ws = check_decode(q, kc, vc, kv_len.tolist(), wl.alpha, calibrated_scale("decode96k"), "decode96k")
+    assert res[1] is not None and res[1]["selected"] > 0
     st = da.dash_decode_stats(ws)
-    print("decode96k", mx, mean, st, "sparsity", 1 - st["selected_pairs"] / st["scored_pairs"])
+    print("decode96k", res, st, "sparsity", 1 - st["selected_pairs"] / st["scored_pairs"])
 
 
 def test_decode_threshold_start_does_not_change_the_result():
