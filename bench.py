@@ -6,7 +6,9 @@
 
 A step is one full prefill (block summaries, coarse scores + alpha-entmax thresholds +
 block lists, prior-weighted fine attention) of the workload (default: the 16K prefill
-at 75 % block sparsity).  `value` is prefill tokens/s over all ranks with inputs resident
+at 75 % block sparsity).  The other prefill configurations (tiny, the 32K alpha sweep and
+the 96K prefill at ~93.75 % block sparsity) are timed with the same steps and warm-up and
+reported in `other_prefill_configs`.  `value` is prefill tokens/s over all ranks with inputs resident
 in HBM; `e2e` is the same through the C ABI's host-buffer entry point (host<->device
 copies inside the timed region).  The `decode` object times one decode step of the 96K
 workload (B=8, cache 98304): its step is replayed from a CUDA graph, as a serving loop
@@ -172,30 +174,35 @@ def max_over_ranks(ws, x):
 
 # ------------------------------------------------------------------ GPU arms
 
-def bench_prefill(args, ws, rank, local):
+def _tile_positions(Hq, Hkv):
+    """Positions per work tile: P = min(64, largest power of two <= 128 / G)."""
+    return min(64, 1 << (max(1, 128 // (Hq // Hkv)).bit_length() - 1))
+
+
+def time_prefill(wl, qd, kd, vd, alpha, cs, steps, warmup, flush, ws, wsb=None, clocks_dev=None):
+    """Times `steps` full prefills (after `warmup` untimed ones) of one workload with the
+    profiled entry point (CUDA events between the three kernels, on the launching stream;
+    L2 flushed before each step) and derives the roofline figures of the fine kernel and of
+    the block-summary kernel from the call's own counters.  Returns a plain dict."""
     import torch
     from sparse_hierarchical_attention_pool_b200 import dash_attn as da
-    from sparse_hierarchical_attention_pool_b200 import inputs
-
-    wl, (q, k, v) = inputs.make(args.workload)
-    cal = calibrated(args.workload)
-    cs, alpha = cal["coarse_scale"], wl.alpha
     B, Hq, Hkv, T, d = wl.B, wl.Hq, wl.Hkv, wl.T, wl.d
-    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     out = torch.empty_like(qd)
-    wsb = da.alloc_workspace(da.prefill_workspace_size(B, Hq, Hkv, T, d))
-    flush = L2Flush()
-    for _ in range(args.warmup):
+    if wsb is None:
+        wsb = da.alloc_workspace(da.prefill_workspace_size(B, Hq, Hkv, T, d))
+    for _ in range(warmup):
         flush()
         da.dash_prefill(qd, kd, vd, out, alpha, cs, wsb)
     torch.cuda.synchronize()
     barrier(ws)
     torch.cuda.synchronize()
-    clk = ClockSampler(local)
-    clk.start()
-    time.sleep(0.3)
+    clk = None
+    if clocks_dev is not None:
+        clk = ClockSampler(clocks_dev)
+        clk.start()
+        time.sleep(0.3)
     evs = []
-    for _ in range(args.steps):
+    for _ in range(steps):
         flush()
         e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
         da.dash_prefill_profiled(qd, kd, vd, out, alpha, cs, wsb, e)
@@ -203,22 +210,21 @@ def bench_prefill(args, ws, rank, local):
     torch.cuda.synchronize()
     barrier(ws)
     torch.cuda.synchronize()
-    clocks = clk.stop()
+    clocks = clk.stop() if clk is not None else None
+    mean = lambda xs: sum(xs) / len(xs)  # noqa: E731
     tot = [e[0].elapsed_time(e[3]) for e in evs]
     summ = [e[0].elapsed_time(e[1]) for e in evs]
     coarse = [e[1].elapsed_time(e[2]) for e in evs]
     fine = [e[2].elapsed_time(e[3]) for e in evs]
-    mean = lambda xs: sum(xs) / len(xs)  # noqa: E731
     step_ms = max_over_ranks(ws, mean(tot))
     st = da.dash_prefill_stats(wsb)
     if da.dash_get_device_status(wsb) != 0:
-        raise RuntimeError("device status not clean after the timed prefill")
-
+        raise RuntimeError(f"device status not clean after the timed prefill of {wl.name}")
     # algorithmic work: fine FLOPs = 4 d * sum_rows |L_row|; coarse FLOPs = 2 d * sum_rows bt
     diag_tokens = sum((t % 64) + 1 for t in range(T)) * B * Hq
     fine_alg = 4.0 * d * (64.0 * st["selected_pairs"] + diag_tokens)
     coarse_alg = 2.0 * d * st["scored_pairs"]
-    P = min(64, 1 << (max(1, 128 // (Hq // Hkv)).bit_length() - 1))
+    P = _tile_positions(Hq, Hkv)
     ntiles = B * Hkv * ((T + P - 1) // P)
     fine_exec = 4.0 * d * 64.0 * 128.0 * (st["union_blocks"] + ntiles)
     pk, pk_kind = peaks()
@@ -229,9 +235,55 @@ def bench_prefill(args, ws, rank, local):
     nb = T // 64
     sum_bytes = B * Hkv * T * d * 2 + B * Hkv * nb * d * (4 + 2 + 2)
     sum_gbs = sum_bytes / (mean(summ) * 1e-3) / 1e9
-    summary_roofline = {"bound": "hbm", "kernel": "block_summary_kernel", "bytes_per_launch": sum_bytes,
-                        "achieved": round(sum_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                        "frac": round(sum_gbs / pk["hbm_gbs"], 4)}
+    G = Hq // Hkv
+    fine_kernel = "fine_tc_kernel" if G <= 16 else "fine_mma_kernel"
+    return {
+        "workload": wl.name, "alpha": alpha, "coarse_scale": cs, "seed": wl.seed,
+        "B": B, "Hq": Hq, "Hkv": Hkv, "T": T, "d": d,
+        "steps": steps, "warmup": warmup,
+        "step_ms": step_ms, "tok_s": ws * B * T / (step_ms * 1e-3),
+        "stage_ms": {"block_summary": mean(summ), "coarse_select": mean(coarse), "fine_attention": fine_ms},
+        "stats": st, "clocks": clocks,
+        "sparsity": 1.0 - st["selected_pairs"] / max(1, st["scored_pairs"]),
+        "roofline": {"bound": "tensor", "kernel": fine_kernel, "achieved": round(achieved, 2),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_source": f"{pk_kind} bf16_tflops (burst)",
+                     "algorithmic_flops_per_launch": fine_alg,
+                     "executed_flops_per_launch": fine_exec,
+                     "executed_tflops": round(fine_exec / (fine_ms * 1e-3) / 1e12, 2),
+                     "executed_frac": round(fine_exec / (fine_ms * 1e-3) / 1e12 / peak, 4),
+                     "inflation": round(fine_exec / fine_alg, 3)},
+        "coarse_algorithmic_flops": coarse_alg,
+        "summary_roofline": {"bound": "hbm", "kernel": "block_summary_kernel", "bytes_per_launch": sum_bytes,
+                             "achieved": round(sum_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                             "frac": round(sum_gbs / pk["hbm_gbs"], 4)},
+        "launches_per_step": 3,
+        "l2": "flushed before every timed step",
+        "_wsb": wsb, "_out": out, "_fine_alg": fine_alg, "_fine_exec": fine_exec,
+    }
+
+
+def public(d):
+    """The JSON-ready part of a time_prefill result."""
+    return {k: v for k, v in d.items() if not k.startswith("_")}
+
+
+def bench_prefill(args, ws, rank, local):
+    import torch
+    from sparse_hierarchical_attention_pool_b200 import dash_attn as da
+    from sparse_hierarchical_attention_pool_b200 import inputs
+
+    wl, (q, k, v) = inputs.make(args.workload)
+    cal = calibrated(args.workload)
+    cs, alpha = cal["coarse_scale"], wl.alpha
+    B, Hq, Hkv, T, d = wl.B, wl.Hq, wl.Hkv, wl.T, wl.d
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    flush = L2Flush()
+    core = time_prefill(wl, qd, kd, vd, alpha, cs, args.steps, args.warmup, flush, ws, clocks_dev=local)
+    wsb, out = core["_wsb"], core["_out"]
+    fine_alg, fine_exec = core["_fine_alg"], core["_fine_exec"]
+    st = core["stats"]
+    mean = lambda xs: sum(xs) / len(xs)  # noqa: E731
     # context only: dense causal attention FLOPs and torch's SDPA (flash) on the same tensors
     dense_flops = 4.0 * d * B * Hq * T * (T + 1) / 2
     import torch.nn.functional as F
@@ -251,27 +303,20 @@ def bench_prefill(args, ws, rank, local):
                "torch_sdpa_tflops": round(dense_flops / (sdpa_ms * 1e-3) / 1e12, 1),
                "note": "library dense attention on the same inputs, for context only"}
     G = Hq // Hkv
-    fine_kernel = "fine_tc_kernel" if G <= 16 else "fine_mma_kernel"
     traffic = (recorded_traffic("fine_tc_kernel", source_sha("fine_tc.cu", "sm100.cuh", "common.cuh"), args.workload)
                if G <= 16 else recorded_traffic("fine_mma_kernel", source_sha("fine_mma.cu", "mma_sync.cuh", "common.cuh"),
                                                 args.workload))
+    core["roofline"]["traffic"] = traffic
     res = {
-        "step_ms": step_ms,
-        "tok_s": ws * B * T / (step_ms * 1e-3),
-        "stage_ms": {"block_summary": mean(summ), "coarse_select": mean(coarse), "fine_attention": fine_ms},
-        "clocks": clocks,
+        "step_ms": core["step_ms"],
+        "tok_s": core["tok_s"],
+        "stage_ms": core["stage_ms"],
+        "clocks": core["clocks"],
         "stats": st,
-        "sparsity": 1.0 - st["selected_pairs"] / max(1, st["scored_pairs"]),
-        "roofline": {"bound": "tensor", "kernel": fine_kernel, "achieved": round(achieved, 2),
-                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "traffic": traffic, "peak_source": f"{pk_kind} bf16_tflops (burst)",
-                     "algorithmic_flops_per_launch": fine_alg,
-                     "executed_flops_per_launch": fine_exec,
-                     "executed_tflops": round(fine_exec / (fine_ms * 1e-3) / 1e12, 2),
-                     "executed_frac": round(fine_exec / (fine_ms * 1e-3) / 1e12 / peak, 4),
-                     "inflation": round(fine_exec / fine_alg, 3)},
-        "coarse_algorithmic_flops": coarse_alg,
-        "summary_roofline": summary_roofline,
+        "sparsity": core["sparsity"],
+        "roofline": core["roofline"],
+        "coarse_algorithmic_flops": core["coarse_algorithmic_flops"],
+        "summary_roofline": core["summary_roofline"],
         "context": context,
         "launches_per_step": 3,
         "wl": wl, "cs": cs,
@@ -301,6 +346,70 @@ def bench_prefill(args, ws, rank, local):
         res["backward"] = bench_backward(args, ws, qd, kd, vd, out, wl, cs, st, fine_alg, fine_exec, flush)
     del flush, wsb
     return res
+
+
+def bench_other_prefills(args, ws, rank):
+    """The prefill configurations besides the headline one, each timed with the same steps
+    and warm-up: the tiny configuration (its oracle timed in full on the host, rank 0 at
+    N = 1), the 32K workload at alpha 1.25 / 1.5 / 2 with one coarse scale, and the 96K
+    workload at ~93.75 % block sparsity (whose block-summary kernel reads 201 MB of keys, a
+    size at which that kernel is not launch-bound)."""
+    import torch
+    from sparse_hierarchical_attention_pool_b200 import inputs
+    flush = L2Flush()
+    res = {}
+    # tiny: B=1, Hq=Hkv=1, T=512, d=64, fp32 N(0, 1) rounded to bf16
+    wl, (q, k, v) = inputs.make("tiny")
+    cs = calibrated("tiny")["coarse_scale"]
+    tiny = public(time_prefill(wl, q.cuda(), k.cuda(), v.cuda(), wl.alpha, cs, args.steps, args.warmup, flush, ws))
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        tiny["cpu_baseline"] = oracle_full_tiny(wl, q, k, v, cs)
+    res["tiny"] = tiny
+    # 32K: one input set and coarse scale, three alphas
+    wl, (q, k, v) = inputs.make("32k")
+    cs = calibrated("32k")["coarse_scale"]
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    del q, k, v
+    sweep = {}
+    wsb = None
+    for alpha in (1.25, 1.5, 2.0):
+        r = time_prefill(wl, qd, kd, vd, alpha, cs, args.steps, args.warmup, flush, ws, wsb=wsb)
+        wsb = r["_wsb"]
+        sweep[str(alpha)] = public(r)
+    res["32k_alpha_sweep"] = sweep
+    del qd, kd, vd, wsb, r
+    torch.cuda.empty_cache()
+    # 96K: B=1, Hq=32, Hkv=8, T=98304
+    wl, (q, k, v) = inputs.make("96k")
+    cs = calibrated("96k")["coarse_scale"]
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    del q, k, v
+    res["96k"] = public(time_prefill(wl, qd, kd, vd, wl.alpha, cs, args.steps, args.warmup, flush, ws))
+    del qd, kd, vd
+    torch.cuda.empty_cache()
+    return res
+
+
+def oracle_full_tiny(wl, q, k, v, cs):
+    """The fp64 oracle over every row of the tiny configuration, timed on the host."""
+    import oracle
+    oracle.build()
+    rows = [(0, 0, t) for t in range(wl.T)]
+    qr = oracle.gather_q_rows(q, rows)
+    threads = len(os.sched_getaffinity(0))
+    oracle.forward_rows(qr, k, v, rows[:8], wl.Hq, 64, wl.alpha, cs, nthreads=threads)
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.forward_rows(qr, k, v, rows, wl.Hq, 64, wl.alpha, cs, nthreads=threads)
+        reps += 1
+        if time.perf_counter() - t0 > 1.0:
+            break
+    dt = (time.perf_counter() - t0) / reps
+    return {"value": wl.T / dt, "unit": "tok/s", "cores": threads, "kind": "oracle",
+            "ms_per_step": dt * 1e3,
+            "sample": f"every row of the tiny configuration (T={wl.T}), fp64 C oracle with OpenMP over rows, "
+                      f"mean of {reps} full passes"}
 
 
 def backward_only(args, ws):
@@ -568,6 +677,8 @@ def main():
                     help="16k-coherent is not a target workload: block-coherent query topics")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the prefill backward measurement")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the tiny, 32K alpha-sweep and 96K prefill measurements")
     ap.add_argument("--backward-only", action="store_true",
                     help="time only the prefill backward and print its object (for profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -604,6 +715,7 @@ def main():
             _REPLICAS.close()
         return
     pre = bench_prefill(args, ws, rank, local)
+    others = None if args.no_other_configs else bench_other_prefills(args, ws, rank)
     dec = None if args.no_decode else bench_decode(args, ws, rank, local)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -631,6 +743,7 @@ def main():
             "prefill_stats": pre["stats"],
             "backward": pre.get("backward"),
             "decode": dec,
+            "other_prefill_configs": others,
         }
         print(json.dumps(line), flush=True)
     if ws > 1:

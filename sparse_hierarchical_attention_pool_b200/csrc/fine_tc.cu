@@ -11,13 +11,17 @@
 //
 // One CTA per tile.  The tile's listed blocks (steps s = 0 .. n-1, own block last) are
 // dealt alternately to two softmax groups (group s & 1), each with its own TMEM S buffer,
-// P buffer, O accumulator, row-sum column and running max; the two partial softmaxes are
-// merged in the epilogue (exactly as split-KV partials).  The per-step work of a row is a
-// serial chain (load S, row stats, weights, exponentials, P), so two groups keep two chains
-// in flight while sharing the Q tile and every K/V load.  Warps:
-//   8 SPLIT            TMA producer (one lane): the Q tile once (one 64-column box per head
-//                      and half of d), then K, the summary rows and V of every listed
-//                      block, 4-stage ring;
+// two P buffers (steps alternate between them), O accumulator, row-sum column and running
+// max; the two partial softmaxes are merged in the epilogue (exactly as split-KV partials).
+// The per-step work of a row is a serial chain (load S, row stats, weights, exponentials,
+// P), so two groups keep two chains in flight while sharing the Q tile and every K/V load;
+// with two P buffers a group writes P_s while the tensor core still reads P_{s-2}, and
+// waits for its previous product only to rescale O.  Warps:
+//   8 SPLIT            K producer (one lane): the Q tile once (one 64-column box per head
+//                      and half of d), then K and the summary rows of every listed block,
+//                      3-stage ring (a stage is free once S of its block is computed);
+//   8 SPLIT + 3        V producer (one lane): V of every listed block, 3-stage ring (a stage
+//                      is free once the block's P V product is done);
 //   8 SPLIT + 1        S issuer (one lane): S_s = Q [K_s | kbar_hi | kbar_lo]^T (M=128, N=80
 //                      with the summary atoms at columns 64 and 72) into the S buffer of
 //                      group s & 1 as soon as block s is loaded and that group has read
@@ -32,7 +36,10 @@
 //                      of one group sharing TMEM lanes 32 (warp % 4).. split the row's keys
 //                      and exchange partial row sums and maxima through shared memory behind
 //                      a named barrier).  Online softmax in the log2 domain; O_g is rescaled
-//                      in TMEM only when the running max grows by more than 2^8.
+//                      in TMEM only when the running max grows by more than 2^8.  Of every 8
+//                      exponentials, 2 kFinePolyPairs run as a polynomial on the FMA pipe
+//                      (poly_exp2) and the rest on the SFU, so that neither unit alone sets
+//                      the pace.
 // Head aggregation (optional): the rows of a position average their block weights
 // through shared memory (one group barrier per step) and share log of the mean as prior.
 // Operands: Q, K, P K-major and V MN-major, all 128-byte swizzled (TMA writes that layout).
@@ -48,9 +55,41 @@
 
 namespace dash {
 
-constexpr int kTcStages = 4;
+constexpr int kKStages = 3;            // K (+ summary rows) ring
+constexpr int kVStages = 3;            // V ring
 constexpr int kFineSplit = 1;          // threads per tile row in each softmax group
+constexpr int kFinePolyPairs = 1;      // pairs of every 4 whose 2^x runs on the FMA pipe
 constexpr float kLazyRescale = 8.0f;   // log2 units: p values stay below 2^8 between rescales
+
+// 2^x for x <= 8 on the FMA and integer pipes.  Cody-Waite style split x = n + f with
+// n = round(x) (added to the exponent field) and f in [-1/2, 1/2], where 2^f comes from a
+// degree-3 polynomial fitted here for the least maximum relative error on that interval
+// (iteratively reweighted least squares: max relative error 7.5e-5 in fp32, far below the
+// bf16 rounding every P value gets).  Arguments below -125 (masked keys, -inf) give
+// 2^-125 (about 2e-38), which no fp32 sum of the row can see.
+__device__ __forceinline__ uint64_t poly_exp2_x2(uint64_t x2) {
+    using namespace sm100;
+    float a, b;
+    f2_unpack(x2, a, b);
+    a = fmaxf(a, -125.0f);
+    b = fmaxf(b, -125.0f);
+    const uint64_t xc = f2_pack(__float_as_uint(a), __float_as_uint(b));
+    const uint32_t kMagic = 0x4B400000u;                          // 1.5 * 2^23: rounds to an integer
+    const uint64_t magic2 = f2_pack(kMagic, kMagic);
+    const uint64_t t2 = f2_add(xc, magic2);                       // n in the low mantissa bits
+    const uint64_t nmagic2 = f2_pack(0xCB400000u, 0xCB400000u);   // -1.5 * 2^23
+    const uint64_t f2 = f2_add(xc, f2_neg(f2_add(t2, nmagic2)));  // f = x - n
+    const uint64_t c3 = f2_pack(0x3D61FBB0u, 0x3D61FBB0u);        // 0.0551716685
+    const uint64_t c2 = f2_pack(0x3E786F0Eu, 0x3E786F0Eu);        // 0.2426111400
+    const uint64_t c1 = f2_pack(0x3F31798Du, 0x3F31798Du);        // 0.6932609677
+    const uint64_t c0 = f2_pack(0x3F7FFB49u, 0x3F7FFB49u);        // 0.9999280572
+    const uint64_t pf = f2_fma(f2_fma(f2_fma(c3, f2, c2), f2, c1), f2, c0);
+    uint32_t plo, phi, tlo, thi;
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(plo), "=r"(phi) : "l"(pf));
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(tlo), "=r"(thi) : "l"(t2));
+    // (bits(t) << 23) == n << 23 modulo 2^32: the magic number's bits vanish in the shift
+    return f2_pack(plo + (tlo << 23), phi + (thi << 23));
+}
 
 template <int D>
 struct TcLayout {
@@ -61,12 +100,12 @@ struct TcLayout {
     static constexpr uint32_t kK = (D / 64) * kKHalf;
     static constexpr uint32_t kVHalf = 64 * 128;                // 64 keys x 64 bf16
     static constexpr uint32_t kV = (D / 64) * kVHalf;
-    static constexpr uint32_t kStage = kK + kV;                 // K (+ summary rows) then V
     static constexpr uint32_t kP = 128 * 128;                   // 128 rows x 64 keys bf16
     static constexpr uint32_t off_q = 0;
-    static constexpr uint32_t off_kv = kQ;
-    static constexpr uint32_t off_p = kQ + kTcStages * kStage;  // one P buffer per group
-    static constexpr uint32_t off_ones = off_p + 2 * kP;        // 16 x 64 bf16 ones (B of the row sum)
+    static constexpr uint32_t off_k = kQ;                       // K ring
+    static constexpr uint32_t off_v = off_k + kKStages * kK;    // V ring
+    static constexpr uint32_t off_p = off_v + kVStages * kV;    // P buffers [group][2]
+    static constexpr uint32_t off_ones = off_p + 4 * kP;        // 16 x 64 bf16 ones (B of the row sum)
     static constexpr uint32_t bytes = off_ones + 2048 + 1024;   // + alignment slack
     // TMEM columns: S of group 0 and 1, O of group 0 and 1, row sums of group 0 and 1
     static constexpr uint32_t colS = 96;                        // S buffer of group g at g * 96 (80 used)
@@ -75,13 +114,14 @@ struct TcLayout {
 };
 constexpr uint32_t kTmemCols = 512;
 
-// barrier slots
-enum : int { B_Q = 0, B_KV_FULL = 1, B_KV_EMPTY = 1 + kTcStages, B_S_FULL = 1 + 2 * kTcStages,
-             B_S_FREE = B_S_FULL + 2, B_P_FULL = B_S_FREE + 2, B_PV_DONE = B_P_FULL + 2,
-             B_DRAIN = B_PV_DONE + 2, B_DRAIN2 = B_DRAIN + 1, B_COUNT = B_DRAIN2 + 1 };
+// barrier slots (P_FULL and PV_DONE per P buffer: index 2 group + buffer)
+enum : int { B_Q = 0, B_K_FULL = 1, B_K_EMPTY = B_K_FULL + kKStages, B_V_FULL = B_K_EMPTY + kKStages,
+             B_V_EMPTY = B_V_FULL + kVStages, B_S_FULL = B_V_EMPTY + kVStages, B_S_FREE = B_S_FULL + 2,
+             B_P_FULL = B_S_FREE + 2, B_PV_DONE = B_P_FULL + 4, B_DRAIN = B_PV_DONE + 4,
+             B_DRAIN2 = B_DRAIN + 1, B_COUNT = B_DRAIN2 + 1 };
 
 template <int D, int SPLIT, bool AGG, bool DUMP>
-__global__ void __launch_bounds__((8 * SPLIT + 3) * 32, 1)
+__global__ void __launch_bounds__((8 * SPLIT + 4) * 32, 1)
 fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_hi,
                const __grid_constant__ CUtensorMap tm_lo, __nv_bfloat16* __restrict__ out,
@@ -97,6 +137,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     constexpr int RCOLS = D / SPLIT;            // O columns a thread rescales in its group
     constexpr int RCW = RCOLS < 32 ? RCOLS : 32;
     constexpr int kProducerWarp = 8 * SPLIT, kMmaSWarp = 8 * SPLIT + 1, kMmaPvWarp = 8 * SPLIT + 2;
+    constexpr int kVProducerWarp = 8 * SPLIT + 3;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t bars[B_COUNT];
     __shared__ uint32_t tmem_base_sh;
@@ -109,7 +150,8 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* const base_ptr = smem_raw + (base - raw);
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
-    auto kv_addr = [&](int st) { return base + L::off_kv + (uint32_t)st * L::kStage; };
+    auto k_addr = [&](int st) { return base + L::off_k + (uint32_t)st * L::kK; };
+    auto v_addr = [&](int st) { return base + L::off_v + (uint32_t)st * L::kV; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // group-major order (longest tiles of a group first): the CTAs in flight share one KV
@@ -128,13 +170,19 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (tid == 0) {
         abort_sh = 0;
         mbar_init(bar(B_Q), 1);
-        for (int st = 0; st < kTcStages; ++st) {
-            mbar_init(bar(B_KV_FULL + st), 1);
-            mbar_init(bar(B_KV_EMPTY + st), 1);
+        for (int st = 0; st < kKStages; ++st) {
+            mbar_init(bar(B_K_FULL + st), 1);
+            mbar_init(bar(B_K_EMPTY + st), 1);
+        }
+        for (int st = 0; st < kVStages; ++st) {
+            mbar_init(bar(B_V_FULL + st), 1);
+            mbar_init(bar(B_V_EMPTY + st), 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar(B_S_FULL + i), 1);
             mbar_init(bar(B_S_FREE + i), kGroupThreads);
+        }
+        for (int i = 0; i < 4; ++i) {
             mbar_init(bar(B_P_FULL + i), kGroupThreads);
             mbar_init(bar(B_PV_DONE + i), 1);
         }
@@ -180,22 +228,21 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 for (int h = 0; h < D / 64; ++h)
                     tma_load_2d(base + L::off_q + h * L::kQHalf + hl * g.P * 128, &tm_q, h * 64, row, bar(B_Q));
             }
-            int last_armed[kTcStages];
-            for (int st = 0; st < kTcStages; ++st) last_armed[st] = -1;
+            int last_armed[kKStages];
+            for (int st = 0; st < kKStages; ++st) last_armed[st] = -1;
             for (int s = 0; s < n; ++s) {
-                const int st = s % kTcStages;
-                if (s >= kTcStages && !mbar_wait(bar(B_KV_EMPTY + st), ((s / kTcStages) - 1) & 1, abort_flag)) break;
+                const int st = s % kKStages;
+                if (s >= kKStages && !mbar_wait(bar(B_K_EMPTY + st), ((s / kKStages) - 1) & 1, abort_flag)) break;
                 const int j = s < U ? lst[s] : bt;
                 const int row = bg * g.T + j * kBlock;
                 // the summary atoms: 8 rows of kbar hi / lo starting at block j (the own block,
                 // whose x is not used, reads a neighbour; rows past the array read zeros)
                 const int srow = g.nbs > 0 ? bg * g.nbs + min(j, g.nbs - 1) : 0;
-                mbar_arrive_expect_tx(bar(B_KV_FULL + st), (uint32_t)((2 * kBlock + 16) * D * 2));
+                mbar_arrive_expect_tx(bar(B_K_FULL + st), (uint32_t)((kBlock + 16) * D * 2));
                 for (int h = 0; h < D / 64; ++h) {
-                    tma_load_2d(kv_addr(st) + h * L::kKHalf, &tm_k, h * 64, row, bar(B_KV_FULL + st));
-                    tma_load_2d(kv_addr(st) + h * L::kKHalf + 64 * 128, &tm_hi, h * 64, srow, bar(B_KV_FULL + st));
-                    tma_load_2d(kv_addr(st) + h * L::kKHalf + 72 * 128, &tm_lo, h * 64, srow, bar(B_KV_FULL + st));
-                    tma_load_2d(kv_addr(st) + L::kK + h * L::kVHalf, &tm_v, h * 64, row, bar(B_KV_FULL + st));
+                    tma_load_2d(k_addr(st) + h * L::kKHalf, &tm_k, h * 64, row, bar(B_K_FULL + st));
+                    tma_load_2d(k_addr(st) + h * L::kKHalf + 64 * 128, &tm_hi, h * 64, srow, bar(B_K_FULL + st));
+                    tma_load_2d(k_addr(st) + h * L::kKHalf + 72 * 128, &tm_lo, h * 64, srow, bar(B_K_FULL + st));
                 }
                 last_armed[st] = s;
             }
@@ -203,8 +250,29 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 // let every load this thread started land before the CTA exits
                 volatile int dummy = 0;
                 mbar_wait(bar(B_Q), 0, &dummy);
-                for (int st = 0; st < kTcStages; ++st)
-                    if (last_armed[st] >= 0) { dummy = 0; mbar_wait(bar(B_KV_FULL + st), (last_armed[st] / kTcStages) & 1, &dummy); }
+                for (int st = 0; st < kKStages; ++st)
+                    if (last_armed[st] >= 0) { dummy = 0; mbar_wait(bar(B_K_FULL + st), (last_armed[st] / kKStages) & 1, &dummy); }
+            }
+        }
+    } else if (warp == kVProducerWarp) {
+        // ------------------------------------------------------------ V producer
+        if (lane == 0) {
+            int last_armed[kVStages];
+            for (int st = 0; st < kVStages; ++st) last_armed[st] = -1;
+            for (int s = 0; s < n; ++s) {
+                const int st = s % kVStages;
+                if (s >= kVStages && !mbar_wait(bar(B_V_EMPTY + st), ((s / kVStages) - 1) & 1, abort_flag)) break;
+                const int j = s < U ? lst[s] : bt;
+                const int row = bg * g.T + j * kBlock;
+                mbar_arrive_expect_tx(bar(B_V_FULL + st), (uint32_t)(kBlock * D * 2));
+                for (int h = 0; h < D / 64; ++h)
+                    tma_load_2d(v_addr(st) + h * L::kVHalf, &tm_v, h * 64, row, bar(B_V_FULL + st));
+                last_armed[st] = s;
+            }
+            if (*abort_flag) {
+                volatile int dummy = 0;
+                for (int st = 0; st < kVStages; ++st)
+                    if (last_armed[st] >= 0) { dummy = 0; mbar_wait(bar(B_V_FULL + st), (last_armed[st] / kVStages) & 1, &dummy); }
             }
         }
     } else if (warp == kMmaSWarp) {
@@ -215,18 +283,19 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint32_t idesc_s = idesc_bf16(128, L::kKRows, false);
             bool ok = mbar_wait(bar(B_Q), 0, abort_flag);
             for (int s = 0; ok && s < n; ++s) {
-                const int st = s % kTcStages, sb = s & 1;
-                if (!mbar_wait(bar(B_KV_FULL + st), (s / kTcStages) & 1, abort_flag)) { ok = false; break; }
+                const int st = s % kKStages, sb = s & 1;
+                if (!mbar_wait(bar(B_K_FULL + st), (s / kKStages) & 1, abort_flag)) { ok = false; break; }
                 if (s >= 2 && !mbar_wait(bar(B_S_FREE + sb), ((s - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const int h = kk >> 2, wk = kk & 3;
                     const uint64_t a = smem_desc_sw128(base + L::off_q + h * L::kQHalf + wk * 32, 16, 1024);
-                    const uint64_t bk = smem_desc_sw128(kv_addr(st) + h * L::kKHalf + wk * 32, 16, 1024);
+                    const uint64_t bk = smem_desc_sw128(k_addr(st) + h * L::kKHalf + wk * 32, 16, 1024);
                     mma_bf16_ss(tmem + sb * L::colS, a, bk, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar(B_S_FULL + sb));
+                mma_commit(bar(B_K_EMPTY + st));
             }
             if (!ok) {
                 // every MMA this thread issued must finish before TMEM is released
@@ -237,31 +306,33 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
     } else if (warp == kMmaPvWarp) {
         // ------------------------------------------------------------ PV issuer
-        // O_g += P_p V_p and L_g += P_p 1 as soon as P_p is written; then the K/V stage of
-        // block p is free (S_p finished before the softmax could write P_p).
+        // O_g += P_p V_p and L_g += P_p 1 as soon as P_p is written and V_p has landed; then
+        // the V stage of block p and P buffer (p & 1, (p >> 1) & 1) are free again.
         if (lane == 0) {
             const uint32_t idesc_pv = idesc_bf16(128, D, true);
             const uint32_t idesc_l = idesc_bf16(128, 16, false);
             bool ok = true;
             for (int p = 0; p < n; ++p) {
-                const int bp = p & 1, stp = p % kTcStages;
-                if (!mbar_wait(bar(B_P_FULL + bp), (p >> 1) & 1, abort_flag)) { ok = false; break; }
+                const int gp = p & 1, pbuf = 2 * gp + ((p >> 1) & 1), stp = p % kVStages;
+                if (!mbar_wait(bar(B_P_FULL + pbuf), (p >> 2) & 1, abort_flag)) { ok = false; break; }
+                if (!mbar_wait(bar(B_V_FULL + stp), (p / kVStages) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t acc = p >= 2 ? 1u : 0u;          // first step of a group overwrites
+                const uint32_t pa = base + L::off_p + pbuf * L::kP;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t a = smem_desc_sw128(base + L::off_p + bp * L::kP + kk * 32, 16, 1024);
-                    const uint64_t bv = smem_desc_sw128(kv_addr(stp) + L::kK + kk * 2048, L::kVHalf, 1024);
-                    mma_bf16_ss(tmem + L::colO + bp * D, a, bv, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                    const uint64_t a = smem_desc_sw128(pa + kk * 32, 16, 1024);
+                    const uint64_t bv = smem_desc_sw128(v_addr(stp) + kk * 2048, L::kVHalf, 1024);
+                    mma_bf16_ss(tmem + L::colO + gp * D, a, bv, idesc_pv, (acc || kk > 0) ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t a = smem_desc_sw128(base + L::off_p + bp * L::kP + kk * 32, 16, 1024);
+                    const uint64_t a = smem_desc_sw128(pa + kk * 32, 16, 1024);
                     const uint64_t bo = smem_desc_sw128(base + L::off_ones + kk * 32, 16, 1024);
-                    mma_bf16_ss(tmem + L::colL + bp * 32, a, bo, idesc_l, (acc || kk > 0) ? 1u : 0u);
+                    mma_bf16_ss(tmem + L::colL + gp * 32, a, bo, idesc_l, (acc || kk > 0) ? 1u : 0u);
                 }
-                mma_commit(bar(B_PV_DONE + bp));
-                mma_commit(bar(B_KV_EMPTY + stp));
+                mma_commit(bar(B_PV_DONE + pbuf));
+                mma_commit(bar(B_V_EMPTY + stp));
             }
             if (!ok) {
                 mma_commit(bar(B_DRAIN2));
@@ -293,7 +364,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const uint32_t s_col = grp * L::colS + sp * KEYS;   // this thread's keys in its group's S buffer
         const uint32_t o_col = L::colO + grp * D + sp * RCOLS;   // O columns it rescales
         const uint32_t l_col = L::colL + grp * 32;
-        uint8_t* const prow = base_ptr + L::off_p + grp * L::kP + (r >> 3) * 1024 + (r & 7) * 128;
+        uint8_t* const prow0 = base_ptr + L::off_p + (2 * grp) * L::kP + (r >> 3) * 1024 + (r & 7) * 128;
         const int row_bar = 1 + grp * 4 + quarter;          // named barrier of the row's SPLIT warps
         float m_run = -INFINITY;
         bool ok = true;
@@ -392,9 +463,12 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     resc = true;
                 }
             }
-            // O_grp, L_grp and the P buffer were last used by this group's previous PV
-            if (i2 >= 1 && !wwait(bar(B_PV_DONE + grp), (i2 - 1) & 1)) { ok = false; continue; }
-            // p = 2^(s sm2 + log2 p_j - m): packed FMA, SFU exponent, bf16 pairs
+            // P buffer pb of this group was last read by its product two steps back
+            const int pb = i2 & 1;
+            uint8_t* const prow = prow0 + pb * L::kP;
+            if (i2 >= 2 && !wwait(bar(B_PV_DONE + 2 * grp + pb), ((i2 - 2) >> 1) & 1)) { ok = false; continue; }
+            // p = 2^(s sm2 + log2 p_j - m): packed FMA, exponent on the SFU or the FMA pipe,
+            // bf16 pairs
             const float c0 = lp2 - m_run;
             const uint64_t sm2x2 = f2_pack(__float_as_uint(sm2), __float_as_uint(sm2));
             const uint64_t c0x2 = f2_pack(__float_as_uint(c0), __float_as_uint(c0));
@@ -404,17 +478,26 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (active) {
 #pragma unroll
                     for (int q2 = 0; q2 < 4; ++q2) {
+                        const uint64_t e2 = f2_fma(f2_pack(sr[c * 8 + 2 * q2], sr[c * 8 + 2 * q2 + 1]), sm2x2, c0x2);
                         float e0, e1;
-                        f2_unpack(f2_fma(f2_pack(sr[c * 8 + 2 * q2], sr[c * 8 + 2 * q2 + 1]), sm2x2, c0x2), e0, e1);
-                        __nv_bfloat162 h2 = __floats2bfloat162_rn(fast_exp2(e0), fast_exp2(e1));
+                        if (q2 < kFinePolyPairs) {
+                            f2_unpack(poly_exp2_x2(e2), e0, e1);
+                        } else {
+                            f2_unpack(e2, e0, e1);
+                            e0 = fast_exp2(e0);
+                            e1 = fast_exp2(e1);
+                        }
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
                         pk[q2] = *reinterpret_cast<uint32_t*>(&h2);
                     }
                 }
                 const int chunk = sp * (KEYS / 8) + c;
                 *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
-            // rescale after P: the S registers are dead by now
+            // rescale after P: the S registers are dead by now; O_grp and L_grp hold the
+            // group's previous product only once that product has landed
             if (__any_sync(0xffffffffu, resc)) {
+                if (i2 >= 1 && !wwait(bar(B_PV_DONE + 2 * grp + (pb ^ 1)), ((i2 - 1) >> 1) & 1)) { ok = false; continue; }
                 tc_fence_after();
 #pragma unroll
                 for (int c = 0; c < RCOLS / RCW; ++c) {
@@ -437,7 +520,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(bar(B_P_FULL + grp));
+            mbar_arrive(bar(B_P_FULL + 2 * grp + pb));
         }
         // ---- merge the two groups: out = (O_0 2^(m_0-M) + O_1 2^(m_1-M)) / (L_0 ... + L_1 ...)
         if (sp == 0) m_sh[grp][r] = m_run;
@@ -445,8 +528,9 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const bool has1 = n >= 2;                           // group 1 ran at least one step
         const int last0 = (n - 1) & ~1;                     // last step of group 0
         const int last1 = (n - 1) - ((n - 1) & 1 ? 0 : 1);  // last step of group 1
-        bool done = ok && wwait(bar(B_PV_DONE + 0), (last0 >> 1) & 1);
-        if (has1) done = done && wwait(bar(B_PV_DONE + 1), (last1 >> 1) & 1);
+        const int i0 = last0 >> 1, i1 = last1 >> 1;       // their step indices within the groups
+        bool done = ok && wwait(bar(B_PV_DONE + (i0 & 1)), (i0 >> 1) & 1);
+        if (has1) done = done && wwait(bar(B_PV_DONE + 2 + (i1 & 1)), (i1 >> 1) & 1);
         if (done) {
             tc_fence_after();
             const float m0 = m_sh[0][r], m1 = has1 ? m_sh[1][r] : -INFINITY;
@@ -519,7 +603,7 @@ cudaError_t launch_fine_tc(const void* q, const void* k, const void* v, void* ou
     const int* count = reinterpret_cast<const int*>(ws + g.off_count);
     WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
     auto* ob = static_cast<__nv_bfloat16*>(out);
-    constexpr int threads = (8 * kFineSplit + 3) * 32;
+    constexpr int threads = (8 * kFineSplit + 4) * 32;
     const FineDump dv = dump ? *dump : FineDump{nullptr, nullptr, nullptr};
     auto go = [&](auto kernel, int sm) -> cudaError_t {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);

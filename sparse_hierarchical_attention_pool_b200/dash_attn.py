@@ -401,22 +401,25 @@ def dash_prefill_dump(q, k, v, rows, alpha=1.5, coarse_scale=1.0, w_summary=None
         out = torch.empty_like(q)
     if workspace is None:
         workspace = alloc_workspace(prefill_workspace_size(B, Hq, Hkv, T, d, block), q.device)
-    slot = torch.full((B, Hq, T), -1, dtype=torch.int32)
+    # one slot per distinct row (a slot has one writer); repeated rows share their slot's dump
     r = torch.as_tensor([list(x) for x in rows], dtype=torch.long).reshape(-1, 3)
-    slot[r[:, 0], r[:, 1], r[:, 2]] = torch.arange(len(r), dtype=torch.int32)
+    uniq, inv = torch.unique((r[:, 0] * Hq + r[:, 1]) * T + r[:, 2], return_inverse=True)
+    slot = torch.full((B * Hq * T,), -1, dtype=torch.int32)
+    slot[uniq] = torch.arange(len(uniq), dtype=torch.int32)
     slot = slot.to(q.device)
     nbs = T // block
-    x = torch.empty(max(len(r), 1), max(nbs, 1), dtype=torch.float32, device=q.device)
+    x = torch.empty(max(len(uniq), 1), max(nbs, 1), dtype=torch.float32, device=q.device)
     p = torch.empty_like(x)
     wp = _dev(w_summary, torch.float32, "w_summary") if w_summary is not None else None
     rc = lib().dash_prefill_dump(_dev(q, torch.bfloat16, "q"), _dev(k, torch.bfloat16, "k"),
                                  _dev(v, torch.bfloat16, "v"), wp, _dev(out, torch.bfloat16, "out"),
                                  B, Hq, Hkv, T, d, block, float(alpha), float(coarse_scale), int(flags),
-                                 _dev(slot, torch.int32, "row_slot"), len(r), _dev(x, torch.float32, "x"),
+                                 _dev(slot, torch.int32, "row_slot"), len(uniq), _dev(x, torch.float32, "x"),
                                  _dev(p, torch.float32, "p"), ctypes.c_void_p(workspace.data_ptr()),
                                  workspace.numel(), _stream(stream))
     _check("dash_prefill_dump", rc)
-    return out, workspace, x[:len(r), :nbs], p[:len(r), :nbs]
+    idx = inv.to(q.device)
+    return out, workspace, x[:, :nbs][idx], p[:, :nbs][idx]
 
 
 def dash_decode_dump(q, k_cache, v_cache, ksum, kv_len, alpha=1.5, coarse_scale=1.0, flags=0, out=None,
