@@ -174,11 +174,6 @@ def max_over_ranks(ws, x):
 
 # ------------------------------------------------------------------ GPU arms
 
-def _tile_positions(Hq, Hkv):
-    """Positions per work tile: P = min(64, largest power of two <= 128 / G)."""
-    return min(64, 1 << (max(1, 128 // (Hq // Hkv)).bit_length() - 1))
-
-
 def time_prefill(wl, qd, kd, vd, alpha, cs, steps, warmup, flush, ws, wsb=None, clocks_dev=None):
     """Times `steps` full prefills (after `warmup` untimed ones) of one workload with the
     profiled entry point (CUDA events between the three kernels, on the launching stream;
@@ -224,9 +219,8 @@ def time_prefill(wl, qd, kd, vd, alpha, cs, steps, warmup, flush, ws, wsb=None, 
     diag_tokens = sum((t % 64) + 1 for t in range(T)) * B * Hq
     fine_alg = 4.0 * d * (64.0 * st["selected_pairs"] + diag_tokens)
     coarse_alg = 2.0 * d * st["scored_pairs"]
-    P = _tile_positions(Hq, Hkv)
-    ntiles = B * Hkv * ((T + P - 1) // P)
-    fine_exec = 4.0 * d * 64.0 * 128.0 * (st["union_blocks"] + ntiles)
+    # executed: every step of a 128-row tile multiplies 64 keys for all 128 rows
+    fine_exec = 4.0 * d * 64.0 * 128.0 * st["fine_steps"]
     pk, pk_kind = peaks()
     peak = pk["bf16_tflops"]
     fine_ms = mean(fine)
@@ -427,8 +421,7 @@ def backward_only(args, ws):
     st = da.dash_prefill_stats(wsb)
     diag_tokens = sum((t % 64) + 1 for t in range(T)) * B * Hq
     fine_alg = 4.0 * d * (64.0 * st["selected_pairs"] + diag_tokens)
-    P = min(64, 1 << (max(1, 128 // (Hq // Hkv)).bit_length() - 1))
-    fine_exec = 4.0 * d * 64.0 * 128.0 * (st["union_blocks"] + B * Hkv * ((T + P - 1) // P))
+    fine_exec = 4.0 * d * 64.0 * 128.0 * st["fine_steps"]
     return bench_backward(args, ws, qd, kd, vd, out, wl, cs, st, fine_alg, fine_exec, L2Flush())
 
 

@@ -209,9 +209,13 @@ DASH_API int dash_prefill_profiled(const void* q, const void* k, const void* v, 
 typedef struct {
     long long scored_pairs;    /* sum over rows of the number of scored past blocks */
     long long selected_pairs;  /* sum over rows of #{j : p_j > 0} */
-    long long union_blocks;    /* sum over work tiles of the union of their rows' blocks */
+    long long union_blocks;    /* sum over work tiles of their block lists: the union of their
+                                  rows' selected past blocks (position tiles; decode groups) or
+                                  of their selected and own blocks (selection-ordered tiles) */
     long long tiles;           /* work tiles with at least one past block */
     int status;                /* device status bits (0 = clean) */
+    long long fine_steps;      /* prefill: key blocks the fine stage processes, summed over its
+                                  tiles (128 rows each); executed fine FLOPs = 4 d 64 128 x this */
 } dash_stats;
 
 /* Synchronises `stream`, then copies the counters out of `workspace` into *out (host). */

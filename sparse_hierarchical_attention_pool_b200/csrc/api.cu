@@ -34,7 +34,16 @@ int read_stats(const void* ws, size_t ws_bytes, dash_stats* out, dash_stream_t s
     out->union_blocks = (long long)h.union_blocks;
     out->tiles = (long long)h.tiles;
     out->status = h.status;
+    out->fine_steps = (long long)h.fine_steps;
     return DASH_OK;
+}
+
+// Selection-ordered tiles apply on the tensor-core path with at least one complete block and
+// per-head priors; DASH_TILES=positions keeps the position tiles (for comparisons).
+bool ordered_tiles_enabled(const PrefillGeom& g, int agg) {
+    if (!g.tc || !coarse_tc_supported(g) || !fine_tc_supported(g) || agg || g.nbs == 0) return false;
+    const char* e = getenv("DASH_TILES");
+    return !(e && strcmp(e, "positions") == 0);
 }
 
 }  // namespace
@@ -113,14 +122,21 @@ static int prefill_impl(const void* q, const void* k, const void* v, void* out, 
                                           ws + g.off_khi, ws + g.off_klo, wsum) != cudaSuccess)
         return DASH_ERR_CUDA;
     if (!mark(1)) return DASH_ERR_CUDA;
-    const cudaError_t ce = g.tc ? (coarse_tc_supported(g) ? launch_coarse_tc(q, g, ws, alpha, coarse_scale, s)
+    // selection-ordered tiles on the tensor-core path (head aggregation averages over the
+    // heads of a position, which position tiles keep together)
+    const bool ordered = ordered_tiles_enabled(g, agg);
+    const cudaError_t ce = g.tc ? (coarse_tc_supported(g) ? launch_coarse_tc(q, g, ws, alpha, coarse_scale, s, ordered)
                                                           : launch_coarse(q, g, ws, alpha, coarse_scale, s))
                                 : launch_coarse(q, g, ws, alpha, coarse_scale, s);
     if (ce != cudaSuccess) return DASH_ERR_CUDA;
+    if (ordered && launch_order_tiles(g, ws, s) != cudaSuccess) return DASH_ERR_CUDA;
     if (!mark(2)) return DASH_ERR_CUDA;
     if (dump) {
         if (launch_dump_fill(dump->x, dump->p, dump_entries, s) != cudaSuccess ||
-            launch_fine_tc(q, k, v, out, g, ws, alpha, coarse_scale, s, agg, dump) != cudaSuccess)
+            launch_fine_tc(q, k, v, out, g, ws, alpha, coarse_scale, s, agg, dump, ordered) != cudaSuccess)
+            return DASH_ERR_CUDA;
+    } else if (ordered) {
+        if (launch_fine_tc(q, k, v, out, g, ws, alpha, coarse_scale, s, agg, nullptr, true) != cudaSuccess)
             return DASH_ERR_CUDA;
     } else if (launch_fine(q, k, v, out, g, ws, alpha, coarse_scale, s, agg, need_tc) != cudaSuccess) {
         return DASH_ERR_CUDA;

@@ -56,7 +56,10 @@ coarse_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ ksu
                 int hl = r / g.P, t = t0 + r % g.P;
                 if (t < g.T) tau_out[((size_t)(b * g.Hq + kvh * g.G + hl)) * g.T + t] = __int_as_float(0x7fc00000);
             }
-            if (tid == 0) count[tile_id] = 0;
+            if (tid == 0) {
+                count[tile_id] = 0;
+                atomicAdd(&hdr->fine_steps, 1ull);            // the own block alone
+            }
             continue;
         }
         // ---- Q tile -> shared, transposed to [d][row], fp32
@@ -170,6 +173,7 @@ coarse_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ ksu
                 atomicAdd(&hdr->scored_pairs, (unsigned long long)rows_valid * bt);
                 atomicAdd(&hdr->union_blocks, (unsigned long long)base);
                 atomicAdd(&hdr->tiles, 1ull);
+                atomicAdd(&hdr->fine_steps, (unsigned long long)base + 1ull);
             }
         }
         __syncthreads();

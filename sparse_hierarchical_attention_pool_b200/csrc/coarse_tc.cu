@@ -85,7 +85,8 @@ __global__ void __launch_bounds__(320, 1)
 coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_hi,
                  const __grid_constant__ CUtensorMap tm_lo, float* __restrict__ tau_out,
                  int* __restrict__ list, int* __restrict__ count, WsHeader* __restrict__ hdr,
-                 PrefillGeom g, float alpha, float cx) {
+                 PrefillGeom g, float alpha, float cx, unsigned* __restrict__ rowbits,
+                 unsigned* __restrict__ wcnt) {
     using L = CtLayout<D>;
     using namespace sm100;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -99,6 +100,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __shared__ float xp[2][2][6][kTileRows];     // [pass parity][half][sum][row]: partial pass sums
     __shared__ float topv[2][kTopK][kTileRows];  // [half][rank][row]: each half-row's largest scores
     __shared__ int wtot_sh[8];
+    __shared__ unsigned bcnt[kMaxT / kBlock / 4];  // per block of a tile: rows selecting it (a byte each)
 
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -242,14 +244,28 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         auto sync8 = [&]() { asm volatile("bar.sync 1, 256;" ::: "memory"); };
         // the two warps (w, w + 4) that share a quarter of the tile rows
         auto sync_pair = [&]() { asm volatile("bar.sync %0, 64;" :: "r"(2 + quarter) : "memory"); };
+        // with row bitmaps: add how many of this warp's rows select each of the nbits blocks
+        // starting at j0 to the tile's byte counters (at most 128 rows per tile: no carry)
+        auto count_blocks = [&](int j0, unsigned mask, int nbits) {
+            unsigned mine = 0u;
+            for (int i = 0; i < nbits; ++i) {
+                const unsigned c = __reduce_add_sync(0xffffffffu, (mask >> i) & 1u);
+                if (lane == i) mine = c;
+            }
+            if (lane < nbits && mine) atomicAdd(&bcnt[(j0 + lane) >> 2], mine << (8 * ((j0 + lane) & 3)));
+        };
         for (int w = blockIdx.x; ok && w < g.ntiles; w += gridDim.x) {
             const TileInfo ti = tile_info(g, w);
             const int hl = r / g.P, t = ti.t0 + r % g.P;
             const bool valid = r < g.M && t < g.T;
             const size_t tau_idx = (size_t)(ti.b * g.Hq + ti.kvh * g.G + hl) * g.T + t;
+            const size_t bits_row = tau_idx * g.nbw;        // this row's selection bitmap
             if (ti.bt == 0) {
                 if (valid && hf == 0) tau_out[tau_idx] = __int_as_float(0x7fc00000);
-                if (r == 0 && hf == 0) count[ti.tile_id] = 0;
+                if (r == 0 && hf == 0) {
+                    count[ti.tile_id] = 0;
+                    if (!rowbits) atomicAdd(&hdr->fine_steps, 1ull);   // the own block alone
+                }
                 continue;
             }
             // chunk c of the current sweep sits in TMEM buffer (sweep_base + c) % 4
@@ -361,6 +377,8 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 else sweep(std::integral_constant<int, 0>{});
                 // ---- union pass: OR of x > tau over the rows, per block
                 for (int i = st; i < nw; i += 256) bitmap[i] = 0u;
+                if (rowbits)
+                    for (int i = st; i < (ti.bt + 3) / 4; i += 256) bcnt[i] = 0u;
                 if (st == 0) sel_sh = 0ull;
                 sync8();
 #pragma unroll
@@ -372,6 +390,10 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
                             if (valid && xc[k][i] > tau) mask |= 1u << i;
+                        if (rowbits) {
+                            if (valid) rowbits[bits_row + (j0 >> 5)] = mask;
+                            count_blocks(j0, mask, 32);
+                        }
                         nsel += (float)__popc(mask);
                         const unsigned wm = __reduce_or_sync(0xffffffffu, mask);
                         if (lane == 0 && wm) atomicOr(&bitmap[j0 >> 5], wm);
@@ -381,6 +403,12 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     unsigned mask = 0u;
                     for (int i = 0; i < 16; ++i)
                         if (i < nv && valid && __fmul_rn(__uint_as_float(v[i]), cx) > tau) mask |= 1u << i;
+                    // 16 blocks: the half word starting at block j0
+                    if (rowbits) {
+                        if (valid)
+                            reinterpret_cast<unsigned short*>(rowbits + bits_row + (j0 >> 5))[(j0 & 31) >> 4] = (unsigned short)mask;
+                        count_blocks(j0, mask, 16);
+                    }
                     nsel += (float)__popc(mask);
                     const unsigned wm = __reduce_or_sync(0xffffffffu, mask);
                     if (lane == 0 && wm) atomicOr(&bitmap[j0 >> 5], wm << (j0 & 31));
@@ -480,12 +508,18 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 if (!ok) break;
                 // ---- union pass: OR of x > tau over the rows, per block
                 for (int i = st; i < nw; i += 256) bitmap[i] = 0u;
+                if (rowbits)
+                    for (int i = st; i < (ti.bt + 3) / 4; i += 256) bcnt[i] = 0u;
                 if (st == 0) sel_sh = 0ull;
                 sync8();
                 if (!run_pass([&](int j0, const uint32_t* v, int nv) {
                         unsigned mask = 0u;
                         for (int i = 0; i < 32; ++i)
                             if (i < nv && valid && __fmul_rn(__uint_as_float(v[i]), cx) > tau) mask |= 1u << i;
+                        if (rowbits) {
+                            if (valid) rowbits[bits_row + (j0 >> 5)] = mask;
+                            count_blocks(j0, mask, 32);
+                        }
                         nsel += (float)__popc(mask);
                         const unsigned wm = __reduce_or_sync(0xffffffffu, mask);
                         if (lane == 0 && wm) atomicOr(&bitmap[j0 >> 5], wm);
@@ -496,6 +530,18 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             nsel = warp_sum(nsel);
             if (lane == 0) atomicAdd(&sel_sh, (unsigned long long)nsel);
             sync8();
+            if (rowbits) {
+                // the tile's block counts into its ordering window's counts
+                unsigned* wc = wcnt + ((size_t)ti.bg * ((g.T + g.W - 1) / g.W) + ti.t0 / g.W) * g.nbs;
+                for (int i = st; i < (ti.bt + 3) / 4; i += 256) {
+                    const unsigned v4 = bcnt[i];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const unsigned c = (v4 >> (8 * q)) & 0xFFu;
+                        if (c) atomicAdd(&wc[4 * i + q], c);
+                    }
+                }
+            }
             // ---- compaction: thread st owns bitmap words 2 st and 2 st + 1; a block-wide
             // scan of their popcounts places them in the tile's ascending list
             {
@@ -536,8 +582,12 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     const int rows_valid = g.G * min(g.P, g.T - ti.t0);
                     atomicAdd(&hdr->selected_pairs, sel_sh);
                     atomicAdd(&hdr->scored_pairs, (unsigned long long)rows_valid * ti.bt);
-                    atomicAdd(&hdr->union_blocks, (unsigned long long)total);
-                    atomicAdd(&hdr->tiles, 1ull);
+                    // with ordered tiles the ordering pass counts the tiles the fine stage runs
+                    if (!rowbits) {
+                        atomicAdd(&hdr->union_blocks, (unsigned long long)total);
+                        atomicAdd(&hdr->tiles, 1ull);
+                        atomicAdd(&hdr->fine_steps, (unsigned long long)total + 1ull);
+                    }
                 }
             }
             sync8();
@@ -568,7 +618,7 @@ int sm_count() {
 bool coarse_tc_supported(const PrefillGeom& g) { return g.P >= 8 && g.nbs > 0; }
 
 cudaError_t launch_coarse_tc(const void* q, const PrefillGeom& g, char* ws, float alpha,
-                             float coarse_scale, cudaStream_t stream) {
+                             float coarse_scale, cudaStream_t stream, bool write_rowbits) {
     const float cx = (alpha - 1.0f) * coarse_scale / sqrtf((float)g.d);
     CUtensorMap tq, thi, tlo;
     const unsigned long long qrows = (unsigned long long)g.B * g.Hq * g.T;
@@ -581,11 +631,18 @@ cudaError_t launch_coarse_tc(const void* q, const PrefillGeom& g, char* ws, floa
     float* tau = reinterpret_cast<float*>(ws + g.off_tau);
     int* list = reinterpret_cast<int*>(ws + g.off_list);
     int* count = reinterpret_cast<int*>(ws + g.off_count);
+    unsigned* rowbits = write_rowbits ? reinterpret_cast<unsigned*>(ws + g.off_rowbits) : nullptr;
+    unsigned* wcnt = write_rowbits ? reinterpret_cast<unsigned*>(ws + g.off_wcnt) : nullptr;
+    if (wcnt) {
+        const size_t nwin = (size_t)((g.T + g.W - 1) / g.W);
+        cudaError_t e0 = cudaMemsetAsync(wcnt, 0, (size_t)g.B * g.Hkv * nwin * g.nbs * sizeof(unsigned), stream);
+        if (e0 != cudaSuccess) return e0;
+    }
     const int grid = g.ntiles < sm_count() ? g.ntiles : sm_count();
     auto go = [&](auto kernel, int sm) -> cudaError_t {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
         if (e != cudaSuccess) return e;
-        kernel<<<grid, 320, sm, stream>>>(tq, thi, tlo, tau, list, count, hdr, g, alpha, cx);
+        kernel<<<grid, 320, sm, stream>>>(tq, thi, tlo, tau, list, count, hdr, g, alpha, cx, rowbits, wcnt);
         return cudaSuccess;
     };
     cudaError_t e;

@@ -25,7 +25,8 @@ struct WsHeader {
     unsigned long long selected_pairs;
     unsigned long long union_blocks;
     unsigned long long tiles;
-    unsigned long long reserved[27];
+    unsigned long long fine_steps;   // key blocks the prefill's fine stage processes, over all its tiles
+    unsigned long long reserved[26];
 };
 static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
 
@@ -43,6 +44,12 @@ inline int solve_cap_from_env() {
 
 // Geometry of a prefill call.  Work tiles are P consecutive positions (inside one key
 // block) x the G query heads of one KV head: rows r = head_local * P + pos_local.
+// Selection-ordered tiles (tensor-core path, G <= 16): the rows of a KV group are cut into
+// windows of kOrderRows rows (W = kOrderRows / G positions x the G heads), each window's rows
+// are sorted by a selection signature, and every 128 consecutive sorted rows form a tile
+// whose block list is the union of its rows' selected blocks and own blocks.
+constexpr int kOrderRows = 4096;
+
 struct PrefillGeom {
     int B, Hq, Hkv, T, d, G, P, M;   // M = G * P rows used of the 128-row tile
     int ntile_bg;                    // tiles per (b, kv head) = ceil(T / P)
@@ -51,7 +58,14 @@ struct PrefillGeom {
     int cap;                         // list capacity per tile = max(1, nbs)
     bool tc;                         // tensor-core Stage 1/2 kernels (needs P >= 8)
     int maxit;                       // iteration cap of the threshold solves
-    size_t off_ksum, off_khi, off_klo, off_tau, off_list, off_count, off_scratch, total;
+    int nbw;                         // 32-bit words of a row's selection bitmap = ceil(nbs / 32)
+    int W;                           // positions per ordering window: a multiple of 64, W G <= 4096
+    int ord_tw;                      // ordered tiles of a full window = ceil(W G / 128)
+    int ord_bg;                      // ordered tiles per (b, kv head)
+    int ord_ntiles;                  // B * Hkv * ord_bg
+    int ord_cap;                     // list capacity of an ordered tile = ceil(T / 64)
+    size_t off_ksum, off_khi, off_klo, off_tau, off_list, off_count, off_scratch;
+    size_t off_rowbits, off_wcnt, off_ord_rows, off_ord_list, off_ord_count, total;
 };
 
 inline int pow2_floor(int x) {
@@ -77,6 +91,18 @@ inline bool make_prefill_geom(int B, int Hq, int Hkv, int T, int d, PrefillGeom*
     g->cap = g->nbs > 0 ? g->nbs : 1;
     g->tc = P >= 8;
     g->maxit = solve_cap_from_env();
+    g->nbw = (g->nbs + 31) / 32;
+    g->W = (kOrderRows / G) / kBlock * kBlock;
+    if (g->W < kBlock) g->W = kBlock;
+    g->ord_tw = (g->W * G + kTileRows - 1) / kTileRows;
+    {
+        // full windows have ord_tw tiles each, the last one ceil(its rows / 128)
+        const int nwin = (T + g->W - 1) / g->W;
+        const long long rlast = (long long)(T - (nwin - 1) * g->W) * G;
+        g->ord_bg = (nwin - 1) * g->ord_tw + (int)((rlast + kTileRows - 1) / kTileRows);
+    }
+    g->ord_ntiles = B * Hkv * g->ord_bg;
+    g->ord_cap = (T + kBlock - 1) / kBlock;
     const size_t nsum = (size_t)B * Hkv * (g->nbs > 0 ? g->nbs : 1) * d;
     size_t off = align256(sizeof(WsHeader));
     g->off_ksum = off;    off = align256(off + nsum * sizeof(float));
@@ -88,6 +114,22 @@ inline bool make_prefill_geom(int B, int Hq, int Hkv, int T, int d, PrefillGeom*
     int cgrid = g->ntiles < kCoarseCTAs ? g->ntiles : kCoarseCTAs;
     g->off_scratch = off; // per-CTA score slabs of the CUDA-core coarse kernel only
     if (!g->tc) off = align256(off + (size_t)cgrid * kTileRows * g->cap * sizeof(float));
+    // selection-ordered tiles (tensor-core path only): per-row selection bitmaps, the rows
+    // of every ordered tile, its block list and count
+    g->off_rowbits = off;
+    g->off_wcnt = off;
+    g->off_ord_rows = off;
+    g->off_ord_list = off;
+    g->off_ord_count = off;
+    if (g->tc && g->nbs > 0) {
+        g->off_rowbits = off;   off = align256(off + (size_t)B * Hq * T * g->nbw * sizeof(unsigned));
+        // per window, how many of its rows select each block (filled by the coarse stage)
+        const int nwin = (T + g->W - 1) / g->W;
+        g->off_wcnt = off;      off = align256(off + (size_t)B * Hkv * nwin * g->nbs * sizeof(unsigned));
+        g->off_ord_rows = off;  off = align256(off + (size_t)g->ord_ntiles * kTileRows * sizeof(int));
+        g->off_ord_list = off;  off = align256(off + (size_t)g->ord_ntiles * g->ord_cap * sizeof(int));
+        g->off_ord_count = off; off = align256(off + (size_t)g->ord_ntiles * sizeof(int));
+    }
     g->total = off;
     return true;
 }

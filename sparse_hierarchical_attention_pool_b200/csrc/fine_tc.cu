@@ -24,8 +24,10 @@
 //                      is free once the block's P V product is done);
 //   8 SPLIT + 1        S issuer (one lane): S_s = Q [K_s | kbar_hi | kbar_lo]^T (M=128, N=80
 //                      with the summary atoms at columns 64 and 72) into the S buffer of
-//                      group s & 1 as soon as block s is loaded and that group has read
-//                      S_{s-2}, so S_{s+2} is computed while the group works on step s;
+//                      group s & 1 as soon as block s is loaded, that group has read
+//                      S_{s-2} and the product of step s-4 (same P buffer) has landed, so
+//                      S_{s+2} is computed while the group works on step s and a group
+//                      that sees S_s may write its P buffer without another wait;
 //   8 SPLIT + 2        PV issuer (one lane): O_g += P_s V_s (M=128, N=d) and L_g += P_s 1
 //                      (N=16, an all-ones B tile: the softmax denominator summed by the
 //                      tensor core over exactly the bf16 P it multiplies) as soon as P_s is
@@ -44,6 +46,10 @@
 // through shared memory (one group barrier per step) and share log of the mean as prior.
 // Operands: Q, K, P K-major and V MN-major, all 128-byte swizzled (TMA writes that layout).
 // Every wait is bounded (~2 s); a CTA that gives up sets a status bit and exits cleanly.
+// Selection-ordered tiles (ORD = true): a tile is 128 rows of one KV group chosen by the
+// ordering pass (order.cu), with any positions; the softmax threads load their rows of Q,
+// every row has its own block (prior 1, causal) and ignores listed blocks after it, and the
+// tile's list (selected and own blocks of its rows, ascending) gives every step.
 // Dump variant (DUMP = true, parity checks only): for rows with a slot in dump.slot, every
 // listed block's x_j (as recomputed here from the summary columns) and the weight p_j the
 // prior applies (0 when x_j <= tau) are written to dump.x / dump.p [slot, T / 64].
@@ -59,7 +65,30 @@ constexpr int kKStages = 3;            // K (+ summary rows) ring
 constexpr int kVStages = 3;            // V ring
 constexpr int kFineSplit = 1;          // threads per tile row in each softmax group
 constexpr int kFinePolyPairs = 1;      // pairs of every 4 whose 2^x runs on the FMA pipe
+constexpr bool kFineIntPack = false;   // fp32 -> bf16 pairs with integer ops instead of cvt
+constexpr bool kFineScalar = false;    // scalar FMA / exponent per key instead of f32x2 pairs
 constexpr float kLazyRescale = 8.0f;   // log2 units: p values stay below 2^8 between rescales
+
+// Two non-negative finite fp32 values rounded to nearest-even bf16 and packed (lo in the low
+// half) with integer operations only: adding 0x7FFF plus the lowest kept bit carries into
+// the kept bits exactly when the dropped half is above one half-ulp, or equal to it with an
+// odd kept part.
+__device__ __forceinline__ uint32_t bf16x2_rne_int(float lo, float hi) {
+    uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
+    a += 0x7FFFu + ((a >> 16) & 1u);
+    b += 0x7FFFu + ((b >> 16) & 1u);
+    return __byte_perm(a, b, 0x7632);
+}
+
+// Scalar form of poly_exp2_x2 below (same steps and constants).
+__device__ __forceinline__ float poly_exp2(float x) {
+    x = fmaxf(x, -125.0f);
+    const float t = x + 12582912.0f;                  // 1.5 * 2^23: n = round(x) in the low bits
+    const float f = x - (t - 12582912.0f);
+    const float p = fmaf(fmaf(fmaf(__uint_as_float(0x3D61FBB0u), f, __uint_as_float(0x3E786F0Eu)), f,
+                              __uint_as_float(0x3F31798Du)), f, __uint_as_float(0x3F7FFB49u));
+    return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+}
 
 // 2^x for x <= 8 on the FMA and integer pipes.  Cody-Waite style split x = n + f with
 // n = round(x) (added to the exponent field) and f in [-1/2, 1/2], where 2^f comes from a
@@ -120,14 +149,15 @@ enum : int { B_Q = 0, B_K_FULL = 1, B_K_EMPTY = B_K_FULL + kKStages, B_V_FULL = 
              B_P_FULL = B_S_FREE + 2, B_PV_DONE = B_P_FULL + 4, B_DRAIN = B_PV_DONE + 4,
              B_DRAIN2 = B_DRAIN + 1, B_COUNT = B_DRAIN2 + 1 };
 
-template <int D, int SPLIT, bool AGG, bool DUMP>
+template <int D, int SPLIT, bool AGG, bool DUMP, bool ORD>
 __global__ void __launch_bounds__((8 * SPLIT + 4) * 32, 1)
 fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_hi,
                const __grid_constant__ CUtensorMap tm_lo, __nv_bfloat16* __restrict__ out,
                const float* __restrict__ tau, const int* __restrict__ list, const int* __restrict__ count,
                WsHeader* __restrict__ hdr, PrefillGeom g, float cx, float e_pow, float sm2,
-               FineDump dump) {
+               FineDump dump, const __nv_bfloat16* __restrict__ qrows, const int* __restrict__ ord_rows) {
+    static_assert(!(ORD && AGG), "head aggregation keeps the position tiles");
     using L = TcLayout<D>;
     using namespace sm100;
     constexpr int kGroupThreads = 128 * SPLIT;  // softmax threads per group
@@ -157,19 +187,21 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // group-major order (longest tiles of a group first): the CTAs in flight share one KV
     // group, whose K and V stay in L2 while its tiles re-read them
     const int w = blockIdx.x;
-    const int bg = w / g.ntile_bg;
-    const int it = g.ntile_bg - 1 - w % g.ntile_bg;
+    const int ntb = ORD ? g.ord_bg : g.ntile_bg;            // tiles per KV group
+    const int bg = w / ntb;
+    const int it = ntb - 1 - w % ntb;
     const int b = bg / g.Hkv, kvh = bg % g.Hkv;
-    const int t0 = it * g.P;
-    const int bt = t0 / kBlock;
-    const size_t tile_id = (size_t)bg * g.ntile_bg + it;
-    const int U = bt > 0 ? count[tile_id] : 0;
-    const int n = U + 1;                                    // listed past blocks, then the own block
-    const int* lst = list + tile_id * g.cap;
+    const int t0 = ORD ? 0 : it * g.P;
+    const int bt = ORD ? 0 : t0 / kBlock;                   // own block of a position tile
+    const size_t tile_id = (size_t)bg * ntb + it;
+    // position tiles: the listed past blocks, then the own block; ordered tiles: the list
+    const int U = (ORD || bt > 0) ? count[tile_id] : 0;
+    const int n = ORD ? U : U + 1;
+    const int* lst = list + tile_id * (ORD ? g.ord_cap : g.cap);
 
     if (tid == 0) {
         abort_sh = 0;
-        mbar_init(bar(B_Q), 1);
+        mbar_init(bar(B_Q), ORD ? kTileRows : 1);          // ordered tiles: the row loads arrive
         for (int st = 0; st < kKStages; ++st) {
             mbar_init(bar(B_K_FULL + st), 1);
             mbar_init(bar(B_K_EMPTY + st), 1);
@@ -191,7 +223,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         fence_mbar_init();
     }
     // rows of the Q tile beyond G * P are never loaded: zero them once
-    if (g.M < kTileRows && tid < kTileRows && tid >= g.M) {
+    if (!ORD && g.M < kTileRows && tid < kTileRows && tid >= g.M) {
         for (int h = 0; h < D / 64; ++h) {
             uint4* p = reinterpret_cast<uint4*>(base_ptr + L::off_q + h * L::kQHalf + tid * 128);
 #pragma unroll
@@ -222,11 +254,13 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             prefetch_tmap(&tm_v);
             prefetch_tmap(&tm_hi);
             prefetch_tmap(&tm_lo);
-            mbar_arrive_expect_tx(bar(B_Q), (uint32_t)(g.M * D * 2));
-            for (int hl = 0; hl < g.G; ++hl) {
-                const int row = (b * g.Hq + kvh * g.G + hl) * g.T + t0;
-                for (int h = 0; h < D / 64; ++h)
-                    tma_load_2d(base + L::off_q + h * L::kQHalf + hl * g.P * 128, &tm_q, h * 64, row, bar(B_Q));
+            if (!ORD) {
+                mbar_arrive_expect_tx(bar(B_Q), (uint32_t)(g.M * D * 2));
+                for (int hl = 0; hl < g.G; ++hl) {
+                    const int row = (b * g.Hq + kvh * g.G + hl) * g.T + t0;
+                    for (int h = 0; h < D / 64; ++h)
+                        tma_load_2d(base + L::off_q + h * L::kQHalf + hl * g.P * 128, &tm_q, h * 64, row, bar(B_Q));
+                }
             }
             int last_armed[kKStages];
             for (int st = 0; st < kKStages; ++st) last_armed[st] = -1;
@@ -249,7 +283,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (*abort_flag) {
                 // let every load this thread started land before the CTA exits
                 volatile int dummy = 0;
-                mbar_wait(bar(B_Q), 0, &dummy);
+                if (!ORD) mbar_wait(bar(B_Q), 0, &dummy);
                 for (int st = 0; st < kKStages; ++st)
                     if (last_armed[st] >= 0) { dummy = 0; mbar_wait(bar(B_K_FULL + st), (last_armed[st] / kKStages) & 1, &dummy); }
             }
@@ -286,6 +320,13 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const int st = s % kKStages, sb = s & 1;
                 if (!mbar_wait(bar(B_K_FULL + st), (s / kKStages) & 1, abort_flag)) { ok = false; break; }
                 if (s >= 2 && !mbar_wait(bar(B_S_FREE + sb), ((s - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
+                // the P buffer step s will use was last read by the product of step s - 4:
+                // S_s is computed only after that product landed, so a softmax group that
+                // sees S_s may overwrite the buffer
+                if (s >= 4 && !mbar_wait(bar(B_PV_DONE + 2 * sb + ((s >> 1) & 1)), (((s >> 1) - 2) >> 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -346,10 +387,30 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int wg = warp % (4 * SPLIT);
         const int quarter = wg & 3, sp = wg >> 2;          // TMEM lane quarter, key split
         const int r = quarter * 32 + lane;                  // tile row = TMEM lane
-        const int hl = r / g.P, t = t0 + r % g.P;
-        const bool valid = r < g.M && t < g.T;
+        // the tile row: (head in group, position); ordered tiles read it from the tile's rows
+        const int rid = ORD ? ord_rows[tile_id * kTileRows + r] : 0;
+        const int hl = ORD ? (rid >= 0 ? rid / g.T : 0) : r / g.P;
+        const int t = ORD ? (rid >= 0 ? rid % g.T : 0) : t0 + r % g.P;
+        const bool valid = ORD ? rid >= 0 : (r < g.M && t < g.T);
         const int tpos = valid ? t : -1;
-        const float tau_r = (valid && bt > 0) ? tau[(size_t)(b * g.Hq + kvh * g.G + hl) * g.T + t] : INFINITY;
+        const int bt_r = ORD ? t / kBlock : bt;             // the row's own block
+        const float tau_r = (valid && bt_r > 0) ? tau[(size_t)(b * g.Hq + kvh * g.G + hl) * g.T + t] : INFINITY;
+        if constexpr (ORD) {
+            // this tile's rows of Q, 128-byte swizzled as the TMA would write them (zeros for
+            // rows the tile does not fill)
+            if (grp == 0 && sp == 0) {
+                const uint4* src = reinterpret_cast<const uint4*>(qrows + ((size_t)(b * g.Hq + kvh * g.G + hl) * g.T + t) * D);
+#pragma unroll
+                for (int h = 0; h < D / 64; ++h)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 v = valid ? src[h * 8 + c] : make_uint4(0u, 0u, 0u, 0u);
+                        *reinterpret_cast<uint4*>(base_ptr + L::off_q + h * L::kQHalf + r * 128 + ((c ^ (r & 7)) << 4)) = v;
+                    }
+                fence_proxy_async_smem();
+                mbar_arrive(bar(B_Q));
+            }
+        }
         const int slot = (DUMP && valid) ? dump.slot[(size_t)(b * g.Hq + kvh * g.G + hl) * g.T + t] : -1;
         // parity dump of one listed past block: x_j and the weight the prior applies
         auto dump_block = [&](int j, float x) {
@@ -382,7 +443,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int s = grp; s < n; s += 2) {
             const int i2 = s >> 1;                          // this group's step index
             const int j = s < U ? lst[s] : bt;
-            const bool diag = (j == bt);
+            const bool diag = (j == bt_r);
             const bool okw = ok && wwait(bar(B_S_FULL + grp), i2 & 1);
             uint32_t sr[KEYS];
             float ps_own = 0.f, pm_own = -INFINITY;
@@ -446,9 +507,10 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             } else {
                 if (!okw) { ok = false; continue; }
                 const float x = __fmul_rn(rs, cx);
+                // past blocks only: an ordered tile also lists blocks after some rows' own
                 lp2 = diag ? (tpos >= 0 ? 0.f : -INFINITY)
-                           : (x > tau_r ? e_pow * __log2f(x - tau_r) : -INFINITY);
-                if (!diag) dump_block(j, x);
+                           : ((j < bt_r && x > tau_r) ? e_pow * __log2f(x - tau_r) : -INFINITY);
+                if (!diag && j < bt_r) dump_block(j, x);
             }
             const bool active = lp2 > -INFINITY;
             const float mx = active ? fmaf(smax, sm2, lp2) : -INFINITY;
@@ -463,10 +525,10 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     resc = true;
                 }
             }
-            // P buffer pb of this group was last read by its product two steps back
+            // P buffer pb of this group was last read by its product two steps back, which
+            // had landed before S_s was computed (the S issuer waits for it)
             const int pb = i2 & 1;
             uint8_t* const prow = prow0 + pb * L::kP;
-            if (i2 >= 2 && !wwait(bar(B_PV_DONE + 2 * grp + pb), ((i2 - 2) >> 1) & 1)) { ok = false; continue; }
             // p = 2^(s sm2 + log2 p_j - m): packed FMA, exponent on the SFU or the FMA pipe,
             // bf16 pairs
             const float c0 = lp2 - m_run;
@@ -475,7 +537,17 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
             for (int c = 0; c < KEYS / 8; ++c) {
                 uint32_t pk[4] = {0u, 0u, 0u, 0u};
-                if (active) {
+                if (active && kFineScalar) {
+#pragma unroll
+                    for (int q2 = 0; q2 < 4; ++q2) {
+                        const float a0 = fmaf(__uint_as_float(sr[c * 8 + 2 * q2]), sm2, c0);
+                        const float a1 = fmaf(__uint_as_float(sr[c * 8 + 2 * q2 + 1]), sm2, c0);
+                        const float e0 = q2 < kFinePolyPairs ? poly_exp2(a0) : fast_exp2(a0);
+                        const float e1 = q2 < kFinePolyPairs ? poly_exp2(a1) : fast_exp2(a1);
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
+                        pk[q2] = *reinterpret_cast<uint32_t*>(&h2);
+                    }
+                } else if (active) {
 #pragma unroll
                     for (int q2 = 0; q2 < 4; ++q2) {
                         const uint64_t e2 = f2_fma(f2_pack(sr[c * 8 + 2 * q2], sr[c * 8 + 2 * q2 + 1]), sm2x2, c0x2);
@@ -487,8 +559,12 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             e0 = fast_exp2(e0);
                             e1 = fast_exp2(e1);
                         }
-                        __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
-                        pk[q2] = *reinterpret_cast<uint32_t*>(&h2);
+                        if constexpr (kFineIntPack) {
+                            pk[q2] = bf16x2_rne_int(e0, e1);
+                        } else {
+                            __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
+                            pk[q2] = *reinterpret_cast<uint32_t*>(&h2);
+                        }
                     }
                 }
                 const int chunk = sp * (KEYS / 8) + c;
@@ -584,7 +660,8 @@ bool fine_tc_supported(const PrefillGeom& g) { return g.P >= 8 && (g.d == 64 || 
 
 cudaError_t launch_fine_tc(const void* q, const void* k, const void* v, void* out, const PrefillGeom& g,
                            char* ws, float alpha, float coarse_scale, cudaStream_t stream, int agg,
-                           const FineDump* dump) {
+                           const FineDump* dump, bool ordered) {
+    if (ordered && (agg || g.nbs == 0)) return cudaErrorInvalidValue;
     const float cx = (alpha - 1.0f) * coarse_scale / sqrtf((float)g.d);
     const float e_pow = 1.0f / (alpha - 1.0f);
     const float sm2 = 1.4426950408889634f / sqrtf((float)g.d);
@@ -599,25 +676,31 @@ cudaError_t launch_fine_tc(const void* q, const void* k, const void* v, void* ou
         !make_tmap_bf16(&tlo, ws + g.off_klo, srows, g.d, 8))
         return cudaErrorInvalidValue;
     const float* tau = reinterpret_cast<const float*>(ws + g.off_tau);
-    const int* list = reinterpret_cast<const int*>(ws + g.off_list);
-    const int* count = reinterpret_cast<const int*>(ws + g.off_count);
+    const int* list = reinterpret_cast<const int*>(ws + (ordered ? g.off_ord_list : g.off_list));
+    const int* count = reinterpret_cast<const int*>(ws + (ordered ? g.off_ord_count : g.off_count));
+    const int* ord_rows = ordered ? reinterpret_cast<const int*>(ws + g.off_ord_rows) : nullptr;
     WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
     auto* ob = static_cast<__nv_bfloat16*>(out);
+    const auto* qb = static_cast<const __nv_bfloat16*>(q);
     constexpr int threads = (8 * kFineSplit + 4) * 32;
     const FineDump dv = dump ? *dump : FineDump{nullptr, nullptr, nullptr};
+    const int grid = ordered ? g.ord_ntiles : g.ntiles;
     auto go = [&](auto kernel, int sm) -> cudaError_t {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
         if (e != cudaSuccess) return e;
-        kernel<<<g.ntiles, threads, sm, stream>>>(tq, tk, tv, thi, tlo, ob, tau, list, count, hdr, g, cx, e_pow, sm2, dv);
+        kernel<<<grid, threads, sm, stream>>>(tq, tk, tv, thi, tlo, ob, tau, list, count, hdr, g, cx, e_pow, sm2, dv,
+                                              qb, ord_rows);
         return cudaSuccess;
     };
     auto pick = [&](auto dcon) -> cudaError_t {
         constexpr int DD = decltype(dcon)::value;
         const int sm = (int)TcLayout<DD>::bytes;
-        if (dump) return agg ? go(fine_tc_kernel<DD, kFineSplit, true, true>, sm)
-                             : go(fine_tc_kernel<DD, kFineSplit, false, true>, sm);
-        return agg ? go(fine_tc_kernel<DD, kFineSplit, true, false>, sm)
-                   : go(fine_tc_kernel<DD, kFineSplit, false, false>, sm);
+        if (ordered) return dump ? go(fine_tc_kernel<DD, kFineSplit, false, true, true>, sm)
+                                 : go(fine_tc_kernel<DD, kFineSplit, false, false, true>, sm);
+        if (dump) return agg ? go(fine_tc_kernel<DD, kFineSplit, true, true, false>, sm)
+                             : go(fine_tc_kernel<DD, kFineSplit, false, true, false>, sm);
+        return agg ? go(fine_tc_kernel<DD, kFineSplit, true, false, false>, sm)
+                   : go(fine_tc_kernel<DD, kFineSplit, false, false, false>, sm);
     };
     cudaError_t e = g.d == 128 ? pick(std::integral_constant<int, 128>{}) : pick(std::integral_constant<int, 64>{});
     if (e != cudaSuccess) return e;

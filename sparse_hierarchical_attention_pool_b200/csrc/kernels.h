@@ -18,10 +18,16 @@ cudaError_t launch_block_summary(const void* k, float* ksum, int B, int Hkv, int
 cudaError_t launch_coarse(const void* q, const PrefillGeom& g, char* ws, float alpha,
                           float coarse_scale, cudaStream_t stream);
 
-// tcgen05 variant of launch_coarse (needs P >= 8 and at least one complete block)
+// tcgen05 variant of launch_coarse (needs P >= 8 and at least one complete block);
+// write_rowbits: also store every row's selection bitmap (for the selection-ordered tiles)
 bool coarse_tc_supported(const PrefillGeom& g);
 cudaError_t launch_coarse_tc(const void* q, const PrefillGeom& g, char* ws, float alpha,
-                             float coarse_scale, cudaStream_t stream);
+                             float coarse_scale, cudaStream_t stream, bool write_rowbits = false);
+
+// Selection-ordered tiles from the per-row bitmaps of the coarse stage: sorts the rows of
+// every window of a KV group by their signature and writes each ordered tile's rows, block
+// list (selected and own blocks, ascending) and count; adds the tiles' unions to the header.
+cudaError_t launch_order_tiles(const PrefillGeom& g, char* ws, cudaStream_t stream);
 
 // Parity dump of the tensor-core fine kernel: rows with slot[row] >= 0 (row = (b Hq + h) T + t)
 // get x_j and the applied weight p_j of every listed past block j at x[slot nbs + j],
@@ -40,11 +46,13 @@ cudaError_t launch_fine(const void* q, const void* k, const void* v, void* out,
                         cudaStream_t stream, int agg = 0, bool need_tc = false);
 
 // tcgen05 variant of launch_fine (needs P >= 8, i.e. at most 16 query heads per KV head);
-// dump != nullptr selects the dump variant
+// dump != nullptr selects the dump variant; ordered: run the selection-ordered tiles of
+// launch_order_tiles instead of the position tiles (not with head aggregation)
 bool fine_tc_supported(const PrefillGeom& g);
 cudaError_t launch_fine_tc(const void* q, const void* k, const void* v, void* out,
                            const PrefillGeom& g, char* ws, float alpha, float coarse_scale,
-                           cudaStream_t stream, int agg = 0, const FineDump* dump = nullptr);
+                           cudaStream_t stream, int agg = 0, const FineDump* dump = nullptr,
+                           bool ordered = false);
 
 // x = NaN and p = 0 for n entries (the "not listed" marks of the parity dumps)
 cudaError_t launch_dump_fill(float* x, float* p, size_t n, cudaStream_t stream);

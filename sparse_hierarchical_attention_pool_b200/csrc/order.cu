@@ -1,0 +1,204 @@
+// order.cu -- selection-ordered tiles for the tensor-core fine stage.
+//
+// The fine stage runs 128 query rows of one KV group per tile over the union of their
+// selected blocks ("DashAttention: Making Sparse Attention Fully Differentiable with Adaptive
+// Block Selection", section "Core Mechanism": the selection is per query row, the gathered
+// key/value blocks are shared by the rows of a tile).  Tiles of consecutive positions carry
+// rows whose selections are nearly independent, so their union approaches every past block.
+// This pass forms tiles from rows with similar selections instead: the rows of a window
+// (W = 4096 / G positions, rounded down to whole blocks, x the G heads of a KV group) are
+// sorted by a signature and cut into
+// tiles of 128.
+//
+// Signature: one power-iteration step towards the leading principal axis of the window's
+// selection matrix S (rows x blocks), started from the block selection counts:
+//     c_j = #{rows r of the window : j in S_r},   score_r = sum_{j in S_r} c_j.
+// Sorting by it places rows that select the window's common blocks next to each other (a
+// spectral ordering of the rows).  The sort is a stable radix sort on (score, row), so the
+// tiles, and every result computed from them, are deterministic.
+//
+// The block counts c_j of every window are accumulated by the coarse stage while it writes
+// the row bitmaps.  order_rows_kernel, one CTA of 1024 threads per window: per-row scores
+// (lanes as bitmap words), then a block-wide radix sort on the bits the scores use, which
+// gives the rows of every tile.  order_union_kernel, one warp per tile: the OR of its rows' bitmaps (plus their own
+// blocks), lanes as bitmap words, compacted into the tile's ascending list.
+#include <cub/block/block_radix_sort.cuh>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dash {
+
+constexpr int kOrdThreads = 512;
+constexpr int kOrdItems = kOrderRows / kOrdThreads;
+
+// Bit mask of the valid blocks of word w of a row with bt complete past blocks.
+__device__ __forceinline__ unsigned row_word_mask(int w, int bt) {
+    const int rem = bt - w * 32;
+    return rem >= 32 ? 0xFFFFFFFFu : (rem <= 0 ? 0u : ((1u << rem) - 1u));
+}
+
+__global__ void __launch_bounds__(kOrdThreads, 1)
+order_rows_kernel(const unsigned* __restrict__ rowbits, const unsigned* __restrict__ wcnt, int* __restrict__ ord_rows,
+                  PrefillGeom g) {
+    using Sort = cub::BlockRadixSort<unsigned, kOrdThreads, kOrdItems, int>;
+    extern __shared__ unsigned dyn[];                   // [kOrderRows] row scores, then [nbw * 32] counts
+    unsigned* const score = dyn;
+    unsigned* const cnt = dyn + kOrderRows;
+    __shared__ union {
+        typename Sort::TempStorage sort_tmp;
+        int sorted[kOrderRows];                         // window row by rank (after the sort)
+    } sh;
+    __shared__ unsigned smax_sh;
+
+    const int nwin = (g.T + g.W - 1) / g.W;
+    const int bg = blockIdx.x / nwin, win = blockIdx.x % nwin;
+    const int b = bg / g.Hkv, kvh = bg % g.Hkv;
+    const int p0 = win * g.W, np = min(g.W, g.T - p0); // positions of the window
+    const int R = np * g.G;                             // rows: ri = hl * np + (t - p0)
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int kWarps = kOrdThreads / 32;
+    const size_t row0 = (size_t)(b * g.Hq + kvh * g.G) * g.T;
+    auto row_bits = [&](int ri) { return rowbits + (row0 + (size_t)(ri / np) * g.T + p0 + ri % np) * g.nbw; };
+    auto row_bt = [&](int ri) { return (p0 + ri % np) / kBlock; };
+
+    const int nbt = (p0 + np - 1) / kBlock + 1;         // blocks 0 .. nbt-1 (own blocks included)
+    const int nwm = min(g.nbw, (nbt + 31) / 32);        // bitmap words any row of the window uses
+    // the window's block counts, accumulated by the coarse stage
+    const unsigned* wc = wcnt + ((size_t)bg * nwin + win) * g.nbs;
+    for (int i = tid; i < nwm * 32; i += kOrdThreads) cnt[i] = i < g.nbs ? wc[i] : 0u;
+    if (tid == 0) smax_sh = 0u;
+    __syncthreads();
+    // ---- signature score_r = sum of the counts of the row's selected blocks: a thread per
+    // row, the row's bitmap words loaded 8 at a time (independent loads in flight)
+    unsigned my_max = 0u;
+    for (int ri = tid; ri < R; ri += kOrdThreads) {
+        const int bt = row_bt(ri), nw = (bt + 31) / 32;
+        const unsigned* rb = row_bits(ri);
+        unsigned sc = 0u;
+        for (int w0 = 0; w0 < nw; w0 += 8) {
+            unsigned wv[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) wv[k] = w0 + k < nw ? rb[w0 + k] & row_word_mask(w0 + k, bt) : 0u;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                unsigned word = wv[k];
+                while (word) {
+                    sc += cnt[(w0 + k) * 32 + __ffs(word) - 1];
+                    word &= word - 1u;
+                }
+            }
+        }
+        score[ri] = sc;
+        my_max = max(my_max, sc);
+    }
+    my_max = __reduce_max_sync(0xffffffffu, my_max);
+    if (lane == 0) atomicMax(&smax_sh, my_max);
+    __syncthreads();
+    // ---- stable sort on the bits the scores use (blocked arrangement: thread i holds ranks
+    // 8 i .. 8 i + 7); padding rows (past R) get the largest key and sort last
+    const int nbits = 33 - __clz((int)(smax_sh | 1u));  // bits of max(score) + 1
+    const unsigned pad = nbits >= 32 ? 0xFFFFFFFFu : (1u << nbits) - 1u;
+    unsigned keys[kOrdItems];
+    int vals[kOrdItems];
+#pragma unroll
+    for (int k = 0; k < kOrdItems; ++k) {
+        const int ri = tid * kOrdItems + k;
+        keys[k] = ri < R ? score[ri] : pad;
+        vals[k] = ri;
+    }
+    Sort(sh.sort_tmp).Sort(keys, vals, 0, nbits > 32 ? 32 : nbits);
+    __syncthreads();                                    // the sort's storage is reused below
+#pragma unroll
+    for (int k = 0; k < kOrdItems; ++k) sh.sorted[tid * kOrdItems + k] = vals[k];
+    __syncthreads();
+    const int ntw = (R + kTileRows - 1) / kTileRows;
+    const size_t tile0 = (size_t)bg * g.ord_bg + (size_t)win * g.ord_tw;
+    for (int i = tid; i < ntw * kTileRows; i += kOrdThreads) {
+        const int ri = i < R ? sh.sorted[i] : -1;
+        ord_rows[tile0 * kTileRows + i] = ri < 0 ? -1 : (ri / np) * g.T + p0 + ri % np;
+    }
+}
+
+// One warp per ordered tile: the union of its rows' selected blocks and own blocks.  Lanes
+// take 32 consecutive bitmap words and OR them over the tile's rows (one coalesced load per
+// row), then a scan of the words' popcounts places their set bits in the ascending list.
+constexpr int kUnionWarps = 8;
+
+__global__ void __launch_bounds__(kUnionWarps * 32)
+order_union_kernel(const unsigned* __restrict__ rowbits, const int* __restrict__ ord_rows, int* __restrict__ ord_list,
+                   int* __restrict__ ord_count, WsHeader* __restrict__ hdr, PrefillGeom g) {
+    __shared__ int bt_sh[kUnionWarps][kTileRows];                    // own block, -1: no row
+    __shared__ const unsigned* rb_sh[kUnionWarps][kTileRows];         // the row's bitmap
+    const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
+    const int tile = blockIdx.x * kUnionWarps + wl;
+    if (tile >= g.ord_ntiles) return;                   // whole warp
+    const int bg = tile / g.ord_bg;
+    const int b = bg / g.Hkv, kvh = bg % g.Hkv;
+    const size_t row0 = (size_t)(b * g.Hq + kvh * g.G) * g.T;
+    int btmax = 0;
+    for (int k = lane; k < kTileRows; k += 32) {
+        const int rid = ord_rows[(size_t)tile * kTileRows + k];
+        const int bt = rid >= 0 ? (rid % g.T) / kBlock : -1;
+        bt_sh[wl][k] = bt;
+        rb_sh[wl][k] = rowbits + (row0 + (size_t)(rid >= 0 ? rid : 0)) * g.nbw;
+        btmax = max(btmax, bt);
+    }
+    btmax = __reduce_max_sync(0xffffffffu, btmax);
+    __syncwarp();
+    const int nwt = btmax / 32 + 1;                     // words holding any listed block
+    int* dst = ord_list + (size_t)tile * g.ord_cap;
+    int total = 0;
+    for (int wb = 0; wb < nwt; wb += 32) {
+        const int w = wb + lane;
+        unsigned word = 0u;
+        for (int k0 = 0; k0 < kTileRows; k0 += 8) {
+            unsigned wv[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {                   // 8 independent loads in flight
+                const int bt = bt_sh[wl][k0 + k];
+                wv[k] = (bt >= 0 && w * 32 < bt) ? rb_sh[wl][k0 + k][w] & row_word_mask(w, bt) : 0u;
+                if (bt >= 0 && (bt >> 5) == w) wv[k] |= 1u << (bt & 31);   // own block
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) word |= wv[k];
+        }
+        const int pc = __popc(word);
+        int incl = pc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int nn = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += nn;
+        }
+        int pos = total + incl - pc;
+        while (word) {
+            dst[pos++] = w * 32 + __ffs(word) - 1;
+            word &= word - 1u;
+        }
+        total += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+        ord_count[tile] = total;
+        atomicAdd(&hdr->union_blocks, (unsigned long long)total);
+        atomicAdd(&hdr->tiles, 1ull);
+        atomicAdd(&hdr->fine_steps, (unsigned long long)total);
+    }
+}
+
+cudaError_t launch_order_tiles(const PrefillGeom& g, char* ws, cudaStream_t stream) {
+    if (!g.tc || g.nbs == 0) return cudaErrorInvalidValue;
+    const int nwin = (g.T + g.W - 1) / g.W;
+    const unsigned* rowbits = reinterpret_cast<const unsigned*>(ws + g.off_rowbits);
+    int* ord_rows = reinterpret_cast<int*>(ws + g.off_ord_rows);
+    const int sm = (kOrderRows + g.nbw * 32) * (int)sizeof(unsigned);
+    cudaError_t e = cudaFuncSetAttribute(order_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
+    if (e != cudaSuccess) return e;
+    order_rows_kernel<<<g.B * g.Hkv * nwin, kOrdThreads, sm, stream>>>(
+        rowbits, reinterpret_cast<const unsigned*>(ws + g.off_wcnt), ord_rows, g);
+    order_union_kernel<<<(g.ord_ntiles + kUnionWarps - 1) / kUnionWarps, kUnionWarps * 32, 0, stream>>>(
+        rowbits, ord_rows, reinterpret_cast<int*>(ws + g.off_ord_list), reinterpret_cast<int*>(ws + g.off_ord_count),
+        reinterpret_cast<WsHeader*>(ws), g);
+    return cudaGetLastError();
+}
+
+}  // namespace dash

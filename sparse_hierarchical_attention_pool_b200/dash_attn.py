@@ -43,7 +43,7 @@ class DashError(RuntimeError):
 class dash_stats(ctypes.Structure):
     _fields_ = [("scored_pairs", ctypes.c_longlong), ("selected_pairs", ctypes.c_longlong),
                 ("union_blocks", ctypes.c_longlong), ("tiles", ctypes.c_longlong),
-                ("status", ctypes.c_int)]
+                ("status", ctypes.c_int), ("fine_steps", ctypes.c_longlong)]
 
 
 _lib = None

@@ -147,7 +147,8 @@ def test_stats_count_selected_pairs():
     near = int(sum((np.abs(sel["x"][r, :sel["bt"][r]] - sel["tau"][r]) < 1e-4).sum() for r in range(len(rows))))
     assert abs(st["selected_pairs"] - int(sel["nsel"].sum())) <= near
     assert st["status"] == 0 and st["tiles"] > 0
-    assert st["union_blocks"] <= st["tiles"] * (T // 64)
+    assert st["union_blocks"] <= st["tiles"] * ((T + 63) // 64)
+    assert st["fine_steps"] >= st["union_blocks"]
 
 
 # ------------------------------------------------------------------ the workloads at full size
