@@ -251,10 +251,23 @@ def time_prefill(wl, qd, kd, vd, alpha, cs, steps, warmup, flush, ws, wsb=None, 
         "summary_roofline": {"bound": "hbm", "kernel": "block_summary_kernel", "bytes_per_launch": sum_bytes,
                              "achieved": round(sum_gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                              "frac": round(sum_gbs / pk["hbm_gbs"], 4)},
-        "launches_per_step": 3,
+        # block summary, coarse, fine; with selection-ordered tiles also the two ordering kernels
+        "launches_per_step": 5 if (Hq // Hkv <= 16 and T >= 64 and os.environ.get("DASH_TILES") != "positions") else 3,
         "l2": "flushed before every timed step",
         "_wsb": wsb, "_out": out, "_fine_alg": fine_alg, "_fine_exec": fine_exec,
     }
+
+
+def tau_start_timings(wl, qd, kd, vd, alpha, cs, steps, warmup, flush, ws, newton_ms):
+    """The coarse stage with the histogram-started threshold solve (AdaSplash-2's
+    initialisation) against the default start, same inputs and steps."""
+    os.environ["DASH_ENTMAX_INIT"] = "histogram"
+    try:
+        r = time_prefill(wl, qd, kd, vd, alpha, cs, steps, warmup, flush, ws)
+    finally:
+        os.environ.pop("DASH_ENTMAX_INIT", None)
+    return {"default_coarse_select_ms": newton_ms, "histogram_coarse_select_ms": r["stage_ms"]["coarse_select"],
+            "note": "default: Newton from u = -1 (scores in TMEM) or from the top-8 subset root (streamed tiles)"}
 
 
 def public(d):
@@ -301,6 +314,8 @@ def bench_prefill(args, ws, rank, local):
                if G <= 16 else recorded_traffic("fine_mma_kernel", source_sha("fine_mma.cu", "mma_sync.cuh", "common.cuh"),
                                                 args.workload))
     core["roofline"]["traffic"] = traffic
+    tau_start = tau_start_timings(wl, qd, kd, vd, alpha, cs, args.steps, args.warmup, flush, ws,
+                                  core["stage_ms"]["coarse_select"])
     res = {
         "step_ms": core["step_ms"],
         "tok_s": core["tok_s"],
@@ -312,7 +327,8 @@ def bench_prefill(args, ws, rank, local):
         "coarse_algorithmic_flops": core["coarse_algorithmic_flops"],
         "summary_roofline": core["summary_roofline"],
         "context": context,
-        "launches_per_step": 3,
+        "launches_per_step": core["launches_per_step"],
+        "tau_start": tau_start,
         "wl": wl, "cs": cs,
     }
     # end-to-end through the host-buffer entry point
@@ -378,7 +394,10 @@ def bench_other_prefills(args, ws, rank):
     cs = calibrated("96k")["coarse_scale"]
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     del q, k, v
-    res["96k"] = public(time_prefill(wl, qd, kd, vd, wl.alpha, cs, args.steps, args.warmup, flush, ws))
+    r96 = public(time_prefill(wl, qd, kd, vd, wl.alpha, cs, args.steps, args.warmup, flush, ws))
+    r96["tau_start"] = tau_start_timings(wl, qd, kd, vd, wl.alpha, cs, args.steps, args.warmup, flush, ws,
+                                         r96["stage_ms"]["coarse_select"])
+    res["96k"] = r96
     del qd, kd, vd
     torch.cuda.empty_cache()
     return res
@@ -731,6 +750,7 @@ def main():
             "clocks": pre["clocks"],
             "gpu_launches": pre["launches_per_step"] * args.steps,
             "stage_ms": pre["stage_ms"],
+            "tau_start": pre["tau_start"],
             "summary_roofline": pre["summary_roofline"],
             "context": pre["context"],
             "prefill_stats": pre["stats"],

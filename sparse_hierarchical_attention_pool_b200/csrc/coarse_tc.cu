@@ -26,9 +26,15 @@
 //                      bitmap) and counts selected pairs; warp 0 compacts the bitmap into
 //                      the tile's ascending block list.
 // Tiles with bt <= 512 keep all their scores in TMEM: one GEMM pass, every further pass
-// reads TMEM.  Longer tiles recompute their score chunks for every pass; the threshold
+// reads TMEM.  Optional histogram start (alpha = 1.5 and 2; "DashAttention: Differentiable and
+// Adaptive Sparse Hierarchical Attention", paper listing page, the AdaSplash-2 abstract): after
+// the max, one pass bins y = x - max over (-1, 0] into 16 bins with integer count, offset and
+// squared-offset sums per row; f at every bin edge follows exactly from them, and Newton starts
+// at the highest edge with f >= 1.  Longer tiles recompute their score chunks for every pass; the threshold
 // warps tell the producer and the MMA issuer after each pass whether another is needed.
 // Every wait is bounded (~2 s); a CTA that gives up sets a status bit and exits cleanly.
+#include <string.h>
+
 #include <type_traits>
 
 #include "common.cuh"
@@ -42,6 +48,7 @@ constexpr int kCtStages = 2;
 constexpr int kCtChunk = 128;        // blocks per score chunk (MMA N)
 constexpr int kCtBufs = 4;           // TMEM chunk buffers (4 x 128 columns)
 constexpr int kTopK = 4;             // largest scores per half-row kept for the threshold start
+constexpr int kHistBins = 16;        // bins of y = x - max over (-1, 0] for the threshold start
 
 template <int D>
 struct CtLayout {
@@ -52,7 +59,12 @@ struct CtLayout {
     static constexpr uint32_t kStage = 2 * kKPart;              // hi then lo
     static constexpr uint32_t off_q = 0;
     static constexpr uint32_t off_k = kQ;
-    static constexpr uint32_t bytes = off_k + kCtStages * kStage + 1024;
+    // per-tile scratch of the threshold warps: the histogram of the start (between the max
+    // pass and the first Newton pass) or the block byte counters (union pass), never both
+    static constexpr uint32_t off_aux = off_k + kCtStages * kStage;
+    static constexpr uint32_t kAux = (3 * kHistBins * kTileRows * 4) > (kMaxT / kBlock)
+                                         ? (3 * kHistBins * kTileRows * 4) : (kMaxT / kBlock);
+    static constexpr uint32_t bytes = off_aux + kAux + 1024;
 };
 
 enum : int { C_Q_FULL = 0, C_Q_EMPTY = 1, C_K_FULL = 2, C_K_EMPTY = C_K_FULL + kCtStages,
@@ -86,7 +98,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                  const __grid_constant__ CUtensorMap tm_lo, float* __restrict__ tau_out,
                  int* __restrict__ list, int* __restrict__ count, WsHeader* __restrict__ hdr,
                  PrefillGeom g, float alpha, float cx, unsigned* __restrict__ rowbits,
-                 unsigned* __restrict__ wcnt) {
+                 unsigned* __restrict__ wcnt, int hist_init) {
     using L = CtLayout<D>;
     using namespace sm100;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -100,12 +112,17 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __shared__ float xp[2][2][6][kTileRows];     // [pass parity][half][sum][row]: partial pass sums
     __shared__ float topv[2][kTopK][kTileRows];  // [half][rank][row]: each half-row's largest scores
     __shared__ int wtot_sh[8];
-    __shared__ unsigned bcnt[kMaxT / kBlock / 4];  // per block of a tile: rows selecting it (a byte each)
+    __shared__ float u0_sh[kTileRows];
 
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
     auto k_addr = [&](int st) { return base + L::off_k + (uint32_t)st * L::kStage; };
+    // per block of a tile: rows selecting it (a byte each, four per word)
+    unsigned* const bcnt = reinterpret_cast<unsigned*>(smem_raw + (base - raw) + L::off_aux);
+    // threshold start (alpha = 1.5 and 2): per row and bin, the count, the sum of the offsets
+    // from the bin's lower edge (2^-20 units) and of their squares (2^-24 units)
+    unsigned (*const hist)[kHistBins][kTileRows] = reinterpret_cast<unsigned (*)[kHistBins][kTileRows]>(bcnt);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
@@ -246,6 +263,40 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         auto sync_pair = [&]() { asm volatile("bar.sync %0, 64;" :: "r"(2 + quarter) : "memory"); };
         // with row bitmaps: add how many of this warp's rows select each of the nbits blocks
         // starting at j0 to the tile's byte counters (at most 128 rows per tile: no carry)
+        // histogram start: y = x - m in (-1, 0] (values at or below -1 are never selected:
+        // p_max <= 1 puts tau at or above m - 1).  Integer sums: the same start on every run.
+        auto hist_zero = [&]() {
+            for (int i = st; i < 3 * kHistBins * kTileRows; i += 256) (&hist[0][0][0])[i] = 0u;
+        };
+        auto hist_add = [&](float y) {
+            if (y > -1.0f) {
+                const float z = y + 1.0f;                   // (0, 1]
+                const int bin = min(kHistBins - 1, (int)(z * (float)kHistBins));
+                const float off = z - (float)bin * (1.0f / kHistBins);   // [0, 1 / 16]
+                atomicAdd(&hist[0][bin][r], 1u);
+                atomicAdd(&hist[1][bin][r], __float2uint_rn(off * 1048576.0f));
+                atomicAdd(&hist[2][bin][r], __float2uint_rn(off * off * 16777216.0f));
+            }
+        };
+        // the highest bin edge e with f(e) = sum_{y > e} (y - e)^e_pow >= 1 (approximately: a
+        // start slightly above the root is corrected by the first Newton step); one thread per
+        // row (hf == 0) writes it to u0_sh
+        auto hist_start = [&](int mode) {
+            if (hf != 0) return;
+            float u0 = -1.0f;
+            for (int k = kHistBins - 1; k > 0; --k) {
+                float f = 0.f;
+                for (int bn = k; bn < kHistBins; ++bn) {
+                    const float c = (float)hist[0][bn][r];
+                    const float s1 = (float)hist[1][bn][r] * (1.0f / 1048576.0f);
+                    const float s2 = (float)hist[2][bn][r] * (1.0f / 16777216.0f);
+                    const float dd = (float)(bn - k) * (1.0f / kHistBins);
+                    f += mode == 1 ? fmaf(c * dd, dd, fmaf(2.0f * dd, s1, s2)) : fmaf(c, dd, s1);
+                }
+                if (f >= 1.0f) { u0 = -1.0f + (float)k * (1.0f / kHistBins); break; }
+            }
+            u0_sh[r] = u0;
+        };
         auto count_blocks = [&](int j0, unsigned mask, int nbits) {
             unsigned mine = 0u;
             for (int i = 0; i < nbits; ++i) {
@@ -338,8 +389,30 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 xp[0][hf][0][r] = m;
                 sync_pair();
                 m = fmaxf(xp[0][0][0][r], xp[0][1][0][r]);
-                // Newton from u = -1: with the scores in registers a pass is cheap, and the
-                // subset start of the streamed tiles costs more here than the passes it saves
+                // Newton from u = -1 (with the scores in registers a pass is cheap), or, with
+                // the histogram start (alpha = 1.5 and 2), from the bin edge below the root
+                const int hmode = !hist_init ? 0 : (alpha == 1.5f ? 1 : (alpha == 2.0f ? 2 : 0));
+                float u_start = -1.0f;
+                if (hmode) {
+                    hist_zero();
+                    sync8();
+                    if (valid) {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) hist_add(xc[k][i] - m);
+                        tail([&](int, const uint32_t* v, int nv) {
+                            for (int i = 0; i < 16; ++i)
+                                if (i < nv) hist_add(__fmul_rn(__uint_as_float(v[i]), cx) - m);
+                        });
+                    } else {
+                        tail([&](int, const uint32_t*, int) {});   // TMEM loads are warp-collective
+                    }
+                    sync8();
+                    hist_start(hmode);
+                    sync8();
+                    u_start = u0_sh[r];
+                }
                 EntmaxSolver sv;
                 bool done = !valid;
                 // ---- Newton / exact-support passes; the pair of warps iterates until all of
@@ -347,7 +420,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 // exchanged through a buffer alternating with the pass parity
                 auto sweep = [&](auto mode) {
                     constexpr int MODE = decltype(mode)::value;
-                    sv.init(m, alpha, -1.0f, g.maxit);
+                    sv.init(m, alpha, u_start, g.maxit);
                     for (int pp = 1; __any_sync(0xffffffffu, !done); ++pp) {
                         EntmaxPass ps;
                         ps.reset();
@@ -464,10 +537,26 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 // the pooled values are read from shared memory on every subset pass (they
                 // would otherwise take registers from the whole kernel)
                 auto ysub = [&](int i) { return topv[i / kTopK][i % kTopK][r] - m; };
-                const float u0 = !valid ? -1.0f
-                               : alpha == 1.5f ? subset_start<2 * kTopK, 1>(ysub, alpha)
-                               : alpha == 2.0f ? subset_start<2 * kTopK, 2>(ysub, alpha)
-                                               : subset_start<2 * kTopK, 0>(ysub, alpha);
+                float u0 = !valid ? -1.0f
+                         : alpha == 1.5f ? subset_start<2 * kTopK, 1>(ysub, alpha)
+                         : alpha == 2.0f ? subset_start<2 * kTopK, 2>(ysub, alpha)
+                                         : subset_start<2 * kTopK, 0>(ysub, alpha);
+                // histogram start (alpha = 1.5 and 2): one more pass places the start at the
+                // bin edge below the root when that is higher than the subset start
+                const int hmode = !hist_init ? 0 : (alpha == 1.5f ? 1 : (alpha == 2.0f ? 2 : 0));
+                if (hmode) {
+                    hist_zero();
+                    sync8();
+                    announce(true);                            // the histogram pass follows
+                    if (!run_pass([&](int, const uint32_t* v, int nv) {
+                            for (int i = 0; i < 32; ++i)
+                                if (i < nv && valid) hist_add(__fmul_rn(__uint_as_float(v[i]), cx) - m);
+                        })) { ok = false; break; }
+                    sync8();
+                    hist_start(hmode);
+                    sync8();
+                    if (valid) u0 = fmaxf(u0, u0_sh[r]);
+                }
                 EntmaxSolver sv;
                 sv.init(m, alpha, u0, g.maxit);
                 bool done = !valid;
@@ -632,6 +721,11 @@ cudaError_t launch_coarse_tc(const void* q, const PrefillGeom& g, char* ws, floa
     int* list = reinterpret_cast<int*>(ws + g.off_list);
     int* count = reinterpret_cast<int*>(ws + g.off_count);
     unsigned* rowbits = write_rowbits ? reinterpret_cast<unsigned*>(ws + g.off_rowbits) : nullptr;
+    // DASH_ENTMAX_INIT=histogram starts the threshold solves at a histogram edge (AdaSplash-2's
+    // initialisation); the default, Newton from u = -1 (resident tiles) or from the subset
+    // start (streamed tiles), is faster on the workloads measured here
+    const char* init = getenv("DASH_ENTMAX_INIT");
+    const int hist_init = (init && strcmp(init, "histogram") == 0) ? 1 : 0;
     unsigned* wcnt = write_rowbits ? reinterpret_cast<unsigned*>(ws + g.off_wcnt) : nullptr;
     if (wcnt) {
         const size_t nwin = (size_t)((g.T + g.W - 1) / g.W);
@@ -642,7 +736,8 @@ cudaError_t launch_coarse_tc(const void* q, const PrefillGeom& g, char* ws, floa
     auto go = [&](auto kernel, int sm) -> cudaError_t {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
         if (e != cudaSuccess) return e;
-        kernel<<<grid, 320, sm, stream>>>(tq, thi, tlo, tau, list, count, hdr, g, alpha, cx, rowbits, wcnt);
+        kernel<<<grid, 320, sm, stream>>>(tq, thi, tlo, tau, list, count, hdr, g, alpha, cx, rowbits, wcnt,
+                                          hist_init);
         return cudaSuccess;
     };
     cudaError_t e;

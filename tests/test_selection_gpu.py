@@ -183,3 +183,40 @@ def test_capped_solve_reports_no_converge_decode(solve_cap):
     solve_cap(64)
     _, ws = da.dash_decode(q.cuda(), kcd, vc.cuda(), ksum, lens, alpha=1.25, coarse_scale=cs)
     assert da.dash_get_device_status(ws) == 0
+
+
+# ------------------------------------------------------------------ histogram-started threshold (F4)
+
+@pytest.fixture
+def histogram_start(monkeypatch):
+    monkeypatch.setenv("DASH_ENTMAX_INIT", "histogram")
+    yield
+    monkeypatch.delenv("DASH_ENTMAX_INIT", raising=False)
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged", "16k", "96k"])
+def test_histogram_start_prefill_vs_oracle(histogram_start, name):
+    """The AdaSplash-2 style start (a histogram edge below the root) reaches the oracle's
+    thresholds, block sets and weights: register-resident rows (tiny, ragged, 16K) and the
+    streamed rows of the 96K workload (more than 512 past blocks)."""
+    from gpu_helpers import all_rows, check_prefill
+    if name == "tiny":
+        wl, (q, k, v) = inputs.make("tiny")
+        res, _, _ = check_prefill(q, k, v, 1.5, calibrated_scale("tiny"), all_rows(1, 1, wl.T), "hist tiny")
+    elif name == "ragged":
+        _, (q, k, v) = inputs.make("16k", B=2, Hq=8, Hkv=2, T=700, d=128, n_topics=16, seed=777)
+        res, _, _ = check_prefill(q, k, v, 2.0, 0.1, all_rows(2, 8, 700), "hist ragged alpha=2")
+    else:
+        wl, (q, k, v) = inputs.make(name)
+        rows = stratified_rows(wl.B, wl.Hq, wl.T, 2048 - 17 * wl.Hq, seed=wl.seed + 11)
+        res, _, _ = check_prefill(q, k, v, wl.alpha, calibrated_scale(name), rows, f"hist {name}")
+    assert res["sel"]["selected"] > 0
+    print(name, res)
+
+
+def test_histogram_start_decode_vs_oracle(histogram_start):
+    from gpu_helpers import check_decode
+    wl, (q, kc, vc, kv_len) = inputs.make("decode96k")
+    res, _, _ = check_decode(q, kc, vc, kv_len.tolist(), wl.alpha, calibrated_scale("decode96k"), "hist decode96k")
+    assert res[1] is not None and res[1]["selected"] > 0
+    print(res)
