@@ -297,12 +297,18 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             u0_sh[r] = u0;
         };
+        // (lane i's mask holds row i's bits; a 32 x 32 bit transpose in five exchange stages
+        // leaves column i, i.e. block j0 + i over the warp's rows, in lane i)
         auto count_blocks = [&](int j0, unsigned mask, int nbits) {
-            unsigned mine = 0u;
-            for (int i = 0; i < nbits; ++i) {
-                const unsigned c = __reduce_add_sync(0xffffffffu, (mask >> i) & 1u);
-                if (lane == i) mine = c;
+            unsigned x = mask;
+#pragma unroll
+            for (int j = 16; j > 0; j >>= 1) {
+                const unsigned lo = j == 16 ? 0x0000FFFFu : j == 8 ? 0x00FF00FFu : j == 4 ? 0x0F0F0F0Fu
+                                  : j == 2 ? 0x33333333u : 0x55555555u;      // columns c with (c & j) == 0
+                const unsigned y = __shfl_xor_sync(0xffffffffu, x, j);
+                x = (lane & j) ? ((x & ~lo) | ((y & ~lo) >> j)) : ((x & lo) | ((y & lo) << j));
             }
+            const unsigned mine = __popc(x);
             if (lane < nbits && mine) atomicAdd(&bcnt[(j0 + lane) >> 2], mine << (8 * ((j0 + lane) & 3)));
         };
         for (int w = blockIdx.x; ok && w < g.ntiles; w += gridDim.x) {
@@ -426,9 +432,12 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         ps.reset();
                         const float mm = sv.m, uu = sv.u;
 #pragma unroll
-                        for (int k = 0; k < 4; ++k)
+                        for (int k = 0; k < 4; ++k) {
+                            // groups wholly past the tile's blocks hold only -inf (warp-uniform)
+                            if ((k >> 1) * kCtChunk + (hf + 2 * (k & 1)) * 32 >= ti.bt) continue;
 #pragma unroll
                             for (int i = 0; i < 32; ++i) ps.add_t<MODE>((xc[k][i] - mm) - uu, sv.e);
+                        }
                         tail([&](int, const uint32_t* v, int nv) {
                             for (int i = 0; i < 16; ++i)
                                 if (i < nv) ps.add_t<MODE>((__fmul_rn(__uint_as_float(v[i]), cx) - mm) - uu, sv.e);
@@ -468,8 +477,10 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             count_blocks(j0, mask, 32);
                         }
                         nsel += (float)__popc(mask);
-                        const unsigned wm = __reduce_or_sync(0xffffffffu, mask);
-                        if (lane == 0 && wm) atomicOr(&bitmap[j0 >> 5], wm);
+                        if (!rowbits) {
+                            const unsigned wm = __reduce_or_sync(0xffffffffu, mask);
+                            if (lane == 0 && wm) atomicOr(&bitmap[j0 >> 5], wm);
+                        }
                     }
                 }
                 tail([&](int j0, const uint32_t* v, int nv) {
@@ -483,8 +494,10 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         count_blocks(j0, mask, 16);
                     }
                     nsel += (float)__popc(mask);
-                    const unsigned wm = __reduce_or_sync(0xffffffffu, mask);
-                    if (lane == 0 && wm) atomicOr(&bitmap[j0 >> 5], wm << (j0 & 31));
+                    if (!rowbits) {
+                        const unsigned wm = __reduce_or_sync(0xffffffffu, mask);
+                        if (lane == 0 && wm) atomicOr(&bitmap[j0 >> 5], wm << (j0 & 31));
+                    }
                 });
                 for (int c = 0; c < ti.nch; ++c) release((sweep_base + c) % kCtBufs);
             } else {
@@ -610,8 +623,10 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             count_blocks(j0, mask, 32);
                         }
                         nsel += (float)__popc(mask);
-                        const unsigned wm = __reduce_or_sync(0xffffffffu, mask);
-                        if (lane == 0 && wm) atomicOr(&bitmap[j0 >> 5], wm);
+                        if (!rowbits) {
+                            const unsigned wm = __reduce_or_sync(0xffffffffu, mask);
+                            if (lane == 0 && wm) atomicOr(&bitmap[j0 >> 5], wm);
+                        }
                     })) { ok = false; break; }
                 announce(false);
             }
@@ -632,8 +647,15 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
             }
             // ---- compaction: thread st owns bitmap words 2 st and 2 st + 1; a block-wide
-            // scan of their popcounts places them in the tile's ascending list
-            {
+            // scan of their popcounts places them in the tile's ascending list.  With row
+            // bitmaps the fine stage runs ordered tiles and reads no position-tile list.
+            if (rowbits) {
+                if (st == 0) {
+                    const int rows_valid = g.G * min(g.P, g.T - ti.t0);
+                    atomicAdd(&hdr->selected_pairs, sel_sh);
+                    atomicAdd(&hdr->scored_pairs, (unsigned long long)rows_valid * ti.bt);
+                }
+            } else {
                 unsigned wv[2];
                 int pc = 0;
 #pragma unroll
