@@ -49,6 +49,10 @@ inline int solve_cap_from_env() {
 // are sorted by a selection signature, and every 128 consecutive sorted rows form a tile
 // whose block list is the union of its rows' selected blocks and own blocks.
 constexpr int kOrderRows = 4096;
+// row ids in the ordered tiles: (head in the KV group << kRowShift) | position (T <= 2^20)
+constexpr int kRowShift = 20;
+constexpr int kRowMask = (1 << kRowShift) - 1;
+static_assert(kMaxT <= (1 << kRowShift), "positions fit the row id");
 
 struct PrefillGeom {
     int B, Hq, Hkv, T, d, G, P, M;   // M = G * P rows used of the 128-row tile

@@ -11,12 +11,12 @@
 //
 // One CTA per tile.  The tile's listed blocks (steps s = 0 .. n-1, own block last) are
 // dealt alternately to two softmax groups (group s & 1), each with its own TMEM S buffer,
-// two P buffers (steps alternate between them), O accumulator, row-sum column and running
+// kPBuf P buffers (its steps take them in turn), O accumulator, row-sum column and running
 // max; the two partial softmaxes are merged in the epilogue (exactly as split-KV partials).
 // The per-step work of a row is a serial chain (load S, row stats, weights, exponentials,
 // P), so two groups keep two chains in flight while sharing the Q tile and every K/V load;
-// with two P buffers a group writes P_s while the tensor core still reads P_{s-2}, and
-// waits for its previous product only to rescale O.  Warps:
+// with kPBuf P buffers a group writes P_s while the tensor core still reads its earlier
+// ones, and waits for its previous product only to rescale O.  Warps:
 //   8 SPLIT            K producer (one lane): the Q tile once (one 64-column box per head
 //                      and half of d), then K and the summary rows of every listed block,
 //                      3-stage ring (a stage is free once S of its block is computed);
@@ -25,7 +25,7 @@
 //   8 SPLIT + 1        S issuer (one lane): S_s = Q [K_s | kbar_hi | kbar_lo]^T (M=128, N=80
 //                      with the summary atoms at columns 64 and 72) into the S buffer of
 //                      group s & 1 as soon as block s is loaded, that group has read
-//                      S_{s-2} and the product of step s-4 (same P buffer) has landed, so
+//                      S_{s-2} and the product of step s - 2 kPBuf (same P buffer) has landed, so
 //                      S_{s+2} is computed while the group works on step s and a group
 //                      that sees S_s may write its P buffer without another wait;
 //   8 SPLIT + 2        PV issuer (one lane): O_g += P_s V_s (M=128, N=d) and L_g += P_s 1
@@ -63,6 +63,7 @@ namespace dash {
 
 constexpr int kKStages = 3;            // K (+ summary rows) ring
 constexpr int kVStages = 3;            // V ring
+constexpr int kPBuf = 2;               // P buffers of each softmax group (its steps take them in turn)
 constexpr int kFineSplit = 1;          // threads per tile row in each softmax group
 constexpr int kFinePolyPairs = 1;      // pairs of every 4 whose 2^x runs on the FMA pipe
 constexpr bool kFineIntPack = false;   // fp32 -> bf16 pairs with integer ops instead of cvt
@@ -133,8 +134,8 @@ struct TcLayout {
     static constexpr uint32_t off_q = 0;
     static constexpr uint32_t off_k = kQ;                       // K ring
     static constexpr uint32_t off_v = off_k + kKStages * kK;    // V ring
-    static constexpr uint32_t off_p = off_v + kVStages * kV;    // P buffers [group][2]
-    static constexpr uint32_t off_ones = off_p + 4 * kP;        // 16 x 64 bf16 ones (B of the row sum)
+    static constexpr uint32_t off_p = off_v + kVStages * kV;    // P buffers [group][kPBuf]
+    static constexpr uint32_t off_ones = off_p + 2 * kPBuf * kP; // 16 x 64 bf16 ones (B of the row sum)
     static constexpr uint32_t bytes = off_ones + 2048 + 1024;   // + alignment slack
     // TMEM columns: S of group 0 and 1, O of group 0 and 1, row sums of group 0 and 1
     static constexpr uint32_t colS = 96;                        // S buffer of group g at g * 96 (80 used)
@@ -143,10 +144,10 @@ struct TcLayout {
 };
 constexpr uint32_t kTmemCols = 512;
 
-// barrier slots (P_FULL and PV_DONE per P buffer: index 2 group + buffer)
+// barrier slots (P_FULL and PV_DONE per P buffer: index kPBuf group + buffer)
 enum : int { B_Q = 0, B_K_FULL = 1, B_K_EMPTY = B_K_FULL + kKStages, B_V_FULL = B_K_EMPTY + kKStages,
              B_V_EMPTY = B_V_FULL + kVStages, B_S_FULL = B_V_EMPTY + kVStages, B_S_FREE = B_S_FULL + 2,
-             B_P_FULL = B_S_FREE + 2, B_PV_DONE = B_P_FULL + 4, B_DRAIN = B_PV_DONE + 4,
+             B_P_FULL = B_S_FREE + 2, B_PV_DONE = B_P_FULL + 2 * kPBuf, B_DRAIN = B_PV_DONE + 2 * kPBuf,
              B_DRAIN2 = B_DRAIN + 1, B_COUNT = B_DRAIN2 + 1 };
 
 template <int D, int SPLIT, bool AGG, bool DUMP, bool ORD>
@@ -214,7 +215,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(bar(B_S_FULL + i), 1);
             mbar_init(bar(B_S_FREE + i), kGroupThreads);
         }
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 2 * kPBuf; ++i) {
             mbar_init(bar(B_P_FULL + i), kGroupThreads);
             mbar_init(bar(B_PV_DONE + i), 1);
         }
@@ -320,10 +321,11 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const int st = s % kKStages, sb = s & 1;
                 if (!mbar_wait(bar(B_K_FULL + st), (s / kKStages) & 1, abort_flag)) { ok = false; break; }
                 if (s >= 2 && !mbar_wait(bar(B_S_FREE + sb), ((s - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
-                // the P buffer step s will use was last read by the product of step s - 4:
-                // S_s is computed only after that product landed, so a softmax group that
-                // sees S_s may overwrite the buffer
-                if (s >= 4 && !mbar_wait(bar(B_PV_DONE + 2 * sb + ((s >> 1) & 1)), (((s >> 1) - 2) >> 1) & 1, abort_flag)) {
+                // the P buffer step s will use was last read by the product of step
+                // s - 2 kPBuf: S_s is computed only after that product landed, so a softmax
+                // group that sees S_s may overwrite the buffer
+                const int i2 = s >> 1;
+                if (i2 >= kPBuf && !mbar_wait(bar(B_PV_DONE + kPBuf * sb + i2 % kPBuf), ((i2 - kPBuf) / kPBuf) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -348,14 +350,14 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     } else if (warp == kMmaPvWarp) {
         // ------------------------------------------------------------ PV issuer
         // O_g += P_p V_p and L_g += P_p 1 as soon as P_p is written and V_p has landed; then
-        // the V stage of block p and P buffer (p & 1, (p >> 1) & 1) are free again.
+        // the V stage of block p and P buffer (p & 1, (p >> 1) % kPBuf) are free again.
         if (lane == 0) {
             const uint32_t idesc_pv = idesc_bf16(128, D, true);
             const uint32_t idesc_l = idesc_bf16(128, 16, false);
             bool ok = true;
             for (int p = 0; p < n; ++p) {
-                const int gp = p & 1, pbuf = 2 * gp + ((p >> 1) & 1), stp = p % kVStages;
-                if (!mbar_wait(bar(B_P_FULL + pbuf), (p >> 2) & 1, abort_flag)) { ok = false; break; }
+                const int gp = p & 1, i2 = p >> 1, pbuf = kPBuf * gp + i2 % kPBuf, stp = p % kVStages;
+                if (!mbar_wait(bar(B_P_FULL + pbuf), (i2 / kPBuf) & 1, abort_flag)) { ok = false; break; }
                 if (!mbar_wait(bar(B_V_FULL + stp), (p / kVStages) & 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t acc = p >= 2 ? 1u : 0u;          // first step of a group overwrites
@@ -389,8 +391,8 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int r = quarter * 32 + lane;                  // tile row = TMEM lane
         // the tile row: (head in group, position); ordered tiles read it from the tile's rows
         const int rid = ORD ? ord_rows[tile_id * kTileRows + r] : 0;
-        const int hl = ORD ? (rid >= 0 ? rid / g.T : 0) : r / g.P;
-        const int t = ORD ? (rid >= 0 ? rid % g.T : 0) : t0 + r % g.P;
+        const int hl = ORD ? (rid >= 0 ? rid >> kRowShift : 0) : r / g.P;
+        const int t = ORD ? (rid >= 0 ? rid & kRowMask : 0) : t0 + r % g.P;
         const bool valid = ORD ? rid >= 0 : (r < g.M && t < g.T);
         const int tpos = valid ? t : -1;
         const int bt_r = ORD ? t / kBlock : bt;             // the row's own block
@@ -425,7 +427,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const uint32_t s_col = grp * L::colS + sp * KEYS;   // this thread's keys in its group's S buffer
         const uint32_t o_col = L::colO + grp * D + sp * RCOLS;   // O columns it rescales
         const uint32_t l_col = L::colL + grp * 32;
-        uint8_t* const prow0 = base_ptr + L::off_p + (2 * grp) * L::kP + (r >> 3) * 1024 + (r & 7) * 128;
+        uint8_t* const prow0 = base_ptr + L::off_p + (kPBuf * grp) * L::kP + (r >> 3) * 1024 + (r & 7) * 128;
         const int row_bar = 1 + grp * 4 + quarter;          // named barrier of the row's SPLIT warps
         float m_run = -INFINITY;
         bool ok = true;
@@ -525,9 +527,9 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     resc = true;
                 }
             }
-            // P buffer pb of this group was last read by its product two steps back, which
+            // P buffer pb of this group was last read by its product kPBuf steps back, which
             // had landed before S_s was computed (the S issuer waits for it)
-            const int pb = i2 & 1;
+            const int pb = i2 % kPBuf;
             uint8_t* const prow = prow0 + pb * L::kP;
             // p = 2^(s sm2 + log2 p_j - m): packed FMA, exponent on the SFU or the FMA pipe,
             // bf16 pairs
@@ -573,7 +575,10 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             // rescale after P: the S registers are dead by now; O_grp and L_grp hold the
             // group's previous product only once that product has landed
             if (__any_sync(0xffffffffu, resc)) {
-                if (i2 >= 1 && !wwait(bar(B_PV_DONE + 2 * grp + (pb ^ 1)), ((i2 - 1) >> 1) & 1)) { ok = false; continue; }
+                if (i2 >= 1 && !wwait(bar(B_PV_DONE + kPBuf * grp + (i2 - 1) % kPBuf), ((i2 - 1) / kPBuf) & 1)) {
+                    ok = false;
+                    continue;
+                }
                 tc_fence_after();
 #pragma unroll
                 for (int c = 0; c < RCOLS / RCW; ++c) {
@@ -596,7 +601,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(bar(B_P_FULL + 2 * grp + pb));
+            mbar_arrive(bar(B_P_FULL + kPBuf * grp + pb));
         }
         // ---- merge the two groups: out = (O_0 2^(m_0-M) + O_1 2^(m_1-M)) / (L_0 ... + L_1 ...)
         if (sp == 0) m_sh[grp][r] = m_run;
@@ -605,8 +610,8 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int last0 = (n - 1) & ~1;                     // last step of group 0
         const int last1 = (n - 1) - ((n - 1) & 1 ? 0 : 1);  // last step of group 1
         const int i0 = last0 >> 1, i1 = last1 >> 1;       // their step indices within the groups
-        bool done = ok && wwait(bar(B_PV_DONE + (i0 & 1)), (i0 >> 1) & 1);
-        if (has1) done = done && wwait(bar(B_PV_DONE + 2 + (i1 & 1)), (i1 >> 1) & 1);
+        bool done = ok && wwait(bar(B_PV_DONE + i0 % kPBuf), (i0 / kPBuf) & 1);
+        if (has1) done = done && wwait(bar(B_PV_DONE + kPBuf + i1 % kPBuf), (i1 / kPBuf) & 1);
         if (done) {
             tc_fence_after();
             const float m0 = m_sh[0][r], m1 = has1 ? m_sh[1][r] : -INFINITY;

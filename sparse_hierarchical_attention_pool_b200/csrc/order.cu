@@ -18,9 +18,10 @@
 // tiles, and every result computed from them, are deterministic.
 //
 // The block counts c_j of every window are accumulated by the coarse stage while it writes
-// the row bitmaps.  order_rows_kernel, one CTA of 1024 threads per window: per-row scores
-// (lanes as bitmap words), then a block-wide radix sort on the bits the scores use, which
-// gives the rows of every tile.  order_union_kernel, one warp per tile: the OR of its rows' bitmaps (plus their own
+// the row bitmaps.  order_rows_kernel, one CTA of 512 threads per window: a score per row (a
+// thread per row, its bitmap words loaded 8 at a time), then a block-wide radix sort on the
+// bits the scores use, which gives the rows of every tile.  A row id is
+// (head in the KV group << kRowShift) | position, decoded with a shift and a mask.  order_union_kernel, one warp per tile: the OR of its rows' bitmaps (plus their own
 // blocks), lanes as bitmap words, compacted into the tile's ascending list.
 #include <cub/block/block_radix_sort.cuh>
 
@@ -57,10 +58,7 @@ order_rows_kernel(const unsigned* __restrict__ rowbits, const unsigned* __restri
     const int p0 = win * g.W, np = min(g.W, g.T - p0); // positions of the window
     const int R = np * g.G;                             // rows: ri = hl * np + (t - p0)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    constexpr int kWarps = kOrdThreads / 32;
     const size_t row0 = (size_t)(b * g.Hq + kvh * g.G) * g.T;
-    auto row_bits = [&](int ri) { return rowbits + (row0 + (size_t)(ri / np) * g.T + p0 + ri % np) * g.nbw; };
-    auto row_bt = [&](int ri) { return (p0 + ri % np) / kBlock; };
 
     const int nbt = (p0 + np - 1) / kBlock + 1;         // blocks 0 .. nbt-1 (own blocks included)
     const int nwm = min(g.nbw, (nbt + 31) / 32);        // bitmap words any row of the window uses
@@ -70,28 +68,29 @@ order_rows_kernel(const unsigned* __restrict__ rowbits, const unsigned* __restri
     if (tid == 0) smax_sh = 0u;
     __syncthreads();
     // ---- signature score_r = sum of the counts of the row's selected blocks: a thread per
-    // row, the row's bitmap words loaded 8 at a time (independent loads in flight)
+    // row (ri = hl np + pl), the row's bitmap words loaded 8 at a time (independent loads)
     unsigned my_max = 0u;
-    for (int ri = tid; ri < R; ri += kOrdThreads) {
-        const int bt = row_bt(ri), nw = (bt + 31) / 32;
-        const unsigned* rb = row_bits(ri);
-        unsigned sc = 0u;
-        for (int w0 = 0; w0 < nw; w0 += 8) {
-            unsigned wv[8];
+    for (int hl = 0; hl < g.G; ++hl)
+        for (int pl = tid; pl < np; pl += kOrdThreads) {
+            const int t = p0 + pl, bt = t / kBlock, nw = (bt + 31) / 32;
+            const unsigned* rb = rowbits + (row0 + (size_t)hl * g.T + t) * g.nbw;
+            unsigned sc = 0u;
+            for (int w0 = 0; w0 < nw; w0 += 8) {
+                unsigned wv[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) wv[k] = w0 + k < nw ? rb[w0 + k] & row_word_mask(w0 + k, bt) : 0u;
+                for (int k = 0; k < 8; ++k) wv[k] = w0 + k < nw ? rb[w0 + k] & row_word_mask(w0 + k, bt) : 0u;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                unsigned word = wv[k];
-                while (word) {
-                    sc += cnt[(w0 + k) * 32 + __ffs(word) - 1];
-                    word &= word - 1u;
+                for (int k = 0; k < 8; ++k) {
+                    unsigned word = wv[k];
+                    while (word) {
+                        sc += cnt[(w0 + k) * 32 + __ffs(word) - 1];
+                        word &= word - 1u;
+                    }
                 }
             }
+            score[hl * np + pl] = sc;
+            my_max = max(my_max, sc);
         }
-        score[ri] = sc;
-        my_max = max(my_max, sc);
-    }
     my_max = __reduce_max_sync(0xffffffffu, my_max);
     if (lane == 0) atomicMax(&smax_sh, my_max);
     __syncthreads();
@@ -99,13 +98,15 @@ order_rows_kernel(const unsigned* __restrict__ rowbits, const unsigned* __restri
     // 8 i .. 8 i + 7); padding rows (past R) get the largest key and sort last
     const int nbits = 33 - __clz((int)(smax_sh | 1u));  // bits of max(score) + 1
     const unsigned pad = nbits >= 32 ? 0xFFFFFFFFu : (1u << nbits) - 1u;
+    // values: the row ids of the ordered-tile lists, (head in group << 20) | position
     unsigned keys[kOrdItems];
     int vals[kOrdItems];
 #pragma unroll
     for (int k = 0; k < kOrdItems; ++k) {
         const int ri = tid * kOrdItems + k;
+        const int hl = ri / np;                         // R <= 4096 rows: one division per item
         keys[k] = ri < R ? score[ri] : pad;
-        vals[k] = ri;
+        vals[k] = ri < R ? (hl << kRowShift) | (p0 + ri - hl * np) : -1;
     }
     Sort(sh.sort_tmp).Sort(keys, vals, 0, nbits > 32 ? 32 : nbits);
     __syncthreads();                                    // the sort's storage is reused below
@@ -114,10 +115,7 @@ order_rows_kernel(const unsigned* __restrict__ rowbits, const unsigned* __restri
     __syncthreads();
     const int ntw = (R + kTileRows - 1) / kTileRows;
     const size_t tile0 = (size_t)bg * g.ord_bg + (size_t)win * g.ord_tw;
-    for (int i = tid; i < ntw * kTileRows; i += kOrdThreads) {
-        const int ri = i < R ? sh.sorted[i] : -1;
-        ord_rows[tile0 * kTileRows + i] = ri < 0 ? -1 : (ri / np) * g.T + p0 + ri % np;
-    }
+    for (int i = tid; i < ntw * kTileRows; i += kOrdThreads) ord_rows[tile0 * kTileRows + i] = i < R ? sh.sorted[i] : -1;
 }
 
 // One warp per ordered tile: the union of its rows' selected blocks and own blocks.  Lanes
@@ -139,9 +137,10 @@ order_union_kernel(const unsigned* __restrict__ rowbits, const int* __restrict__
     int btmax = 0;
     for (int k = lane; k < kTileRows; k += 32) {
         const int rid = ord_rows[(size_t)tile * kTileRows + k];
-        const int bt = rid >= 0 ? (rid % g.T) / kBlock : -1;
+        const int t = rid & kRowMask, hl = rid >> kRowShift;
+        const int bt = rid >= 0 ? t / kBlock : -1;
         bt_sh[wl][k] = bt;
-        rb_sh[wl][k] = rowbits + (row0 + (size_t)(rid >= 0 ? rid : 0)) * g.nbw;
+        rb_sh[wl][k] = rowbits + (row0 + (rid >= 0 ? (size_t)hl * g.T + t : 0)) * g.nbw;
         btmax = max(btmax, bt);
     }
     btmax = __reduce_max_sync(0xffffffffu, btmax);
