@@ -26,7 +26,10 @@
 //                      bitmap) and counts selected pairs; warp 0 compacts the bitmap into
 //                      the tile's ascending block list.
 // Tiles with bt <= 512 keep all their scores in TMEM: one GEMM pass, every further pass
-// reads TMEM.  Optional histogram start (alpha = 1.5 and 2; "DashAttention: Differentiable and
+// reads TMEM (and registers).  Newton starts at a subset root (entmax.cuh): of the maxima of
+// every 16 register values (resident tiles, free in the max pass) or of the 4 largest scores
+// of each half-row (streamed tiles).  For alpha = 1.5 and 2 a pass takes z = (x - m) - u in
+// the saturating form (EntmaxPass::add_sat).  Optional histogram start (alpha = 1.5 and 2; "DashAttention: Differentiable and
 // Adaptive Sparse Hierarchical Attention", paper listing page, the AdaSplash-2 abstract): after
 // the max, one pass bins y = x - max over (-1, 0] into 16 bins with integer count, offset and
 // squared-offset sums per row; f at every bin edge follows exactly from them, and Newton starts
@@ -111,6 +114,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __shared__ unsigned long long sel_sh;
     __shared__ float xp[2][2][6][kTileRows];     // [pass parity][half][sum][row]: partial pass sums
     __shared__ float topv[2][kTopK][kTileRows];  // [half][rank][row]: each half-row's largest scores
+    __shared__ float gsub[2][8][kTileRows];      // [half][group][row]: maxima of the register groups
     __shared__ int wtot_sh[8];
     __shared__ float u0_sh[kTileRows];
 
@@ -383,11 +387,19 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             }
                     }
                 };
+                // the maximum of every 16 register values (a subset of the row for the
+                // threshold start below), then the row maximum
                 float m = -INFINITY;
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) m = fmaxf(m, xc[k][i]);
+                    for (int h = 0; h < 2; ++h) {
+                        float a = xc[k][16 * h];
+#pragma unroll
+                        for (int i = 1; i < 16; ++i) a = fmaxf(a, xc[k][16 * h + i]);
+                        gsub[hf][2 * k + h][r] = a;
+                        m = fmaxf(m, a);
+                    }
                 tail([&](int, const uint32_t* v, int nv) {
                     for (int i = 0; i < 16; ++i)
                         if (i < nv) m = fmaxf(m, __fmul_rn(__uint_as_float(v[i]), cx));
@@ -395,10 +407,18 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 xp[0][hf][0][r] = m;
                 sync_pair();
                 m = fmaxf(xp[0][0][0][r], xp[0][1][0][r]);
-                // Newton from u = -1 (with the scores in registers a pass is cheap), or, with
-                // the histogram start (alpha = 1.5 and 2), from the bin edge below the root
+                // Newton starts at the root of the subset of the 16 group maxima (at or below
+                // the row's root, entmax.cuh), or, with the histogram start (alpha = 1.5 and 2),
+                // at the bin edge below the root when that is higher
+                float ys[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) ys[i] = gsub[i >> 3][i & 7][r] - m;
+                auto ysub = [&](int i) { return ys[i]; };
+                float u_start = !valid ? -1.0f
+                              : alpha == 1.5f ? subset_start<16, 1>(ysub, alpha)
+                              : alpha == 2.0f ? subset_start<16, 2>(ysub, alpha)
+                                              : subset_start<16, 0>(ysub, alpha);
                 const int hmode = !hist_init ? 0 : (alpha == 1.5f ? 1 : (alpha == 2.0f ? 2 : 0));
-                float u_start = -1.0f;
                 if (hmode) {
                     hist_zero();
                     sync8();
@@ -417,7 +437,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     sync8();
                     hist_start(hmode);
                     sync8();
-                    u_start = u0_sh[r];
+                    if (valid) u_start = fmaxf(u_start, u0_sh[r]);
                 }
                 EntmaxSolver sv;
                 bool done = !valid;
@@ -431,17 +451,41 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         EntmaxPass ps;
                         ps.reset();
                         const float mm = sv.m, uu = sv.u;
+                        if constexpr (MODE == 0) {
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            // groups wholly past the tile's blocks hold only -inf (warp-uniform)
-                            if ((k >> 1) * kCtChunk + (hf + 2 * (k & 1)) * 32 >= ti.bt) continue;
+                            for (int k = 0; k < 4; ++k) {
+                                // groups wholly past the tile's blocks hold only -inf (warp-uniform)
+                                if ((k >> 1) * kCtChunk + (hf + 2 * (k & 1)) * 32 >= ti.bt) continue;
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) ps.add_t<MODE>((xc[k][i] - mm) - uu, sv.e);
+                                for (int i = 0; i < 32; ++i) ps.add_t<MODE>((xc[k][i] - mm) - uu, sv.e);
+                            }
+                            tail([&](int, const uint32_t* v, int nv) {
+                                for (int i = 0; i < 16; ++i)
+                                    if (i < nv) ps.add_t<MODE>((__fmul_rn(__uint_as_float(v[i]), cx) - mm) - uu, sv.e);
+                            });
+                        } else {
+                            // pairs of values, f32x2 (EntmaxPassX2); -inf pads a group's tail
+                            EntmaxPassX2 px;
+                            px.reset();
+                            const uint64_t nm2 = f2_pack(__float_as_uint(-mm), __float_as_uint(-mm));
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                if ((k >> 1) * kCtChunk + (hf + 2 * (k & 1)) * 32 >= ti.bt) continue;
+#pragma unroll
+                                for (int i = 0; i < 32; i += 2)
+                                    px.add2<MODE>(f2_pack(__float_as_uint(xc[k][i]), __float_as_uint(xc[k][i + 1])), nm2, uu);
+                            }
+                            const uint64_t cx2 = f2_pack(__float_as_uint(cx), __float_as_uint(cx));
+                            tail([&](int, const uint32_t* v, int nv) {
+#pragma unroll
+                                for (int i = 0; i < 16; i += 2) {
+                                    uint64_t x2 = f2_mul(f2_pack(v[i], v[i + 1]), cx2);
+                                    if (i + 1 >= nv) x2 = f2_pack(i < nv ? (uint32_t)x2 : 0xFF800000u, 0xFF800000u);
+                                    px.add2<MODE>(x2, nm2, uu);
+                                }
+                            });
+                            ps = px.finish();
                         }
-                        tail([&](int, const uint32_t* v, int nv) {
-                            for (int i = 0; i < 16; ++i)
-                                if (i < nv) ps.add_t<MODE>((__fmul_rn(__uint_as_float(v[i]), cx) - mm) - uu, sv.e);
-                        });
                         float* xb = &xp[pp & 1][hf][0][0];
                         xb[0 * kTileRows + r] = ps.z0; xb[1 * kTileRows + r] = ps.z1; xb[2 * kTileRows + r] = ps.z2;
                         xb[3 * kTileRows + r] = ps.fe; xb[4 * kTileRows + r] = ps.de; xb[5 * kTileRows + r] = ps.minz;
@@ -535,6 +579,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
                 for (int i = 0; i < kTopK; ++i) tk[i] = -INFINITY;
                 if (!run_pass([&](int, const uint32_t* v, int nv) {
+#pragma unroll
                         for (int i = 0; i < 32; ++i)
                             if (i < nv) {
                                 const float x = __fmul_rn(__uint_as_float(v[i]), cx);
@@ -562,6 +607,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     sync8();
                     announce(true);                            // the histogram pass follows
                     if (!run_pass([&](int, const uint32_t* v, int nv) {
+#pragma unroll
                             for (int i = 0; i < 32; ++i)
                                 if (i < nv && valid) hist_add(__fmul_rn(__uint_as_float(v[i]), cx) - m);
                         })) { ok = false; break; }
@@ -585,19 +631,35 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     if (!more) break;
                     EntmaxPass ps;
                     ps.reset();
-                    // z = (x - m) - u with x rounded exactly as in pass 0 (__fmul_rn is never
-                    // fused into an FMA), so the maximum gives z = -u exactly
+                    EntmaxPassX2 px;
+                    px.reset();
+                    const uint64_t nm2 = f2_pack(__float_as_uint(-sv.m), __float_as_uint(-sv.m));
+                    const uint64_t cx2 = f2_pack(__float_as_uint(cx), __float_as_uint(cx));
+                    // z = (x - m) - u with x rounded exactly as in pass 0 (a multiply, never
+                    // fused into an FMA), so the maximum gives z = -u exactly; alpha = 1.5 and 2
+                    // take pairs in the saturating form
                     if (!run_pass([&](int, const uint32_t* v, int nv) {
                             auto acc = [&](auto mode) {
                                 constexpr int MODE = decltype(mode)::value;
+                                if constexpr (MODE == 0) {
 #pragma unroll
-                                for (int i = 0; i < 32; ++i)
-                                    if (i < nv) ps.add_t<MODE>((__fmul_rn(__uint_as_float(v[i]), cx) - sv.m) - sv.u, sv.e);
+                                    for (int i = 0; i < 32; ++i)
+                                        if (i < nv) ps.add_t<MODE>((__fmul_rn(__uint_as_float(v[i]), cx) - sv.m) - sv.u, sv.e);
+                                } else {
+                                    // pairs, f32x2: x = v cx (one rounding, as in pass 0), -inf past nv
+#pragma unroll
+                                    for (int i = 0; i < 32; i += 2) {
+                                        uint64_t x2 = f2_mul(f2_pack(v[i], v[i + 1]), cx2);
+                                        if (i + 1 >= nv) x2 = f2_pack(i < nv ? (uint32_t)x2 : 0xFF800000u, 0xFF800000u);
+                                        px.add2<MODE>(x2, nm2, sv.u);
+                                    }
+                                }
                             };
                             if (sv.mode == 1) acc(std::integral_constant<int, 1>{});
                             else if (sv.mode == 2) acc(std::integral_constant<int, 2>{});
                             else acc(std::integral_constant<int, 0>{});
                         })) { ok = false; break; }
+                    if (sv.mode != 0) ps = px.finish();
                     xp[0][hf][0][r] = ps.z0; xp[0][hf][1][r] = ps.z1; xp[0][hf][2][r] = ps.z2;
                     xp[0][hf][3][r] = ps.fe; xp[0][hf][4][r] = ps.de; xp[0][hf][5][r] = ps.minz;
                     sync8();
@@ -616,6 +678,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 sync8();
                 if (!run_pass([&](int j0, const uint32_t* v, int nv) {
                         unsigned mask = 0u;
+#pragma unroll
                         for (int i = 0; i < 32; ++i)
                             if (i < nv && valid && __fmul_rn(__uint_as_float(v[i]), cx) > tau) mask |= 1u << i;
                         if (rowbits) {
@@ -744,8 +807,9 @@ cudaError_t launch_coarse_tc(const void* q, const PrefillGeom& g, char* ws, floa
     int* count = reinterpret_cast<int*>(ws + g.off_count);
     unsigned* rowbits = write_rowbits ? reinterpret_cast<unsigned*>(ws + g.off_rowbits) : nullptr;
     // DASH_ENTMAX_INIT=histogram starts the threshold solves at a histogram edge (AdaSplash-2's
-    // initialisation); the default, Newton from u = -1 (resident tiles) or from the subset
-    // start (streamed tiles), is faster on the workloads measured here
+    // initialisation); the default, Newton from a subset root (the 16 group maxima of a
+    // resident row, the 8 largest scores of a streamed one), is faster on the workloads
+    // measured here
     const char* init = getenv("DASH_ENTMAX_INIT");
     const int hist_init = (init && strcmp(init, "histogram") == 0) ? 1 : 0;
     unsigned* wcnt = write_rowbits ? reinterpret_cast<unsigned*>(ws + g.off_wcnt) : nullptr;

@@ -26,13 +26,38 @@
 #pragma once
 
 #include "common.cuh"
+#include "sm100.cuh"
 
 namespace dash {
 
 // Power sums of one pass over (part of) a row at the current shifted threshold u.
 struct EntmaxPass {
     float z0, z1, z2, fe, de, minz;
-    __device__ __forceinline__ void reset() { z0 = z1 = z2 = fe = de = 0.f; minz = INFINITY; }
+    unsigned mb;                                   // add_sat: least bits(z) - 1 over the values
+    __device__ __forceinline__ void reset() { z0 = z1 = z2 = fe = de = 0.f; minz = INFINITY; mb = 0xFFFFFFFFu; }
+    // Saturating form of add_t for alpha = 1.5 (MODE 1) and alpha = 2 (MODE 2), taking
+    // y = x - m <= 0 and u >= -1: z = y - u is at most -u <= 1, so [z]_+ is the saturated
+    // difference, one instruction, rounded exactly as y - u.  The count of positive z is
+    // sat(sat(z+ 2^127) 2^127), exactly 1 for every positive fp32 (denormals included), and
+    // the least positive z comes from an unsigned minimum of bits(z+) - 1, in which z+ = 0
+    // wraps to the largest value.  The sums equal add_t's, with fewer compare and select
+    // instructions.
+    template <int MODE>
+    __device__ __forceinline__ void add_sat(float y, float u) {
+        static_assert(MODE == 1 || MODE == 2, "closed-form modes only");
+        float zp, t, cnt;
+        asm("sub.sat.f32 %0, %1, %2;" : "=f"(zp) : "f"(y), "f"(u));
+        asm("mul.sat.f32 %0, %1, 0f7F000000;" : "=f"(t) : "f"(zp));
+        asm("mul.sat.f32 %0, %1, 0f7F000000;" : "=f"(cnt) : "f"(t));
+        z0 += cnt;
+        z1 += zp;
+        if constexpr (MODE == 1) z2 = fmaf(zp, zp, z2);
+        mb = min(mb, __float_as_uint(zp) - 1u);
+    }
+    // after add_sat: the least positive z into minz
+    __device__ __forceinline__ void seal() {
+        if (mb != 0xFFFFFFFFu) minz = fminf(minz, __uint_as_float(mb + 1u));
+    }
     // z = y - u for one value (mode 0 = general alpha needs the powers)
     __device__ __forceinline__ void add(float z, int mode, float e) {
         if (z > 0.f) {
@@ -77,6 +102,49 @@ struct EntmaxPass {
     __device__ __forceinline__ void warp_reduce() {
         z0 = warp_sum(z0); z1 = warp_sum(z1); z2 = warp_sum(z2);
         fe = warp_sum(fe); de = warp_sum(de); minz = warp_min(minz);
+    }
+};
+
+// Pairs of values through add_sat's steps with f32x2 arithmetic for the shift x - m and the
+// three sums (f32x2 has no saturating forms: [z]_+ and the count stay scalar).  Each sum is
+// kept in two lanes, added in finish(), so its order of additions differs from add_t's.  The
+// count takes one saturating multiply, sat(z 2^127), which is exactly 1 for every positive z
+// that occurs: the largest weight (-u*)^e is at least 1 / n for n blocks, every iterate stays
+// at or below u* / 2 (Newton from below, bisection midpoints), so |u| >= (1/n)^(alpha-1) / 2
+// (above 2^-16 for n <= 2^14), and z = y - u > 0 with y in (u, 0] is at least one unit in the
+// last place of u, far above 2^-127.
+struct EntmaxPassX2 {
+    uint64_t s0, s1, s2;                           // (lane a, lane b): count, sum z, sum z^2
+    unsigned mb;
+    __device__ __forceinline__ void reset() { s0 = s1 = s2 = 0ull; mb = 0xFFFFFFFFu; }
+    // x2 = (x_a, x_b), nm2 = (-m, -m)
+    template <int MODE>
+    __device__ __forceinline__ void add2(uint64_t x2, uint64_t nm2, float u) {
+        static_assert(MODE == 1 || MODE == 2, "closed-form modes only");
+        using namespace sm100;
+        float ya, yb, za, zb, ca, cb;
+        f2_unpack(f2_add(x2, nm2), ya, yb);
+        asm("sub.sat.f32 %0, %1, %2;" : "=f"(za) : "f"(ya), "f"(u));
+        asm("sub.sat.f32 %0, %1, %2;" : "=f"(zb) : "f"(yb), "f"(u));
+        asm("mul.sat.f32 %0, %1, 0f7F000000;" : "=f"(ca) : "f"(za));
+        asm("mul.sat.f32 %0, %1, 0f7F000000;" : "=f"(cb) : "f"(zb));
+        const uint64_t z2 = f2_pack(__float_as_uint(za), __float_as_uint(zb));
+        s0 = f2_add(s0, f2_pack(__float_as_uint(ca), __float_as_uint(cb)));
+        s1 = f2_add(s1, z2);
+        if constexpr (MODE == 1) s2 = f2_fma(z2, z2, s2);
+        mb = min(mb, min(__float_as_uint(za) - 1u, __float_as_uint(zb) - 1u));
+    }
+    __device__ __forceinline__ EntmaxPass finish() const {
+        using namespace sm100;
+        EntmaxPass p;
+        p.reset();
+        float a, b;
+        f2_unpack(s0, a, b); p.z0 = a + b;
+        f2_unpack(s1, a, b); p.z1 = a + b;
+        f2_unpack(s2, a, b); p.z2 = a + b;
+        p.mb = mb;
+        p.seal();
+        return p;
     }
 };
 
