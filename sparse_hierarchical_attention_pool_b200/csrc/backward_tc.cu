@@ -487,11 +487,14 @@ bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     auto do_addr = [&](int st) { return base + L::off_ring + (uint32_t)st * L::kStage + L::kT; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int BH = g.B * g.Hkv;
-    const int jp = blockIdx.x / BH;            // low pairs (listed by the most tiles) first
-    const int bg = blockIdx.x % BH;
-    const int b = bg / g.Hkv, kvh = bg % g.Hkv;
+    // group-major order: the CTAs in flight share one KV group, whose Q and dout tiles stay
+    // in L2 while its pairs re-read them; within a group, low pairs (listed by the most
+    // tiles) first
     const int nb = (g.T + kBlock - 1) / kBlock;
+    const int npairs = (nb + 1) / 2;
+    const int bg = blockIdx.x / npairs;
+    const int jp = blockIdx.x % npairs;
+    const int b = bg / g.Hkv, kvh = bg % g.Hkv;
     const int j0 = 2 * jp, j1 = 2 * jp + 1;
     const bool has1 = j1 < nb;
 
