@@ -31,7 +31,10 @@
 namespace dash {
 
 constexpr int kOrdThreads = 512;
-constexpr int kOrdItems = kOrderRows / kOrdThreads;
+constexpr int kOrdItems = kOrderRows / kOrdThreads;   // rows per thread (scoring) and sort items
+constexpr int kTabWords = 16;                           // bitmap words per chunk of lookup tables
+constexpr int kKeyBits = 12;                            // sort key: the score's leading 12 bits
+constexpr int kSortRadix = 6;                           // radix bits per sort pass
 
 // Bit mask of the valid blocks of word w of a row with bt complete past blocks.
 __device__ __forceinline__ unsigned row_word_mask(int w, int bt) {
@@ -39,17 +42,23 @@ __device__ __forceinline__ unsigned row_word_mask(int w, int bt) {
     return rem >= 32 ? 0xFFFFFFFFu : (rem <= 0 ? 0u : ((1u << rem) - 1u));
 }
 
+// bytes of the block sort's storage, rounded up to 16
+__host__ __device__ constexpr int order_sort_bytes() {
+    return (int)((sizeof(typename cub::BlockRadixSort<unsigned, kOrdThreads, kOrdItems, int, kSortRadix>::TempStorage) + 15) / 16 * 16);
+}
+
 __global__ void __launch_bounds__(kOrdThreads, 1)
 order_rows_kernel(const unsigned* __restrict__ rowbits, const unsigned* __restrict__ wcnt, int* __restrict__ ord_rows,
                   PrefillGeom g) {
-    using Sort = cub::BlockRadixSort<unsigned, kOrdThreads, kOrdItems, int>;
-    extern __shared__ unsigned dyn[];                   // [kOrderRows] row scores, then [nbw * 32] counts
-    unsigned* const score = dyn;
-    unsigned* const cnt = dyn + kOrderRows;
-    __shared__ union {
-        typename Sort::TempStorage sort_tmp;
-        int sorted[kOrderRows];                         // window row by rank (after the sort)
-    } sh;
+    using Sort = cub::BlockRadixSort<unsigned, kOrdThreads, kOrdItems, int, kSortRadix>;
+    // dynamic: the sort's storage, [kOrderRows] row scores (then the window's rows by rank),
+    // [kTabWords][4][256] tables, [nbw * 32] block counts
+    extern __shared__ __align__(16) unsigned char dyn_raw[];
+    typename Sort::TempStorage& sort_tmp = *reinterpret_cast<typename Sort::TempStorage*>(dyn_raw);
+    unsigned* const score = reinterpret_cast<unsigned*>(dyn_raw + order_sort_bytes());
+    int* const sorted = reinterpret_cast<int*>(score);
+    unsigned short* const tab = reinterpret_cast<unsigned short*>(score + kOrderRows);
+    unsigned* const cnt = reinterpret_cast<unsigned*>(tab + kTabWords * 1024);
     __shared__ unsigned smax_sh;
 
     const int nwin = (g.T + g.W - 1) / g.W;
@@ -57,7 +66,7 @@ order_rows_kernel(const unsigned* __restrict__ rowbits, const unsigned* __restri
     const int b = bg / g.Hkv, kvh = bg % g.Hkv;
     const int p0 = win * g.W, np = min(g.W, g.T - p0); // positions of the window
     const int R = np * g.G;                             // rows: ri = hl * np + (t - p0)
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x, lane = tid & 31;
     const size_t row0 = (size_t)(b * g.Hq + kvh * g.G) * g.T;
 
     const int nbt = (p0 + np - 1) / kBlock + 1;         // blocks 0 .. nbt-1 (own blocks included)
@@ -66,56 +75,88 @@ order_rows_kernel(const unsigned* __restrict__ rowbits, const unsigned* __restri
     const unsigned* wc = wcnt + ((size_t)bg * nwin + win) * g.nbs;
     for (int i = tid; i < nwm * 32; i += kOrdThreads) cnt[i] = i < g.nbs ? wc[i] : 0u;
     if (tid == 0) smax_sh = 0u;
-    __syncthreads();
-    // ---- signature score_r = sum of the counts of the row's selected blocks: a thread per
-    // row (ri = hl np + pl), the row's bitmap words loaded 8 at a time (independent loads)
-    unsigned my_max = 0u;
-    for (int hl = 0; hl < g.G; ++hl)
-        for (int pl = tid; pl < np; pl += kOrdThreads) {
-            const int t = p0 + pl, bt = t / kBlock, nw = (bt + 31) / 32;
-            const unsigned* rb = rowbits + (row0 + (size_t)hl * g.T + t) * g.nbw;
-            unsigned sc = 0u;
-            for (int w0 = 0; w0 < nw; w0 += 8) {
-                unsigned wv[8];
+    // this thread's rows ri = tid + 512 k: (head in group, position), one division each
+    int rh[kOrdItems], rt[kOrdItems];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) wv[k] = w0 + k < nw ? rb[w0 + k] & row_word_mask(w0 + k, bt) : 0u;
+    for (int k = 0; k < kOrdItems; ++k) {
+        const int ri = tid + k * kOrdThreads;
+        rh[k] = ri < R ? ri / np : -1;
+        rt[k] = ri < R ? p0 + ri - rh[k] * np : 0;
+    }
+    // ---- signature score_r = sum of the counts of the row's selected blocks, through tables
+    // of 256 entries per bitmap byte (entry v = the sum of the counts of the byte's set bits;
+    // at most 8 x 4096, so 16 bits): four lookups per 32-block word, in chunks of kTabWords
+    // words whose tables are rebuilt per chunk
+    unsigned sc[kOrdItems];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    unsigned word = wv[k];
-                    while (word) {
-                        sc += cnt[(w0 + k) * 32 + __ffs(word) - 1];
-                        word &= word - 1u;
-                    }
-                }
+    for (int k = 0; k < kOrdItems; ++k) sc[k] = 0u;
+    for (int w0 = 0; w0 < nwm; w0 += kTabWords) {
+        const int nwc = min(kTabWords, nwm - w0);
+        __syncthreads();                                // counts loaded; previous tables read
+        for (int e = tid; e < nwc * 1024; e += kOrdThreads) {
+            const unsigned* cc = cnt + 32 * (w0 + (e >> 10)) + 8 * ((e >> 8) & 3);
+            const unsigned v = e & 255u;
+            unsigned sum = 0u;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sum += ((v >> i) & 1u) ? cc[i] : 0u;
+            tab[e] = (unsigned short)sum;
+        }
+        __syncthreads();
+#pragma unroll 1
+        for (int k = 0; k < kOrdItems; ++k) {
+            if (rh[k] < 0) continue;
+            const int t = rt[k], bt = t / kBlock, nwr = (bt + 31) / 32;
+            const unsigned* rb = rowbits + (row0 + (size_t)rh[k] * g.T + t) * g.nbw;
+            unsigned wv[kTabWords];
+#pragma unroll
+            for (int w = 0; w < kTabWords; ++w)         // independent loads in flight
+                wv[w] = (w < nwc && w0 + w < nwr) ? rb[w0 + w] & row_word_mask(w0 + w, bt) : 0u;
+            unsigned s = 0u;
+#pragma unroll
+            for (int w = 0; w < kTabWords; ++w) {
+                if (w >= nwc) break;
+                const unsigned short* tw = tab + w * 1024;
+                s += tw[wv[w] & 255u] + tw[256 + ((wv[w] >> 8) & 255u)] + tw[512 + ((wv[w] >> 16) & 255u)]
+                   + tw[768 + (wv[w] >> 24)];
             }
-            score[hl * np + pl] = sc;
-            my_max = max(my_max, sc);
+            sc[k] += s;
+        }
+    }
+    unsigned my_max = 0u;
+#pragma unroll
+    for (int k = 0; k < kOrdItems; ++k)
+        if (rh[k] >= 0) {
+            score[tid + k * kOrdThreads] = sc[k];
+            my_max = max(my_max, sc[k]);
         }
     my_max = __reduce_max_sync(0xffffffffu, my_max);
     if (lane == 0) atomicMax(&smax_sh, my_max);
     __syncthreads();
-    // ---- stable sort on the bits the scores use (blocked arrangement: thread i holds ranks
-    // 8 i .. 8 i + 7); padding rows (past R) get the largest key and sort last
-    const int nbits = 33 - __clz((int)(smax_sh | 1u));  // bits of max(score) + 1
-    const unsigned pad = nbits >= 32 ? 0xFFFFFFFFu : (1u << nbits) - 1u;
+    // ---- stable sort on the score's leading kKeyBits bits (rows of nearly equal score keep
+    // their window order; blocked arrangement: thread i holds ranks 8 i .. 8 i + 7); padding
+    // rows (past R) take the largest key and, being last, sort after every row
+    const int nbits = 32 - __clz((int)(smax_sh | 1u));  // bits of max(score)
+    const int shift = nbits > kKeyBits ? nbits - kKeyBits : 0;
+    const int kbits = nbits - shift;                     // <= kKeyBits
+    const unsigned pad = (1u << kbits) - 1u;
     // values: the row ids of the ordered-tile lists, (head in group << 20) | position
     unsigned keys[kOrdItems];
     int vals[kOrdItems];
 #pragma unroll
     for (int k = 0; k < kOrdItems; ++k) {
         const int ri = tid * kOrdItems + k;
-        const int hl = ri / np;                         // R <= 4096 rows: one division per item
-        keys[k] = ri < R ? score[ri] : pad;
+        const int hl = ri / np;                         // one division per item
+        keys[k] = ri < R ? score[ri] >> shift : pad;
         vals[k] = ri < R ? (hl << kRowShift) | (p0 + ri - hl * np) : -1;
     }
-    Sort(sh.sort_tmp).Sort(keys, vals, 0, nbits > 32 ? 32 : nbits);
-    __syncthreads();                                    // the sort's storage is reused below
+    Sort(sort_tmp).Sort(keys, vals, 0, kbits);
+    // the scores were read into keys before the sort: their space takes the sorted rows
 #pragma unroll
-    for (int k = 0; k < kOrdItems; ++k) sh.sorted[tid * kOrdItems + k] = vals[k];
+    for (int k = 0; k < kOrdItems; ++k) sorted[tid * kOrdItems + k] = vals[k];
     __syncthreads();
     const int ntw = (R + kTileRows - 1) / kTileRows;
     const size_t tile0 = (size_t)bg * g.ord_bg + (size_t)win * g.ord_tw;
-    for (int i = tid; i < ntw * kTileRows; i += kOrdThreads) ord_rows[tile0 * kTileRows + i] = i < R ? sh.sorted[i] : -1;
+    for (int i = tid; i < ntw * kTileRows; i += kOrdThreads) ord_rows[tile0 * kTileRows + i] = i < R ? sorted[i] : -1;
 }
 
 // One warp per ordered tile: the union of its rows' selected blocks and own blocks.  Lanes
@@ -189,7 +230,8 @@ cudaError_t launch_order_tiles(const PrefillGeom& g, char* ws, cudaStream_t stre
     const int nwin = (g.T + g.W - 1) / g.W;
     const unsigned* rowbits = reinterpret_cast<const unsigned*>(ws + g.off_rowbits);
     int* ord_rows = reinterpret_cast<int*>(ws + g.off_ord_rows);
-    const int sm = (kOrderRows + g.nbw * 32) * (int)sizeof(unsigned);
+    const int sm = order_sort_bytes() + (kOrderRows + g.nbw * 32) * (int)sizeof(unsigned) +
+                   kTabWords * 1024 * (int)sizeof(unsigned short);
     cudaError_t e = cudaFuncSetAttribute(order_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
     if (e != cudaSuccess) return e;
     order_rows_kernel<<<g.B * g.Hkv * nwin, kOrdThreads, sm, stream>>>(
