@@ -33,7 +33,7 @@ namespace dash {
 constexpr int kOrdThreads = 512;
 constexpr int kOrdItems = kOrderRows / kOrdThreads;   // rows per thread (scoring) and sort items
 constexpr int kTabWords = 16;                           // bitmap words per chunk of lookup tables
-constexpr int kKeyBits = 12;                            // sort key: the score's leading 12 bits
+constexpr int kKeyBits = 18;                            // sort key: the score's leading 18 bits
 constexpr int kSortRadix = 6;                           // radix bits per sort pass
 
 // Bit mask of the valid blocks of word w of a row with bt complete past blocks.
