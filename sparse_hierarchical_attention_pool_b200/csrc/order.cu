@@ -169,8 +169,8 @@ order_union_kernel(const unsigned* __restrict__ rowbits, const int* __restrict__
                    int* __restrict__ ord_count, WsHeader* __restrict__ hdr, PrefillGeom g) {
     __shared__ int bt_sh[kUnionWarps][kTileRows];                    // own block, -1: no row
     __shared__ const unsigned* rb_sh[kUnionWarps][kTileRows];         // the row's bitmap
-    const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
-    const int tile = blockIdx.x * kUnionWarps + wl;
+    const int lane = threadIdx.x & 31, wl_ = threadIdx.x >> 5;
+    const int tile = blockIdx.x * kUnionWarps + wl_;
     if (tile >= g.ord_ntiles) return;                   // whole warp
     const int bg = tile / g.ord_bg;
     const int b = bg / g.Hkv, kvh = bg % g.Hkv;
@@ -180,8 +180,8 @@ order_union_kernel(const unsigned* __restrict__ rowbits, const int* __restrict__
         const int rid = ord_rows[(size_t)tile * kTileRows + k];
         const int t = rid & kRowMask, hl = rid >> kRowShift;
         const int bt = rid >= 0 ? t / kBlock : -1;
-        bt_sh[wl][k] = bt;
-        rb_sh[wl][k] = rowbits + (row0 + (rid >= 0 ? (size_t)hl * g.T + t : 0)) * g.nbw;
+        bt_sh[wl_][k] = bt;
+        rb_sh[wl_][k] = rowbits + (row0 + (rid >= 0 ? (size_t)hl * g.T + t : 0)) * g.nbw;
         btmax = max(btmax, bt);
     }
     btmax = __reduce_max_sync(0xffffffffu, btmax);
@@ -190,30 +190,42 @@ order_union_kernel(const unsigned* __restrict__ rowbits, const int* __restrict__
     int* dst = ord_list + (size_t)tile * g.ord_cap;
     int total = 0;
     for (int wb = 0; wb < nwt; wb += 32) {
-        const int w = wb + lane;
+        // lanes = (row offset, word): nwp lanes (a power of two >= the chunk's words) per row,
+        // 32 / nwp rows per load, 8 loads in flight; an OR over the row offsets follows
+        const int nww = min(32, nwt - wb);
+        const int nwp = nww <= 1 ? 1 : 1 << (32 - __clz(nww - 1));
+        const int rpl = 32 / nwp;
+        const int wl = lane & (nwp - 1), ro = lane / nwp;
+        const int w = wb + wl;
+        const bool wok = wl < nww;
         unsigned word = 0u;
-        for (int k0 = 0; k0 < kTileRows; k0 += 8) {
+        for (int k0 = 0; k0 < kTileRows; k0 += 8 * rpl) {
             unsigned wv[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) {                   // 8 independent loads in flight
-                const int bt = bt_sh[wl][k0 + k];
-                wv[k] = (bt >= 0 && w * 32 < bt) ? rb_sh[wl][k0 + k][w] & row_word_mask(w, bt) : 0u;
-                if (bt >= 0 && (bt >> 5) == w) wv[k] |= 1u << (bt & 31);   // own block
+                const int row = k0 + k * rpl + ro;
+                const int bt = row < kTileRows ? bt_sh[wl_][row] : -1;
+                wv[k] = (wok && bt >= 0 && w * 32 < bt) ? rb_sh[wl_][row][w] & row_word_mask(w, bt) : 0u;
+                if (wok && bt >= 0 && (bt >> 5) == w) wv[k] |= 1u << (bt & 31);   // own block
             }
 #pragma unroll
             for (int k = 0; k < 8; ++k) word |= wv[k];
         }
-        const int pc = __popc(word);
+        for (int o = nwp; o < 32; o <<= 1) word |= __shfl_xor_sync(0xffffffffu, word, o);
+        // lanes 0 .. nww-1 hold words wb .. wb + nww - 1
+        const int pc = lane < nww ? __popc(word) : 0;
         int incl = pc;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int nn = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += nn;
         }
-        int pos = total + incl - pc;
-        while (word) {
-            dst[pos++] = w * 32 + __ffs(word) - 1;
-            word &= word - 1u;
+        if (lane < nww) {
+            int pos = total + incl - pc;
+            while (word) {
+                dst[pos++] = (wb + lane) * 32 + __ffs(word) - 1;
+                word &= word - 1u;
+            }
         }
         total += __shfl_sync(0xffffffffu, incl, 31);
     }
