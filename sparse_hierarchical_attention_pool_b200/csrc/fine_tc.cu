@@ -140,7 +140,15 @@ struct TcLayout {
     // TMEM columns: S of group 0 and 1, O of group 0 and 1, row sums of group 0 and 1
     static constexpr uint32_t colS = 96;                        // S buffer of group g at g * 96 (80 used)
     static constexpr uint32_t colO = 192;
-    static constexpr uint32_t colL = 192 + 2 * D;
+    static constexpr uint32_t colL = 192 + 2 * D;               // row sums of group g at + g * 32 (16 used)
+    // Selection-ordered tiles keep Q in TMEM as the A operand of S (the tensor core then reads
+    // only K from shared memory): K step kk (8 columns) in the unused 16-column gaps after
+    // the S buffers and the row sums
+    __host__ __device__ static constexpr uint32_t colQ(int kk) {
+        return ((kk >> 1) == 0 ? 80u : (kk >> 1) == 1 ? 176u : (kk >> 1) == 2 ? 464u : 496u) + (uint32_t)(kk & 1) * 8u;
+    }
+    static_assert(kKRows <= 80 && colO >= 192 && colL + 32 + 16 <= 496, "Q gaps of TMEM");
+    static_assert(D == 64 || colL == 448, "the last two Q gaps follow the row sums of d = 128");
 };
 constexpr uint32_t kTmemCols = 512;
 
@@ -333,9 +341,13 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const int h = kk >> 2, wk = kk & 3;
-                    const uint64_t a = smem_desc_sw128(base + L::off_q + h * L::kQHalf + wk * 32, 16, 1024);
                     const uint64_t bk = smem_desc_sw128(k_addr(st) + h * L::kKHalf + wk * 32, 16, 1024);
-                    mma_bf16_ss(tmem + sb * L::colS, a, bk, idesc_s, kk > 0 ? 1u : 0u);
+                    if constexpr (ORD) {
+                        mma_bf16_ts(tmem + sb * L::colS, tmem + L::colQ(kk), bk, idesc_s, kk > 0 ? 1u : 0u);
+                    } else {
+                        const uint64_t a = smem_desc_sw128(base + L::off_q + h * L::kQHalf + wk * 32, 16, 1024);
+                        mma_bf16_ss(tmem + sb * L::colS, a, bk, idesc_s, kk > 0 ? 1u : 0u);
+                    }
                 }
                 mma_commit(bar(B_S_FULL + sb));
                 mma_commit(bar(B_K_EMPTY + st));
@@ -397,19 +409,24 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int tpos = valid ? t : -1;
         const int bt_r = ORD ? t / kBlock : bt;             // the row's own block
         const float tau_r = (valid && bt_r > 0) ? tau[(size_t)(b * g.Hq + kvh * g.G + hl) * g.T + t] : INFINITY;
+        const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
         if constexpr (ORD) {
-            // this tile's rows of Q, 128-byte swizzled as the TMA would write them (zeros for
-            // rows the tile does not fill)
+            // this tile's rows of Q into TMEM, the A operand of S (row r in lane r; zeros for
+            // rows the tile does not fill): 16 columns (two K steps, 32 elements) per store
             if (grp == 0 && sp == 0) {
                 const uint4* src = reinterpret_cast<const uint4*>(qrows + ((size_t)(b * g.Hq + kvh * g.G + hl) * g.T + t) * D);
 #pragma unroll
-                for (int h = 0; h < D / 64; ++h)
+                for (int f = 0; f < D / 32; ++f) {
+                    uint32_t w16[16];
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint4 v = valid ? src[h * 8 + c] : make_uint4(0u, 0u, 0u, 0u);
-                        *reinterpret_cast<uint4*>(base_ptr + L::off_q + h * L::kQHalf + r * 128 + ((c ^ (r & 7)) << 4)) = v;
+                    for (int c = 0; c < 4; ++c) {
+                        const uint4 v = valid ? src[f * 4 + c] : make_uint4(0u, 0u, 0u, 0u);
+                        w16[4 * c] = v.x; w16[4 * c + 1] = v.y; w16[4 * c + 2] = v.z; w16[4 * c + 3] = v.w;
                     }
-                fence_proxy_async_smem();
+                    tmem_st16(lane_addr + L::colQ(2 * f), w16);
+                }
+                tmem_wait_st();
+                tc_fence_before();
                 mbar_arrive(bar(B_Q));
             }
         }
@@ -423,7 +440,6 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
             }
         };
-        const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
         const uint32_t s_col = grp * L::colS + sp * KEYS;   // this thread's keys in its group's S buffer
         const uint32_t o_col = L::colO + grp * D + sp * RCOLS;   // O columns it rescales
         const uint32_t l_col = L::colL + grp * 32;
