@@ -182,10 +182,13 @@ DASH_API int dash_prefill_ex(const void* q, const void* k, const void* v, const 
  * for the last copy (host buffers should be pinned for the copies to overlap).
  * Host pointers: q_host, k_host, v_host (read), out_host (written).  Device pointers:
  * q_dev, k_dev, v_dev, out_dev (same shapes as dash_prefill) and the workspace.
- * The (b, kv head) groups are independent, so with B * Hkv > 1 the call pipelines them:
- * the copies of one group overlap the kernels of the previous one (two short-lived helper
- * streams).  The workspace then holds the state of the last group only (its statistics and
- * thresholds are those of a prefill with B = 1, Hq = Hq / Hkv, Hkv = 1).
+ * The rows of a query head depend only on its queries and its (b, kv head) group's keys and
+ * values, so the call pipelines units of one group and a chunk of its heads (about 8 MiB of
+ * queries each): the copies of one unit overlap the kernels of the previous one (two
+ * short-lived helper streams; a group's keys and values are copied once, with its first
+ * chunk).  With more than one unit the workspace then holds the state of the last unit only
+ * (its statistics and thresholds are those of a prefill with B = 1, Hkv = 1 and that chunk's
+ * heads).
  */
 DASH_API int dash_prefill_host(const void* q_host, const void* k_host, const void* v_host, void* out_host,
                       void* q_dev, void* k_dev, void* v_dev, void* out_dev,

@@ -3,6 +3,7 @@
 // Argument checks happen here, before any launch; kernels live in summary.cu, coarse.cu,
 // coarse_tc.cu, fine_mma.cu, fine_tc.cu, backward.cu, decode.cu, decode_tc.cu and dump.cu.
 // Nothing here allocates memory.
+#include <algorithm>
 #include <math.h>
 
 #include <new>
@@ -232,18 +233,25 @@ int dash_prefill_host(const void* q_host, const void* k_host, const void* v_host
     if (!good_params(alpha, coarse_scale)) return DASH_ERR_ARG;
     if (!workspace || !al256(workspace) || ws_bytes < g.total) return DASH_ERR_WORKSPACE;
     cudaStream_t s = S(stream);
-    // The (b, kv head) groups are independent prefills on contiguous slices of q, k, v and
-    // out, so the copies of one group overlap the kernels of another: copies in on one
-    // helper stream, the groups' kernels in order on `stream` (sharing the workspace),
-    // copies out on a second helper stream; `stream` finally waits for the last copy out.
+    // The rows of one query head depend only on that head's queries and its KV group's keys and
+    // values, so any set of heads of one (b, kv head) group is an independent prefill on
+    // contiguous slices of q, k, v and out.  The work is cut into units of one group and a chunk
+    // of its heads (about 8 MiB of queries each), so the copies of one unit overlap the kernels
+    // of another: copies in on one helper stream (a group's keys and values with its first
+    // chunk), the units' kernels in order on `stream` (sharing the workspace), copies out on a
+    // second helper stream; `stream` finally waits for the last copy out.
     const int ng = B * Hkv, G = Hq / Hkv;
-    const size_t qg = (size_t)G * T * d * 2, kg = (size_t)T * d * 2;    // bytes per group
+    const size_t hb = (size_t)T * d * 2;                                   // bytes per head
+    const size_t qg = (size_t)G * hb, kg = hb;                             // bytes per group
+    const int gc = (int)std::min<size_t>((size_t)G, std::max<size_t>(1, ((size_t)8 << 20) / std::max<size_t>(hb, 1)));
+    const int nch = (G + gc - 1) / gc;                                     // head chunks per group
+    const int nu = ng * nch;                                               // units
     auto cp = [](void* dst, const void* src, size_t n, cudaMemcpyKind kind, cudaStream_t st) {
         return cudaMemcpyAsync(dst, src, n, kind, st) == cudaSuccess;
     };
     auto at = [](const void* p, size_t off) { return static_cast<const char*>(p) + off; };
     auto atw = [](void* p, size_t off) { return static_cast<char*>(p) + off; };
-    if (ng == 1) {
+    if (nu == 1) {
         if (!cp(k_dev, k_host, kg, cudaMemcpyHostToDevice, s) || !cp(v_dev, v_host, kg, cudaMemcpyHostToDevice, s) ||
             !cp(q_dev, q_host, qg, cudaMemcpyHostToDevice, s))
             return DASH_ERR_CUDA;
@@ -254,39 +262,40 @@ int dash_prefill_host(const void* q_host, const void* k_host, const void* v_host
     }
     cudaStream_t sin = nullptr, sout = nullptr;
     cudaEvent_t start = nullptr, fin = nullptr;
-    cudaEvent_t* ev = new (std::nothrow) cudaEvent_t[2 * (size_t)ng]();
+    cudaEvent_t* ev = new (std::nothrow) cudaEvent_t[2 * (size_t)nu]();
     int rc = DASH_OK;
     auto mkev = [](cudaEvent_t* e) { return cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess; };
     if (!ev || cudaStreamCreateWithFlags(&sin, cudaStreamNonBlocking) != cudaSuccess ||
         cudaStreamCreateWithFlags(&sout, cudaStreamNonBlocking) != cudaSuccess || !mkev(&start) || !mkev(&fin))
         rc = DASH_ERR_CUDA;
-    for (int i = 0; rc == DASH_OK && i < 2 * ng; ++i)
+    for (int i = 0; rc == DASH_OK && i < 2 * nu; ++i)
         if (!mkev(&ev[i])) rc = DASH_ERR_CUDA;
     // the helper streams start after the work already queued on `stream`
     if (rc == DASH_OK && (cudaEventRecord(start, s) != cudaSuccess || cudaStreamWaitEvent(sin, start, 0) != cudaSuccess ||
                           cudaStreamWaitEvent(sout, start, 0) != cudaSuccess))
         rc = DASH_ERR_CUDA;
-    for (int gi = 0; rc == DASH_OK && gi < ng; ++gi) {
-        const size_t oq = (size_t)gi * qg, ok = (size_t)gi * kg;
-        if (!cp(atw(k_dev, ok), at(k_host, ok), kg, cudaMemcpyHostToDevice, sin) ||
-            !cp(atw(v_dev, ok), at(v_host, ok), kg, cudaMemcpyHostToDevice, sin) ||
-            !cp(atw(q_dev, oq), at(q_host, oq), qg, cudaMemcpyHostToDevice, sin) ||
-            cudaEventRecord(ev[2 * gi], sin) != cudaSuccess || cudaStreamWaitEvent(s, ev[2 * gi], 0) != cudaSuccess) {
+    for (int u = 0; rc == DASH_OK && u < nu; ++u) {
+        const int gi = u / nch, c = u % nch, h0 = c * gc, hc = std::min(gc, G - h0);
+        const size_t ok = (size_t)gi * kg, oq = (size_t)gi * qg + (size_t)h0 * hb, nq = (size_t)hc * hb;
+        if ((c == 0 && (!cp(atw(k_dev, ok), at(k_host, ok), kg, cudaMemcpyHostToDevice, sin) ||
+                        !cp(atw(v_dev, ok), at(v_host, ok), kg, cudaMemcpyHostToDevice, sin))) ||
+            !cp(atw(q_dev, oq), at(q_host, oq), nq, cudaMemcpyHostToDevice, sin) ||
+            cudaEventRecord(ev[2 * u], sin) != cudaSuccess || cudaStreamWaitEvent(s, ev[2 * u], 0) != cudaSuccess) {
             rc = DASH_ERR_CUDA;
             break;
         }
-        rc = dash_prefill(atw(q_dev, oq), atw(k_dev, ok), atw(v_dev, ok), atw(out_dev, oq), 1, G, 1, T, d, block,
+        rc = dash_prefill(atw(q_dev, oq), atw(k_dev, ok), atw(v_dev, ok), atw(out_dev, oq), 1, hc, 1, T, d, block,
                           alpha, coarse_scale, workspace, ws_bytes, stream);
         if (rc != DASH_OK) break;
-        if (cudaEventRecord(ev[2 * gi + 1], s) != cudaSuccess || cudaStreamWaitEvent(sout, ev[2 * gi + 1], 0) != cudaSuccess ||
-            !cp(atw(out_host, oq), at(out_dev, oq), qg, cudaMemcpyDeviceToHost, sout))
+        if (cudaEventRecord(ev[2 * u + 1], s) != cudaSuccess || cudaStreamWaitEvent(sout, ev[2 * u + 1], 0) != cudaSuccess ||
+            !cp(atw(out_host, oq), at(out_dev, oq), nq, cudaMemcpyDeviceToHost, sout))
             rc = DASH_ERR_CUDA;
     }
     // `stream` waits for everything issued on the helper streams, also after an error
     if (sout && fin && cudaEventRecord(fin, sout) == cudaSuccess) cudaStreamWaitEvent(s, fin, 0);
     if (sin && start && cudaEventRecord(start, sin) == cudaSuccess) cudaStreamWaitEvent(s, start, 0);
     // destroying a stream or event with work pending releases it once the work completes
-    for (int i = 0; ev && i < 2 * ng; ++i)
+    for (int i = 0; ev && i < 2 * nu; ++i)
         if (ev[i]) cudaEventDestroy(ev[i]);
     delete[] ev;
     if (start) cudaEventDestroy(start);

@@ -136,6 +136,24 @@ def test_host_entry_point_matches_device_path():
     assert torch.equal(oh, out.cpu())
 
 
+def test_host_entry_point_head_chunks():
+    # 4 MiB of queries per head: the host entry point cuts each KV group (4 heads) into chunks
+    # of 2 heads, each its own prefill on the group's keys and values
+    wl, (q, k, v) = inputs.make("16k", Hq=8, Hkv=2)
+    cs = calibrated_scale("16k")
+    qd, kd, vd, out, ws = gpu_prefill(q, k, v, 1.5, cs)
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = torch.empty_like(q).pin_memory()
+    da.dash_prefill_host(qh, kh, vh, oh, torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd),
+                         torch.empty_like(out), 1.5, cs, ws)
+    torch.cuda.synchronize()
+    assert da.dash_get_device_status(ws) == 0
+    compare_out(oh.float().numpy(), out.float().cpu().numpy(), "host chunks against the device path")
+    rows = stratified_rows(1, 8, wl.T, 512, seed=17)
+    ref, _, _ = oracle.forward_rows(oracle.gather_q_rows(q, rows), k, v, rows, 8, 64, 1.5, cs)
+    compare_out(rows_of(oh, rows).float().numpy(), ref, "host chunks against the oracle")
+
+
 def test_stats_count_selected_pairs():
     B, Hq, Hkv, T, d = 1, 8, 2, 1000, 128
     _, (q, k, v) = inputs.make("16k", B=B, Hq=Hq, Hkv=Hkv, T=T, d=d, n_topics=16, seed=91)
