@@ -95,8 +95,13 @@ __device__ __forceinline__ TileInfo tile_info(const PrefillGeom& g, int w) {
     return ti;
 }
 
-template <int D>
-__global__ void __launch_bounds__(320, 1)
+// Tiles whose scores stay in TMEM (bt <= 512) and streamed tiles run as two instantiations:
+// STREAM = false, two threads per tile row (8 threshold warps, the first 128 scores of each in
+// registers); STREAM = true, four threads per tile row (16 threshold warps, one 32-column group
+// of every score chunk each), so that more warps cover the latency of the per-pass chains.
+// Each instantiation skips the other's tiles.
+template <int D, bool STREAM>
+__global__ void __launch_bounds__(STREAM ? 576 : 320, 1)
 coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_hi,
                  const __grid_constant__ CUtensorMap tm_lo, float* __restrict__ tau_out,
                  int* __restrict__ list, int* __restrict__ count, WsHeader* __restrict__ hdr,
@@ -104,6 +109,11 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                  unsigned* __restrict__ wcnt, int hist_init) {
     using L = CtLayout<D>;
     using namespace sm100;
+    constexpr int RT = STREAM ? 4 : 2;                  // threads per tile row
+    constexpr int kThr = 128 * RT;                      // threshold threads
+    constexpr int kThrWarps = kThr / 32;
+    constexpr int kMmaWarp = kThrWarps, kProdWarp = kThrWarps + 1;
+    constexpr int kCW = (kMaxT / kBlock / 32) / kThr;   // bitmap words per thread in the compaction
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t bars[C_COUNT];
     __shared__ uint32_t tmem_base_sh;
@@ -112,10 +122,10 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __shared__ int unconverged_sh;
     __shared__ unsigned bitmap[kMaxT / kBlock / 32];
     __shared__ unsigned long long sel_sh;
-    __shared__ float xp[2][2][6][kTileRows];     // [pass parity][half][sum][row]: partial pass sums
-    __shared__ float topv[2][kTopK][kTileRows];  // [half][rank][row]: each half-row's largest scores
-    __shared__ float gsub[2][8][kTileRows];      // [half][group][row]: maxima of the register groups
-    __shared__ int wtot_sh[8];
+    __shared__ float xp[STREAM ? 1 : 2][RT][6][kTileRows];  // [pass parity][part][sum][row]: partial pass sums
+    __shared__ float topv[RT][kTopK][kTileRows]; // [part][rank][row]: each part-row's largest scores
+    __shared__ float gsub[STREAM ? 1 : 2][8][kTileRows];    // [half][group][row]: maxima of the register groups
+    __shared__ int wtot_sh[kThrWarps];
     __shared__ float u0_sh[kTileRows];
 
     const uint32_t raw = smem_u32(smem_raw);
@@ -139,7 +149,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         for (int i = 0; i < kCtBufs; ++i) {
             mbar_init(bar(C_C_FULL + i), 1);
-            mbar_init(bar(C_C_FREE + i), 256);
+            mbar_init(bar(C_C_FREE + i), kThr);
         }
         mbar_init(bar(C_DEC), 1);
         mbar_init(bar(C_DRAIN), 1);
@@ -155,7 +165,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t tmem = tmem_base_sh;
     volatile int* abort_flag = &abort_sh;
 
-    if (warp == 9) {
+    if (warp == kProdWarp) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             prefetch_tmap(&tm_q);
@@ -166,7 +176,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             bool ok = true;
             for (int w = blockIdx.x; ok && w < g.ntiles; w += gridDim.x) {
                 const TileInfo ti = tile_info(g, w);
-                if (ti.bt == 0) continue;
+                if (ti.bt == 0 || ti.resident == STREAM) continue;
                 if (ntile > 0 && !mbar_wait(bar(C_Q_EMPTY), (ntile - 1) & 1, abort_flag)) { ok = false; break; }
                 mbar_arrive_expect_tx(bar(C_Q_FULL), (uint32_t)(g.M * D * 2));
                 for (int hl = 0; hl < g.G; ++hl) {
@@ -202,7 +212,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     if (last_armed[st] >= 0) { dummy = 0; mbar_wait(bar(C_K_FULL + st), (last_armed[st] / kCtStages) & 1, &dummy); }
             }
         }
-    } else if (warp == 8) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(128, kCtChunk, false);
@@ -211,7 +221,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             bool ok = true;
             for (int w = blockIdx.x; ok && w < g.ntiles; w += gridDim.x) {
                 const TileInfo ti = tile_info(g, w);
-                if (ti.bt == 0) continue;
+                if (ti.bt == 0 || ti.resident == STREAM) continue;
                 if (!mbar_wait(bar(C_Q_FULL), ntile & 1, abort_flag)) { ok = false; break; }
                 ++ntile;
                 while (ok) {
@@ -249,8 +259,8 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
         }
     } else {
-        // ------------------------------------------------------------ threshold warps 0-7
-        const int quarter = warp & 3, hf = warp >> 2;
+        // ------------------------------------------------------------ threshold warps
+        const int quarter = warp & 3, hf = warp >> 2;      // TMEM lane quarter, part of the row (< RT)
         const int r = quarter * 32 + lane;                  // tile row = TMEM lane
         const int st = warp * 32 + lane;                    // 0 .. 255
         const uint32_t lane_addr = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -262,7 +272,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const bool got = mbar_wait(bar_addr, parity, abort_flag);
             return __all_sync(0xffffffffu, got);
         };
-        auto sync8 = [&]() { asm volatile("bar.sync 1, 256;" ::: "memory"); };
+        auto sync8 = [&]() { asm volatile("bar.sync 1, %0;" :: "n"(kThr) : "memory"); };
         // the two warps (w, w + 4) that share a quarter of the tile rows
         auto sync_pair = [&]() { asm volatile("bar.sync %0, 64;" :: "r"(2 + quarter) : "memory"); };
         // with row bitmaps: add how many of this warp's rows select each of the nbits blocks
@@ -270,7 +280,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // histogram start: y = x - m in (-1, 0] (values at or below -1 are never selected:
         // p_max <= 1 puts tau at or above m - 1).  Integer sums: the same start on every run.
         auto hist_zero = [&]() {
-            for (int i = st; i < 3 * kHistBins * kTileRows; i += 256) (&hist[0][0][0])[i] = 0u;
+            for (int i = st; i < 3 * kHistBins * kTileRows; i += kThr) (&hist[0][0][0])[i] = 0u;
         };
         auto hist_add = [&](float y) {
             if (y > -1.0f) {
@@ -317,6 +327,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         };
         for (int w = blockIdx.x; ok && w < g.ntiles; w += gridDim.x) {
             const TileInfo ti = tile_info(g, w);
+            if (ti.resident == STREAM) continue;           // the other instantiation's tile
             const int hl = r / g.P, t = ti.t0 + r % g.P;
             const bool valid = r < g.M && t < g.T;
             const size_t tau_idx = (size_t)(ti.b * g.Hq + ti.kvh * g.G + hl) * g.T + t;
@@ -345,7 +356,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const int nw = (ti.bt + 31) / 32;
             float tau = INFINITY;
             float nsel = 0.f;
-            if (ti.resident) {
+            if constexpr (!STREAM) {
                 // ---- every chunk stays in TMEM for the whole tile.  This thread's first four
                 // 32-column groups (chunks 0 and 1: blocks below 256) are read once into
                 // registers (-inf past bt); groups of chunks 2 and 3 are read from TMEM per pass.
@@ -502,9 +513,9 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 else if (alpha == 2.0f) sweep(std::integral_constant<int, 2>{});
                 else sweep(std::integral_constant<int, 0>{});
                 // ---- union pass: OR of x > tau over the rows, per block
-                for (int i = st; i < nw; i += 256) bitmap[i] = 0u;
+                for (int i = st; i < nw; i += kThr) bitmap[i] = 0u;
                 if (rowbits)
-                    for (int i = st; i < (ti.bt + 3) / 4; i += 256) bcnt[i] = 0u;
+                    for (int i = st; i < (ti.bt + 3) / 4; i += kThr) bcnt[i] = 0u;
                 if (st == 0) sel_sh = 0ull;
                 sync8();
 #pragma unroll
@@ -553,7 +564,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         const int bf = (sweep_base + c) % kCtBufs;
                         if (!acquire(bf)) return false;
                         const int ncol = min(kCtChunk, ti.bt - c * kCtChunk);
-                        for (int g32 = hf; g32 < (ncol + 31) / 32; g32 += 2) {
+                        for (int g32 = hf; g32 < (ncol + 31) / 32; g32 += RT) {
                             uint32_t v[32];
                             tmem_ld32(lane_addr + bf * kCtChunk + g32 * 32, v);
                             tmem_wait_ld();
@@ -591,14 +602,15 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
                 for (int i = 0; i < kTopK; ++i) topv[hf][i][r] = tk[i];
                 sync8();
-                m = fmaxf(xp[0][0][0][r], xp[0][1][0][r]);
+#pragma unroll
+                for (int h = 0; h < RT; ++h) m = fmaxf(m, xp[0][h][0][r]);
                 // the pooled values are read from shared memory on every subset pass (they
                 // would otherwise take registers from the whole kernel)
                 auto ysub = [&](int i) { return topv[i / kTopK][i % kTopK][r] - m; };
                 float u0 = !valid ? -1.0f
-                         : alpha == 1.5f ? subset_start<2 * kTopK, 1>(ysub, alpha)
-                         : alpha == 2.0f ? subset_start<2 * kTopK, 2>(ysub, alpha)
-                                         : subset_start<2 * kTopK, 0>(ysub, alpha);
+                         : alpha == 1.5f ? subset_start<RT * kTopK, 1>(ysub, alpha)
+                         : alpha == 2.0f ? subset_start<RT * kTopK, 2>(ysub, alpha)
+                                         : subset_start<RT * kTopK, 0>(ysub, alpha);
                 // histogram start (alpha = 1.5 and 2): one more pass places the start at the
                 // bin edge below the root when that is higher than the subset start
                 const int hmode = !hist_init ? 0 : (alpha == 1.5f ? 1 : (alpha == 2.0f ? 2 : 0));
@@ -663,17 +675,22 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     xp[0][hf][0][r] = ps.z0; xp[0][hf][1][r] = ps.z1; xp[0][hf][2][r] = ps.z2;
                     xp[0][hf][3][r] = ps.fe; xp[0][hf][4][r] = ps.de; xp[0][hf][5][r] = ps.minz;
                     sync8();
+                    // every thread of the row merges the parts in the same order
                     EntmaxPass tot;
-                    tot.z0 = xp[0][0][0][r] + xp[0][1][0][r]; tot.z1 = xp[0][0][1][r] + xp[0][1][1][r];
-                    tot.z2 = xp[0][0][2][r] + xp[0][1][2][r]; tot.fe = xp[0][0][3][r] + xp[0][1][3][r];
-                    tot.de = xp[0][0][4][r] + xp[0][1][4][r]; tot.minz = fminf(xp[0][0][5][r], xp[0][1][5][r]);
+                    tot.z0 = xp[0][0][0][r]; tot.z1 = xp[0][0][1][r]; tot.z2 = xp[0][0][2][r];
+                    tot.fe = xp[0][0][3][r]; tot.de = xp[0][0][4][r]; tot.minz = xp[0][0][5][r];
+#pragma unroll
+                    for (int h = 1; h < RT; ++h) {
+                        tot.z0 += xp[0][h][0][r]; tot.z1 += xp[0][h][1][r]; tot.z2 += xp[0][h][2][r];
+                        tot.fe += xp[0][h][3][r]; tot.de += xp[0][h][4][r]; tot.minz = fminf(tot.minz, xp[0][h][5][r]);
+                    }
                     if (!done) done = sv.update(tot, &tau, &no_conv);
                 }
                 if (!ok) break;
                 // ---- union pass: OR of x > tau over the rows, per block
-                for (int i = st; i < nw; i += 256) bitmap[i] = 0u;
+                for (int i = st; i < nw; i += kThr) bitmap[i] = 0u;
                 if (rowbits)
-                    for (int i = st; i < (ti.bt + 3) / 4; i += 256) bcnt[i] = 0u;
+                    for (int i = st; i < (ti.bt + 3) / 4; i += kThr) bcnt[i] = 0u;
                 if (st == 0) sel_sh = 0ull;
                 sync8();
                 if (!run_pass([&](int j0, const uint32_t* v, int nv) {
@@ -700,7 +717,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (rowbits) {
                 // the tile's block counts into its ordering window's counts
                 unsigned* wc = wcnt + ((size_t)ti.bg * ((g.T + g.W - 1) / g.W) + ti.t0 / g.W) * g.nbs;
-                for (int i = st; i < (ti.bt + 3) / 4; i += 256) {
+                for (int i = st; i < (ti.bt + 3) / 4; i += kThr) {
                     const unsigned v4 = bcnt[i];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
@@ -709,7 +726,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     }
                 }
             }
-            // ---- compaction: thread st owns bitmap words 2 st and 2 st + 1; a block-wide
+            // ---- compaction: thread st owns bitmap words kCW st .. kCW st + kCW - 1; a block-wide
             // scan of their popcounts places them in the tile's ascending list.  With row
             // bitmaps the fine stage runs ordered tiles and reads no position-tile list.
             if (rowbits) {
@@ -719,11 +736,11 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     atomicAdd(&hdr->scored_pairs, (unsigned long long)rows_valid * ti.bt);
                 }
             } else {
-                unsigned wv[2];
+                unsigned wv[kCW];
                 int pc = 0;
 #pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    const int wi = 2 * st + k;
+                for (int k = 0; k < kCW; ++k) {
+                    const int wi = kCW * st + k;
                     wv[k] = wi < nw ? bitmap[wi] : 0u;
                     pc += __popc(wv[k]);
                 }
@@ -736,18 +753,18 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 if (lane == 31) wtot_sh[warp] = incl;
                 sync8();
                 int basei = 0, total = 0;
-                for (int wv8 = 0; wv8 < 8; ++wv8) {
+                for (int wv8 = 0; wv8 < kThrWarps; ++wv8) {
                     if (wv8 < warp) basei += wtot_sh[wv8];
                     total += wtot_sh[wv8];
                 }
                 int pos = basei + incl - pc;
                 int* dst = list + ti.tile_id * g.cap;
 #pragma unroll
-                for (int k = 0; k < 2; ++k) {
+                for (int k = 0; k < kCW; ++k) {
                     unsigned word = wv[k];
                     while (word) {
                         const int bit = __ffs(word) - 1;
-                        dst[pos++] = (2 * st + k) * 32 + bit;
+                        dst[pos++] = (kCW * st + k) * 32 + bit;
                         word &= word - 1;
                     }
                 }
@@ -819,23 +836,26 @@ cudaError_t launch_coarse_tc(const void* q, const PrefillGeom& g, char* ws, floa
         if (e0 != cudaSuccess) return e0;
     }
     const int grid = g.ntiles < sm_count() ? g.ntiles : sm_count();
-    auto go = [&](auto kernel, int sm) -> cudaError_t {
+    auto go = [&](auto kernel, int threads, int sm) -> cudaError_t {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
         if (e != cudaSuccess) return e;
-        kernel<<<grid, 320, sm, stream>>>(tq, thi, tlo, tau, list, count, hdr, g, alpha, cx, rowbits, wcnt,
-                                          hist_init);
-        return cudaSuccess;
+        kernel<<<grid, threads, sm, stream>>>(tq, thi, tlo, tau, list, count, hdr, g, alpha, cx, rowbits, wcnt,
+                                              hist_init);
+        return cudaGetLastError();
     };
+    // streamed tiles (more than kCtBufs chunks of past blocks) exist once T exceeds 32768
+    const bool streamed = g.nbs > kCtBufs * kCtChunk;
     cudaError_t e;
     if (g.d == 128) {
         const int sm = (int)CtLayout<128>::bytes;
-        e = go(coarse_tc_kernel<128>, sm);
+        e = streamed ? go(coarse_tc_kernel<128, true>, 576, sm) : cudaSuccess;
+        if (e == cudaSuccess) e = go(coarse_tc_kernel<128, false>, 320, sm);
     } else {
         const int sm = (int)CtLayout<64>::bytes;
-        e = go(coarse_tc_kernel<64>, sm);
+        e = streamed ? go(coarse_tc_kernel<64, true>, 576, sm) : cudaSuccess;
+        if (e == cudaSuccess) e = go(coarse_tc_kernel<64, false>, 320, sm);
     }
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace dash

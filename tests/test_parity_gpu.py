@@ -154,6 +154,20 @@ def test_host_entry_point_head_chunks():
     compare_out(rows_of(oh, rows).float().numpy(), ref, "host chunks against the oracle")
 
 
+@pytest.mark.parametrize("tiles", ["ordered", "positions"])
+def test_streamed_tiles_both_tilings(tiles, monkeypatch):
+    # T = 40960: tiles past position 32768 have more than 512 past blocks, so their scores are
+    # recomputed for every threshold pass (the streamed instantiation of the coarse kernel,
+    # four threads per row), with row bitmaps (ordered tiles) or tile lists (position tiles)
+    if tiles == "positions":
+        monkeypatch.setenv("DASH_TILES", "positions")
+    T = 40960
+    _, (q, k, v) = inputs.make("16k", T=T, Hq=4, Hkv=1, n_topics=32, seed=77)
+    rows = stratified_rows(1, 4, T, 384, seed=5)
+    assert sum(t > 32768 for _, _, t in rows) >= 50
+    check_prefill(q, k, v, 1.5, calibrated_scale("16k"), rows, f"T={T}, {tiles} tiles")
+
+
 def test_stats_count_selected_pairs():
     B, Hq, Hkv, T, d = 1, 8, 2, 1000, 128
     _, (q, k, v) = inputs.make("16k", B=B, Hq=Hq, Hkv=Hkv, T=T, d=d, n_topics=16, seed=91)
