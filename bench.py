@@ -267,7 +267,7 @@ def tau_start_timings(wl, qd, kd, vd, alpha, cs, steps, warmup, flush, ws, newto
     finally:
         os.environ.pop("DASH_ENTMAX_INIT", None)
     return {"default_coarse_select_ms": newton_ms, "histogram_coarse_select_ms": r["stage_ms"]["coarse_select"],
-            "note": "default: Newton from the root of a subset (the 16 group maxima of a row whose scores stay in TMEM, the 8 largest scores of a streamed row)"}
+            "note": "default: Newton from the root of a subset (the 16 group maxima of a row whose scores stay in TMEM, the 4 largest scores of each quarter of a streamed row)"}
 
 
 def public(d):

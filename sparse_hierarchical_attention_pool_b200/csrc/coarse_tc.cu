@@ -10,31 +10,35 @@
 // computed as Q (bf16, exact) times kbar split into bf16 hi + lo parts (kbar = hi + lo to
 // 2^-17 relative), so the fp32 accumulation matches an fp32 dot product closely.
 //
-// Persistent kernel, one CTA per SM, 320 threads:
-//   warp 9 (one lane)  TMA producer: Q tile, then 128-block chunks of kbar hi and lo
+// Persistent kernel, one CTA per SM, 576 threads:
+//   warp 17 (one lane) TMA producer: Q tile, then 128-block chunks of kbar hi and lo
 //                      through a 2-stage ring;
-//   warp 8 (one lane)  MMA issuer: S_chunk = Q [hi | lo]^T (M=128, N=128, K=2d) into a
+//   warp 16 (one lane) MMA issuer: S_chunk = Q [hi | lo]^T (M=128, N=128, K=2d) into a
 //                      4-chunk TMEM ring (512 columns) whose buffers rotate across tiles,
 //                      so a short tile's scores are computed while the previous tile is
 //                      still being solved;
-//   warps 0-7          two threads per row (warps w and w+4 share TMEM lanes 32 (w%4)..
-//                      and take alternate 32-block groups; their pass sums are merged in
-//                      shared memory in a fixed order): pass 0 takes the row maximum;
-//                      then Newton / exact-support passes for tau (entmax.cuh) until every
-//                      row of the tile has its final threshold; a last pass ORs each
-//                      block's "x > tau" over the rows (warp OR-reductions into a shared
-//                      bitmap) and counts selected pairs; warp 0 compacts the bitmap into
-//                      the tile's ascending block list.
-// Tiles with bt <= 512 keep all their scores in TMEM: one GEMM pass, every further pass
-// reads TMEM (and registers).  Newton starts at a subset root (entmax.cuh): of the maxima of
-// every 16 register values (resident tiles, free in the max pass) or of the 4 largest scores
-// of each half-row (streamed tiles).  For alpha = 1.5 and 2 a pass takes z = (x - m) - u in
-// the saturating form (EntmaxPass::add_sat).  Optional histogram start (alpha = 1.5 and 2; "DashAttention: Differentiable and
-// Adaptive Sparse Hierarchical Attention", paper listing page, the AdaSplash-2 abstract): after
-// the max, one pass bins y = x - max over (-1, 0] into 16 bins with integer count, offset and
-// squared-offset sums per row; f at every bin edge follows exactly from them, and Newton starts
-// at the highest edge with f >= 1.  Longer tiles recompute their score chunks for every pass; the threshold
-// warps tell the producer and the MMA issuer after each pass whether another is needed.
+//   warps 0-15         four threads per row (warps w, w+4, w+8, w+12 share TMEM lanes
+//                      32 (w%4).. and take the 32-block groups hf = w/4 of every chunk;
+//                      their pass sums are merged in shared memory in a fixed order): pass 0
+//                      takes the row maximum; then Newton / exact-support passes for tau
+//                      (entmax.cuh) until every row of the tile has its final threshold; a
+//                      last pass marks each block's "x > tau": row selection bitmaps and
+//                      per-block counts for the ordering pass, or (position tiles) warp
+//                      OR-reductions into a shared bitmap compacted into the tile's
+//                      ascending block list.
+// Tiles with bt <= 512 keep all their scores in TMEM: one GEMM pass, every further pass reads
+// TMEM, and the four warps of a quarter iterate on their own.  Longer tiles recompute their
+// score chunks for every pass; the threshold warps tell the producer and the MMA issuer
+// after each pass whether another is needed.  Newton starts at a subset root (entmax.cuh):
+// of the maxima of every 16 scores of the first two chunks (resident tiles, free in the max
+// pass) or of the 4 largest scores of each part-row (streamed tiles).  For alpha = 1.5 and 2 a
+// pass takes value pairs in f32x2 with saturating steps (EntmaxPassX2).  Four threads per row
+// (not two) keep four warps per SM sub-partition to cover the latency of each pass's chains.
+// Optional histogram start (alpha = 1.5 and 2; "DashAttention: Differentiable and Adaptive
+// Sparse Hierarchical Attention", paper listing page, the AdaSplash-2 abstract): after the
+// max, one pass bins y = x - max over (-1, 0] into 16 bins with integer count, offset and
+// squared-offset sums per row; f at every bin edge follows exactly from them, and Newton
+// starts at the highest edge with f >= 1.
 // Every wait is bounded (~2 s); a CTA that gives up sets a status bit and exits cleanly.
 #include <string.h>
 
@@ -48,6 +52,8 @@
 namespace dash {
 
 constexpr int kCtStages = 2;
+constexpr int kCtRowThreads = 4;     // threshold threads per tile row
+constexpr int kCtThreads = 128 * kCtRowThreads + 64;   // + the MMA and TMA producer warps
 constexpr int kCtChunk = 128;        // blocks per score chunk (MMA N)
 constexpr int kCtBufs = 4;           // TMEM chunk buffers (4 x 128 columns)
 constexpr int kTopK = 4;             // largest scores per half-row kept for the threshold start
@@ -95,13 +101,8 @@ __device__ __forceinline__ TileInfo tile_info(const PrefillGeom& g, int w) {
     return ti;
 }
 
-// Tiles whose scores stay in TMEM (bt <= 512) and streamed tiles run as two instantiations:
-// STREAM = false, two threads per tile row (8 threshold warps, the first 128 scores of each in
-// registers); STREAM = true, four threads per tile row (16 threshold warps, one 32-column group
-// of every score chunk each), so that more warps cover the latency of the per-pass chains.
-// Each instantiation skips the other's tiles.
-template <int D, bool STREAM>
-__global__ void __launch_bounds__(STREAM ? 576 : 320, 1)
+template <int D>
+__global__ void __launch_bounds__(kCtThreads, 1)
 coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_hi,
                  const __grid_constant__ CUtensorMap tm_lo, float* __restrict__ tau_out,
                  int* __restrict__ list, int* __restrict__ count, WsHeader* __restrict__ hdr,
@@ -109,7 +110,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                  unsigned* __restrict__ wcnt, int hist_init) {
     using L = CtLayout<D>;
     using namespace sm100;
-    constexpr int RT = STREAM ? 4 : 2;                  // threads per tile row
+    constexpr int RT = kCtRowThreads;                   // threads per tile row
     constexpr int kThr = 128 * RT;                      // threshold threads
     constexpr int kThrWarps = kThr / 32;
     constexpr int kMmaWarp = kThrWarps, kProdWarp = kThrWarps + 1;
@@ -122,9 +123,9 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __shared__ int unconverged_sh;
     __shared__ unsigned bitmap[kMaxT / kBlock / 32];
     __shared__ unsigned long long sel_sh;
-    __shared__ float xp[STREAM ? 1 : 2][RT][6][kTileRows];  // [pass parity][part][sum][row]: partial pass sums
+    __shared__ float xp[1][RT][6][kTileRows];    // [.][part][sum][row]: partial pass sums
     __shared__ float topv[RT][kTopK][kTileRows]; // [part][rank][row]: each part-row's largest scores
-    __shared__ float gsub[STREAM ? 1 : 2][8][kTileRows];    // [half][group][row]: maxima of the register groups
+    __shared__ float gsub[RT][4][kTileRows];     // [part][group][row]: maxima of 16-score groups
     __shared__ int wtot_sh[kThrWarps];
     __shared__ float u0_sh[kTileRows];
 
@@ -176,7 +177,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             bool ok = true;
             for (int w = blockIdx.x; ok && w < g.ntiles; w += gridDim.x) {
                 const TileInfo ti = tile_info(g, w);
-                if (ti.bt == 0 || ti.resident == STREAM) continue;
+                if (ti.bt == 0) continue;
                 if (ntile > 0 && !mbar_wait(bar(C_Q_EMPTY), (ntile - 1) & 1, abort_flag)) { ok = false; break; }
                 mbar_arrive_expect_tx(bar(C_Q_FULL), (uint32_t)(g.M * D * 2));
                 for (int hl = 0; hl < g.G; ++hl) {
@@ -221,7 +222,7 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             bool ok = true;
             for (int w = blockIdx.x; ok && w < g.ntiles; w += gridDim.x) {
                 const TileInfo ti = tile_info(g, w);
-                if (ti.bt == 0 || ti.resident == STREAM) continue;
+                if (ti.bt == 0) continue;
                 if (!mbar_wait(bar(C_Q_FULL), ntile & 1, abort_flag)) { ok = false; break; }
                 ++ntile;
                 while (ok) {
@@ -273,8 +274,6 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             return __all_sync(0xffffffffu, got);
         };
         auto sync8 = [&]() { asm volatile("bar.sync 1, %0;" :: "n"(kThr) : "memory"); };
-        // the two warps (w, w + 4) that share a quarter of the tile rows
-        auto sync_pair = [&]() { asm volatile("bar.sync %0, 64;" :: "r"(2 + quarter) : "memory"); };
         // with row bitmaps: add how many of this warp's rows select each of the nbits blocks
         // starting at j0 to the tile's byte counters (at most 128 rows per tile: no carry)
         // histogram start: y = x - m in (-1, 0] (values at or below -1 are never selected:
@@ -327,7 +326,6 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         };
         for (int w = blockIdx.x; ok && w < g.ntiles; w += gridDim.x) {
             const TileInfo ti = tile_info(g, w);
-            if (ti.resident == STREAM) continue;           // the other instantiation's tile
             const int hl = r / g.P, t = ti.t0 + r % g.P;
             const bool valid = r < g.M && t < g.T;
             const size_t tau_idx = (size_t)(ti.b * g.Hq + ti.kvh * g.G + hl) * g.T + t;
@@ -356,74 +354,50 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const int nw = (ti.bt + 31) / 32;
             float tau = INFINITY;
             float nsel = 0.f;
-            if constexpr (!STREAM) {
-                // ---- every chunk stays in TMEM for the whole tile.  This thread's first four
-                // 32-column groups (chunks 0 and 1: blocks below 256) are read once into
-                // registers (-inf past bt); groups of chunks 2 and 3 are read from TMEM per pass.
+            if (ti.resident) {
+                // ---- scores in TMEM for the whole tile: every pass reads this thread's 32-column
+                // group of each chunk (g32 = hf) from TMEM; the four warps of a quarter iterate
+                // together (a named barrier per quarter)
                 sweep_base = gch;
                 gch += ti.nch;
                 bool got = true;
                 for (int c = 0; c < ti.nch && got; ++c) got = acquire((sweep_base + c) % kCtBufs);
                 if (!got) { ok = false; break; }
-                float xc[4][32];
-#pragma unroll
-                for (int kp = 0; kp < 2; ++kp) {               // two groups in flight at a time
-                    uint32_t v[2][32];
-#pragma unroll
-                    for (int kk = 0; kk < 2; ++kk) {
-                        const int k = 2 * kp + kk, c = k >> 1, g32 = hf + 2 * (k & 1);
-                        if (c < ti.nch && c * kCtChunk + g32 * 32 < ti.bt)
-                            tmem_ld32(lane_addr + ((sweep_base + c) % kCtBufs) * kCtChunk + g32 * 32, v[kk]);
-                    }
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int kk = 0; kk < 2; ++kk) {
-                        const int k = 2 * kp + kk, c = k >> 1, g32 = hf + 2 * (k & 1);
-                        const int nv = ti.bt - (c * kCtChunk + g32 * 32);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            xc[k][i] = (c < ti.nch && i < nv) ? __fmul_rn(__uint_as_float(v[kk][i]), cx) : -INFINITY;
-                    }
-                }
-                // groups past the register cache (chunks 2 and 3), 16 columns per TMEM load
-                auto tail = [&](auto&& fn) {
-                    for (int c = 2; c < ti.nch; ++c) {
-                        const int ncol = min(kCtChunk, ti.bt - c * kCtChunk);
-                        for (int g32 = hf; g32 < (ncol + 31) / 32; g32 += 2)
-                            for (int h16 = 0; h16 < 2 && g32 * 32 + h16 * 16 < ncol; ++h16) {
-                                uint32_t v[16];
-                                tmem_ld16(lane_addr + ((sweep_base + c) % kCtBufs) * kCtChunk + g32 * 32 + h16 * 16, v);
-                                tmem_wait_ld();
-                                fn(c * kCtChunk + g32 * 32 + h16 * 16, v, min(16, ncol - g32 * 32 - h16 * 16));
-                            }
+                auto sync_row = [&]() { asm volatile("bar.sync %0, %1;" :: "r"(2 + quarter), "n"(32 * RT) : "memory"); };
+                auto groups = [&](auto&& fn) {
+                    for (int c = 0; c < ti.nch; ++c) {
+                        const int j0 = c * kCtChunk + hf * 32;
+                        if (j0 >= ti.bt) continue;                      // warp-uniform
+                        uint32_t v[32];
+                        tmem_ld32(lane_addr + ((sweep_base + c) % kCtBufs) * kCtChunk + hf * 32, v);
+                        tmem_wait_ld();
+                        fn(c, j0, v, min(32, ti.bt - j0));
                     }
                 };
-                // the maximum of every 16 register values (a subset of the row for the
-                // threshold start below), then the row maximum
+                // the row maximum and the maxima of every 16 scores of the first two chunks (a
+                // subset of the row: Newton starts at its root)
                 float m = -INFINITY;
+                float gm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                groups([&](int c, int, const uint32_t* v, int nv) {
+                    float a0 = -INFINITY, a1 = -INFINITY;
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        float a = xc[k][16 * h];
-#pragma unroll
-                        for (int i = 1; i < 16; ++i) a = fmaxf(a, xc[k][16 * h + i]);
-                        gsub[hf][2 * k + h][r] = a;
-                        m = fmaxf(m, a);
+                    for (int i = 0; i < 16; ++i) {
+                        if (i < nv) a0 = fmaxf(a0, __fmul_rn(__uint_as_float(v[i]), cx));
+                        if (i + 16 < nv) a1 = fmaxf(a1, __fmul_rn(__uint_as_float(v[i + 16]), cx));
                     }
-                tail([&](int, const uint32_t* v, int nv) {
-                    for (int i = 0; i < 16; ++i)
-                        if (i < nv) m = fmaxf(m, __fmul_rn(__uint_as_float(v[i]), cx));
+                    m = fmaxf(m, fmaxf(a0, a1));
+                    if (c == 0) { gm[0] = a0; gm[1] = a1; }
+                    else if (c == 1) { gm[2] = a0; gm[3] = a1; }
                 });
+#pragma unroll
+                for (int k = 0; k < 4; ++k) gsub[hf][k][r] = gm[k];
                 xp[0][hf][0][r] = m;
-                sync_pair();
-                m = fmaxf(xp[0][0][0][r], xp[0][1][0][r]);
-                // Newton starts at the root of the subset of the 16 group maxima (at or below
-                // the row's root, entmax.cuh), or, with the histogram start (alpha = 1.5 and 2),
-                // at the bin edge below the root when that is higher
+                sync_row();
+#pragma unroll
+                for (int h = 0; h < RT; ++h) m = fmaxf(m, xp[0][h][0][r]);
                 float ys[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) ys[i] = gsub[i >> 3][i & 7][r] - m;
+                for (int i = 0; i < 16; ++i) ys[i] = gsub[i >> 2][i & 3][r] - m;
                 auto ysub = [&](int i) { return ys[i]; };
                 float u_start = !valid ? -1.0f
                               : alpha == 1.5f ? subset_start<16, 1>(ysub, alpha)
@@ -433,18 +407,11 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 if (hmode) {
                     hist_zero();
                     sync8();
-                    if (valid) {
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) hist_add(xc[k][i] - m);
-                        tail([&](int, const uint32_t* v, int nv) {
-                            for (int i = 0; i < 16; ++i)
+                    groups([&](int, int, const uint32_t* v, int nv) {   // TMEM loads are warp-collective
+                        if (valid)
+                            for (int i = 0; i < 32; ++i)
                                 if (i < nv) hist_add(__fmul_rn(__uint_as_float(v[i]), cx) - m);
-                        });
-                    } else {
-                        tail([&](int, const uint32_t*, int) {});   // TMEM loads are warp-collective
-                    }
+                    });
                     sync8();
                     hist_start(hmode);
                     sync8();
@@ -452,106 +419,70 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
                 EntmaxSolver sv;
                 bool done = !valid;
-                // ---- Newton / exact-support passes; the pair of warps iterates until all of
-                // its 32 rows are final (both warps see the same flags), partial sums are
-                // exchanged through a buffer alternating with the pass parity
                 auto sweep = [&](auto mode) {
                     constexpr int MODE = decltype(mode)::value;
                     sv.init(m, alpha, u_start, g.maxit);
-                    for (int pp = 1; __any_sync(0xffffffffu, !done); ++pp) {
+                    while (__any_sync(0xffffffffu, !done)) {   // the quarter's four warps agree
                         EntmaxPass ps;
                         ps.reset();
-                        const float mm = sv.m, uu = sv.u;
                         if constexpr (MODE == 0) {
-#pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                // groups wholly past the tile's blocks hold only -inf (warp-uniform)
-                                if ((k >> 1) * kCtChunk + (hf + 2 * (k & 1)) * 32 >= ti.bt) continue;
-#pragma unroll
-                                for (int i = 0; i < 32; ++i) ps.add_t<MODE>((xc[k][i] - mm) - uu, sv.e);
-                            }
-                            tail([&](int, const uint32_t* v, int nv) {
-                                for (int i = 0; i < 16; ++i)
-                                    if (i < nv) ps.add_t<MODE>((__fmul_rn(__uint_as_float(v[i]), cx) - mm) - uu, sv.e);
+                            groups([&](int, int, const uint32_t* v, int nv) {
+                                for (int i = 0; i < 32; ++i)
+                                    if (i < nv) ps.add_t<MODE>((__fmul_rn(__uint_as_float(v[i]), cx) - sv.m) - sv.u, sv.e);
                             });
                         } else {
-                            // pairs of values, f32x2 (EntmaxPassX2); -inf pads a group's tail
                             EntmaxPassX2 px;
                             px.reset();
-                            const uint64_t nm2 = f2_pack(__float_as_uint(-mm), __float_as_uint(-mm));
-#pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                if ((k >> 1) * kCtChunk + (hf + 2 * (k & 1)) * 32 >= ti.bt) continue;
-#pragma unroll
-                                for (int i = 0; i < 32; i += 2)
-                                    px.add2<MODE>(f2_pack(__float_as_uint(xc[k][i]), __float_as_uint(xc[k][i + 1])), nm2, uu);
-                            }
+                            const uint64_t nm2 = f2_pack(__float_as_uint(-sv.m), __float_as_uint(-sv.m));
                             const uint64_t cx2 = f2_pack(__float_as_uint(cx), __float_as_uint(cx));
-                            tail([&](int, const uint32_t* v, int nv) {
+                            groups([&](int, int, const uint32_t* v, int nv) {
 #pragma unroll
-                                for (int i = 0; i < 16; i += 2) {
+                                for (int i = 0; i < 32; i += 2) {
                                     uint64_t x2 = f2_mul(f2_pack(v[i], v[i + 1]), cx2);
                                     if (i + 1 >= nv) x2 = f2_pack(i < nv ? (uint32_t)x2 : 0xFF800000u, 0xFF800000u);
-                                    px.add2<MODE>(x2, nm2, uu);
+                                    px.add2<MODE>(x2, nm2, sv.u);
                                 }
                             });
                             ps = px.finish();
                         }
-                        float* xb = &xp[pp & 1][hf][0][0];
-                        xb[0 * kTileRows + r] = ps.z0; xb[1 * kTileRows + r] = ps.z1; xb[2 * kTileRows + r] = ps.z2;
-                        xb[3 * kTileRows + r] = ps.fe; xb[4 * kTileRows + r] = ps.de; xb[5 * kTileRows + r] = ps.minz;
-                        sync_pair();
-                        // both threads of the row merge the halves in the same order
+                        sync_row();                             // the previous sums have been read
+                        xp[0][hf][0][r] = ps.z0; xp[0][hf][1][r] = ps.z1; xp[0][hf][2][r] = ps.z2;
+                        xp[0][hf][3][r] = ps.fe; xp[0][hf][4][r] = ps.de; xp[0][hf][5][r] = ps.minz;
+                        sync_row();
+                        // every thread of the row merges the parts in the same order
                         EntmaxPass tot;
-                        tot.z0 = xp[pp & 1][0][0][r] + xp[pp & 1][1][0][r]; tot.z1 = xp[pp & 1][0][1][r] + xp[pp & 1][1][1][r];
-                        tot.z2 = xp[pp & 1][0][2][r] + xp[pp & 1][1][2][r]; tot.fe = xp[pp & 1][0][3][r] + xp[pp & 1][1][3][r];
-                        tot.de = xp[pp & 1][0][4][r] + xp[pp & 1][1][4][r]; tot.minz = fminf(xp[pp & 1][0][5][r], xp[pp & 1][1][5][r]);
+                        tot.z0 = xp[0][0][0][r]; tot.z1 = xp[0][0][1][r]; tot.z2 = xp[0][0][2][r];
+                        tot.fe = xp[0][0][3][r]; tot.de = xp[0][0][4][r]; tot.minz = xp[0][0][5][r];
+#pragma unroll
+                        for (int h = 1; h < RT; ++h) {
+                            tot.z0 += xp[0][h][0][r]; tot.z1 += xp[0][h][1][r]; tot.z2 += xp[0][h][2][r];
+                            tot.fe += xp[0][h][3][r]; tot.de += xp[0][h][4][r]; tot.minz = fminf(tot.minz, xp[0][h][5][r]);
+                        }
                         if (!done) done = sv.update(tot, &tau, &no_conv);
                     }
                 };
                 if (alpha == 1.5f) sweep(std::integral_constant<int, 1>{});
                 else if (alpha == 2.0f) sweep(std::integral_constant<int, 2>{});
                 else sweep(std::integral_constant<int, 0>{});
-                // ---- union pass: OR of x > tau over the rows, per block
+                // ---- union pass: x > tau per block
                 for (int i = st; i < nw; i += kThr) bitmap[i] = 0u;
                 if (rowbits)
                     for (int i = st; i < (ti.bt + 3) / 4; i += kThr) bcnt[i] = 0u;
                 if (st == 0) sel_sh = 0ull;
                 sync8();
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int c = k >> 1, g32 = hf + 2 * (k & 1);
-                    const int j0 = c * kCtChunk + g32 * 32;
-                    if (j0 < ti.bt) {                           // warp-uniform
-                        unsigned mask = 0u;
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (valid && xc[k][i] > tau) mask |= 1u << i;
-                        if (rowbits) {
-                            if (valid) rowbits[bits_row + (j0 >> 5)] = mask;
-                            count_blocks(j0, mask, 32);
-                        }
-                        nsel += (float)__popc(mask);
-                        if (!rowbits) {
-                            const unsigned wm = __reduce_or_sync(0xffffffffu, mask);
-                            if (lane == 0 && wm) atomicOr(&bitmap[j0 >> 5], wm);
-                        }
-                    }
-                }
-                tail([&](int j0, const uint32_t* v, int nv) {
+                groups([&](int, int j0, const uint32_t* v, int nv) {
                     unsigned mask = 0u;
-                    for (int i = 0; i < 16; ++i)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
                         if (i < nv && valid && __fmul_rn(__uint_as_float(v[i]), cx) > tau) mask |= 1u << i;
-                    // 16 blocks: the half word starting at block j0
                     if (rowbits) {
-                        if (valid)
-                            reinterpret_cast<unsigned short*>(rowbits + bits_row + (j0 >> 5))[(j0 & 31) >> 4] = (unsigned short)mask;
-                        count_blocks(j0, mask, 16);
+                        if (valid) rowbits[bits_row + (j0 >> 5)] = mask;
+                        count_blocks(j0, mask, 32);
                     }
                     nsel += (float)__popc(mask);
                     if (!rowbits) {
                         const unsigned wm = __reduce_or_sync(0xffffffffu, mask);
-                        if (lane == 0 && wm) atomicOr(&bitmap[j0 >> 5], wm << (j0 & 31));
+                        if (lane == 0 && wm) atomicOr(&bitmap[j0 >> 5], wm);
                     }
                 });
                 for (int c = 0; c < ti.nch; ++c) release((sweep_base + c) % kCtBufs);
@@ -825,8 +756,8 @@ cudaError_t launch_coarse_tc(const void* q, const PrefillGeom& g, char* ws, floa
     unsigned* rowbits = write_rowbits ? reinterpret_cast<unsigned*>(ws + g.off_rowbits) : nullptr;
     // DASH_ENTMAX_INIT=histogram starts the threshold solves at a histogram edge (AdaSplash-2's
     // initialisation); the default, Newton from a subset root (the 16 group maxima of a
-    // resident row, the 8 largest scores of a streamed one), is faster on the workloads
-    // measured here
+    // resident row, the 16 largest part-row scores of a streamed one), is faster on the
+    // workloads measured here
     const char* init = getenv("DASH_ENTMAX_INIT");
     const int hist_init = (init && strcmp(init, "histogram") == 0) ? 1 : 0;
     unsigned* wcnt = write_rowbits ? reinterpret_cast<unsigned*>(ws + g.off_wcnt) : nullptr;
@@ -836,26 +767,15 @@ cudaError_t launch_coarse_tc(const void* q, const PrefillGeom& g, char* ws, floa
         if (e0 != cudaSuccess) return e0;
     }
     const int grid = g.ntiles < sm_count() ? g.ntiles : sm_count();
-    auto go = [&](auto kernel, int threads, int sm) -> cudaError_t {
+    auto go = [&](auto kernel, int sm) -> cudaError_t {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, sm);
         if (e != cudaSuccess) return e;
-        kernel<<<grid, threads, sm, stream>>>(tq, thi, tlo, tau, list, count, hdr, g, alpha, cx, rowbits, wcnt,
-                                              hist_init);
+        kernel<<<grid, kCtThreads, sm, stream>>>(tq, thi, tlo, tau, list, count, hdr, g, alpha, cx, rowbits, wcnt,
+                                                 hist_init);
         return cudaGetLastError();
     };
-    // streamed tiles (more than kCtBufs chunks of past blocks) exist once T exceeds 32768
-    const bool streamed = g.nbs > kCtBufs * kCtChunk;
-    cudaError_t e;
-    if (g.d == 128) {
-        const int sm = (int)CtLayout<128>::bytes;
-        e = streamed ? go(coarse_tc_kernel<128, true>, 576, sm) : cudaSuccess;
-        if (e == cudaSuccess) e = go(coarse_tc_kernel<128, false>, 320, sm);
-    } else {
-        const int sm = (int)CtLayout<64>::bytes;
-        e = streamed ? go(coarse_tc_kernel<64, true>, 576, sm) : cudaSuccess;
-        if (e == cudaSuccess) e = go(coarse_tc_kernel<64, false>, 320, sm);
-    }
-    return e;
+    return g.d == 128 ? go(coarse_tc_kernel<128>, (int)CtLayout<128>::bytes)
+                      : go(coarse_tc_kernel<64>, (int)CtLayout<64>::bytes);
 }
 
 }  // namespace dash
