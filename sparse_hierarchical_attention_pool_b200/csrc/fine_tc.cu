@@ -66,30 +66,7 @@ constexpr int kVStages = 3;            // V ring
 constexpr int kPBuf = 2;               // P buffers of each softmax group (its steps take them in turn)
 constexpr int kFineSplit = 1;          // threads per tile row in each softmax group
 constexpr int kFinePolyPairs = 1;      // pairs of every 4 whose 2^x runs on the FMA pipe
-constexpr bool kFineIntPack = false;   // fp32 -> bf16 pairs with integer ops instead of cvt
-constexpr bool kFineScalar = false;    // scalar FMA / exponent per key instead of f32x2 pairs
 constexpr float kLazyRescale = 8.0f;   // log2 units: p values stay below 2^8 between rescales
-
-// Two non-negative finite fp32 values rounded to nearest-even bf16 and packed (lo in the low
-// half) with integer operations only: adding 0x7FFF plus the lowest kept bit carries into
-// the kept bits exactly when the dropped half is above one half-ulp, or equal to it with an
-// odd kept part.
-__device__ __forceinline__ uint32_t bf16x2_rne_int(float lo, float hi) {
-    uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
-    a += 0x7FFFu + ((a >> 16) & 1u);
-    b += 0x7FFFu + ((b >> 16) & 1u);
-    return __byte_perm(a, b, 0x7632);
-}
-
-// Scalar form of poly_exp2_x2 below (same steps and constants).
-__device__ __forceinline__ float poly_exp2(float x) {
-    x = fmaxf(x, -125.0f);
-    const float t = x + 12582912.0f;                  // 1.5 * 2^23: n = round(x) in the low bits
-    const float f = x - (t - 12582912.0f);
-    const float p = fmaf(fmaf(fmaf(__uint_as_float(0x3D61FBB0u), f, __uint_as_float(0x3E786F0Eu)), f,
-                              __uint_as_float(0x3F31798Du)), f, __uint_as_float(0x3F7FFB49u));
-    return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
 
 // 2^x for x <= 8 on the FMA and integer pipes.  Cody-Waite style split x = n + f with
 // n = round(x) (added to the exponent field) and f in [-1/2, 1/2], where 2^f comes from a
@@ -555,17 +532,7 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
             for (int c = 0; c < KEYS / 8; ++c) {
                 uint32_t pk[4] = {0u, 0u, 0u, 0u};
-                if (active && kFineScalar) {
-#pragma unroll
-                    for (int q2 = 0; q2 < 4; ++q2) {
-                        const float a0 = fmaf(__uint_as_float(sr[c * 8 + 2 * q2]), sm2, c0);
-                        const float a1 = fmaf(__uint_as_float(sr[c * 8 + 2 * q2 + 1]), sm2, c0);
-                        const float e0 = q2 < kFinePolyPairs ? poly_exp2(a0) : fast_exp2(a0);
-                        const float e1 = q2 < kFinePolyPairs ? poly_exp2(a1) : fast_exp2(a1);
-                        __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
-                        pk[q2] = *reinterpret_cast<uint32_t*>(&h2);
-                    }
-                } else if (active) {
+                if (active) {
 #pragma unroll
                     for (int q2 = 0; q2 < 4; ++q2) {
                         const uint64_t e2 = f2_fma(f2_pack(sr[c * 8 + 2 * q2], sr[c * 8 + 2 * q2 + 1]), sm2x2, c0x2);
@@ -577,12 +544,8 @@ fine_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             e0 = fast_exp2(e0);
                             e1 = fast_exp2(e1);
                         }
-                        if constexpr (kFineIntPack) {
-                            pk[q2] = bf16x2_rne_int(e0, e1);
-                        } else {
-                            __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
-                            pk[q2] = *reinterpret_cast<uint32_t*>(&h2);
-                        }
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(e0, e1);
+                        pk[q2] = *reinterpret_cast<uint32_t*>(&h2);
                     }
                 }
                 const int chunk = sp * (KEYS / 8) + c;
