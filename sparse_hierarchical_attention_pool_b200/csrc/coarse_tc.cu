@@ -123,9 +123,11 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __shared__ int unconverged_sh;
     __shared__ unsigned bitmap[kMaxT / kBlock / 32];
     __shared__ unsigned long long sel_sh;
-    __shared__ float xp[1][RT][6][kTileRows];    // [.][part][sum][row]: partial pass sums
-    __shared__ float topv[RT][kTopK][kTileRows]; // [part][rank][row]: each part-row's largest scores
-    __shared__ float gsub[RT][4][kTileRows];     // [part][group][row]: maxima of 16-score groups
+    __shared__ float xp[2][RT][6][kTileRows];    // [pass parity][part][sum][row]: partial pass sums
+    // [part][k][row]: the subset of the threshold start, the maxima of 16-score groups (tiles
+    // whose scores stay in TMEM) or each part-row's largest scores (streamed tiles)
+    __shared__ float subset_sh[RT][4][kTileRows];
+    static_assert(kTopK == 4, "one subset array for both starts");
     __shared__ int wtot_sh[kThrWarps];
     __shared__ float u0_sh[kTileRows];
 
@@ -390,14 +392,14 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     else if (c == 1) { gm[2] = a0; gm[3] = a1; }
                 });
 #pragma unroll
-                for (int k = 0; k < 4; ++k) gsub[hf][k][r] = gm[k];
+                for (int k = 0; k < 4; ++k) subset_sh[hf][k][r] = gm[k];
                 xp[0][hf][0][r] = m;
                 sync_row();
 #pragma unroll
                 for (int h = 0; h < RT; ++h) m = fmaxf(m, xp[0][h][0][r]);
                 float ys[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) ys[i] = gsub[i >> 2][i & 3][r] - m;
+                for (int i = 0; i < 16; ++i) ys[i] = subset_sh[i >> 2][i & 3][r] - m;
                 auto ysub = [&](int i) { return ys[i]; };
                 float u_start = !valid ? -1.0f
                               : alpha == 1.5f ? subset_start<16, 1>(ysub, alpha)
@@ -422,7 +424,11 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 auto sweep = [&](auto mode) {
                     constexpr int MODE = decltype(mode)::value;
                     sv.init(m, alpha, u_start, g.maxit);
-                    while (__any_sync(0xffffffffu, !done)) {   // the quarter's four warps agree
+                    // partial sums alternate between two buffers with the pass parity (pass 1
+                    // first: the maximum went through buffer 0), so one barrier per pass
+                    // suffices: a buffer is rewritten two passes later, after every thread of
+                    // the quarter has passed the barrier in between
+                    for (int pp = 1; __any_sync(0xffffffffu, !done); ++pp) {   // the quarter's four warps agree
                         EntmaxPass ps;
                         ps.reset();
                         if constexpr (MODE == 0) {
@@ -445,18 +451,18 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                             });
                             ps = px.finish();
                         }
-                        sync_row();                             // the previous sums have been read
-                        xp[0][hf][0][r] = ps.z0; xp[0][hf][1][r] = ps.z1; xp[0][hf][2][r] = ps.z2;
-                        xp[0][hf][3][r] = ps.fe; xp[0][hf][4][r] = ps.de; xp[0][hf][5][r] = ps.minz;
+                        float (*const xb)[6][kTileRows] = xp[pp & 1];
+                        xb[hf][0][r] = ps.z0; xb[hf][1][r] = ps.z1; xb[hf][2][r] = ps.z2;
+                        xb[hf][3][r] = ps.fe; xb[hf][4][r] = ps.de; xb[hf][5][r] = ps.minz;
                         sync_row();
                         // every thread of the row merges the parts in the same order
                         EntmaxPass tot;
-                        tot.z0 = xp[0][0][0][r]; tot.z1 = xp[0][0][1][r]; tot.z2 = xp[0][0][2][r];
-                        tot.fe = xp[0][0][3][r]; tot.de = xp[0][0][4][r]; tot.minz = xp[0][0][5][r];
+                        tot.z0 = xb[0][0][r]; tot.z1 = xb[0][1][r]; tot.z2 = xb[0][2][r];
+                        tot.fe = xb[0][3][r]; tot.de = xb[0][4][r]; tot.minz = xb[0][5][r];
 #pragma unroll
                         for (int h = 1; h < RT; ++h) {
-                            tot.z0 += xp[0][h][0][r]; tot.z1 += xp[0][h][1][r]; tot.z2 += xp[0][h][2][r];
-                            tot.fe += xp[0][h][3][r]; tot.de += xp[0][h][4][r]; tot.minz = fminf(tot.minz, xp[0][h][5][r]);
+                            tot.z0 += xb[h][0][r]; tot.z1 += xb[h][1][r]; tot.z2 += xb[h][2][r];
+                            tot.fe += xb[h][3][r]; tot.de += xb[h][4][r]; tot.minz = fminf(tot.minz, xb[h][5][r]);
                         }
                         if (!done) done = sv.update(tot, &tau, &no_conv);
                     }
@@ -531,13 +537,13 @@ coarse_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     })) { ok = false; break; }
                 xp[0][hf][0][r] = m;
 #pragma unroll
-                for (int i = 0; i < kTopK; ++i) topv[hf][i][r] = tk[i];
+                for (int i = 0; i < kTopK; ++i) subset_sh[hf][i][r] = tk[i];
                 sync8();
 #pragma unroll
                 for (int h = 0; h < RT; ++h) m = fmaxf(m, xp[0][h][0][r]);
                 // the pooled values are read from shared memory on every subset pass (they
                 // would otherwise take registers from the whole kernel)
-                auto ysub = [&](int i) { return topv[i / kTopK][i % kTopK][r] - m; };
+                auto ysub = [&](int i) { return subset_sh[i / kTopK][i % kTopK][r] - m; };
                 float u0 = !valid ? -1.0f
                          : alpha == 1.5f ? subset_start<RT * kTopK, 1>(ysub, alpha)
                          : alpha == 2.0f ? subset_start<RT * kTopK, 2>(ysub, alpha)
