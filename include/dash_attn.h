@@ -184,11 +184,13 @@ DASH_API int dash_prefill_ex(const void* q, const void* k, const void* v, const 
  * q_dev, k_dev, v_dev, out_dev (same shapes as dash_prefill) and the workspace.
  * The rows of a query head depend only on its queries and its (b, kv head) group's keys and
  * values, so the call pipelines units of one group and a chunk of its heads (about 8 MiB of
- * queries each): the copies of one unit overlap the kernels of the previous one (two
- * short-lived helper streams; a group's keys and values are copied once, with its first
- * chunk).  With more than one unit the workspace then holds the state of the last unit only
- * (its statistics and thresholds are those of a prefill with B = 1, Hkv = 1 and that chunk's
- * heads).
+ * queries each): the copies of one unit overlap the kernels of others (short-lived helper
+ * streams: copies in, copies out, and up to four compute streams, so that the kernels of
+ * several units run at once; a group's keys and values are copied once, with its first
+ * chunk).  With more than one unit each compute stream works in its own slice of the
+ * workspace (after its 256-byte header); the header then holds the OR of every unit's device
+ * status bits (dash_get_device_status) and the sums of their statistics (dash_prefill_stats),
+ * and the rest of the workspace (thresholds) is unspecified.
  */
 DASH_API int dash_prefill_host(const void* q_host, const void* k_host, const void* v_host, void* out_host,
                       void* q_dev, void* k_dev, void* v_dev, void* out_dev,

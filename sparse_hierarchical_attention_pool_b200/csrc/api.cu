@@ -222,6 +222,21 @@ int dash_prefill_profiled(const void* q, const void* k, const void* v, void* out
                         ws_bytes, stream, events);
 }
 
+namespace {
+// Adds a finished unit's header (status bits, statistics) into the header of the whole call.
+// Units on different streams may finish together: atomics.
+__global__ void accumulate_header_kernel(WsHeader* dst, const WsHeader* src) {
+    if (threadIdx.x != 0) return;
+    if (src->status) atomicOr(&dst->status, src->status);
+    atomicAdd(&dst->scored_pairs, src->scored_pairs);
+    atomicAdd(&dst->selected_pairs, src->selected_pairs);
+    atomicAdd(&dst->union_blocks, src->union_blocks);
+    atomicAdd(&dst->tiles, src->tiles);
+    atomicAdd(&dst->fine_steps, src->fine_steps);
+}
+constexpr int kHostComputeStreams = 4;   // units of a host-buffer prefill in flight at once
+}  // namespace
+
 int dash_prefill_host(const void* q_host, const void* k_host, const void* v_host, void* out_host,
                       void* q_dev, void* k_dev, void* v_dev, void* out_dev, int B, int Hq, int Hkv,
                       int T, int d, int block, float alpha, float coarse_scale, void* workspace,
@@ -237,9 +252,12 @@ int dash_prefill_host(const void* q_host, const void* k_host, const void* v_host
     // values, so any set of heads of one (b, kv head) group is an independent prefill on
     // contiguous slices of q, k, v and out.  The work is cut into units of one group and a chunk
     // of its heads (about 8 MiB of queries each), so the copies of one unit overlap the kernels
-    // of another: copies in on one helper stream (a group's keys and values with its first
-    // chunk), the units' kernels in order on `stream` (sharing the workspace), copies out on a
-    // second helper stream; `stream` finally waits for the last copy out.
+    // of others: copies in on one helper stream (a group's keys and values with its first
+    // chunk), copies out on a second.  A unit's kernels take about the same time whatever its
+    // head count (the rows at the end of the sequence, with the most blocks, set their
+    // length), so up to kHostComputeStreams units run at once, each on its own compute stream
+    // with its own slice of the workspace, and their tails overlap.  The workspace's header
+    // collects every unit's status bits and statistics; `stream` finally waits for all of it.
     const int ng = B * Hkv, G = Hq / Hkv;
     const size_t hb = (size_t)T * d * 2;                                   // bytes per head
     const size_t qg = (size_t)G * hb, kg = hb;                             // bytes per group
@@ -260,7 +278,17 @@ int dash_prefill_host(const void* q_host, const void* k_host, const void* v_host
         if (rc != DASH_OK) return rc;
         return cp(out_host, out_dev, qg, cudaMemcpyDeviceToHost, s) ? DASH_OK : DASH_ERR_CUDA;
     }
+    // a unit's workspace: the largest unit (gc heads of one group); slices after the header
+    PrefillGeom gu;
+    if (!make_prefill_geom(1, gc, 1, T, d, &gu)) return DASH_ERR_SHAPE;
+    const size_t wsu = align256(gu.total);
+    const int ns = (int)std::min<size_t>({(size_t)kHostComputeStreams, (size_t)nu,
+                                          (ws_bytes - sizeof(WsHeader)) / wsu});
+    if (ns < 1) return DASH_ERR_WORKSPACE;
+    char* const ws0 = static_cast<char*>(workspace);
+    auto unit_ws = [&](int i) { return ws0 + sizeof(WsHeader) + (size_t)i * wsu; };
     cudaStream_t sin = nullptr, sout = nullptr;
+    cudaStream_t sc[kHostComputeStreams] = {};
     cudaEvent_t start = nullptr, fin = nullptr;
     cudaEvent_t* ev = new (std::nothrow) cudaEvent_t[2 * (size_t)nu]();
     int rc = DASH_OK;
@@ -268,32 +296,46 @@ int dash_prefill_host(const void* q_host, const void* k_host, const void* v_host
     if (!ev || cudaStreamCreateWithFlags(&sin, cudaStreamNonBlocking) != cudaSuccess ||
         cudaStreamCreateWithFlags(&sout, cudaStreamNonBlocking) != cudaSuccess || !mkev(&start) || !mkev(&fin))
         rc = DASH_ERR_CUDA;
+    for (int i = 0; rc == DASH_OK && i < ns; ++i)
+        if (cudaStreamCreateWithFlags(&sc[i], cudaStreamNonBlocking) != cudaSuccess) rc = DASH_ERR_CUDA;
     for (int i = 0; rc == DASH_OK && i < 2 * nu; ++i)
         if (!mkev(&ev[i])) rc = DASH_ERR_CUDA;
-    // the helper streams start after the work already queued on `stream`
-    if (rc == DASH_OK && (cudaEventRecord(start, s) != cudaSuccess || cudaStreamWaitEvent(sin, start, 0) != cudaSuccess ||
+    // the helper streams start after the work already queued on `stream`, which clears the
+    // call's header first
+    if (rc == DASH_OK && (cudaMemsetAsync(ws0, 0, sizeof(WsHeader), s) != cudaSuccess ||
+                          cudaEventRecord(start, s) != cudaSuccess || cudaStreamWaitEvent(sin, start, 0) != cudaSuccess ||
                           cudaStreamWaitEvent(sout, start, 0) != cudaSuccess))
         rc = DASH_ERR_CUDA;
+    for (int i = 0; rc == DASH_OK && i < ns; ++i)
+        if (cudaStreamWaitEvent(sc[i], start, 0) != cudaSuccess) rc = DASH_ERR_CUDA;
     for (int u = 0; rc == DASH_OK && u < nu; ++u) {
         const int gi = u / nch, c = u % nch, h0 = c * gc, hc = std::min(gc, G - h0);
         const size_t ok = (size_t)gi * kg, oq = (size_t)gi * qg + (size_t)h0 * hb, nq = (size_t)hc * hb;
+        cudaStream_t cs = sc[u % ns];                                 // units on one stream share a slice
+        char* const wsi = unit_ws(u % ns);
+        // copies in are in order on `sin`: a unit's event also covers its group's keys and values
         if ((c == 0 && (!cp(atw(k_dev, ok), at(k_host, ok), kg, cudaMemcpyHostToDevice, sin) ||
                         !cp(atw(v_dev, ok), at(v_host, ok), kg, cudaMemcpyHostToDevice, sin))) ||
             !cp(atw(q_dev, oq), at(q_host, oq), nq, cudaMemcpyHostToDevice, sin) ||
-            cudaEventRecord(ev[2 * u], sin) != cudaSuccess || cudaStreamWaitEvent(s, ev[2 * u], 0) != cudaSuccess) {
+            cudaEventRecord(ev[2 * u], sin) != cudaSuccess || cudaStreamWaitEvent(cs, ev[2 * u], 0) != cudaSuccess) {
             rc = DASH_ERR_CUDA;
             break;
         }
         rc = dash_prefill(atw(q_dev, oq), atw(k_dev, ok), atw(v_dev, ok), atw(out_dev, oq), 1, hc, 1, T, d, block,
-                          alpha, coarse_scale, workspace, ws_bytes, stream);
+                          alpha, coarse_scale, wsi, wsu, reinterpret_cast<dash_stream_t>(cs));
         if (rc != DASH_OK) break;
-        if (cudaEventRecord(ev[2 * u + 1], s) != cudaSuccess || cudaStreamWaitEvent(sout, ev[2 * u + 1], 0) != cudaSuccess ||
+        accumulate_header_kernel<<<1, 32, 0, cs>>>(reinterpret_cast<WsHeader*>(ws0), reinterpret_cast<const WsHeader*>(wsi));
+        if (cudaGetLastError() != cudaSuccess || cudaEventRecord(ev[2 * u + 1], cs) != cudaSuccess ||
+            cudaStreamWaitEvent(sout, ev[2 * u + 1], 0) != cudaSuccess ||
             !cp(atw(out_host, oq), at(out_dev, oq), nq, cudaMemcpyDeviceToHost, sout))
             rc = DASH_ERR_CUDA;
     }
-    // `stream` waits for everything issued on the helper streams, also after an error
+    // `stream` waits for everything issued on the helper streams, also after an error (each
+    // compute stream's work precedes a copy out it ordered, or is joined here)
     if (sout && fin && cudaEventRecord(fin, sout) == cudaSuccess) cudaStreamWaitEvent(s, fin, 0);
     if (sin && start && cudaEventRecord(start, sin) == cudaSuccess) cudaStreamWaitEvent(s, start, 0);
+    for (int i = 0; i < ns; ++i)
+        if (sc[i] && start && cudaEventRecord(start, sc[i]) == cudaSuccess) cudaStreamWaitEvent(s, start, 0);
     // destroying a stream or event with work pending releases it once the work completes
     for (int i = 0; ev && i < 2 * nu; ++i)
         if (ev[i]) cudaEventDestroy(ev[i]);
@@ -302,6 +344,8 @@ int dash_prefill_host(const void* q_host, const void* k_host, const void* v_host
     if (fin) cudaEventDestroy(fin);
     if (sin) cudaStreamDestroy(sin);
     if (sout) cudaStreamDestroy(sout);
+    for (int i = 0; i < ns; ++i)
+        if (sc[i]) cudaStreamDestroy(sc[i]);
     return rc;
 }
 

@@ -138,16 +138,23 @@ def test_host_entry_point_matches_device_path():
 
 def test_host_entry_point_head_chunks():
     # 4 MiB of queries per head: the host entry point cuts each KV group (4 heads) into chunks
-    # of 2 heads, each its own prefill on the group's keys and values
+    # of 2 heads, each its own prefill on the group's keys and values; the units run on
+    # several compute streams at once
     wl, (q, k, v) = inputs.make("16k", Hq=8, Hkv=2)
     cs = calibrated_scale("16k")
     qd, kd, vd, out, ws = gpu_prefill(q, k, v, 1.5, cs)
+    st_dev = da.dash_prefill_stats(ws)
     qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
     oh = torch.empty_like(q).pin_memory()
     da.dash_prefill_host(qh, kh, vh, oh, torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd),
                          torch.empty_like(out), 1.5, cs, ws)
     torch.cuda.synchronize()
+    # the units run on several streams with their own workspace slices; the call's header
+    # holds the OR of their status bits and the sums of their statistics
     assert da.dash_get_device_status(ws) == 0
+    st = da.dash_prefill_stats(ws)
+    assert st["scored_pairs"] == st_dev["scored_pairs"]
+    assert st["selected_pairs"] == st_dev["selected_pairs"]
     compare_out(oh.float().numpy(), out.float().cpu().numpy(), "host chunks against the device path")
     rows = stratified_rows(1, 8, wl.T, 512, seed=17)
     ref, _, _ = oracle.forward_rows(oracle.gather_q_rows(q, rows), k, v, rows, 8, 64, 1.5, cs)
