@@ -84,6 +84,16 @@ def test_argument_errors_return_before_launch(L):
     assert L.dash_select_dump(fake, fake, fake, -1, 4, fake, fake, fake, fake, 1, 1, 1, 128, 64, 64,
                               1.5, 1.0, None) == -1
     assert L.dash_get_device_status(None, None) == -1
+    # host-buffer prefill: host pointers, shape, device pointers, parameters, workspace
+    h = lambda *a: L.dash_prefill_host(*a)
+    assert h(None, fake, fake, fake, fake, fake, fake, fake, 1, 2, 1, 128, 64, 64, 1.5, 1.0, fake, big, None) == -1
+    assert h(fake, fake, fake, None, fake, fake, fake, fake, 1, 2, 1, 128, 64, 64, 1.5, 1.0, fake, big, None) == -1
+    assert h(fake, fake, fake, fake, fake, fake, fake, fake, 1, 3, 2, 128, 64, 64, 1.5, 1.0, fake, big, None) == -2
+    assert h(fake, fake, fake, fake, fake, fake, fake, fake, 1, 2, 1, 128, 64, 32, 1.5, 1.0, fake, big, None) == -2
+    assert h(fake, fake, fake, fake, None, fake, fake, fake, 1, 2, 1, 128, 64, 64, 1.5, 1.0, fake, big, None) == -1
+    assert h(fake, fake, fake, fake, fake, fake, fake, fake, 1, 2, 1, 128, 64, 64, 1.0, 1.0, fake, big, None) == -1
+    assert h(fake, fake, fake, fake, fake, fake, fake, fake, 1, 2, 1, 128, 64, 64, 1.5, 1.0, None, big, None) == -5
+    assert h(fake, fake, fake, fake, fake, fake, fake, fake, 1, 2, 1, 128, 64, 64, 1.5, 1.0, fake, 16, None) == -5
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
