@@ -31,6 +31,16 @@
  *     variable DASH_DEBUG_SOLVE_CAP=n (1 <= n < 64), read at each call, lowers that cap to
  *     n iterations so that the status path can be exercised with a normal launch; rows
  *     whose solve is cut short get an inexact threshold.
+ *   - Other environment switches (all off by default; they choose among kernels that compute
+ *     the same result, for comparisons):
+ *       DASH_TILES=positions      (read at each prefill) the fine stage runs tiles of
+ *                                 consecutive positions instead of selection-ordered tiles;
+ *       DASH_ENTMAX_INIT=histogram (read at each call) the threshold solves start at a
+ *                                 histogram edge below the root (AdaSplash-2's start) instead
+ *                                 of the default subset root (prefill) or u = -1 (decode);
+ *       DASH_FINE_KERNEL=mma, DASH_BWD_KERNEL=mma (read once per process) the prefill's fine
+ *                                 stage, or its backward, on the mma.sync kernels that serve
+ *                                 more than 16 query heads per KV head.
  *   - No C++ exception crosses this interface.
  */
 #ifndef DASH_ATTN_H
